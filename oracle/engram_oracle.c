@@ -1,0 +1,271 @@
+/*
+ * engram_oracle.c -- plain, slow, single-threaded CPU definition of the
+ * Engram conditional-memory forward (lookup and gate).
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load this file.  It shares no code, header, table or
+ * constant generator with the CUDA path, and it includes none of its files.
+ *
+ * Every step follows "Conditional Memory via Scalable Lookup: A New Axis of
+ * Sparsity for Large Language Models" (DeepSeek-AI & Peking University),
+ * section 2, in the order the paper gives it:
+ *
+ *   compress   x'_t = P(x_t)                          section 2.2, "Tokenizer compression"
+ *   n-grams    g_{t,n} = (x'_{t-n+1}, ..., x'_t)      section 2.2
+ *   hash       z_{t,n,k} = phi_{n,k}(g_{t,n})         section 2.2, Eq. (1)
+ *   gather     e_t = concat_n concat_k E_{n,k}[z]     section 2.2, Eq. (1)-(2)
+ *   project    k_t = W_K e_t,  v_t = W_V e_t          section 2.3, Eq. (3)
+ *   gate       alpha_t = sigmoid(RMSNorm(h_t) . RMSNorm(k_t) / sqrt(d))
+ *                                                     section 2.3, Eq. (4);
+ *                                                     per branch, section 2.4, Eq. (6)
+ *   output     out = h + alpha * v                    section 2.3 (gated value,
+ *                                                     residual H <- H + Y) and
+ *                                                     section 2.4 (u = alpha (W_V e))
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - phi is called a "lightweight multiplicative-XOR hash" and nothing more.
+ *    The form used: x = 0; for j < n: x ^= c[t-j] * m[s][j] (wrapping 64-bit),
+ *    z = x mod p[s].  j = 0 is the current token.
+ *  - multipliers m[s][j] = splitmix64_next() | 1, drawn from one SplitMix64
+ *    stream seeded with the hash seed, slot s ascending, then j ascending,
+ *    max_order draws per slot.  SplitMix64 is the published generator of
+ *    Steele, Lea and Flood, "Fast splittable pseudorandom number generators"
+ *    (OOPSLA 2014), in the 64-bit mixing form of Vigna's reference code.
+ *  - table sizes: "prime size" only.  The primes are the ascending primes
+ *    >= a target, one per slot, slot order = order ascending, head ascending.
+ *  - positions before the start of a sequence read the pad id; n-grams never
+ *    cross sequences.
+ *  - RMSNorm(x) = x / sqrt(mean(x^2) + eps) * w, with a learnable weight w
+ *    per branch for the query and for the key; the key is normalised after
+ *    the projection (Eq. 4), the scale is 1/sqrt(d) with d the hidden size.
+ *  - ShortConv (Eq. 5) is zero-initialised in the paper (Table 5), so at
+ *    initialisation its output equals the gated value and out = h + alpha v.
+ *
+ * Floating point: every sum is accumulated in double over the exact values of
+ * the fp32 or bf16 inputs.  bf16 outputs are rounded to nearest-even
+ * (through float: double -> float -> bf16).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define EO_F32 0
+#define EO_BF16 1
+
+/* ---------------------------------------------------------------- SplitMix64 */
+
+uint64_t eo_splitmix64_next(uint64_t *state)
+{
+    uint64_t z;
+    *state += 0x9E3779B97F4A7C15ULL;
+    z = *state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+    return z ^ (z >> 31);
+}
+
+/* mult[s * max_order + j], s < num_tables, j < max_order; every value odd. */
+void eo_hash_multipliers(uint64_t seed, int32_t num_tables, int32_t max_order, uint64_t *mult)
+{
+    uint64_t st = seed;
+    int32_t s, j;
+    for (s = 0; s < num_tables; ++s)
+        for (j = 0; j < max_order; ++j)
+            mult[(int64_t)s * max_order + j] = eo_splitmix64_next(&st) | 1ULL;
+}
+
+/* ------------------------------------------------------------------- primes */
+
+int eo_is_prime(int64_t n)
+{
+    int64_t f;
+    if (n < 2) return 0;
+    if (n < 4) return 1;
+    if (n % 2 == 0) return 0;
+    for (f = 3; f * f <= n; f += 2)
+        if (n % f == 0) return 0;
+    return 1;
+}
+
+/* The num_tables ascending primes >= target.  Returns 0, or -1 if target < 2. */
+int eo_table_primes(int64_t target, int32_t num_tables, int64_t *primes)
+{
+    int64_t n = target;
+    int32_t s;
+    if (target < 2) return -1;
+    for (s = 0; s < num_tables; ++s) {
+        while (!eo_is_prime(n)) ++n;
+        primes[s] = n;
+        ++n;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------ compression */
+
+/* c[i] = map[x[i]].  Returns the number of tokens outside [0, V) (their c is -1). */
+int64_t eo_compress(const int32_t *x, int64_t n, const int32_t *map, int32_t V, int32_t *c)
+{
+    int64_t i, bad = 0;
+    for (i = 0; i < n; ++i) {
+        if (x[i] < 0 || x[i] >= V) { c[i] = -1; ++bad; continue; }
+        c[i] = map[x[i]];
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------ hashing */
+
+/*
+ * z[(b * (T - t_begin) + (t - t_begin)) * S + s] for t in [t_begin, T),
+ * slot s = order_index * heads + head.  c is the compressed sequence [B, T].
+ */
+void eo_hash(const int32_t *c, int32_t B, int32_t T, int32_t t_begin, int32_t pad,
+             int32_t num_orders, const int32_t *orders, int32_t heads,
+             const uint64_t *mult, int32_t max_order, const int64_t *primes, int64_t *z)
+{
+    int32_t S = num_orders * heads;
+    int32_t b, t, oi, k, j;
+    for (b = 0; b < B; ++b) {
+        for (t = t_begin; t < T; ++t) {
+            int64_t row = (int64_t)b * (T - t_begin) + (t - t_begin);
+            for (oi = 0; oi < num_orders; ++oi) {
+                int32_t n = orders[oi];
+                for (k = 0; k < heads; ++k) {
+                    int32_t s = oi * heads + k;
+                    uint64_t x = 0;
+                    for (j = 0; j < n; ++j) {
+                        int32_t pos = t - j;
+                        int32_t tok = pos >= 0 ? c[(int64_t)b * T + pos] : pad;
+                        x ^= (uint64_t)(uint32_t)tok * mult[(int64_t)s * max_order + j];
+                    }
+                    z[row * S + s] = (int64_t)(x % (uint64_t)primes[s]);
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ gather */
+
+/* e[r][s * d_head + i] = tables[s][z[r][s]][i], copied byte for byte. */
+void eo_gather(const void *const *tables, int32_t elem_bytes, int32_t d_head,
+               const int64_t *z, int64_t rows, int32_t S, void *e)
+{
+    int64_t r;
+    int32_t s;
+    size_t row_bytes = (size_t)d_head * (size_t)elem_bytes;
+    for (r = 0; r < rows; ++r)
+        for (s = 0; s < S; ++s) {
+            const char *src = (const char *)tables[s] + (size_t)z[r * S + s] * row_bytes;
+            char *dst = (char *)e + ((size_t)r * S + s) * row_bytes;
+            memcpy(dst, src, row_bytes);
+        }
+}
+
+/* --------------------------------------------------------- element access */
+
+static double eo_load(const void *p, int32_t dtype, int64_t i)
+{
+    if (dtype == EO_F32) return (double)((const float *)p)[i];
+    {
+        uint32_t u = (uint32_t)((const uint16_t *)p)[i] << 16;
+        float f;
+        memcpy(&f, &u, 4);
+        return (double)f;
+    }
+}
+
+static uint16_t eo_bf16_rne(double v)
+{
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x40);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------- projection */
+
+/* y[r][o] = sum_j w[o][j] * e[r][j], accumulated in double (Eq. 3). */
+void eo_project(const void *e, int32_t dtype, int64_t rows, int32_t d_mem,
+                const void *w, int32_t n_out, double *y)
+{
+    int64_t r;
+    int32_t o, j;
+    for (r = 0; r < rows; ++r)
+        for (o = 0; o < n_out; ++o) {
+            double acc = 0.0;
+            for (j = 0; j < d_mem; ++j)
+                acc += eo_load(w, dtype, (int64_t)o * d_mem + j) * eo_load(e, dtype, r * d_mem + j);
+            y[r * n_out + o] = acc;
+        }
+}
+
+/* ------------------------------------------------------------------- gate */
+
+/*
+ * alpha = sigmoid( RMSNorm_q(h) . RMSNorm_k(k) / sqrt(d) )        (Eq. 4)
+ * RMSNorm_w(x)_i = x_i / sqrt(mean(x^2) + eps) * w_i.
+ */
+double eo_gate(const double *h, const double *k, const float *wq, const float *wk,
+               int32_t d, double eps)
+{
+    double sh = 0.0, sk = 0.0, dot = 0.0, rh, rk, s;
+    int32_t i;
+    for (i = 0; i < d; ++i) { sh += h[i] * h[i]; sk += k[i] * k[i]; }
+    rh = 1.0 / sqrt(sh / d + eps);
+    rk = 1.0 / sqrt(sk / d + eps);
+    for (i = 0; i < d; ++i) {
+        double q = h[i] * rh * (double)wq[i];
+        double kn = k[i] * rk * (double)wk[i];
+        dot += q * kn;
+    }
+    s = dot / sqrt((double)d);
+    return 1.0 / (1.0 + exp(-s));
+}
+
+/* ---------------------------------------------------------------- forward */
+
+/*
+ * Projection, gate and output for `rows` rows whose memory vectors e are given
+ * (Eq. 3, Eq. 4 / Eq. 6, gated residual).
+ *   e     [rows, d_mem]          dtype
+ *   w_k   [M, d, d_mem]          dtype   (one key projection per branch)
+ *   w_v   [d, d_mem]             dtype   (shared value projection)
+ *   wq,wk [M, d]                 float   (RMSNorm weights of query and key)
+ *   h     [rows, M, d]           dtype
+ *   alpha [rows, M]              double  (out)
+ *   delta [rows, M, d]           double  (out; alpha * v; may be NULL)
+ *   out   [rows, M, d]           dtype   (out; h + alpha * v rounded to dtype)
+ * Scratch: kbuf [M * d], vbuf [d], hbuf [d] doubles supplied by the caller.
+ */
+void eo_project_gate(const void *e, int32_t dtype, int64_t rows, int32_t d_mem,
+                     const void *w_k, const void *w_v, const float *wq, const float *wk,
+                     int32_t M, int32_t d, double eps, const void *h,
+                     double *alpha, double *delta, void *out,
+                     double *kbuf, double *vbuf, double *hbuf)
+{
+    int64_t r;
+    int32_t m, i;
+    for (r = 0; r < rows; ++r) {
+        const char *er = (const char *)e + (size_t)r * d_mem * (dtype == EO_F32 ? 4 : 2);
+        eo_project(er, dtype, 1, d_mem, w_k, M * d, kbuf);
+        eo_project(er, dtype, 1, d_mem, w_v, d, vbuf);
+        for (m = 0; m < M; ++m) {
+            int64_t base = (r * M + m) * (int64_t)d;
+            double a;
+            for (i = 0; i < d; ++i) hbuf[i] = eo_load(h, dtype, base + i);
+            a = eo_gate(hbuf, kbuf + (int64_t)m * d, wq + (int64_t)m * d, wk + (int64_t)m * d, d, eps);
+            alpha[r * M + m] = a;
+            for (i = 0; i < d; ++i) {
+                double dl = a * vbuf[i];
+                double o = hbuf[i] + dl;
+                if (delta) delta[base + i] = dl;
+                if (dtype == EO_F32) ((float *)out)[base + i] = (float)o;
+                else ((uint16_t *)out)[base + i] = eo_bf16_rne(o);
+            }
+        }
+    }
+}

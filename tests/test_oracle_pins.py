@@ -1,0 +1,256 @@
+"""Pins of the CPU oracle against what the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: a published
+test sequence, hand-derived worked examples, closed forms of Eq. (4), an
+independent library (sympy, numpy indexing, torch fp64 matmul), brute-force
+enumeration and the uniform-hash expectation.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import sympy
+import torch
+
+import oracle
+
+
+def _sig(x):
+    return 1.0 / (1.0 + math.exp(-x))
+
+
+# --------------------------------------------------------------- SplitMix64
+
+def test_splitmix64_published_sequence(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "splitmix64_seed1234567.json")))
+    assert oracle.splitmix64_stream(g["seed"], 5) == [int(v) for v in g["outputs"]]
+
+
+def test_multipliers_are_the_stream_forced_odd():
+    seed, S, J = 1234567, 3, 3
+    m = oracle.hash_multipliers(seed, S, J)
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                    "splitmix64_seed1234567.json")))
+    first = [int(v) | 1 for v in g["outputs"]]
+    assert [int(x) for x in m.reshape(-1)[:5]] == first
+    assert all(int(x) & 1 for x in m.reshape(-1))
+    assert len({int(x) for x in m.reshape(-1)}) == S * J
+
+
+# ------------------------------------------------------------------- primes
+
+@pytest.mark.parametrize("target,S", [(10007, 8), (1 << 20, 16), (1 << 24, 16), (2, 5), (90, 4)])
+def test_table_primes_match_sympy(target, S):
+    p = oracle.table_primes(target, S)
+    want, n = [], target - 1
+    for _ in range(S):
+        n = sympy.nextprime(n)
+        want.append(n)
+    assert [int(x) for x in p] == want
+
+
+def test_known_primes_above_powers_of_two():
+    # smallest primes above 2^20 and 2^24 are 2^20 + 7 and 2^24 + 43
+    assert int(oracle.table_primes(1 << 20, 1)[0]) == (1 << 20) + 7
+    assert int(oracle.table_primes(1 << 24, 1)[0]) == (1 << 24) + 43
+    assert oracle.is_prime(10007) and not oracle.is_prime(10005) and not oracle.is_prime(1)
+
+
+# -------------------------------------------------------------- compression
+
+def test_compress_lookup_and_range_error():
+    m = np.array([2, 0, 1, 0], dtype=np.int32)
+    x = np.array([[0, 1, 2, 3, 3]], dtype=np.int32)
+    assert oracle.compress(x, m).tolist() == [[2, 0, 1, 0, 0]]
+    with pytest.raises(ValueError):
+        oracle.compress(np.array([[4]], dtype=np.int32), m)
+    with pytest.raises(ValueError):
+        oracle.compress(np.array([[-1]], dtype=np.int32), m)
+
+
+# ------------------------------------------------------------------ hashing
+
+def test_hash_worked_examples(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "hash_worked_examples.json")))
+    for case in g["cases"]:
+        mult = np.array([[int(v) for v in row] for row in case["mult"]], dtype=np.uint64)
+        z = oracle.hash_indices(np.array(case["c"], dtype=np.int32), case["pad"], case["orders"],
+                                case["heads"], mult, np.array(case["primes"], dtype=np.int64))
+        assert z.tolist() == case["z"], case["name"]
+
+
+def test_hash_t_begin_emits_suffix_rows_only():
+    rng = np.random.default_rng(0)
+    c = rng.integers(0, 50, size=(3, 7)).astype(np.int32)
+    mult = oracle.hash_multipliers(99, 4, 3)
+    primes = oracle.table_primes(211, 4)
+    full = oracle.hash_indices(c, 50, (2, 3), 2, mult, primes).reshape(3, 7, 4)
+    tail = oracle.hash_indices(c, 50, (2, 3), 2, mult, primes, t_begin=5).reshape(3, 2, 4)
+    assert np.array_equal(full[:, 5:], tail)
+
+
+def test_hash_invariants_identical_ngrams_same_rows():
+    rng = np.random.default_rng(1)
+    B, T, V = 4, 200, 12
+    c = rng.integers(0, V, size=(B, T)).astype(np.int32)
+    mult = oracle.hash_multipliers(7, 6, 3)
+    primes = oracle.table_primes(1009, 6)
+    z = oracle.hash_indices(c, V, (2, 3), 3, mult, primes).reshape(B, T, 6)
+    assert (z >= 0).all() and (z < primes[None, None, :]).all()
+    padded = np.concatenate([np.full((B, 2), V, np.int32), c], axis=1)
+    seen = {}
+    for b in range(B):
+        for t in range(T):
+            g2 = tuple(padded[b, t + 1:t + 3])
+            g3 = tuple(padded[b, t:t + 3])
+            for key, val in (((2,) + g2, tuple(z[b, t, :3])), ((3,) + g3, tuple(z[b, t, 3:]))):
+                assert seen.setdefault(key, val) == val
+    # different heads of one order use different multipliers, so they disagree somewhere
+    assert (z[:, :, 0] != z[:, :, 1]).any()
+
+
+def _all_ngrams(V, n):
+    grid = np.stack(np.meshgrid(*[np.arange(V)] * n, indexing="ij"), -1).reshape(-1, n)
+    return grid.astype(np.int32)
+
+
+@pytest.mark.parametrize("n,p", [(2, 101), (2, 1009), (3, 100003), (3, 1009)])
+def test_hash_collisions_brute_force_and_uniform_expectation(n, p):
+    V = 41  # 40 compressed ids and the pad id
+    seqs = _all_ngrams(V, n)
+    D = seqs.shape[0]
+    mult = oracle.hash_multipliers(20261202, 1, 3)
+    z = oracle.hash_indices(seqs, V - 1, (n,), 1, mult, np.array([p], np.int64),
+                            t_begin=n - 1)[:, 0]
+    # brute-force enumeration of colliding pairs
+    pairs = 0
+    for i in range(0, D, 4096):
+        blk = z[i:i + 4096]
+        pairs += int((blk[:, None] == z[None, :]).sum()) - blk.size
+    pairs //= 2
+    counts = np.bincount(z, minlength=p)
+    assert pairs == int((counts * (counts - 1) // 2).sum())
+    # uniform hashing: E[pairs] = C(D,2)/p, Var ~ E (1 - 1/p)
+    exp_pairs = D * (D - 1) / 2 / p
+    assert abs(pairs - exp_pairs) < 5 * math.sqrt(exp_pairs * (1 - 1 / p)) + 1
+    occ = int((counts > 0).sum())
+    exp_occ = p * (1 - (1 - 1 / p) ** D)
+    assert abs(occ - exp_occ) < 5 * math.sqrt(max(exp_occ * (1 - exp_occ / p), 1.0)) + 2
+
+
+# ------------------------------------------------------------------- gather
+
+@pytest.mark.parametrize("dtype", [np.float32, np.uint16])
+def test_gather_matches_numpy_indexing(dtype):
+    rng = np.random.default_rng(2)
+    S, d_h, rows = 5, 7, 33
+    tabs = [rng.integers(0, 60000, size=(97 + s, d_h)).astype(dtype) for s in range(S)]
+    z = np.stack([rng.integers(0, 97 + s, size=rows) for s in range(S)], 1)
+    e = oracle.gather(tabs, z)
+    want = np.concatenate([tabs[s][z[:, s]] for s in range(S)], axis=1)
+    assert e.dtype == want.dtype and np.array_equal(e, want)
+    with pytest.raises(IndexError):
+        oracle.gather(tabs, np.full((1, S), 97 + S, dtype=np.int64))
+
+
+# --------------------------------------------------------------- projection
+
+def _bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_project_matches_torch_fp64():
+    g = torch.Generator().manual_seed(3)
+    e = torch.randn(9, 40, generator=g)
+    w = torch.randn(13, 40, generator=g)
+    y = oracle.project(e.numpy(), w.numpy())
+    ref = (e.double() @ w.double().T).numpy()
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-13)
+    yb = oracle.project(_bf16_bits(e), _bf16_bits(w))
+    refb = (e.bfloat16().double() @ w.bfloat16().double().T).numpy()
+    assert np.allclose(yb, refb, rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------------------------- gate
+
+def test_gate_worked_examples(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "gate_worked_examples.json")))
+    for case in g["cases"]:
+        s = eval(case["s"], {"sqrt": math.sqrt})
+        a = oracle.gate(np.array(case["h"], float), np.array(case["k"], float),
+                        np.array(case["wq"], np.float32), np.array(case["wk"], np.float32),
+                        case["eps"])
+        assert abs(a - _sig(s)) < 1e-14, case["name"]
+
+
+def test_gate_scale_invariance_and_range():
+    rng = np.random.default_rng(4)
+    d = 64
+    h, k = rng.normal(size=d), rng.normal(size=d)
+    wq = (1 + 0.1 * rng.normal(size=d)).astype(np.float32)
+    wk = (1 + 0.1 * rng.normal(size=d)).astype(np.float32)
+    a = oracle.gate(h, k, wq, wk, 0.0)
+    assert 0.0 < a < 1.0
+    assert abs(oracle.gate(5.0 * h, 0.25 * k, wq, wk, 0.0) - a) < 1e-14
+    assert abs(oracle.gate(-h, k, wq, wk, 0.0) - (1 - a)) < 1e-14
+
+
+# --------------------------------------------------------------- full gate
+
+def _small_problem(M=2, d=16, dm=24, rows=5, seed=5, bf16=False):
+    g = torch.Generator().manual_seed(seed)
+    e = torch.randn(rows, dm, generator=g) * 0.5
+    wk = torch.randn(M, d, dm, generator=g) / math.sqrt(dm)
+    wv = torch.randn(d, dm, generator=g) / math.sqrt(dm)
+    h = torch.randn(rows, M, d, generator=g)
+    nq = 1 + 0.1 * torch.randn(M, d, generator=g)
+    nk = 1 + 0.1 * torch.randn(M, d, generator=g)
+    if bf16:
+        cv = _bf16_bits
+    else:
+        cv = lambda t: t.float().numpy()
+    return cv(e), cv(wk), cv(wv), nq.numpy(), nk.numpy(), cv(h), (e, wk, wv, h)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_project_gate_against_torch_fp64(bf16):
+    e, wk, wv, nq, nk, h, raw = _small_problem(bf16=bf16)
+    alpha, delta, out = oracle.project_gate(e, wk, wv, nq, nk, h, 1e-6)
+    conv = (lambda t: t.bfloat16().double()) if bf16 else (lambda t: t.double())
+    E, WK, WV, H = [conv(t) for t in raw]
+    k = torch.einsum("rj,mij->rmi", E, WK)
+    v = E @ WV.T
+    d = H.shape[-1]
+    qn = H / torch.sqrt(H.pow(2).mean(-1, keepdim=True) + 1e-6) * torch.from_numpy(nq).double()
+    kn = k / torch.sqrt(k.pow(2).mean(-1, keepdim=True) + 1e-6) * torch.from_numpy(nk).double()
+    a_ref = torch.sigmoid((qn * kn).sum(-1) / math.sqrt(d))
+    assert np.allclose(alpha, a_ref.numpy(), rtol=1e-12, atol=1e-12)
+    d_ref = a_ref[..., None] * v[:, None, :]
+    assert np.allclose(delta, d_ref.numpy(), rtol=1e-12, atol=1e-12)
+    o_ref = H + d_ref
+    if bf16:
+        want = _bf16_bits(o_ref.float())
+        assert np.array_equal(out, want)
+    else:
+        assert np.array_equal(out, o_ref.float().numpy())
+
+
+def test_project_gate_zero_value_projection_keeps_h():
+    e, wk, wv, nq, nk, h, _ = _small_problem()
+    alpha, delta, out = oracle.project_gate(e, wk, np.zeros_like(wv), nq, nk, h, 1e-6)
+    assert np.array_equal(out, h) and (delta == 0).all()
+    assert ((alpha > 0) & (alpha < 1)).all()
+
+
+def test_project_gate_shared_value_per_branch():
+    # Eq. (6): branches share W_V; identical W_K and h in both branches give equal alpha
+    e, wk, wv, nq, nk, h, _ = _small_problem(M=2)
+    wk[1] = wk[0]
+    h[:, 1] = h[:, 0]
+    nq[1] = nq[0]
+    nk[1] = nk[0]
+    alpha, delta, _ = oracle.project_gate(e, wk, wv, nq, nk, h, 1e-6)
+    assert np.array_equal(alpha[:, 0], alpha[:, 1])
+    assert np.array_equal(delta[:, 0], delta[:, 1])
