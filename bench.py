@@ -1,0 +1,417 @@
+"""Throughput of the Engram forward (hash + gather + projections + gate) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one engram_forward over one batch of the prefill workload
+(B=8 sequences x T=4096 tokens, 16 tables of ~2^20 rows x 80 bf16, d=2560,
+M=1): compress, hash, gather, key and value projections, gate, residual.
+`value` is tokens/s with every input resident in HBM; `e2e` is the same call
+with the inputs in pinned host memory, copied in and the output copied out
+inside the timed region.  Inputs are larger than L2 (h 168 MB in, 168 MB out,
+tables 2.7 GB), so no L2 flush runs between steps.
+
+With N > 1 (torchrun), every rank runs its own replica on its own seeded batch
+(the forward has no cross-rank exchange); the time is the max over ranks.
+
+--impl reference times the CPU oracle (plain single-threaded C, fp64) on a
+bounded sample of the same workload: the reference arm of this build.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Engram fwd tokens/s (hash+gather+gate); gather GB/s as % of HBM peak"
+WORKLOAD = "prefill_bf16"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ the workload
+
+def setup(rank: int, device):
+    import torch
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    from hashed_gram_embedding_compress_b200 import synth
+
+    sh = synth.SHAPES[WORKLOAD]
+    seeds = synth.stream_seeds(sh, extra=rank)
+    tokens = synth.make_tokens(sh, seeds)
+    comp_map = synth.make_comp_map(sh, seeds)
+    cfg = eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=comp_map, orders=sh.orders,
+                         heads=sh.heads, d_head=sh.d_head, d_hidden=sh.d_hidden,
+                         branches=sh.branches, dtype=sh.dtype, eps=1e-6,
+                         table_rows_target=sh.rows_target, hash_seed=synth.make_hash_seed(seeds))
+    m = eg.Engram(cfg)
+    primes, _ = m.hash_params()
+    tables = synth.make_tables([int(p) for p in primes], sh.d_head, sh.dtype, seeds, device=device)
+    w_k, w_v, nq, nk = synth.make_weights(sh, seeds)
+    w_k, w_v, nq, nk = w_k.to(device), w_v.to(device), nq.to(device), nk.to(device)
+    m.set_params(tables, w_k, w_v, nq, nk)
+    h = synth.make_hidden(sh, seeds, device=device)
+    m.reserve(sh.rows_out)
+    return dict(sh=sh, m=m, tokens=tokens, comp_map=comp_map, tables=tables, w_k=w_k, w_v=w_v,
+                nq=nq, nk=nk, h=h, seeds=seeds, hash_seed=synth.make_hash_seed(seeds),
+                primes=primes)
+
+
+def algorithmic(sh):
+    """Per-step algorithmic work (measurement section)."""
+    R, S, dm, d, M = sh.rows_out, sh.num_tables, sh.d_mem, sh.d_hidden, sh.branches
+    elt = 2 if sh.dtype == "bf16" else 4
+    row_bytes = sh.d_head * elt
+    gather_bytes = R * S * (row_bytes * 2 + 8)       # rows read, e written, indices read
+    hash_bytes = R * S * 8 + sh.B * sh.T * 4         # indices written, tokens read
+    gemm_flops = 2.0 * R * dm * (M * d + d)          # [W_K^(1..M); W_V] e
+    # key kernel: e read, W_K read, h read; value kernel: e, W_V, h read, out written
+    gemm_bytes = (2 * R * dm * elt + (M * d + d) * dm * elt + 3 * R * M * d * elt)
+    return dict(gather_bytes=gather_bytes, hash_bytes=hash_bytes, gemm_flops=gemm_flops,
+                gemm_bytes=gemm_bytes)
+
+
+def kernel_traffic():
+    """DRAM bytes per launch of the projection kernel from a committed ncu
+    capture, or None when the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = os.path.join(ROOT, "hashed_gram_embedding_compress_b200", "csrc", "k_proj_gate_sm100.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("source_sha256_16") != h:
+        return None
+    return d.get("proj_gate_bytes_per_step")
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    P = setup(rank, device)
+    sh, m = P["sh"], P["m"]
+    tok_d = P["tokens"].to(device)
+    h = P["h"]
+    out = torch.empty_like(h)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m.forward(tok_d, h, out, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if m.check_errors(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = m.kernel_launches()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for k in range(K):
+            m.profile_next_forward(evs[k])
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = m.kernel_launches() - launches0
+    ms = t0.elapsed_time(t1)
+    if dist:
+        tt = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    stage = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)]
+    st_mean = [sum(s[i] for s in stage) / K for i in range(4)]  # hash, gather, key, value (ms)
+    if m.check_errors(stream) != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    # ------------------------------------------------------------- e2e
+    E = max(1, args.e2e_steps)
+    tok_h = P["tokens"].pin_memory()
+    h_h = h.cpu().pin_memory()
+    out_h = torch.empty_like(h_h).pin_memory()
+    tok_buf = torch.empty_like(tok_d)
+    h_buf = torch.empty_like(h)
+    out_buf = torch.empty_like(h)
+
+    def e2e_step():
+        tok_buf.copy_(tok_h, non_blocking=True)
+        h_buf.copy_(h_h, non_blocking=True)
+        m.forward(tok_buf, h_buf, out_buf, stream=stream)
+        out_h.copy_(out_buf, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+    if rank != 0:
+        return None
+
+    hbm, tflops, peak_kind = load_peaks()
+    A = algorithmic(sh)
+    tokens_per_step = sh.rows_out
+    value = tokens_per_step * world * K / (ms / 1e3)
+    gemm_s = (st_mean[2] + st_mean[3]) / 1e3
+    gemm_tflops = A["gemm_flops"] / gemm_s / 1e12
+    gather_gbs = A["gather_bytes"] / (st_mean[1] / 1e3) / 1e9
+    traffic = kernel_traffic()
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "prefill_bf16: B=8 x T=4096 tokens, vocab 32768->25231, orders {2,3} x 8 "
+                        "heads, 16 tables of primes >= 2^20 rows x 80 bf16 (d_mem 1280), d=2560, "
+                        "M=1, fp32 accumulate",
+            "global_batch": tokens_per_step * world,
+            "seq_len": sh.T,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "no flush: inputs larger than L2 (h 168 MB read, out 168 MB written, "
+                  "tables 2.7 GB)",
+        },
+        "roofline": {
+            "kernel": "proj_gate_kernel (tcgen05 key + value launches)",
+            "bound": "tensor",
+            "achieved": gemm_tflops,
+            "peak": tflops,
+            "unit": "TFLOP/s",
+            "frac": gemm_tflops / tflops,
+            "traffic": traffic,
+            "peak_source": "%s bf16 burst" % peak_kind,
+        },
+        "gather": {
+            "achieved_gbs": gather_gbs,
+            "frac_of_hbm": gather_gbs / hbm,
+            "peak_gbs": hbm,
+            "bytes_per_step": A["gather_bytes"],
+        },
+        "stages_ms": {"hash": st_mean[0], "gather": st_mean[1], "key_proj_gate": st_mean[2],
+                      "value_proj_gate": st_mean[3]},
+        "e2e": {
+            "value": tokens_per_step * world * E / (e2e_ms / 1e3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": tok_h.numel() * 4 + h_h.numel() * h_h.element_size(),
+            "d2h_bytes_per_step": out_h.numel() * out_h.element_size(),
+            "steps": E,
+        },
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(P, args.cpu_seconds)
+    return res
+
+
+# ----------------------------------------------------------- CPU oracle leg
+
+def cpu_baseline(P, budget_s: float):
+    """The oracle, as it stands, on a bounded sample of the same workload.
+
+    Compress + hash run on every position; gather, projections and gate on
+    the first n rows, n grown until the sample takes about `budget_s` seconds.
+    tokens/s = 1 / (hash time per position + gather+fp time per row)."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    sh = P["sh"]
+    tokens = P["tokens"].numpy()
+    t0 = time.perf_counter()
+    c, z, mult, primes = oracle.forward_indices(tokens, P["comp_map"].numpy(), sh.cvocab,
+                                                sh.orders, sh.heads, P["hash_seed"],
+                                                sh.rows_target)
+    t_hash = (time.perf_counter() - t0) / sh.rows_out
+
+    def to_np(t):
+        t = t.detach().contiguous().cpu()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    wk, wv = to_np(P["w_k"]), to_np(P["w_v"])
+    nq, nk = P["nq"].cpu().numpy(), P["nk"].cpu().numpy()
+    n, spent, total_rows, total_t = 8, 0.0, 0, 0.0
+    while spent < budget_s and total_rows < sh.rows_out:
+        rows = np.arange(total_rows, min(sh.rows_out, total_rows + n))
+        zr = z[rows]
+        mini = [to_np(t[torch.from_numpy(zr[:, s]).to(t.device)]) for s, t in enumerate(P["tables"])]
+        zz = np.tile(np.arange(len(rows))[:, None], (1, sh.num_tables))
+        hr = to_np(P["h"][torch.from_numpy(rows).to(P["h"].device)])
+        t0 = time.perf_counter()
+        e = oracle.gather(mini, zz)
+        oracle.project_gate(e, wk, wv, nq, nk, hr, 1e-6, want_delta=False)
+        dt = time.perf_counter() - t0
+        total_rows += len(rows)
+        total_t += dt
+        spent += dt
+        n *= 2
+    per_row = t_hash + total_t / total_rows
+    return {"value": 1.0 / per_row, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "compress+hash on all %d positions; gather+projection+gate on the first "
+                      "%d rows (%.1f s); single-threaded C, fp64" % (sh.rows_out, total_rows,
+                                                                    total_t)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    P = setup(0, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))))
+    sh = P["sh"]
+    budget = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(P, budget)
+    vals = [cpu_baseline(P, budget) for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sh.rows_out / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "prefill_bf16 (as the ours arm)", "global_batch": sh.rows_out,
+                   "seq_len": sh.T, "parallelism": "single"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": vals[-1]["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_ours(args, rank, world, dist)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,686 @@
+// C ABI of libengram.so (declared in include/engram.h): configuration checks,
+// the handle and its scratch, tensor maps, and the launch sequence of the
+// Engram forward ("Conditional Memory via Scalable Lookup", section 2).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "../../include/engram.h"
+#include "engram_internal.cuh"
+
+using namespace engram;
+
+struct engram_handle {
+  engram_config cfg{};
+  int device = 0, sms = 148;
+  int S = 0, max_order = 0, d_mem = 0, elt = 4;
+  int64_t primes[kMaxTables] = {};
+  uint64_t mult[kMaxTables * kMaxOrders] = {};
+  std::string last_error;
+
+  // device copies of the configuration
+  int32_t* d_map = nullptr;
+  int64_t* d_primes = nullptr;
+  uint64_t* d_mult = nullptr;
+  unsigned* d_err = nullptr;
+
+  // borrowed parameters
+  bool have_params = false;
+  const void* tables[kMaxTables] = {};
+  const void** d_tables = nullptr;  // device array of S table pointers
+  const void* w_k = nullptr;
+  const void* w_v = nullptr;
+  float* d_wqk = nullptr;           // norm_q * norm_k, [M, d]
+  CUtensorMap map_wk[3], map_wv[3]; // box widths 64, 128, 256
+
+  // scratch, sized for cap_rows emitted positions
+  int64_t cap_rows = 0;
+  int64_t* z = nullptr;
+  void* e = nullptr;
+  float4* partials = nullptr;
+
+  // host-resident tables: prefetch state, double-buffered
+  int64_t pf_cap_rows = 0;
+  uint32_t set_cap = 0;
+  unsigned long long* d_keys = nullptr;
+  int32_t* d_vals = nullptr;
+  unsigned long long* d_count[2] = {nullptr, nullptr};
+  int2* d_uniq = nullptr;
+  int64_t* d_remap[2] = {nullptr, nullptr};
+  void* d_staging[2] = {nullptr, nullptr};
+  const void** d_stage_tables[2] = {nullptr, nullptr};
+  int64_t* d_stage_bound = nullptr;
+  cudaEvent_t ev_ready[2] = {nullptr, nullptr};
+  cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
+  int64_t pf_rows[2] = {0, 0};
+  uint64_t n_prefetch = 0, n_consumed = 0;
+
+  // instrumentation
+  int64_t launches = 0;
+  cudaEvent_t prof[5] = {};
+  bool prof_armed = false;
+};
+
+namespace {
+
+thread_local std::string g_create_error;
+
+int fail(engram_handle* h, int code, const std::string& msg) {
+  if (h)
+    h->last_error = msg;
+  else
+    g_create_error = msg;
+  return code;
+}
+
+int cuda_fail(engram_handle* h, cudaError_t e, const char* what) {
+  return fail(h, e == cudaErrorMemoryAllocation ? ENGRAM_ERR_OOM : ENGRAM_ERR_CUDA,
+              std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(h, call)                                       \
+  do {                                                    \
+    cudaError_t e__ = (call);                             \
+    if (e__ != cudaSuccess) return cuda_fail(h, e__, #call); \
+  } while (0)
+
+// SplitMix64 (Steele, Lea and Flood, OOPSLA 2014): the multiplier stream.
+uint64_t splitmix64(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+bool prime(int64_t n) {
+  if (n < 2) return false;
+  if (n % 2 == 0) return n == 2;
+  for (int64_t f = 3; f <= n / f; f += 2)
+    if (n % f == 0) return false;
+  return true;
+}
+
+template <class T>
+void free_dev(T*& p) {
+  if (p) cudaFree((void*)p);
+  p = nullptr;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `rows` rows of `cols` elements, box 64 x box_rows, 128-B swizzle.
+int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
+             int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  return ENGRAM_OK;
+}
+
+int bn_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
+
+// Widest tile (fewest B re-reads) that still gives every SM a tile; else 64.
+int choose_bn(int64_t R, int n_total, int sms) {
+  const int64_t mblk = (R + 127) / 128;
+  for (int bn : {256, 128}) {
+    if (n_total % bn == 0 && mblk * (n_total / bn) >= sms) return bn;
+  }
+  return 64;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int ensure_scratch(engram_handle* h, int64_t rows) {
+  if (rows <= h->cap_rows) return ENGRAM_OK;
+  free_dev(h->z);
+  free_dev(h->e);
+  free_dev(h->partials);
+  h->cap_rows = 0;
+  const int64_t key_tiles = (int64_t)h->cfg.branches * h->cfg.d_hidden / 64;
+  CK(h, cudaMalloc(&h->z, (size_t)rows * h->S * sizeof(int64_t)));
+  CK(h, cudaMalloc(&h->e, (size_t)rows * h->d_mem * h->elt));
+  CK(h, cudaMalloc(&h->partials, (size_t)rows * key_tiles * sizeof(float4)));
+  h->cap_rows = rows;
+  return ENGRAM_OK;
+}
+
+int check_shape(engram_handle* h, int32_t B, int32_t T, int32_t t_begin) {
+  if (B < 0 || T < 0) return fail(h, ENGRAM_ERR_INVALID, "B and T must be >= 0");
+  if (B > 0 && T > 0 && (t_begin < 0 || t_begin >= T))
+    return fail(h, ENGRAM_ERR_INVALID, "t_begin must lie in [0, T)");
+  const int64_t rows = (int64_t)B * (T - t_begin);
+  if (rows > (int64_t)1 << 31) return fail(h, ENGRAM_ERR_INVALID, "too many rows");
+  return ENGRAM_OK;
+}
+
+HashArgs hash_args(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T, int32_t t_begin,
+                   int64_t* idx) {
+  HashArgs a{};
+  a.tokens = tokens;
+  a.map = h->d_map;
+  a.mult = h->d_mult;
+  a.primes = h->d_primes;
+  a.idx = idx;
+  a.err = h->d_err;
+  a.V = h->cfg.vocab;
+  a.pad = h->cfg.pad_id;
+  a.B = B;
+  a.T = T;
+  a.t_begin = t_begin;
+  a.S = h->S;
+  a.heads = h->cfg.heads;
+  a.num_orders = h->cfg.num_orders;
+  a.max_order = h->max_order;
+  for (int i = 0; i < kMaxOrders; ++i) a.orders[i] = h->cfg.orders[i];
+  return a;
+}
+
+int ensure_prefetch_scratch(engram_handle* h, int64_t rows) {
+  if (rows <= h->pf_cap_rows) return ENGRAM_OK;
+  // the staging buffers may still be in use by queued work
+  CK(h, cudaDeviceSynchronize());
+  free_dev(h->d_keys);
+  free_dev(h->d_vals);
+  free_dev(h->d_uniq);
+  free_dev(h->d_stage_bound);
+  for (int i = 0; i < 2; ++i) {
+    free_dev(h->d_count[i]);
+    free_dev(h->d_remap[i]);
+    free_dev(h->d_staging[i]);
+    free_dev(h->d_stage_tables[i]);
+  }
+  h->pf_cap_rows = 0;
+  const int64_t entries = rows * h->S;
+  uint64_t cap = 1;
+  while (cap < (uint64_t)(2 * entries)) cap <<= 1;
+  if (cap > (1ull << 31)) return fail(h, ENGRAM_ERR_INVALID, "prefetch batch too large");
+  h->set_cap = (uint32_t)cap;
+  const size_t row_bytes = (size_t)h->cfg.d_head * h->elt;
+  CK(h, cudaMalloc(&h->d_keys, cap * sizeof(unsigned long long)));
+  CK(h, cudaMalloc(&h->d_vals, cap * sizeof(int32_t)));
+  CK(h, cudaMalloc(&h->d_uniq, (size_t)entries * sizeof(int2)));
+  CK(h, cudaMalloc(&h->d_stage_bound, h->S * sizeof(int64_t)));
+  int64_t bound[kMaxTables];
+  for (int s = 0; s < h->S; ++s) bound[s] = entries;
+  CK(h, cudaMemcpy(h->d_stage_bound, bound, h->S * sizeof(int64_t), cudaMemcpyHostToDevice));
+  for (int i = 0; i < 2; ++i) {
+    CK(h, cudaMalloc(&h->d_count[i], sizeof(unsigned long long)));
+    CK(h, cudaMalloc(&h->d_remap[i], (size_t)entries * sizeof(int64_t)));
+    CK(h, cudaMalloc(&h->d_staging[i], (size_t)entries * row_bytes));
+    CK(h, cudaMalloc(&h->d_stage_tables[i], h->S * sizeof(void*)));
+    const void* ptrs[kMaxTables];
+    for (int s = 0; s < h->S; ++s) ptrs[s] = h->d_staging[i];
+    CK(h, cudaMemcpy(h->d_stage_tables[i], ptrs, h->S * sizeof(void*), cudaMemcpyHostToDevice));
+  }
+  h->pf_cap_rows = rows;
+  return ENGRAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t engram_config_size(void) { return sizeof(engram_config); }
+
+const char* engram_last_error(const engram_handle* h) {
+  return h ? h->last_error.c_str() : g_create_error.c_str();
+}
+
+int engram_create(const engram_config* cfg, engram_handle** out) {
+  if (!cfg || !out) return fail(nullptr, ENGRAM_ERR_INVALID, "null argument");
+  *out = nullptr;
+  const engram_config& c = *cfg;
+  if (c.vocab < 1 || c.cvocab < 1 || c.cvocab > c.vocab)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "need 1 <= cvocab <= vocab");
+  if (!c.comp_map) return fail(nullptr, ENGRAM_ERR_INVALID, "comp_map is required");
+  if (c.num_orders < 1 || c.num_orders > ENGRAM_MAX_ORDERS)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "num_orders must lie in [1, 4]");
+  for (int i = 0; i < c.num_orders; ++i) {
+    if (c.orders[i] < 1 || c.orders[i] > ENGRAM_MAX_ORDERS)
+      return fail(nullptr, ENGRAM_ERR_INVALID, "n-gram orders must lie in [1, 4]");
+    if (i > 0 && c.orders[i] <= c.orders[i - 1])
+      return fail(nullptr, ENGRAM_ERR_INVALID, "n-gram orders must be strictly ascending");
+  }
+  if (c.heads < 1 || c.num_orders * c.heads > ENGRAM_MAX_TABLES)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "need 1 <= heads and orders*heads <= 64");
+  if (c.dtype != ENGRAM_F32 && c.dtype != ENGRAM_BF16)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "dtype must be ENGRAM_F32 or ENGRAM_BF16");
+  const int elt = c.dtype == ENGRAM_F32 ? 4 : 2;
+  if (c.d_head < 1 || (c.d_head * elt) % 16 != 0)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "d_head * element size must be a multiple of 16");
+  if (c.d_hidden < 64 || c.d_hidden % 64 != 0)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "d_hidden must be a positive multiple of 64");
+  if (c.branches < 1 || c.branches > ENGRAM_MAX_BRANCHES)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "branches must lie in [1, 4]");
+  if (!(c.eps >= 0.f) || !std::isfinite(c.eps))
+    return fail(nullptr, ENGRAM_ERR_INVALID, "eps must be finite and >= 0");
+  if (c.table_location != ENGRAM_DEVICE && c.table_location != ENGRAM_PINNED_HOST)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "bad table_location");
+  if (c.pad_id < -1) return fail(nullptr, ENGRAM_ERR_INVALID, "pad_id must be >= -1");
+  const int S = c.num_orders * c.heads;
+  const int64_t d_mem = (int64_t)S * c.d_head;
+  if (d_mem > (1 << 20)) return fail(nullptr, ENGRAM_ERR_INVALID, "d_mem too large");
+
+  int64_t primes[kMaxTables];
+  int given = 0;
+  for (int s = 0; s < S; ++s) given += c.primes[s] != 0;
+  if (given != 0 && given != S)
+    return fail(nullptr, ENGRAM_ERR_INVALID, "give all table sizes or none");
+  if (given == S) {
+    for (int s = 0; s < S; ++s) {
+      if (c.primes[s] < 2 || c.primes[s] >= ((int64_t)1 << 31))
+        return fail(nullptr, ENGRAM_ERR_INVALID, "table sizes must lie in [2, 2^31)");
+      primes[s] = c.primes[s];
+    }
+  } else {
+    if (c.table_rows_target < 2 || c.table_rows_target >= ((int64_t)1 << 31) - 4096)
+      return fail(nullptr, ENGRAM_ERR_INVALID, "table_rows_target must lie in [2, 2^31 - 4096)");
+    int64_t n = c.table_rows_target;
+    for (int s = 0; s < S; ++s) {
+      while (!prime(n)) ++n;
+      primes[s] = n++;
+    }
+  }
+  for (int i = 0; i < c.vocab; ++i)
+    if (c.comp_map[i] < 0 || c.comp_map[i] >= c.cvocab)
+      return fail(nullptr, ENGRAM_ERR_INVALID, "comp_map values must lie in [0, cvocab)");
+
+  engram_handle* h = new (std::nothrow) engram_handle();
+  if (!h) return fail(nullptr, ENGRAM_ERR_OOM, "host allocation failed");
+  h->cfg = c;
+  h->cfg.comp_map = nullptr;
+  if (h->cfg.pad_id == -1) h->cfg.pad_id = c.cvocab;
+  h->S = S;
+  h->elt = elt;
+  h->d_mem = (int)d_mem;
+  h->max_order = c.orders[c.num_orders - 1];
+  for (int s = 0; s < S; ++s) h->primes[s] = primes[s];
+  uint64_t st = c.hash_seed;
+  for (int s = 0; s < S; ++s)
+    for (int j = 0; j < h->max_order; ++j) h->mult[s * h->max_order + j] = splitmix64(st) | 1ull;
+
+  auto bail = [&](int code) {
+    g_create_error = h->last_error;
+    engram_destroy(h);
+    return code;
+  };
+  int rc;
+  if ((rc = [&]() -> int {
+         CK(h, cudaGetDevice(&h->device));
+         CK(h, cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device));
+         CK(h, cudaMalloc(&h->d_map, (size_t)c.vocab * sizeof(int32_t)));
+         CK(h, cudaMemcpy(h->d_map, c.comp_map, (size_t)c.vocab * sizeof(int32_t),
+                          cudaMemcpyHostToDevice));
+         CK(h, cudaMalloc(&h->d_primes, S * sizeof(int64_t)));
+         CK(h, cudaMemcpy(h->d_primes, h->primes, S * sizeof(int64_t), cudaMemcpyHostToDevice));
+         CK(h, cudaMalloc(&h->d_mult, (size_t)S * h->max_order * sizeof(uint64_t)));
+         CK(h, cudaMemcpy(h->d_mult, h->mult, (size_t)S * h->max_order * sizeof(uint64_t),
+                          cudaMemcpyHostToDevice));
+         CK(h, cudaMalloc(&h->d_err, sizeof(unsigned)));
+         CK(h, cudaMemset(h->d_err, 0, sizeof(unsigned)));
+         CK(h, cudaMalloc(&h->d_tables, S * sizeof(void*)));
+         CK(h, cudaMalloc(&h->d_wqk, (size_t)c.branches * c.d_hidden * sizeof(float)));
+         for (int i = 0; i < 2; ++i) {
+           CK(h, cudaEventCreateWithFlags(&h->ev_ready[i], cudaEventDisableTiming));
+           CK(h, cudaEventCreateWithFlags(&h->ev_consumed[i], cudaEventDisableTiming));
+         }
+         return ENGRAM_OK;
+       }()) != ENGRAM_OK)
+    return bail(rc);
+  *out = h;
+  return ENGRAM_OK;
+}
+
+void engram_destroy(engram_handle* h) {
+  if (!h) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  free_dev(h->d_map);
+  free_dev(h->d_primes);
+  free_dev(h->d_mult);
+  free_dev(h->d_err);
+  free_dev(h->d_tables);
+  free_dev(h->d_wqk);
+  free_dev(h->z);
+  free_dev(h->e);
+  free_dev(h->partials);
+  free_dev(h->d_keys);
+  free_dev(h->d_vals);
+  free_dev(h->d_uniq);
+  free_dev(h->d_stage_bound);
+  for (int i = 0; i < 2; ++i) {
+    free_dev(h->d_count[i]);
+    free_dev(h->d_remap[i]);
+    free_dev(h->d_staging[i]);
+    free_dev(h->d_stage_tables[i]);
+    if (h->ev_ready[i]) cudaEventDestroy(h->ev_ready[i]);
+    if (h->ev_consumed[i]) cudaEventDestroy(h->ev_consumed[i]);
+  }
+  cudaSetDevice(cur);
+  delete h;
+}
+
+int engram_set_params(engram_handle* h, const void* const* tables, const void* w_k, const void* w_v,
+                      const float* norm_q, const float* norm_k) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!tables || !w_k || !w_v || !norm_q || !norm_k)
+    return fail(h, ENGRAM_ERR_INVALID, "null parameter pointer");
+  for (int s = 0; s < h->S; ++s) {
+    if (!tables[s] || !aligned16(tables[s]))
+      return fail(h, ENGRAM_ERR_INVALID, "table pointers must be non-null and 16-byte aligned");
+  }
+  if (!aligned16(w_k) || !aligned16(w_v) || !aligned16(norm_q) || !aligned16(norm_k))
+    return fail(h, ENGRAM_ERR_INVALID, "parameter pointers must be 16-byte aligned");
+  if (h->cfg.table_location == ENGRAM_PINNED_HOST) {
+    for (int s = 0; s < h->S; ++s) {
+      cudaPointerAttributes at;
+      if (cudaPointerGetAttributes(&at, tables[s]) != cudaSuccess || at.type != cudaMemoryTypeHost ||
+          at.devicePointer == nullptr) {
+        cudaGetLastError();
+        return fail(h, ENGRAM_ERR_INVALID, "host tables must be pinned and mapped");
+      }
+    }
+  }
+  const int M = h->cfg.branches, d = h->cfg.d_hidden;
+  const void* dev_tab[kMaxTables];
+  for (int s = 0; s < h->S; ++s) {
+    h->tables[s] = tables[s];
+    dev_tab[s] = tables[s];
+    if (h->cfg.table_location == ENGRAM_PINNED_HOST) {
+      void* dp = nullptr;
+      CK(h, cudaHostGetDevicePointer(&dp, const_cast<void*>(tables[s]), 0));
+      dev_tab[s] = dp;
+    }
+  }
+  CK(h, cudaMemcpy(h->d_tables, dev_tab, h->S * sizeof(void*), cudaMemcpyHostToDevice));
+  CK(h, launch_mul(norm_q, norm_k, h->d_wqk, (int64_t)M * d, 0));
+  CK(h, cudaDeviceSynchronize());
+  h->w_k = w_k;
+  h->w_v = w_v;
+  if (h->cfg.dtype == ENGRAM_BF16) {
+    for (int bn : {64, 128, 256}) {
+      if (d % bn) continue;
+      int rc = make_map(h, &h->map_wk[bn_index(bn)], w_k, h->d_mem, (int64_t)M * d, bn);
+      if (rc) return rc;
+      rc = make_map(h, &h->map_wv[bn_index(bn)], w_v, h->d_mem, d, bn);
+      if (rc) return rc;
+    }
+  }
+  h->have_params = true;
+  return ENGRAM_OK;
+}
+
+int engram_reserve(engram_handle* h, int64_t max_rows) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (max_rows < 0 || max_rows > ((int64_t)1 << 31))
+    return fail(h, ENGRAM_ERR_INVALID, "max_rows out of range");
+  int rc = ensure_scratch(h, max_rows);
+  if (rc) return rc;
+  if (h->cfg.table_location == ENGRAM_PINNED_HOST) return ensure_prefetch_scratch(h, max_rows);
+  return ENGRAM_OK;
+}
+
+int engram_get_hash_params(const engram_handle* h, int64_t* primes, uint64_t* mult) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (primes) std::memcpy(primes, h->primes, h->S * sizeof(int64_t));
+  if (mult) std::memcpy(mult, h->mult, (size_t)h->S * h->max_order * sizeof(uint64_t));
+  return ENGRAM_OK;
+}
+
+int engram_hash(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T, int32_t t_begin,
+                int64_t* idx, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  int rc = check_shape(h, B, T, t_begin);
+  if (rc) return rc;
+  if ((int64_t)B * T == 0) return ENGRAM_OK;
+  if (!tokens || !idx) return fail(h, ENGRAM_ERR_INVALID, "null tokens or idx");
+  CK(h, launch_hash(hash_args(h, tokens, B, T, t_begin, idx), (cudaStream_t)stream));
+  h->launches += 1;
+  return ENGRAM_OK;
+}
+
+int engram_gather(engram_handle* h, const int64_t* idx, int64_t rows, void* e, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (h->cfg.table_location != ENGRAM_DEVICE)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED, "engram_gather reads device-resident tables only");
+  if (rows < 0) return fail(h, ENGRAM_ERR_INVALID, "rows < 0");
+  if (rows == 0) return ENGRAM_OK;
+  if (!idx || !e || !aligned16(e)) return fail(h, ENGRAM_ERR_INVALID, "null or misaligned buffer");
+  GatherArgs g{};
+  g.tables = h->d_tables;
+  g.primes = h->d_primes;
+  g.idx = idx;
+  g.e = e;
+  g.err = h->d_err;
+  g.rows = rows;
+  g.S = h->S;
+  g.row_bytes = h->cfg.d_head * h->elt;
+  CK(h, launch_gather(g, (cudaStream_t)stream));
+  h->launches += 1;
+  return ENGRAM_OK;
+}
+
+int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T, int32_t t_begin,
+                    void* side_stream, int64_t* unique_rows) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (h->cfg.table_location != ENGRAM_PINNED_HOST)
+    return fail(h, ENGRAM_ERR_STATE, "engram_prefetch needs ENGRAM_PINNED_HOST tables");
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  int rc = check_shape(h, B, T, t_begin);
+  if (rc) return rc;
+  if (h->n_prefetch - h->n_consumed >= 2)
+    return fail(h, ENGRAM_ERR_STATE, "two prefetches already pending; run engram_forward first");
+  const int64_t rows = (int64_t)B * (T - t_begin);
+  if (rows > 0 && !tokens) return fail(h, ENGRAM_ERR_INVALID, "null tokens");
+  if ((rc = ensure_prefetch_scratch(h, rows))) return rc;
+  cudaStream_t st = (cudaStream_t)side_stream;
+  const int slot = (int)(h->n_prefetch & 1);
+  // the staging slot must no longer be read by the forward that used it last
+  if (h->n_prefetch >= 2) CK(h, cudaStreamWaitEvent(st, h->ev_consumed[slot], 0));
+  if (rows > 0) {
+    // hash into this slot's index buffer; the prefetch then rewrites each
+    // index in place with its staging slot
+    CK(h, launch_hash(hash_args(h, tokens, B, T, t_begin, h->d_remap[slot]), st));
+    h->launches += 1;
+  }
+  PrefetchArgs a{};
+  a.idx = h->d_remap[slot];
+  a.rows = rows;
+  a.S = h->S;
+  a.keys = h->d_keys;
+  a.vals = h->d_vals;
+  a.cap = h->set_cap;
+  a.count = h->d_count[slot];
+  a.uniq = h->d_uniq;
+  a.remapped = h->d_remap[slot];
+  a.tables = h->d_tables;
+  a.row_bytes = h->cfg.d_head * h->elt;
+  a.staging = h->d_staging[slot];
+  a.sms = h->sms;
+  a.fetch_blocks = h->sms * 8;
+  CK(h, launch_prefetch(a, st));
+  h->launches += rows > 0 ? 5 : 1;
+  CK(h, cudaEventRecord(h->ev_ready[slot], st));
+  h->pf_rows[slot] = rows;
+  ++h->n_prefetch;
+  if (unique_rows) {
+    unsigned long long n = 0;
+    CK(h, cudaMemcpyAsync(&n, h->d_count[slot], sizeof(n), cudaMemcpyDeviceToHost, st));
+    CK(h, cudaStreamSynchronize(st));
+    *unique_rows = rows > 0 ? (int64_t)n : 0;
+  }
+  return ENGRAM_OK;
+}
+
+int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, int32_t B,
+                   int32_t T, int32_t t_begin, const void* hid, void* out, float* alpha,
+                   float* delta, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  int rc = check_shape(h, B, T, t_begin);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int64_t R = (int64_t)B * (T - t_begin);
+  const bool host_tables = h->cfg.table_location == ENGRAM_PINNED_HOST;
+  int slot = 0;
+  if (host_tables) {
+    if (h->n_prefetch == h->n_consumed)
+      return fail(h, ENGRAM_ERR_STATE, "host-resident tables: call engram_prefetch first");
+    slot = (int)(h->n_consumed & 1);
+    if (h->pf_rows[slot] != R)
+      return fail(h, ENGRAM_ERR_INVALID, "forward shape differs from the pending prefetch");
+  }
+  if (R == 0) {
+    if (host_tables) {
+      CK(h, cudaStreamWaitEvent(st, h->ev_ready[slot], 0));
+      CK(h, cudaEventRecord(h->ev_consumed[slot], st));
+      ++h->n_consumed;
+    }
+    return ENGRAM_OK;
+  }
+  if (!hid || !out || !aligned16(hid) || !aligned16(out))
+    return fail(h, ENGRAM_ERR_INVALID, "h and out must be non-null and 16-byte aligned");
+  if ((alpha && !aligned16(alpha)) || (delta && !aligned16(delta)))
+    return fail(h, ENGRAM_ERR_INVALID, "alpha and delta must be 16-byte aligned");
+  if (!idx && !tokens && !host_tables) return fail(h, ENGRAM_ERR_INVALID, "need tokens or idx");
+  if (R > (int64_t)65535 * 64 && h->cfg.dtype == ENGRAM_F32)
+    return fail(h, ENGRAM_ERR_INVALID, "fp32 path limited to 4194240 rows per call");
+  if ((rc = ensure_scratch(h, R))) return rc;
+  const bool prof = h->prof_armed;
+  h->prof_armed = false;
+  auto mark = [&](int i) -> cudaError_t {
+    return prof ? cudaEventRecord(h->prof[i], st) : cudaSuccess;
+  };
+  CK(h, mark(0));
+
+  // steps 1-4: indices, then the gathered memory vectors e
+  GatherArgs ga{};
+  ga.e = h->e;
+  ga.err = h->d_err;
+  ga.rows = R;
+  ga.S = h->S;
+  ga.row_bytes = h->cfg.d_head * h->elt;
+  if (host_tables) {
+    CK(h, cudaStreamWaitEvent(st, h->ev_ready[slot], 0));
+    ga.tables = h->d_stage_tables[slot];
+    ga.primes = h->d_stage_bound;
+    ga.idx = h->d_remap[slot];
+  } else {
+    if (!idx) {
+      CK(h, launch_hash(hash_args(h, tokens, B, T, t_begin, h->z), st));
+      h->launches += 1;
+      idx = h->z;
+    }
+    ga.tables = h->d_tables;
+    ga.primes = h->d_primes;
+    ga.idx = idx;
+  }
+  CK(h, mark(1));
+  CK(h, launch_gather(ga, st));
+  h->launches += 1;
+  CK(h, mark(2));
+  if (host_tables) {
+    CK(h, cudaEventRecord(h->ev_consumed[slot], st));
+    ++h->n_consumed;
+  }
+
+  // steps 5-7: projections, gate, residual
+  GateArgs g{};
+  g.h = hid;
+  g.out = out;
+  g.w_qk = h->d_wqk;
+  g.partials = h->partials;
+  g.alpha = alpha;
+  g.delta = delta;
+  g.err = h->d_err;
+  g.R = (int32_t)R;
+  g.M = h->cfg.branches;
+  g.d = h->cfg.d_hidden;
+  g.d_mem = h->d_mem;
+  g.eps = h->cfg.eps;
+  g.inv_sqrt_d = (float)(1.0 / std::sqrt((double)h->cfg.d_hidden));
+  if (h->cfg.dtype == ENGRAM_F32) {
+    g.key_tile = kF32Tile;
+    CK(h, launch_proj_gate_f32(0, (const float*)h->e, (const float*)h->w_k, g, st));
+    CK(h, mark(3));
+    CK(h, launch_proj_gate_f32(1, (const float*)h->e, (const float*)h->w_v, g, st));
+    CK(h, mark(4));
+    h->launches += 2;
+    return ENGRAM_OK;
+  }
+  CUtensorMap map_e;
+  if ((rc = make_map(h, &map_e, h->e, h->d_mem, R, 128))) return rc;
+  const int64_t mblk = (R + 127) / 128;
+  const int bn0 = choose_bn(R, g.M * g.d, h->sms);
+  g.key_tile = bn0;
+  const int64_t tiles0 = mblk * (g.M * g.d / bn0);
+  CK(h, launch_proj_gate_sm100(0, bn0, map_e, h->map_wk[bn_index(bn0)], g,
+                               (int)(tiles0 < h->sms ? tiles0 : h->sms), st));
+  CK(h, mark(3));
+  const int bn1 = choose_bn(R, g.d, h->sms);
+  const int64_t tiles1 = mblk * (g.d / bn1);
+  CK(h, launch_proj_gate_sm100(1, bn1, map_e, h->map_wv[bn_index(bn1)], g,
+                               (int)(tiles1 < h->sms ? tiles1 : h->sms), st));
+  CK(h, mark(4));
+  h->launches += 2;
+  return ENGRAM_OK;
+}
+
+int engram_profile_next_forward(engram_handle* h, void* const* events, int32_t n_events) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!events) {
+    h->prof_armed = false;
+    return ENGRAM_OK;
+  }
+  if (n_events != 5) return fail(h, ENGRAM_ERR_INVALID, "n_events must be 5");
+  for (int i = 0; i < 5; ++i) {
+    if (!events[i]) return fail(h, ENGRAM_ERR_INVALID, "null event");
+    h->prof[i] = (cudaEvent_t)events[i];
+  }
+  h->prof_armed = true;
+  return ENGRAM_OK;
+}
+
+int64_t engram_kernel_launches(const engram_handle* h) { return h ? h->launches : -1; }
+
+int engram_check_errors(engram_handle* h, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  CK(h, cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned w = 0;
+  CK(h, cudaMemcpy(&w, h->d_err, sizeof(w), cudaMemcpyDeviceToHost));
+  CK(h, cudaMemset(h->d_err, 0, sizeof(unsigned)));
+  if (w & kDevErrTimeout) return fail(h, ENGRAM_ERR_TIMEOUT, "a kernel's bounded wait expired");
+  if (w & (kDevErrToken | kDevErrIndex))
+    return fail(h, ENGRAM_ERR_BOUNDS,
+                (w & kDevErrToken) ? "token id outside [0, vocab) replaced by the pad id"
+                                   : "table index outside the table: zero row used");
+  return ENGRAM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// Internal interface between the C-ABI layer (engram_api.cu) and the kernels.
+// Not installed; callers use include/engram.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace engram {
+
+// Bits of the handle's device error word.
+constexpr unsigned kDevErrToken = 1u;    // token id outside [0, V): pad used instead
+constexpr unsigned kDevErrIndex = 2u;    // table index outside [0, p): zero row used
+constexpr unsigned kDevErrTimeout = 4u;  // a bounded mbarrier wait expired
+
+constexpr int kMaxTables = 64;
+constexpr int kMaxOrders = 4;
+constexpr int kMaxBranches = 4;
+
+// Everything the compress+hash kernel needs (section 2.2, Eq. 1).
+struct HashArgs {
+  const int32_t* tokens;   // [B, T] raw ids
+  const int32_t* map;      // [V] compression map
+  const uint64_t* mult;    // [S, max_order] odd multipliers
+  const int64_t* primes;   // [S]
+  int64_t* idx;            // [B*(T-t_begin), S]
+  unsigned* err;
+  int32_t V, pad, B, T, t_begin, S, heads, num_orders, max_order;
+  int32_t orders[kMaxOrders];
+};
+
+// Row gather (Eq. 2).  Tables are addressed through a device array of S pointers.
+struct GatherArgs {
+  const void* const* tables;  // device array [S] of table base pointers
+  const int64_t* primes;      // [S]
+  const int64_t* idx;         // [rows, S]
+  void* e;                    // [rows, S*d_head]
+  unsigned* err;
+  int64_t rows;
+  int32_t S;
+  int32_t row_bytes;          // d_head * element size, a multiple of 16
+};
+
+// Projection + gate epilogue arguments (Eq. 3, 4, 6).
+struct GateArgs {
+  const void* h;        // [R, M, d]
+  void* out;            // [R, M, d]
+  const float* w_qk;    // [M, d]: norm_q * norm_k (the two RMSNorm weights multiply)
+  float4* partials;     // [num key tiles][R]: (sum k^2, sum h w_q w_k k, sum h^2, 0)
+  float* alpha;         // [R, M] or null
+  float* delta;         // [R, M, d] or null
+  unsigned* err;
+  int32_t R, M, d, d_mem;
+  int32_t key_tile;     // width of the key-phase tiles that wrote `partials`
+  float eps;
+  float inv_sqrt_d;
+};
+
+// Prefetch of host-resident rows into an HBM staging buffer (section 2.5).
+struct PrefetchArgs {
+  const int64_t* idx;           // [rows, S] table indices of the upcoming step
+  int64_t rows;
+  int32_t S;
+  unsigned long long* keys;     // [cap] open-addressing set, cap a power of two >= 2*rows*S
+  int32_t* vals;                // [cap] staging slot of each occupied bucket
+  uint32_t cap;
+  unsigned long long* count;    // distinct rows found
+  int2* uniq;                   // [rows*S] (slot s, row z) of each staging slot
+  int64_t* remapped;            // [rows, S] staging slot of each index
+  const void* const* tables;    // device array [S] of pinned host table pointers
+  int32_t row_bytes;
+  void* staging;                // [rows*S, row_bytes] device
+  int sms;
+  int fetch_blocks;             // grid cap of the PCIe copy kernel
+};
+
+// Launchers (all asynchronous on `stream`; return the launch error).
+cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);
+cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
+cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream);
+cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);
+
+// fp32 path (SIMT FFMA; 64-column tiles).  phase 0 = key tiles over W_K
+// [M*d, d_mem], phase 1 = value tiles over W_V [d, d_mem].
+constexpr int kF32Tile = 64;
+cudaError_t launch_proj_gate_f32(int phase, const float* e, const float* w, const GateArgs& g,
+                                 cudaStream_t stream);
+
+// bf16 path (tcgen05 / TMEM / TMA, sm_100a).  `bn` in {64, 128, 256}.
+int sm100_stages(int bn);
+size_t sm100_smem_bytes(int bn);
+cudaError_t launch_proj_gate_sm100(int phase, int bn, const CUtensorMap& map_e, const CUtensorMap& map_w,
+                                   const GateArgs& g, int grid, cudaStream_t stream);
+
+}  // namespace engram

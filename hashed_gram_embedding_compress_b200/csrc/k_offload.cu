@@ -1,0 +1,148 @@
+// Deterministic prefetch of host-resident table rows.
+//
+// "Conditional Memory via Scalable Lookup", section 2.5 and Figure 2(b): the
+// retrieval indices depend only on the token sequence, so they are known
+// before the layer runs; the rows are fetched asynchronously from host memory
+// over PCIe and the transfer overlaps the preceding blocks' compute.  The
+// paper's Table 4 run sends every retrieval over PCIe, and notes that the
+// traffic scales with the active rows, not the table size.
+//
+// Steps (all on the prefetch stream):
+//   1. clear an open-addressing set of 64-bit keys (slot s << 40 | row z);
+//   2. insert every (s, z[r, s]) with atomicCAS: one key per distinct row;
+//   3. number the occupied buckets with an atomic counter: a staging slot per
+//      distinct row, and a list of (s, z) per slot;
+//   4. remap every index to its staging slot (a lookup, no waiting on other
+//      threads: the slot numbers are final after step 3);
+//   5. copy each distinct row once from pinned host memory (zero-copy loads
+//      over PCIe, 16 bytes per thread, whole rows per run of threads) into
+//      the HBM staging buffer.
+// The forward then gathers from the staging buffer with the remapped indices.
+#include "engram_internal.cuh"
+
+namespace engram {
+
+namespace {
+
+constexpr unsigned long long kEmpty = 0xFFFFFFFFFFFFFFFFull;
+
+__device__ __forceinline__ uint32_t mix_bucket(unsigned long long key, uint32_t mask) {
+  // 64-bit finaliser (the SplitMix64 output mix) spreads consecutive rows
+  unsigned long long z = key + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return (uint32_t)z & mask;
+}
+
+__global__ void clear_kernel(unsigned long long* keys, int32_t* vals, uint32_t cap,
+                             unsigned long long* count) {
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < cap; i += gridDim.x * blockDim.x) {
+    keys[i] = kEmpty;
+    vals[i] = -1;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *count = 0;
+}
+
+// Linear probing; the set holds at least twice as many buckets as inserted
+// keys, so a probe sequence always meets an empty bucket or its key.
+__global__ void insert_kernel(const int64_t* idx, int64_t n, int32_t S, unsigned long long* keys,
+                              uint32_t mask) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int s = (int)(i % S);
+    const unsigned long long key = ((unsigned long long)s << 40) | (unsigned long long)idx[i];
+    uint32_t b = mix_bucket(key, mask);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+      const unsigned long long prev = atomicCAS(keys + b, kEmpty, key);
+      if (prev == kEmpty || prev == key) break;
+      b = (b + 1) & mask;
+    }
+  }
+}
+
+__global__ void number_kernel(const unsigned long long* keys, int32_t* vals, uint32_t cap,
+                              unsigned long long* count, int2* uniq) {
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < cap; i += gridDim.x * blockDim.x) {
+    const unsigned long long k = keys[i];
+    if (k == kEmpty) continue;
+    const int32_t slot = (int32_t)atomicAdd(count, 1ull);
+    vals[i] = slot;
+    uniq[slot] = make_int2((int)(k >> 40), (int)(k & 0xFFFFFFFFFFull));
+  }
+}
+
+__global__ void remap_kernel(const int64_t* idx, int64_t n, int32_t S,
+                             const unsigned long long* keys, const int32_t* vals, uint32_t mask,
+                             int64_t* out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int s = (int)(i % S);
+    const unsigned long long key = ((unsigned long long)s << 40) | (unsigned long long)idx[i];
+    uint32_t b = mix_bucket(key, mask);
+    int64_t v = -1;
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+      const unsigned long long k = keys[b];
+      if (k == key) {
+        v = vals[b];
+        break;
+      }
+      if (k == kEmpty) break;
+      b = (b + 1) & mask;
+    }
+    out[i] = v;  // -1 never happens for a key inserted above; the gather bounds-checks it
+  }
+}
+
+__device__ __forceinline__ uint4 ld_host_16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// One thread per 16-byte chunk of a distinct row; threads past the distinct
+// count (known only on the device) return at once.
+__global__ void fetch_kernel(const void* const* tables, const int2* uniq,
+                             const unsigned long long* count, int32_t row_bytes, char* staging) {
+  const int cpr = row_bytes >> 4;
+  const int64_t total = (int64_t)(*count) * cpr;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = i / cpr;
+    const int c = (int)(i - u * cpr);
+    const int2 sz = uniq[u];
+    const char* src = (const char*)tables[sz.x] + (int64_t)sz.y * row_bytes + c * 16;
+    *reinterpret_cast<uint4*>(staging + u * row_bytes + c * 16) = ld_host_16(src);
+  }
+}
+
+int blocks_for(int64_t n, int threads, int cap) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b > cap) b = cap;
+  return b < 1 ? 1 : (int)b;
+}
+
+}  // namespace
+
+cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream) {
+  const int n = 256;
+  const int cap_blocks = a.sms * 16;
+  const int64_t entries = a.rows * a.S;
+  clear_kernel<<<blocks_for(a.cap, n, cap_blocks), n, 0, stream>>>(a.keys, a.vals, a.cap, a.count);
+  if (entries > 0) {
+    insert_kernel<<<blocks_for(entries, n, cap_blocks), n, 0, stream>>>(a.idx, entries, a.S,
+                                                                       a.keys, a.cap - 1);
+    number_kernel<<<blocks_for(a.cap, n, cap_blocks), n, 0, stream>>>(a.keys, a.vals, a.cap,
+                                                                     a.count, a.uniq);
+    remap_kernel<<<blocks_for(entries, n, cap_blocks), n, 0, stream>>>(
+        a.idx, entries, a.S, a.keys, a.vals, a.cap - 1, a.remapped);
+    // at most `entries` distinct rows
+    fetch_kernel<<<blocks_for(entries * (a.row_bytes >> 4), n, a.fetch_blocks), n, 0, stream>>>(
+        a.tables, a.uniq, a.count, a.row_bytes, (char*)a.staging);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace engram

@@ -1,0 +1,478 @@
+// bf16 projection + context-aware gate on the 5th-generation tensor cores.
+//
+// "Conditional Memory via Scalable Lookup", section 2.3 Eq. (3)-(4) and
+// section 2.4 Eq. (6): k^(m) = W_K^(m) e, v = W_V e,
+//   alpha^(m) = sigmoid(RMSNorm_q(h^(m)) . RMSNorm_k(k^(m)) / sqrt(d)),
+//   out^(m)   = h^(m) + alpha^(m) v.
+// The paper fuses all projections into one dense matmul (section 2.4).  Here
+// both are one persistent warp-specialised GEMM kernel, launched twice:
+//
+//   phase 0 (keys):   N = M*d columns of [W_K^(1); ...; W_K^(M)].  The
+//                     epilogue never stores k: it reduces each 128 x BN tile
+//                     to per-row partial sums (sum k^2, sum h w_q w_k k,
+//                     sum h^2), which decompose RMSNorm(h).RMSNorm(k) over
+//                     column tiles because both norms are per-row scalars.
+//   phase 1 (values): N = d columns of W_V.  The epilogue finishes alpha from
+//                     the partials of every key tile of the branch and writes
+//                     out = h + alpha v for each branch directly from TMEM.
+//
+// Per CTA (one per SM, persistent, 192 threads):
+//   warp 4      TMA producer: A = e tile [128 x 64], B = W tile [BN x 64],
+//               128-byte swizzle, STAGES-deep ring of smem slots;
+//   warp 5      TMEM allocator and MMA issuer: tcgen05.mma.cta_group::1
+//               kind::f16 (bf16 in, fp32 accumulate), M=128, N=BN, K=16,
+//               accumulators double-buffered in TMEM (2*BN columns);
+//   warps 0-3   epilogue: tcgen05.ld 32 columns at a time (warp w owns TMEM
+//               lanes 32w..32w+31, i.e. rows of the tile), fused gate math,
+//               global loads of h and stores of out.
+// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel records
+// kDevErrTimeout, every role leaves its loop, outstanding MMAs are drained and
+// TMEM is freed before the CTA exits.
+#include <cuda_bf16.h>
+
+#include "engram_internal.cuh"
+
+namespace engram {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                    // 64 bf16 = one 128-byte swizzle row
+constexpr uint32_t A_BYTES = BM * BK * 2; // 16 KB
+constexpr int kThreads = 192;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs.
+// Returns false (and raises the CTA's abort flag) on expiry or if another role
+// has already aborted.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Same, ignoring the abort flag (used only to drain on the way out).
+__device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() - t0 > kWaitLimitNs) return;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (SBO),
+// descriptor version 1 (sm_100), layout type 2 = SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9 and 10-12 = 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
+template <int N>
+__host__ __device__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+__device__ __forceinline__ float sigmoid_f(float s) { return 1.0f / (1.0f + expf(-s)); }
+
+template <int BN>
+struct Cfg {
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+template <int BN, int PHASE>
+__global__ void __launch_bounds__(kThreads, 1)
+    proj_gate_kernel(const __grid_constant__ CUtensorMap map_e,
+                     const __grid_constant__ CUtensorMap map_w, GateArgs g) {
+  using C = Cfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int R = g.R;
+  const int n_total = PHASE == 0 ? g.M * g.d : g.d;
+  const int num_n = n_total / BN;
+  const int num_tiles = ((R + BM - 1) / BM) * num_n;
+  const int num_kb = (g.d_mem + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_e) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (lane == 0) ok = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(full_bar(stage), C::STAGE_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, &map_e, full_bar(stage), kb * BK, m_blk * BM);
+          tma_load_2d(sB + stage * C::B_BYTES, &map_w, full_bar(stage), kb * BK, n_blk * BN);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // give any copy already issued time to land before the CTA's smem is released
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 100000ull) {
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16<BN>();
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      if (lane == 0) ok = wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, g.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (lane == 0) ok = wait_bounded(full_bar(stage), phase, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t ad = sw128_desc(sA + stage * A_BYTES);
+          const uint64_t bd = sw128_desc(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(d_tmem, ad + 2u * k, bd + 2u * k, idesc, (kb | k) != 0);
+          umma_commit(empty_bar(stage));  // slot free once these MMAs have read it
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(tfull_bar(acc));  // accumulator complete
+      __syncwarp();
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) {
+      umma_commit(drain_bar);  // arrives once every MMA issued above has finished
+      wait_drain(drain_bar, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int d = g.d, M = g.M;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    const int tiles_per_branch = d / g.key_tile;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
+      if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, g.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = m_blk * BM + warp * 32 + lane;
+      const bool valid = row < R;
+      const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BN);
+      const int n0 = n_blk * BN;
+      float v[32];
+      if (PHASE == 0) {
+        const int mb = n0 / d, j0 = n0 - mb * d;
+        const __nv_bfloat16* hrow =
+            (const __nv_bfloat16*)g.h + ((int64_t)(valid ? row : 0) * M + mb) * d + j0;
+        const float* wrow = g.w_qk + (int64_t)mb * d + j0;
+        float skk = 0.f, shk = 0.f, shh = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          __syncwarp();
+          tmem_ld32(taddr + c * 32, v);
+          if (valid) {
+            const uint4* hp = reinterpret_cast<const uint4*>(hrow + c * 32);
+            const float4* wp = reinterpret_cast<const float4*>(wrow + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float hf[8];
+              unpack8(__ldg(hp + q), hf);
+              const float4 w0 = __ldg(wp + 2 * q), w1 = __ldg(wp + 2 * q + 1);
+              const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float k = v[q * 8 + i];
+                skk = fmaf(k, k, skk);
+                shh = fmaf(hf[i], hf[i], shh);
+                shk = fmaf(hf[i] * wf[i], k, shk);
+              }
+            }
+          }
+        }
+        if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
+      } else {
+        float al[kMaxBranches];
+#pragma unroll
+        for (int mb = 0; mb < kMaxBranches; ++mb) {
+          al[mb] = 0.f;
+          if (mb < M && valid) {
+            float skk = 0.f, shk = 0.f, shh = 0.f;
+            for (int tb = mb * tiles_per_branch; tb < (mb + 1) * tiles_per_branch; ++tb) {
+              const float4 p = g.partials[(int64_t)tb * R + row];
+              skk += p.x;
+              shk += p.y;
+              shh += p.z;
+            }
+            const float rh = 1.0f / sqrtf(shh / (float)d + g.eps);
+            const float rk = 1.0f / sqrtf(skk / (float)d + g.eps);
+            al[mb] = sigmoid_f(shk * rh * rk * g.inv_sqrt_d);
+            if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          __syncwarp();
+          tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+          for (int mb = 0; mb < kMaxBranches; ++mb) {
+            if (mb >= M || !valid) break;
+            const int64_t base = ((int64_t)row * M + mb) * d + n0 + c * 32;
+            const uint4* hp = reinterpret_cast<const uint4*>((const __nv_bfloat16*)g.h + base);
+            uint4* op = reinterpret_cast<uint4*>((__nv_bfloat16*)g.out + base);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float hf[8];
+              unpack8(__ldg(hp + q), hf);
+              float o[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = fmaf(al[mb], v[q * 8 + i], hf[i]);
+              op[q] = make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]),
+                                 pack2(o[6], o[7]));
+            }
+            if (g.delta) {
+              float4* dp = reinterpret_cast<float4*>(g.delta + base);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dp[q] = make_float4(al[mb] * v[4 * q], al[mb] * v[4 * q + 1],
+                                    al[mb] * v[4 * q + 2], al[mb] * v[4 * q + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::TMEM_COLS));
+  }
+}
+
+template <int BN, int PHASE>
+cudaError_t launch_bn(const CUtensorMap& me, const CUtensorMap& mw, const GateArgs& g, int grid,
+                      cudaStream_t stream) {
+  auto kern = proj_gate_kernel<BN, PHASE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Cfg<BN>::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, Cfg<BN>::SMEM, stream>>>(me, mw, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int sm100_stages(int bn) {
+  return bn == 256 ? Cfg<256>::STAGES : bn == 128 ? Cfg<128>::STAGES : Cfg<64>::STAGES;
+}
+
+size_t sm100_smem_bytes(int bn) {
+  return bn == 256 ? Cfg<256>::SMEM : bn == 128 ? Cfg<128>::SMEM : Cfg<64>::SMEM;
+}
+
+cudaError_t launch_proj_gate_sm100(int phase, int bn, const CUtensorMap& map_e,
+                                   const CUtensorMap& map_w, const GateArgs& g, int grid,
+                                   cudaStream_t stream) {
+  if (g.R == 0) return cudaSuccess;
+  switch (bn * 2 + phase) {
+    case 512: return launch_bn<256, 0>(map_e, map_w, g, grid, stream);
+    case 513: return launch_bn<256, 1>(map_e, map_w, g, grid, stream);
+    case 256: return launch_bn<128, 0>(map_e, map_w, g, grid, stream);
+    case 257: return launch_bn<128, 1>(map_e, map_w, g, grid, stream);
+    case 128: return launch_bn<64, 0>(map_e, map_w, g, grid, stream);
+    case 129: return launch_bn<64, 1>(map_e, map_w, g, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace engram

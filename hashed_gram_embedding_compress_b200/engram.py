@@ -1,0 +1,203 @@
+"""Thin ctypes binding of libengram.so (include/engram.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  Functions keep the C names; ``Engram`` wraps a handle and
+accepts torch tensors (device memory, streams) and passes their pointers.
+There is no CPU fallback: if the library is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libengram.so")
+
+ENGRAM_F32, ENGRAM_BF16 = 0, 1
+ENGRAM_DEVICE, ENGRAM_PINNED_HOST = 0, 1
+ENGRAM_OK, ENGRAM_ERR_INVALID, ENGRAM_ERR_BOUNDS, ENGRAM_ERR_CUDA = 0, 1, 2, 3
+ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_UNSUPPORTED, ENGRAM_ERR_STATE = 4, 5, 6, 7
+MAX_ORDERS, MAX_TABLES, MAX_BRANCHES = 4, 64, 4
+
+#: every symbol include/engram.h declares
+EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last_error",
+           "engram_set_params", "engram_reserve", "engram_get_hash_params", "engram_hash",
+           "engram_gather", "engram_forward", "engram_prefetch", "engram_check_errors",
+           "engram_profile_next_forward", "engram_kernel_launches")
+
+
+class engram_config(ctypes.Structure):
+    _fields_ = [
+        ("vocab", ctypes.c_int32), ("cvocab", ctypes.c_int32), ("pad_id", ctypes.c_int32),
+        ("num_orders", ctypes.c_int32), ("orders", ctypes.c_int32 * MAX_ORDERS),
+        ("heads", ctypes.c_int32), ("d_head", ctypes.c_int32), ("d_hidden", ctypes.c_int32),
+        ("branches", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("table_location", ctypes.c_int32), ("eps", ctypes.c_float),
+        ("reserved0", ctypes.c_int32), ("table_rows_target", ctypes.c_int64),
+        ("hash_seed", ctypes.c_uint64), ("primes", ctypes.c_int64 * MAX_TABLES),
+        ("comp_map", ctypes.POINTER(ctypes.c_int32)),
+    ]
+
+
+class EngramError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("engram error %d: %s" % (code, msg))
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libengram.so is not built (run hashed_gram_embedding_compress_b200."
+                          "build.build() or __graft_entry__.build()); there is no fallback")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    H = ctypes.c_void_p
+    sig = {
+        "engram_create": ([ctypes.POINTER(engram_config), ctypes.POINTER(H)], ctypes.c_int),
+        "engram_destroy": ([H], None),
+        "engram_config_size": ([], ctypes.c_size_t),
+        "engram_last_error": ([H], ctypes.c_char_p),
+        "engram_set_params": ([H, P, P, P, P, P], ctypes.c_int),
+        "engram_reserve": ([H, i64], ctypes.c_int),
+        "engram_get_hash_params": ([H, P, P], ctypes.c_int),
+        "engram_hash": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
+        "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
+        "engram_forward": ([H, P, P, i32, i32, i32, P, P, P, P, P], ctypes.c_int),
+        "engram_prefetch": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
+        "engram_check_errors": ([H, P], ctypes.c_int),
+        "engram_profile_next_forward": ([H, P, i32], ctypes.c_int),
+        "engram_kernel_launches": ([H], ctypes.c_int64),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    if L.engram_config_size() != ctypes.sizeof(engram_config):
+        raise ImportError("engram_config layout mismatch between binding and library")
+    return L
+
+
+lib = _load()
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_config(*, vocab, cvocab, comp_map: torch.Tensor, orders: Sequence[int] = (2, 3),
+                heads=8, d_head=80, d_hidden=2560, branches=1, dtype="bf16", eps=1e-6,
+                table_rows_target=1 << 20, primes: Optional[Sequence[int]] = None,
+                hash_seed=0, pad_id=-1, table_location="device"):
+    """Fill an engram_config; keeps the host map alive on the returned object."""
+    c = engram_config()
+    c.vocab, c.cvocab, c.pad_id = vocab, cvocab, pad_id
+    c.num_orders = len(orders)
+    for i, o in enumerate(orders):
+        c.orders[i] = o
+    c.heads, c.d_head, c.d_hidden, c.branches = heads, d_head, d_hidden, branches
+    c.dtype = {"f32": ENGRAM_F32, "bf16": ENGRAM_BF16}[dtype]
+    c.table_location = {"device": ENGRAM_DEVICE, "pinned_host": ENGRAM_PINNED_HOST}[table_location]
+    c.eps = eps
+    c.table_rows_target = table_rows_target
+    c.hash_seed = hash_seed & 0xFFFFFFFFFFFFFFFF
+    if primes is not None:
+        for i, p in enumerate(primes):
+            c.primes[i] = p
+    m = comp_map.to(torch.int32).contiguous().cpu()
+    c._map_keepalive = m
+    c.comp_map = ctypes.cast(m.data_ptr(), ctypes.POINTER(ctypes.c_int32))
+    return c
+
+
+class Engram:
+    """One handle of the forward lookup-and-gate module."""
+
+    def __init__(self, cfg: engram_config):
+        self._h = ctypes.c_void_p()
+        rc = lib.engram_create(ctypes.byref(cfg), ctypes.byref(self._h))
+        if rc != ENGRAM_OK:
+            raise EngramError(rc, lib.engram_last_error(None).decode())
+        self.cfg = cfg
+        self.S = cfg.num_orders * cfg.heads
+        self.max_order = cfg.orders[cfg.num_orders - 1]
+        self.d_mem = self.S * cfg.d_head
+        self._params = None
+
+    def _check(self, rc):
+        if rc != ENGRAM_OK:
+            raise EngramError(rc, lib.engram_last_error(self._h).decode())
+
+    def close(self):
+        if self._h:
+            lib.engram_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # --------------------------------------------------------------- calls
+    def hash_params(self):
+        primes = torch.zeros(self.S, dtype=torch.int64)
+        mult = torch.zeros(self.S * self.max_order, dtype=torch.int64)
+        self._check(lib.engram_get_hash_params(self._h, primes.data_ptr(), mult.data_ptr()))
+        return primes, mult.view(self.S, self.max_order)
+
+    def set_params(self, tables: Sequence[torch.Tensor], w_k, w_v, norm_q, norm_k):
+        arr = (ctypes.c_void_p * self.S)(*[t.data_ptr() for t in tables])
+        self._check(lib.engram_set_params(self._h, ctypes.cast(arr, ctypes.c_void_p), _ptr(w_k),
+                                          _ptr(w_v), _ptr(norm_q), _ptr(norm_k)))
+        self._params = (list(tables), w_k, w_v, norm_q, norm_k)  # borrowed: keep alive
+
+    def reserve(self, max_rows: int):
+        self._check(lib.engram_reserve(self._h, max_rows))
+
+    def hash(self, tokens, idx, t_begin=0, stream=None):
+        B, T = tokens.shape
+        self._check(lib.engram_hash(self._h, _ptr(tokens), B, T, t_begin, _ptr(idx),
+                                    _stream_ptr(stream)))
+
+    def gather(self, idx, e, stream=None):
+        self._check(lib.engram_gather(self._h, _ptr(idx), idx.shape[0], _ptr(e),
+                                      _stream_ptr(stream)))
+
+    def forward(self, tokens, h, out, idx=None, t_begin=0, alpha=None, delta=None, stream=None):
+        B, T = tokens.shape
+        self._check(lib.engram_forward(self._h, _ptr(tokens), _ptr(idx), B, T, t_begin, _ptr(h),
+                                       _ptr(out), _ptr(alpha), _ptr(delta), _stream_ptr(stream)))
+
+    def prefetch(self, tokens, t_begin=0, stream=None, want_count=False):
+        B, T = tokens.shape
+        n = ctypes.c_int64(0)
+        self._check(lib.engram_prefetch(self._h, _ptr(tokens), B, T, t_begin, _stream_ptr(stream),
+                                        ctypes.byref(n) if want_count else None))
+        return n.value if want_count else None
+
+    def profile_next_forward(self, events):
+        """Record 5 CUDA events inside the next forward (stage boundaries)."""
+        self._prof_keep = list(events)
+        arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+        self._check(lib.engram_profile_next_forward(self._h, ctypes.cast(arr, ctypes.c_void_p), 5))
+
+    def kernel_launches(self) -> int:
+        return int(lib.engram_kernel_launches(self._h))
+
+    def check_errors(self, stream=None) -> int:
+        """Synchronise the stream; return the device error status (0 = none)."""
+        return lib.engram_check_errors(self._h, _stream_ptr(stream))

@@ -1,0 +1,253 @@
+/*
+ * engram.h -- C ABI of libengram.so: the forward lookup-and-gate step of the
+ * Engram conditional-memory module on one NVIDIA B200 (sm_100a).
+ *
+ * Method: "Conditional Memory via Scalable Lookup: A New Axis of Sparsity for
+ * Large Language Models" (DeepSeek-AI & Peking University), section 2:
+ *   2.2  tokenizer compression x' = P(x), suffix n-grams g_{t,n},
+ *        multi-head hashing z_{t,n,k} = phi_{n,k}(g_{t,n}) into tables of
+ *        prime size (Eq. 1), concatenation e_t of the addressed rows (Eq. 2);
+ *   2.3  k_t = W_K e_t, v_t = W_V e_t (Eq. 3);
+ *        alpha_t = sigmoid(RMSNorm(h_t) . RMSNorm(k_t) / sqrt(d)) (Eq. 4);
+ *        gated value alpha_t v_t added to the hidden state;
+ *   2.4  multi-branch form: one W_K per branch, W_V shared (Eq. 6);
+ *   2.5  tables offloaded to host memory, rows prefetched over PCIe
+ *        because the indices depend on the tokens only (Figure 2b).
+ *
+ * Conventions for every call:
+ *  - Return value: ENGRAM_OK (0) or one of the ENGRAM_ERR_* codes below.  No
+ *    call aborts or throws; engram_last_error() gives a message for the last
+ *    failure on that handle.
+ *  - "device" pointers point into the memory of the device that was current
+ *    at engram_create; "host" pointers are ordinary CPU memory; "pinned host"
+ *    is page-locked host memory (cudaHostAlloc / cudaHostRegister).
+ *  - All tensors are row-major and densely packed; shapes are given in
+ *    brackets, outermost first.  Every buffer is owned by the caller and is
+ *    only borrowed for the duration of the call, except the parameter
+ *    pointers given to engram_set_params, which must stay valid until the
+ *    handle is destroyed or new parameters are set.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is enqueued asynchronously on it; results are ready when
+ *    the stream reaches that point.  A handle must not be used from two
+ *    streams at once: its scratch buffers are shared by its calls.
+ *  - Device-side range violations (a token id outside [0, V)) never lead to
+ *    an out-of-bounds access: the kernel substitutes the pad id, sets a bit in
+ *    the handle's device error word, and engram_check_errors() reports it.
+ */
+#ifndef ENGRAM_H
+#define ENGRAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define ENGRAM_API __attribute__((visibility("default")))
+#else
+#define ENGRAM_API
+#endif
+
+#define ENGRAM_MAX_ORDERS 4   /* n-gram orders per module            */
+#define ENGRAM_MAX_TABLES 64  /* orders x heads                      */
+#define ENGRAM_MAX_BRANCHES 4 /* M of the multi-branch form (Eq. 6)  */
+
+/* element types */
+#define ENGRAM_F32 0
+#define ENGRAM_BF16 1
+
+/* where the embedding tables live */
+#define ENGRAM_DEVICE 0      /* HBM of the handle's device            */
+#define ENGRAM_PINNED_HOST 1 /* page-locked host memory, read over PCIe */
+
+/* status codes */
+#define ENGRAM_OK 0
+#define ENGRAM_ERR_INVALID 1     /* bad argument or configuration                 */
+#define ENGRAM_ERR_BOUNDS 2      /* a token id outside [0, V) was seen on device  */
+#define ENGRAM_ERR_CUDA 3        /* a CUDA runtime call failed                     */
+#define ENGRAM_ERR_OOM 4         /* device or pinned allocation failed             */
+#define ENGRAM_ERR_TIMEOUT 5     /* a bounded device-side or prefetch wait expired */
+#define ENGRAM_ERR_UNSUPPORTED 6 /* valid request this build does not implement   */
+#define ENGRAM_ERR_STATE 7       /* call out of order (e.g. forward before params) */
+
+typedef struct engram_handle engram_handle;
+
+/*
+ * Module configuration (section 2.2 and Table 5 of the paper; the paper's
+ * Engram-27B uses orders {2,3}, 8 heads, d_mem 1280, M = 4).
+ *
+ *  vocab, cvocab   V and V' of the compression map P: V -> V' (section 2.2,
+ *                  "Tokenizer compression").  comp_map is a HOST int32 [vocab]
+ *                  array with values in [0, cvocab); it is copied at create.
+ *  pad_id          compressed id read for positions before a sequence's start;
+ *                  -1 selects the default cvocab (outside the image of P, so a
+ *                  padded n-gram never aliases a real one).
+ *  num_orders,     the n-gram orders, ascending, each in [1, 4] (paper: {2,3}).
+ *  orders
+ *  heads           K hash heads per order.  Table slot s = order_index*K + k;
+ *                  e_t concatenates the slots in that order (Eq. 2).
+ *  primes          rows of table s.  All zero: derived as the ascending primes
+ *                  >= table_rows_target, one per slot in slot order.  Non-zero
+ *                  entries must all be given and be >= 2 (primality of given
+ *                  sizes is not checked; the paper asks for primes).
+ *  hash_seed       seed of the hash multipliers.  The pages name phi only a
+ *                  "lightweight multiplicative-XOR hash"; this library fixes
+ *                     x = 0; for j < n: x ^= c[t-j] * m[s][j]   (mod 2^64)
+ *                     z = x mod primes[s]
+ *                  with m[s][j] = SplitMix64(hash_seed) | 1 drawn for s
+ *                  ascending, then j ascending, max(orders) draws per slot
+ *                  (SplitMix64: Steele, Lea and Flood, OOPSLA 2014).
+ *  d_head          d_h, columns of every table; d_mem = S * d_h.
+ *  d_hidden        d, the backbone hidden size (also the 1/sqrt(d) scale).
+ *  branches        M (1 = single stream, Eq. 4; > 1 = Eq. 6).
+ *  dtype           ENGRAM_F32 or ENGRAM_BF16: type of tables, W_K, W_V, h and
+ *                  out.  Accumulation is always fp32.
+ *  eps             RMSNorm epsilon (the pages give none; 1e-6 is typical).
+ *  table_location  ENGRAM_DEVICE or ENGRAM_PINNED_HOST.
+ */
+typedef struct engram_config {
+  int32_t vocab;
+  int32_t cvocab;
+  int32_t pad_id;
+  int32_t num_orders;
+  int32_t orders[ENGRAM_MAX_ORDERS];
+  int32_t heads;
+  int32_t d_head;
+  int32_t d_hidden;
+  int32_t branches;
+  int32_t dtype;
+  int32_t table_location;
+  float eps;
+  int32_t reserved0;
+  int64_t table_rows_target;
+  uint64_t hash_seed;
+  int64_t primes[ENGRAM_MAX_TABLES];
+  const int32_t *comp_map;
+} engram_config;
+
+/*
+ * Validate `cfg`, derive primes and multipliers, copy the compression map to
+ * the current device, and return a new handle in *out.  Requirements:
+ * 1 <= cvocab <= vocab; 1 <= heads; num_orders * heads <= 64; d_head >= 1 with
+ * d_head * element size a multiple of 16 bytes; d_hidden a multiple of 64;
+ * 1 <= branches <= 4.  Errors: ENGRAM_ERR_INVALID, _OOM, _CUDA.
+ */
+ENGRAM_API int engram_create(const engram_config *cfg, engram_handle **out);
+
+/* Release everything the handle owns (not the caller's buffers).  NULL is a no-op. */
+ENGRAM_API void engram_destroy(engram_handle *h);
+
+/* sizeof(engram_config) as compiled into the library (for bindings to check their layout). */
+ENGRAM_API size_t engram_config_size(void);
+
+/* Message of the last failure on `h` (or of the last failed create if h is NULL). */
+ENGRAM_API const char *engram_last_error(const engram_handle *h);
+
+/*
+ * Borrow the learned parameters (section 2.2 and 2.3).
+ *  tables  array of S pointers; table s is [primes[s], d_head] of dtype,
+ *          device memory or pinned host memory according to table_location.
+ *          Rows must start 16-byte aligned.
+ *  w_k     device [M, d, d_mem] dtype: one key projection per branch (Eq. 6).
+ *  w_v     device [d, d_mem] dtype: the shared value projection (Eq. 3).
+ *  norm_q  device fp32 [M, d]: RMSNorm weight of the query h (Eq. 4).
+ *  norm_k  device fp32 [M, d]: RMSNorm weight of the key k (Eq. 4).
+ * Errors: ENGRAM_ERR_INVALID (NULL or misaligned pointer), _CUDA.
+ */
+ENGRAM_API int engram_set_params(engram_handle *h, const void *const *tables, const void *w_k,
+                      const void *w_v, const float *norm_q, const float *norm_k);
+
+/*
+ * Pre-allocate the handle's device scratch for calls of up to `max_rows`
+ * emitted positions (rows = B * (T - t_begin)).  Calls with more rows grow the
+ * scratch themselves; reserving first keeps allocation out of timed or
+ * captured regions.  Scratch per row: S int64 indices, d_mem gathered
+ * elements, and 16 bytes per (row, key tile).  Errors: _INVALID, _OOM.
+ */
+ENGRAM_API int engram_reserve(engram_handle *h, int64_t max_rows);
+
+/* Table sizes and multipliers in use: primes [S], mult [S, max(orders)] (host). */
+ENGRAM_API int engram_get_hash_params(const engram_handle *h, int64_t *primes, uint64_t *mult);
+
+/*
+ * Steps 1-3 (section 2.2, Eq. 1): compress, form suffix n-grams (pad before
+ * each sequence's start; n-grams never cross sequences) and hash.
+ *  tokens  device int32 [B, T] raw ids.
+ *  idx     device int64 [B*(T-t_begin), S]: row (b, t) for t >= t_begin.
+ * 0 <= t_begin < T (decode: t_begin = T-1 emits only the newest position,
+ * the earlier tokens being its history).  Errors: _INVALID, _CUDA.
+ */
+ENGRAM_API int engram_hash(engram_handle *h, const int32_t *tokens, int32_t B, int32_t T, int32_t t_begin,
+                int64_t *idx, void *stream);
+
+/*
+ * Step 4 (Eq. 2): e[r, s*d_h:(s+1)*d_h] = table_s[idx[r, s]], bit-exact copy.
+ *  idx  device int64 [rows, S], every entry in [0, primes[s]).
+ *  e    device [rows, d_mem] dtype.
+ * Indices outside a table set ENGRAM_ERR_BOUNDS in the device error word and
+ * the row is filled with zeros instead.  Device-resident tables only.
+ */
+ENGRAM_API int engram_gather(engram_handle *h, const int64_t *idx, int64_t rows, void *e, void *stream);
+
+/*
+ * The whole forward (steps 1-7): out = h + alpha * (W_V e) per branch, with
+ * alpha = sigmoid(RMSNorm_q(h) . RMSNorm_k(W_K e) / sqrt(d)) (Eq. 3, 4, 6).
+ * At the paper's zero-initialised ShortConv (Eq. 5, Table 5) this equals the
+ * module output added to the residual stream.
+ *  tokens  device int32 [B, T].
+ *  idx     device int64 [rows, S] precomputed by engram_hash, or NULL to hash
+ *          inside this call.
+ *  hid     device [rows, M, d] dtype, rows = B*(T-t_begin).
+ *  out     device [rows, M, d] dtype (may alias hid for an in-place update).
+ *  alpha   device fp32 [rows, M] or NULL.
+ *  delta   device fp32 [rows, M, d] or NULL: alpha * v before the residual add.
+ * With ENGRAM_PINNED_HOST tables, the rows must have been staged by
+ * engram_prefetch for the same tokens; the call waits (on the stream) for
+ * that prefetch.  Errors: _INVALID, _STATE, _OOM, _CUDA.
+ */
+ENGRAM_API int engram_forward(engram_handle *h, const int32_t *tokens, const int64_t *idx, int32_t B,
+                   int32_t T, int32_t t_begin, const void *hid, void *out, float *alpha,
+                   float *delta, void *stream);
+
+/*
+ * Deterministic prefetch for host-resident tables (section 2.5, Figure 2b):
+ * hash the tokens of an upcoming step, de-duplicate the addressed rows per
+ * table, and copy each distinct row once from pinned host memory over PCIe
+ * into a device staging buffer, all on `side_stream`.  The next
+ * engram_forward with the same tokens reads the staged rows; its stream waits
+ * for this prefetch through an event, so the copy overlaps whatever runs on
+ * other streams meanwhile.  ENGRAM_PINNED_HOST handles only.
+ * *unique_rows (host, may be NULL) receives the number of distinct rows once
+ * the prefetch has completed (this synchronises side_stream when non-NULL).
+ */
+ENGRAM_API int engram_prefetch(engram_handle *h, const int32_t *tokens, int32_t B, int32_t T,
+                    int32_t t_begin, void *side_stream, int64_t *unique_rows);
+
+/*
+ * Synchronise `stream`, then read and clear the handle's device error word.
+ * Returns ENGRAM_OK, ENGRAM_ERR_BOUNDS (a token or index out of range was
+ * replaced) or ENGRAM_ERR_TIMEOUT (a kernel's bounded wait expired and the
+ * kernel returned early; its outputs are invalid).
+ */
+ENGRAM_API int engram_check_errors(engram_handle *h, void *stream);
+
+/*
+ * Stage timing for the NEXT engram_forward on this handle (one-shot).
+ * `events` holds 5 cudaEvent_t (as void*), created by the caller with timing
+ * enabled.  That forward records them on its stream at: start, after hashing,
+ * after the gather, after the key-projection kernel, after the value-
+ * projection kernel (consecutive events coincide for a stage that does not
+ * run, e.g. hashing when idx is given).  n_events must be 5; NULL clears.
+ */
+ENGRAM_API int engram_profile_next_forward(engram_handle *h, void *const *events, int32_t n_events);
+
+/* Number of CUDA kernels this handle has launched since it was created. */
+ENGRAM_API int64_t engram_kernel_launches(const engram_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENGRAM_H */

@@ -1,0 +1,192 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar: compressed ids and hash indices bit-exact, gathered rows bit-exact;
+fp32 configs max-abs <= 1e-5 on alpha, alpha*v and out; bf16 configs
+relative-L2 <= 1e-3 on alpha and alpha*v (fp32 on the device, fp64 in the
+oracle) and on out against the oracle's out rounded to bf16.
+"""
+import numpy as np
+import pytest
+import torch
+
+from engram_cases import Problem, from_bits, out_close, rel_l2, to_oracle
+from hashed_gram_embedding_compress_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-5
+BF16_REL = 1e-3
+
+
+def run_forward(p: Problem, m, idx=None, alpha=True, delta=True):
+    sh = p.shape
+    R, M, d = sh.rows_out, sh.branches, sh.d_hidden
+    out = torch.empty_like(p.h)
+    a = torch.full((R, M), -1.0, device="cuda") if alpha else None
+    dl = torch.full((R, M, d), float("nan"), device="cuda") if delta else None
+    m.forward(p.tokens.cuda(), p.h, out, idx=idx, t_begin=sh.t_begin, alpha=a, delta=dl)
+    torch.cuda.synchronize()
+    assert m.check_errors() == 0
+    return out, a, dl
+
+
+def check_indices(p: Problem, m):
+    sh = p.shape
+    idx = torch.empty((sh.rows_out, sh.num_tables), dtype=torch.int64, device="cuda")
+    m.hash(p.tokens.cuda(), idx, t_begin=sh.t_begin)
+    torch.cuda.synchronize()
+    primes, mult = m.hash_params()
+    assert np.array_equal(primes.numpy(), p.primes)
+    assert np.array_equal(mult.numpy().view(np.uint64), p.mult)
+    assert np.array_equal(idx.cpu().numpy(), p.z), "hash indices differ from the oracle"
+    return idx
+
+
+def check_rows(p: Problem, m, idx, rows, out, alpha, delta):
+    sh = p.shape
+    e_ref, a_ref, d_ref, o_ref = p.oracle_forward(rows)
+    # gathered memory vectors, bit-exact
+    e = torch.empty((len(rows), sh.d_mem), dtype=synth.torch_dtype(sh.dtype), device="cuda")
+    m.gather(idx[torch.from_numpy(rows).cuda()].contiguous(), e)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_oracle(e), e_ref), "gathered rows differ"
+    rs = torch.from_numpy(rows).cuda()
+    a = alpha[rs].double().cpu().numpy()
+    dl = delta[rs].double().cpu().numpy()
+    o = to_oracle(out[rs])
+    assert np.all((a >= 0) & (a <= 1))
+    if sh.dtype == "f32":
+        assert np.abs(a - a_ref).max() <= F32_TOL
+        assert np.abs(dl - d_ref).max() <= F32_TOL
+        assert out_close(o, o_ref, "f32") <= F32_TOL
+    else:
+        ea, ed, eo = rel_l2(a, a_ref), rel_l2(dl, d_ref), out_close(o, o_ref, "bf16")
+        assert ea <= BF16_REL and ed <= BF16_REL and eo <= BF16_REL, (ea, ed, eo)
+        # bf16 outputs: nearly every element rounds to the same bf16 value
+        assert np.mean(o == o_ref) > 0.98
+
+
+def test_tiny_f32_all_rows():
+    p = Problem(synth.SHAPES["tiny_f32"])
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    rows = np.arange(p.shape.rows_out)
+    check_rows(p, m, idx, rows, out, a, dl)
+
+
+def test_prefill_reduced_all_rows_ragged():
+    # prefill structure at a size the oracle finishes in seconds: 600 rows
+    # (not a multiple of the 128-row tile), several N tiles per branch
+    sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=300, rows_target=4099, d_hidden=512)
+    p = Problem(sh)
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, np.arange(sh.rows_out), out, a, dl)
+
+
+def test_prefill_full_size_sampled():
+    # the benchmarked workload and launch configuration
+    p = Problem(synth.SHAPES["prefill_bf16"])
+    m = p.engram()
+    m.reserve(p.shape.rows_out)
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, p.sample_rows(96), out, a, dl)
+    # without the optional outputs and with caller-supplied indices: same out
+    out2, _, _ = run_forward(p, m, idx=idx, alpha=False, delta=False)
+    assert torch.equal(out, out2)
+
+
+def test_decode_multibranch():
+    p = Problem(synth.SHAPES["decode_mb"])
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, p.sample_rows(48), out, a, dl)
+
+
+@pytest.mark.parametrize("R_B,R_T", [(1, 20000), (1, 10000), (1, 2000), (3, 5), (1, 1)])
+def test_tile_widths_and_ragged_rows(R_B, R_T):
+    # d = 256 lets the launcher pick 256-, 128- and 64-column tiles by row count
+    sh = synth.SHAPES["prefill_bf16"].replace(B=R_B, T=R_T, rows_target=2053, d_hidden=256,
+                                              branches=2)
+    p = Problem(sh)
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, p.sample_rows(64), out, a, dl)
+
+
+def test_hidden_not_multiple_of_128_and_three_branches():
+    sh = synth.SHAPES["decode_mb"].replace(B=37, T=9, t_begin=4, rows_target=1031, d_hidden=192,
+                                           branches=3)
+    p = Problem(sh)
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, np.arange(sh.rows_out), out, a, dl)
+
+
+def test_f32_multibranch_and_t_begin():
+    sh = synth.SHAPES["tiny_f32"].replace(B=5, T=33, t_begin=7, branches=4, d_hidden=192)
+    p = Problem(sh)
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, np.arange(sh.rows_out), out, a, dl)
+
+
+def test_large_hbm_sampled():
+    p = Problem(synth.SHAPES["large_hbm"])
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m, delta=False)
+    rows = p.sample_rows(24)
+    e_ref, a_ref, d_ref, o_ref = p.oracle_forward(rows)
+    rs = torch.from_numpy(rows).cuda()
+    assert rel_l2(a[rs].double().cpu(), a_ref) <= BF16_REL
+    assert out_close(to_oracle(out[rs]), o_ref, "bf16") <= BF16_REL
+    e = torch.empty((len(rows), p.shape.d_mem), dtype=torch.bfloat16, device="cuda")
+    m.gather(idx[rs].contiguous(), e)
+    assert np.array_equal(to_oracle(e), e_ref)
+
+
+def test_in_place_update_and_empty_batch():
+    sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=70, rows_target=3001, d_hidden=256)
+    p = Problem(sh)
+    m = p.engram()
+    out_ref, _, _ = run_forward(p, m, alpha=False, delta=False)
+    h2 = p.h.clone()
+    m.forward(p.tokens.cuda(), h2, h2)  # out aliases h
+    torch.cuda.synchronize()
+    assert torch.equal(h2, out_ref)
+    empty = torch.empty((0, 5), dtype=torch.int32, device="cuda")
+    m.forward(empty, h2[:0], h2[:0])
+    m.hash(empty, torch.empty((0, sh.num_tables), dtype=torch.int64, device="cuda"))
+    assert m.check_errors() == 0
+
+
+def test_out_of_range_tokens_are_reported_not_read():
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["tiny_f32"]
+    p = Problem(sh)
+    m = p.engram()
+    bad = p.tokens.clone()
+    bad[0, 5] = sh.vocab + 7
+    bad[1, 0] = -3
+    idx = torch.empty((sh.rows_out, sh.num_tables), dtype=torch.int64, device="cuda")
+    m.hash(bad.cuda(), idx)
+    assert m.check_errors() == eg.ENGRAM_ERR_BOUNDS
+    assert m.check_errors() == 0  # the error word is cleared by reading it
+    # rows whose n-grams avoid the bad positions are unaffected
+    good = idx.cpu().numpy().reshape(sh.B, sh.T, -1)
+    ref = p.z.reshape(sh.B, sh.T, -1)
+    assert np.array_equal(good[0, :5], ref[0, :5]) and np.array_equal(good[0, 8:], ref[0, 8:])
+    # indices outside a table: zero rows, flagged
+    idx[3, 2] = int(p.primes[2]) + 5
+    e = torch.ones((sh.rows_out, sh.d_mem), device="cuda")
+    m.gather(idx, e)
+    assert m.check_errors() == eg.ENGRAM_ERR_BOUNDS
+    assert torch.all(e[3, 2 * sh.d_head:3 * sh.d_head] == 0)
