@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows-target", type=int, default=None,
+                    help="smaller tables for profiling captures (same kernel shapes); "
+                         "not the benchmarked workload")
     return ap.parse_args()
 
 
@@ -115,12 +118,14 @@ class ClockSampler:
 
 # ------------------------------------------------------------ the workload
 
-def setup(rank: int, device):
+def setup(rank: int, device, rows_target=None):
     import torch
     from hashed_gram_embedding_compress_b200 import engram as eg
     from hashed_gram_embedding_compress_b200 import synth
 
     sh = synth.SHAPES[WORKLOAD]
+    if rows_target:
+        sh = sh.replace(rows_target=rows_target)
     seeds = synth.stream_seeds(sh, extra=rank)
     tokens = synth.make_tokens(sh, seeds)
     comp_map = synth.make_comp_map(sh, seeds)
@@ -175,7 +180,7 @@ def run_ours(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    P = setup(rank, device)
+    P = setup(rank, device, args.rows_target)
     sh, m = P["sh"], P["m"]
     tok_d = P["tokens"].to(device)
     h = P["h"]
@@ -193,6 +198,9 @@ def run_ours(args, rank, world, dist):
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for row in evs:  # torch creates the CUDA event at its first record
+        for ev in row:
+            ev.record(stream)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = m.kernel_launches()
     if dist:
@@ -311,6 +319,8 @@ def run_ours(args, rank, world, dist):
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
+    if args.rows_target:
+        res["config"]["workload"] += " [profiling variant: tables of %d rows]" % args.rows_target
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(P, args.cpu_seconds)
     return res
