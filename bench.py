@@ -87,7 +87,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def __exit__(self, *exc):
         if self.proc:
@@ -97,10 +97,13 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and active throttle reasons of samples in [t0, t1]."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.lines:
+            if (t0 is not None and ts < t0) or (t1 is not None and ts > t1):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -190,11 +193,19 @@ def run_ours(args, rank, world, dist):
     def step():
         m.forward(tok_d, h, out, stream=stream)
 
+    clk = ClockSampler(local).__enter__()
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
     if m.check_errors(stream) != 0:
         raise RuntimeError("device error during warm-up")
+    # keep the GPU under the same back-to-back load for >= 1.5 s before the
+    # timed steps, so that the clock sampler sees the loaded state
+    t_load = time.monotonic()
+    while time.monotonic() - t_load < 1.5:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize()
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
@@ -206,13 +217,15 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record(stream)
-        for k in range(K):
-            m.profile_next_forward(evs[k])
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(K):
+        m.profile_next_forward(evs[k])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    t_end = time.monotonic()
+    time.sleep(0.3)
+    clk.__exit__(None, None, None)
     if dist:
         dist.barrier()
     launches = m.kernel_launches() - launches0
@@ -317,7 +330,8 @@ def run_ours(args, rank, world, dist):
             "steps": E,
         },
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": dict(clk.summary(t_load + 0.5, t_end + 0.15),
+                       window="last 1 s of back-to-back warm-up steps and the timed steps"),
     }
     if args.rows_target:
         res["config"]["workload"] += " [profiling variant: tables of %d rows]" % args.rows_target

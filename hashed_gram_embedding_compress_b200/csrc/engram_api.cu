@@ -634,19 +634,22 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     h->launches += 2;
     return ENGRAM_OK;
   }
-  CUtensorMap map_e;
-  if ((rc = make_map(h, &map_e, h->e, h->d_mem, R, 128))) return rc;
+  ProjMaps maps;
+  const int64_t hcols = (int64_t)g.M * g.d;
+  if ((rc = make_map(h, &maps.e, h->e, h->d_mem, R, 128))) return rc;
+  if ((rc = make_map(h, &maps.h, hid, hcols, R, 128))) return rc;
+  if ((rc = make_map(h, &maps.out, out, hcols, R, 128))) return rc;
   const int64_t mblk = (R + 127) / 128;
   const int bn0 = choose_bn(R, g.M * g.d, h->sms);
   g.key_tile = bn0;
   const int64_t tiles0 = mblk * (g.M * g.d / bn0);
-  CK(h, launch_proj_gate_sm100(0, bn0, map_e, h->map_wk[bn_index(bn0)], g,
-                               (int)(tiles0 < h->sms ? tiles0 : h->sms), st));
+  maps.w = h->map_wk[bn_index(bn0)];
+  CK(h, launch_proj_gate_sm100(0, bn0, maps, g, (int)(tiles0 < h->sms ? tiles0 : h->sms), st));
   CK(h, mark(3));
   const int bn1 = choose_bn(R, g.d, h->sms);
   const int64_t tiles1 = mblk * (g.d / bn1);
-  CK(h, launch_proj_gate_sm100(1, bn1, map_e, h->map_wv[bn_index(bn1)], g,
-                               (int)(tiles1 < h->sms ? tiles1 : h->sms), st));
+  maps.w = h->map_wv[bn_index(bn1)];
+  CK(h, launch_proj_gate_sm100(1, bn1, maps, g, (int)(tiles1 < h->sms ? tiles1 : h->sms), st));
   CK(h, mark(4));
   h->launches += 2;
   return ENGRAM_OK;

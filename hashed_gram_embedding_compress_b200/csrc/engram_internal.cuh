@@ -89,7 +89,12 @@ cudaError_t launch_proj_gate_f32(int phase, const float* e, const float* w, cons
 // bf16 path (tcgen05 / TMEM / TMA, sm_100a).  `bn` in {64, 128, 256}.
 int sm100_stages(int bn);
 size_t sm100_smem_bytes(int bn);
-cudaError_t launch_proj_gate_sm100(int phase, int bn, const CUtensorMap& map_e, const CUtensorMap& map_w,
-                                   const GateArgs& g, int grid, cudaStream_t stream);
+// Tensor maps of one launch: e [R, d_mem], W [N, d_mem] (box 64 x BN), and
+// h / out viewed as [R, M*d] (box 64 x 128); all bf16 with the 128-B swizzle.
+struct ProjMaps {
+  CUtensorMap e, w, h, out;
+};
+cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
+                                   int grid, cudaStream_t stream);
 
 }  // namespace engram

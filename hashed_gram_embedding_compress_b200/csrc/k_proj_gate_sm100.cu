@@ -39,7 +39,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;                    // 64 bf16 = one 128-byte swizzle row
 constexpr uint32_t A_BYTES = BM * BK * 2; // 16 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // 7 warps
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -184,20 +184,46 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 
 __device__ __forceinline__ float sigmoid_f(float s) { return 1.0f / (1.0f + expf(-s)); }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          (uint64_t)map),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+constexpr int H_SLOTS = 2;                  // ring of h / out sub-tiles
+constexpr uint32_t H_BYTES = BM * 64 * 2;   // one sub-tile: 128 rows x 64 bf16, 128-B swizzle
+
 template <int BN>
 struct Cfg {
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static constexpr uint32_t BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 3 * H_SLOTS + 1;
+  static constexpr uint32_t BAR_BYTES = 8 * NUM_BARS + 16;
+  static constexpr size_t SMEM =
+      1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * H_BYTES + BAR_BYTES;
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
+
+// Byte offset of 16-byte chunk c of tile row r in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
 
 template <int BN, int PHASE>
 __global__ void __launch_bounds__(kThreads, 1)
     proj_gate_kernel(const __grid_constant__ CUtensorMap map_e,
-                     const __grid_constant__ CUtensorMap map_w, GateArgs g) {
+                     const __grid_constant__ CUtensorMap map_w,
+                     const __grid_constant__ CUtensorMap map_h,
+                     const __grid_constant__ CUtensorMap map_out, GateArgs g) {
   using C = Cfg<BN>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -205,22 +231,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * C::STAGE_BYTES);
+  uint8_t* hbuf = smem + (size_t)STAGES * C::STAGE_BYTES;
+  const uint32_t sH = smem_u32(hbuf);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(hbuf + (size_t)H_SLOTS * H_BYTES);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  auto hfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + s); };
+  auto hempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + H_SLOTS + s); };
+  auto hdone_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + 2 * H_SLOTS + s); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4 + 3 * H_SLOTS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int R = g.R;
-  const int n_total = PHASE == 0 ? g.M * g.d : g.d;
+  const int R = g.R, d = g.d, M = g.M;
+  const int n_total = PHASE == 0 ? M * d : d;
   const int num_n = n_total / BN;
   const int num_tiles = ((R + BM - 1) / BM) * num_n;
   const int num_kb = (g.d_mem + BK - 1) / BK;
+  // h sub-tiles per output tile: the key phase reads one branch, the value
+  // phase every branch (v is shared, Eq. 6)
+  const int nsub = (BN / 64) * (PHASE == 0 ? 1 : M);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -230,6 +264,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
       mbar_init(tempty_bar(a), 4);
+    }
+    for (int s = 0; s < H_SLOTS; ++s) {
+      mbar_init(hfull_bar(s), 1);
+      mbar_init(hempty_bar(s), PHASE == 0 ? 4 : 1);
+      mbar_init(hdone_bar(s), 4);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -247,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 4) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------- e / W producer (TMA)
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_e) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
@@ -275,6 +314,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok && lane == 0) {
       // give any copy already issued time to land before the CTA's smem is released
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 100000ull) {
+      }
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------- h sub-tile producer (TMA)
+    if (lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_h) : "memory");
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const int m_blk = tile / num_n, n0 = (tile - m_blk * num_n) * BN;
+      for (int i = 0; i < nsub; ++i) {
+        // columns of h viewed as [R, M*d]: key phase n0 + 64q; value phase mb*d + n0 + 64q
+        const int x = PHASE == 0 ? n0 + 64 * i : (i % M) * d + n0 + 64 * (i / M);
+        if (lane == 0) ok = wait_bounded(hempty_bar(slot), phase ^ 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(hfull_bar(slot), H_BYTES);
+          tma_load_2d(sH + slot * H_BYTES, &map_h, hfull_bar(slot), x, m_blk * BM);
+        }
+        __syncwarp();
+        if (++slot == H_SLOTS) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
       const uint64_t t0 = globaltimer();
       while (globaltimer() - t0 < 100000ull) {
       }
@@ -325,54 +394,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int d = g.d, M = g.M;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    // Thread (warp w, lane l) owns tile row r = 32w + l: TMEM lane r and
+    // row r of every h sub-tile in shared memory.
+    const int r = warp * 32 + lane;
+    int acc = 0, hslot = 0;
+    uint32_t acc_phase = 0, hphase = 0;
     bool ok = true;
     const int tiles_per_branch = d / g.key_tile;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
-      if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, g.err);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      const int row = m_blk * BM + warp * 32 + lane;
+      const int row = m_blk * BM + r;
       const bool valid = row < R;
-      const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BN);
       const int n0 = n_blk * BN;
-      float v[32];
-      if (PHASE == 0) {
-        const int mb = n0 / d, j0 = n0 - mb * d;
-        const __nv_bfloat16* hrow =
-            (const __nv_bfloat16*)g.h + ((int64_t)(valid ? row : 0) * M + mb) * d + j0;
-        const float* wrow = g.w_qk + (int64_t)mb * d + j0;
-        float skk = 0.f, shk = 0.f, shh = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          __syncwarp();
-          tmem_ld32(taddr + c * 32, v);
-          if (valid) {
-            const uint4* hp = reinterpret_cast<const uint4*>(hrow + c * 32);
-            const float4* wp = reinterpret_cast<const float4*>(wrow + c * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float hf[8];
-              unpack8(__ldg(hp + q), hf);
-              const float4 w0 = __ldg(wp + 2 * q), w1 = __ldg(wp + 2 * q + 1);
-              const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float k = v[q * 8 + i];
-                skk = fmaf(k, k, skk);
-                shh = fmaf(hf[i], hf[i], shh);
-                shk = fmaf(hf[i] * wf[i], k, shk);
-              }
-            }
-          }
-        }
-        if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
-      } else {
-        float al[kMaxBranches];
+      float al[kMaxBranches];
+      if (PHASE == 1) {
+        // alpha from the key phase's per-tile partial sums (Eq. 4 / Eq. 6)
 #pragma unroll
         for (int mb = 0; mb < kMaxBranches; ++mb) {
           al[mb] = 0.f;
@@ -390,35 +426,108 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
           }
         }
+      }
+      if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, g.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * BN);
+      float v[64];
+      if (PHASE == 0) {
+        const int mb = n0 / d, j0 = n0 - mb * d;
+        const float* wrow = g.w_qk + (int64_t)mb * d + j0;
+        float skk = 0.f, shk = 0.f, shh = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int q = 0; q < BN / 64; ++q) {
           __syncwarp();
-          tmem_ld32(taddr + c * 32, v);
+          tmem_ld32(taddr + q * 64, v);
+          tmem_ld32(taddr + q * 64 + 32, v + 32);
+          if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          const uint8_t* hs = hbuf + hslot * H_BYTES;
+          const float4* wp = reinterpret_cast<const float4*>(wrow + q * 64);
 #pragma unroll
-          for (int mb = 0; mb < kMaxBranches; ++mb) {
-            if (mb >= M || !valid) break;
-            const int64_t base = ((int64_t)row * M + mb) * d + n0 + c * 32;
-            const uint4* hp = reinterpret_cast<const uint4*>((const __nv_bfloat16*)g.h + base);
-            uint4* op = reinterpret_cast<uint4*>((__nv_bfloat16*)g.out + base);
+          for (int c = 0; c < 8; ++c) {
+            float hf[8];
+            unpack8(*reinterpret_cast<const uint4*>(hs + sw128_off(r, c)), hf);
+            const float4 w0 = __ldg(wp + 2 * c), w1 = __ldg(wp + 2 * c + 1);
+            const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float hf[8];
-              unpack8(__ldg(hp + q), hf);
-              float o[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] = fmaf(al[mb], v[q * 8 + i], hf[i]);
-              op[q] = make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]),
-                                 pack2(o[6], o[7]));
-            }
-            if (g.delta) {
-              float4* dp = reinterpret_cast<float4*>(g.delta + base);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dp[q] = make_float4(al[mb] * v[4 * q], al[mb] * v[4 * q + 1],
-                                    al[mb] * v[4 * q + 2], al[mb] * v[4 * q + 3]);
+            for (int i = 0; i < 8; ++i) {
+              const float k = v[c * 8 + i];
+              skk = fmaf(k, k, skk);
+              shh = fmaf(hf[i], hf[i], shh);
+              shk = fmaf(hf[i] * wf[i], k, shk);
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(hempty_bar(hslot));
+          if (++hslot == H_SLOTS) {
+            hslot = 0;
+            hphase ^= 1u;
+          }
         }
+        if (!ok) break;
+        if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
+      } else {
+#pragma unroll 1
+        for (int q = 0; q < BN / 64; ++q) {
+          __syncwarp();
+          tmem_ld32(taddr + q * 64, v);
+          tmem_ld32(taddr + q * 64 + 32, v + 32);
+#pragma unroll 1
+          for (int mb = 0; mb < M; ++mb) {
+            if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            uint8_t* hs = hbuf + hslot * H_BYTES;
+            float a = 0.f;
+#pragma unroll
+            for (int b = 0; b < kMaxBranches; ++b)
+              if (b == mb) a = al[b];
+            // out = h + alpha v, written over h in place, then stored by TMA
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4* p = reinterpret_cast<uint4*>(hs + sw128_off(r, c));
+              float hf[8], o[8];
+              unpack8(*p, hf);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = fmaf(a, v[c * 8 + i], hf[i]);
+              *p = make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]),
+                              pack2(o[6], o[7]));
+            }
+            if (g.delta && valid) {
+              float4* dp = reinterpret_cast<float4*>(g.delta + ((int64_t)row * M + mb) * d + n0 +
+                                                     q * 64);
+#pragma unroll
+              for (int c = 0; c < 16; ++c)
+                dp[c] = make_float4(a * v[4 * c], a * v[4 * c + 1], a * v[4 * c + 2],
+                                    a * v[4 * c + 3]);
+            }
+            fence_async_smem();  // generic-proxy writes -> visible to the TMA store
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hdone_bar(hslot));
+            if (warp == 0) {
+              if (lane == 0) {
+                ok = wait_bounded(hdone_bar(hslot), hphase, abort_flag, g.err);
+                if (ok) {
+                  tma_store_2d(&map_out, sH + hslot * H_BYTES, mb * d + n0 + q * 64, m_blk * BM);
+                  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                  mbar_arrive(hempty_bar(hslot));
+                }
+              }
+              ok = __shfl_sync(0xffffffffu, ok, 0);
+              if (!ok) break;
+            }
+            if (++hslot == H_SLOTS) {
+              hslot = 0;
+              hphase ^= 1u;
+            }
+          }
+          if (!ok) break;
+        }
+        if (!ok) break;
       }
       tc_fence_before();
       __syncwarp();
@@ -428,6 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (PHASE == 1 && warp == 0 && lane == 0)
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   tc_fence_before();
@@ -440,13 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int BN, int PHASE>
-cudaError_t launch_bn(const CUtensorMap& me, const CUtensorMap& mw, const GateArgs& g, int grid,
-                      cudaStream_t stream) {
+cudaError_t launch_bn(const ProjMaps& maps, const GateArgs& g, int grid, cudaStream_t stream) {
   auto kern = proj_gate_kernel<BN, PHASE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg<BN>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, Cfg<BN>::SMEM, stream>>>(me, mw, g);
+  kern<<<grid, kThreads, Cfg<BN>::SMEM, stream>>>(maps.e, maps.w, maps.h, maps.out, g);
   return cudaGetLastError();
 }
 
@@ -460,17 +570,16 @@ size_t sm100_smem_bytes(int bn) {
   return bn == 256 ? Cfg<256>::SMEM : bn == 128 ? Cfg<128>::SMEM : Cfg<64>::SMEM;
 }
 
-cudaError_t launch_proj_gate_sm100(int phase, int bn, const CUtensorMap& map_e,
-                                   const CUtensorMap& map_w, const GateArgs& g, int grid,
-                                   cudaStream_t stream) {
+cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
+                                   int grid, cudaStream_t stream) {
   if (g.R == 0) return cudaSuccess;
   switch (bn * 2 + phase) {
-    case 512: return launch_bn<256, 0>(map_e, map_w, g, grid, stream);
-    case 513: return launch_bn<256, 1>(map_e, map_w, g, grid, stream);
-    case 256: return launch_bn<128, 0>(map_e, map_w, g, grid, stream);
-    case 257: return launch_bn<128, 1>(map_e, map_w, g, grid, stream);
-    case 128: return launch_bn<64, 0>(map_e, map_w, g, grid, stream);
-    case 129: return launch_bn<64, 1>(map_e, map_w, g, grid, stream);
+    case 512: return launch_bn<256, 0>(maps, g, grid, stream);
+    case 513: return launch_bn<256, 1>(maps, g, grid, stream);
+    case 256: return launch_bn<128, 0>(maps, g, grid, stream);
+    case 257: return launch_bn<128, 1>(maps, g, grid, stream);
+    case 128: return launch_bn<64, 0>(maps, g, grid, stream);
+    case 129: return launch_bn<64, 1>(maps, g, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }
