@@ -280,6 +280,7 @@ int engram_create(const engram_config* cfg, engram_handle** out) {
   if (c.table_location != ENGRAM_DEVICE && c.table_location != ENGRAM_PINNED_HOST)
     return fail(nullptr, ENGRAM_ERR_INVALID, "bad table_location");
   if (c.pad_id < -1) return fail(nullptr, ENGRAM_ERR_INVALID, "pad_id must be >= -1");
+  if (c.flags & ~ENGRAM_FLAG_NO_CTA_PAIRS) return fail(nullptr, ENGRAM_ERR_INVALID, "unknown flags");
   const int S = c.num_orders * c.heads;
   const int64_t d_mem = (int64_t)S * c.d_head;
   if (d_mem > (1 << 20)) return fail(nullptr, ENGRAM_ERR_INVALID, "d_mem too large");
@@ -639,18 +640,29 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   if ((rc = make_map(h, &maps.e, h->e, h->d_mem, R, 128))) return rc;
   if ((rc = make_map(h, &maps.h, hid, hcols, R, 128))) return rc;
   if ((rc = make_map(h, &maps.out, out, hcols, R, 128))) return rc;
-  const int64_t mblk = (R + 127) / 128;
-  const int bn0 = choose_bn(R, g.M * g.d, h->sms);
-  g.key_tile = bn0;
-  const int64_t tiles0 = mblk * (g.M * g.d / bn0);
-  maps.w = h->map_wk[bn_index(bn0)];
-  CK(h, launch_proj_gate_sm100(0, bn0, maps, g, (int)(tiles0 < h->sms ? tiles0 : h->sms), st));
-  CK(h, mark(3));
-  const int bn1 = choose_bn(R, g.d, h->sms);
-  const int64_t tiles1 = mblk * (g.d / bn1);
-  maps.w = h->map_wv[bn_index(bn1)];
-  CK(h, launch_proj_gate_sm100(1, bn1, maps, g, (int)(tiles1 < h->sms ? tiles1 : h->sms), st));
-  CK(h, mark(4));
+  const bool pairs_ok = !(h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS);
+  for (int phase = 0; phase < 2; ++phase) {
+    const int n_total = phase == 0 ? g.M * g.d : g.d;
+    const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
+    int bn, grid;
+    bool pair = false;
+    const int64_t ptiles = (R + 255) / 256 * (n_total / 256);
+    if (pairs_ok && n_total % 256 == 0 && ptiles >= h->sms / 2) {
+      // 256 x 256 tiles on CTA pairs; each CTA loads 128 rows of W
+      pair = true;
+      bn = 256;
+      grid = 2 * (int)(ptiles < h->sms / 2 ? ptiles : h->sms / 2);
+      maps.w = wmaps[bn_index(128)];
+    } else {
+      bn = choose_bn(R, n_total, h->sms);
+      const int64_t tiles = (R + 127) / 128 * (n_total / bn);
+      grid = (int)(tiles < h->sms ? tiles : h->sms);
+      maps.w = wmaps[bn_index(bn)];
+    }
+    if (phase == 0) g.key_tile = bn;
+    CK(h, launch_proj_gate_sm100(phase, bn, pair, maps, g, grid, st));
+    CK(h, mark(3 + phase));
+  }
   h->launches += 2;
   return ENGRAM_OK;
 }

@@ -94,7 +94,8 @@ size_t sm100_smem_bytes(int bn);
 struct ProjMaps {
   CUtensorMap e, w, h, out;
 };
-cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
-                                   int grid, cudaStream_t stream);
+// pair: 256 x 256 tiles on CTA pairs (cta_group::2; bn must be 256, grid even).
+cudaError_t launch_proj_gate_sm100(int phase, int bn, bool pair, const ProjMaps& maps,
+                                   const GateArgs& g, int grid, cudaStream_t stream);
 
 }  // namespace engram

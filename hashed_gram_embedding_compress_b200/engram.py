@@ -22,6 +22,7 @@ ENGRAM_DEVICE, ENGRAM_PINNED_HOST = 0, 1
 ENGRAM_OK, ENGRAM_ERR_INVALID, ENGRAM_ERR_BOUNDS, ENGRAM_ERR_CUDA = 0, 1, 2, 3
 ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_UNSUPPORTED, ENGRAM_ERR_STATE = 4, 5, 6, 7
 MAX_ORDERS, MAX_TABLES, MAX_BRANCHES = 4, 64, 4
+ENGRAM_FLAG_NO_CTA_PAIRS = 1
 
 #: every symbol include/engram.h declares
 EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last_error",
@@ -37,7 +38,7 @@ class engram_config(ctypes.Structure):
         ("heads", ctypes.c_int32), ("d_head", ctypes.c_int32), ("d_hidden", ctypes.c_int32),
         ("branches", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("table_location", ctypes.c_int32), ("eps", ctypes.c_float),
-        ("reserved0", ctypes.c_int32), ("table_rows_target", ctypes.c_int64),
+        ("flags", ctypes.c_int32), ("table_rows_target", ctypes.c_int64),
         ("hash_seed", ctypes.c_uint64), ("primes", ctypes.c_int64 * MAX_TABLES),
         ("comp_map", ctypes.POINTER(ctypes.c_int32)),
     ]
@@ -101,7 +102,7 @@ def _stream_ptr(stream) -> Optional[int]:
 def make_config(*, vocab, cvocab, comp_map: torch.Tensor, orders: Sequence[int] = (2, 3),
                 heads=8, d_head=80, d_hidden=2560, branches=1, dtype="bf16", eps=1e-6,
                 table_rows_target=1 << 20, primes: Optional[Sequence[int]] = None,
-                hash_seed=0, pad_id=-1, table_location="device"):
+                hash_seed=0, pad_id=-1, table_location="device", flags=0):
     """Fill an engram_config; keeps the host map alive on the returned object."""
     c = engram_config()
     c.vocab, c.cvocab, c.pad_id = vocab, cvocab, pad_id
@@ -112,6 +113,7 @@ def make_config(*, vocab, cvocab, comp_map: torch.Tensor, orders: Sequence[int] 
     c.dtype = {"f32": ENGRAM_F32, "bf16": ENGRAM_BF16}[dtype]
     c.table_location = {"device": ENGRAM_DEVICE, "pinned_host": ENGRAM_PINNED_HOST}[table_location]
     c.eps = eps
+    c.flags = flags
     c.table_rows_target = table_rows_target
     c.hash_seed = hash_seed & 0xFFFFFFFFFFFFFFFF
     if primes is not None:

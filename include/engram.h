@@ -62,6 +62,9 @@ extern "C" {
 #define ENGRAM_DEVICE 0      /* HBM of the handle's device            */
 #define ENGRAM_PINNED_HOST 1 /* page-locked host memory, read over PCIe */
 
+/* config flags */
+#define ENGRAM_FLAG_NO_CTA_PAIRS 1
+
 /* status codes */
 #define ENGRAM_OK 0
 #define ENGRAM_ERR_INVALID 1     /* bad argument or configuration                 */
@@ -106,6 +109,9 @@ typedef struct engram_handle engram_handle;
  *                  out.  Accumulation is always fp32.
  *  eps             RMSNorm epsilon (the pages give none; 1e-6 is typical).
  *  table_location  ENGRAM_DEVICE or ENGRAM_PINNED_HOST.
+ *  flags           0, or ENGRAM_FLAG_NO_CTA_PAIRS to keep the bf16 projection
+ *                  on single-CTA 128-row tiles (the default uses 256 x 256
+ *                  tiles on CTA pairs when the shape fills the GPU).
  */
 typedef struct engram_config {
   int32_t vocab;
@@ -120,7 +126,7 @@ typedef struct engram_config {
   int32_t dtype;
   int32_t table_location;
   float eps;
-  int32_t reserved0;
+  int32_t flags;
   int64_t table_rows_target;
   uint64_t hash_seed;
   int64_t primes[ENGRAM_MAX_TABLES];

@@ -67,14 +67,14 @@ class Problem:
         self.h = synth.make_hidden(sh, self.seeds, device=self.device)
 
     # ------------------------------------------------------------ CUDA path
-    def engram(self, eps: float = 1e-6):
+    def engram(self, eps: float = 1e-6, flags: int = 0):
         from hashed_gram_embedding_compress_b200 import engram as eg
         sh = self.shape
         cfg = eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=self.comp_map,
                              orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
                              d_hidden=sh.d_hidden, branches=sh.branches, dtype=sh.dtype, eps=eps,
                              table_rows_target=sh.rows_target, hash_seed=self.hash_seed,
-                             table_location=sh.table_location)
+                             table_location=sh.table_location, flags=flags)
         m = eg.Engram(cfg)
         m.set_params(self.tables, self.w_k, self.w_v, self.norm_q, self.norm_k)
         return m
