@@ -124,17 +124,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `rows` rows of `cols` elements, box 64 x box_rows, 128-B swizzle.
+// 2-D bf16 tensor map: `rows` rows of `cols` elements, box box_cols x box_rows;
+// the swizzle width is the box row width (64 columns = 128 B, 32 columns = 64 B).
 int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
-             int box_rows) {
+             int box_rows, int box_cols = 64) {
   auto fn = encode_fn();
   if (!fn) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapSwizzle sw =
+      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   return ENGRAM_OK;
@@ -635,32 +638,42 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     h->launches += 2;
     return ENGRAM_OK;
   }
-  ProjMaps maps;
+  // Tensor maps are built for whichever kernel each phase uses: 512 x 256
+  // tiles on CTA pairs when the tile count fills every pair at least once,
+  // else single-CTA 128-row tiles of the widest N that fills the SMs.
   const int64_t hcols = (int64_t)g.M * g.d;
-  if ((rc = make_map(h, &maps.e, h->e, h->d_mem, R, 128))) return rc;
-  if ((rc = make_map(h, &maps.h, hid, hcols, R, 128))) return rc;
-  if ((rc = make_map(h, &maps.out, out, hcols, R, 128))) return rc;
   const bool pairs_ok = !(h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS);
+  ProjMaps single, wide;
+  bool have_single = false, have_wide = false;
   for (int phase = 0; phase < 2; ++phase) {
     const int n_total = phase == 0 ? g.M * g.d : g.d;
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
-    int bn, grid;
-    bool pair = false;
-    const int64_t ptiles = (R + 255) / 256 * (n_total / 256);
-    if (pairs_ok && n_total % 256 == 0 && ptiles >= h->sms / 2) {
-      // 256 x 256 tiles on CTA pairs; each CTA loads 128 rows of W
-      pair = true;
-      bn = 256;
-      grid = 2 * (int)(ptiles < h->sms / 2 ? ptiles : h->sms / 2);
-      maps.w = wmaps[bn_index(128)];
+    const int64_t wtiles = (R + 511) / 512 * (n_total / 256);
+    if (pairs_ok && n_total % 256 == 0 && wtiles >= h->sms / 2) {
+      if (!have_wide) {
+        if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
+        if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
+        if ((rc = make_map(h, &wide.out, out, hcols, R, 256, 32))) return rc;
+        have_wide = true;
+      }
+      wide.w = wmaps[bn_index(128)];  // each CTA of a pair loads 128 of the tile's 256 W rows
+      if (phase == 0) g.key_tile = 256;
+      const int pairs = (int)(wtiles < h->sms / 2 ? wtiles : h->sms / 2);
+      CK(h, launch_proj_gate_wide(phase, wide, g, 2 * pairs, st));
     } else {
-      bn = choose_bn(R, n_total, h->sms);
+      if (!have_single) {
+        if ((rc = make_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;
+        if ((rc = make_map(h, &single.h, hid, hcols, R, 128))) return rc;
+        if ((rc = make_map(h, &single.out, out, hcols, R, 128))) return rc;
+        have_single = true;
+      }
+      const int bn = choose_bn(R, n_total, h->sms);
       const int64_t tiles = (R + 127) / 128 * (n_total / bn);
-      grid = (int)(tiles < h->sms ? tiles : h->sms);
-      maps.w = wmaps[bn_index(bn)];
+      single.w = wmaps[bn_index(bn)];
+      if (phase == 0) g.key_tile = bn;
+      CK(h, launch_proj_gate_sm100(phase, bn, single, g, (int)(tiles < h->sms ? tiles : h->sms),
+                                   st));
     }
-    if (phase == 0) g.key_tile = bn;
-    CK(h, launch_proj_gate_sm100(phase, bn, pair, maps, g, grid, st));
     CK(h, mark(3 + phase));
   }
   h->launches += 2;

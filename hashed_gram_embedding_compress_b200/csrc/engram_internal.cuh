@@ -88,14 +88,17 @@ cudaError_t launch_proj_gate_f32(int phase, const float* e, const float* w, cons
 
 // bf16 path (tcgen05 / TMEM / TMA, sm_100a).  `bn` in {64, 128, 256}.
 int sm100_stages(int bn);
-size_t sm100_smem_bytes(int bn);
-// Tensor maps of one launch: e [R, d_mem], W [N, d_mem] (box 64 x BN), and
-// h / out viewed as [R, M*d] (box 64 x 128); all bf16 with the 128-B swizzle.
+// Tensor maps of one launch, all bf16: e [R, d_mem] and W [N, d_mem] with the
+// 128-byte swizzle, h and out viewed as [R, M*d].
+//   single-CTA kernel: e box 64 x 128, W box 64 x BN, h/out box 64 x 128 (128-B swizzle)
+//   CTA-pair kernel:   e box 64 x 256, W box 64 x 128, h/out box 32 x 256 (64-B swizzle)
 struct ProjMaps {
   CUtensorMap e, w, h, out;
 };
-// pair: 256 x 256 tiles on CTA pairs (cta_group::2; bn must be 256, grid even).
-cudaError_t launch_proj_gate_sm100(int phase, int bn, bool pair, const ProjMaps& maps,
-                                   const GateArgs& g, int grid, cudaStream_t stream);
+cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
+                                   int grid, cudaStream_t stream);
+// 512 x 256 tiles on CTA pairs (tcgen05 cta_group::2); grid = 2 x pairs.
+cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
+                                  cudaStream_t stream);
 
 }  // namespace engram

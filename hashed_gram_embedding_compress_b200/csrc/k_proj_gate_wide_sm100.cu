@@ -1,0 +1,438 @@
+// bf16 projection + context-aware gate on CTA pairs: the large-batch path.
+//
+// Same computation as k_proj_gate_sm100.cu ("Conditional Memory via Scalable
+// Lookup", section 2.3 Eq. (3)-(4), section 2.4 Eq. (6)); only the tiling
+// differs.  A cluster of two CTAs on one TPC computes a 512 x 256 tile of
+// e . W^T with tcgen05.mma.cta_group::2 (M = 256 per instruction):
+//
+//   CTA rank r holds rows [256 r, 256 r + 256) of the tile: it loads those
+//   256 rows of e (one 256 x 64 TMA box per K step) and rows
+//   [128 r, 128 r + 128) of the 256 W rows (the pair's B operand is split by
+//   N), and keeps two 128 x 256 fp32 accumulators in its 512 TMEM columns
+//   (tile rows 0-127 in columns 0-255, rows 128-255 in columns 256-511).
+//   The leader (rank 0) issues, per 16-wide K step, two pair MMAs that share
+//   B: rows 0-127 of both CTAs, then rows 128-255 of both CTAs.
+//
+// Each byte brought from L2 feeds 1.5x the FLOPs of a 128-row tile, which is
+// what the mainloop is bound by on this part: the operand stream from L2
+// into shared memory, not the tensor pipe.  TMEM holds one tile, so the
+// epilogue runs between tiles; eight epilogue warps keep it short, and h is
+// prefetched into a 5-slot ring during the mainloop.
+//
+// Roles (352 threads per CTA):
+//   warps 0-7   epilogue: warp w reads TMEM lanes 32(w%4).. of accumulator
+//               w/4, i.e. tile row 128(w/4) + 32(w%4) + lane;
+//   warp 8      TMA producer of e and W (3 stages x 48 KB);
+//   warp 9      TMEM allocator; MMA issuer on the leader;
+//   warp 10     TMA producer of h sub-tiles [256 rows x 32 columns, 64-byte
+//               swizzle], shared by both epilogue warpgroups; in the value
+//               phase out is written over h in the slot and stored by TMA.
+// Waits are bounded as in the single-CTA kernel; the pair leaves together
+// through a bounded handshake, then frees TMEM (cta_group::2).
+#include "sm100_ptx.cuh"
+
+namespace engram {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 256;                           // tile rows per CTA
+constexpr int kCols = 256;                           // tile columns
+constexpr int BK = 64;
+constexpr uint32_t A_BYTES = kRows * BK * 2;         // 32 KB
+constexpr uint32_t B_BYTES = (kCols / 2) * BK * 2;   // 16 KB: this CTA's half of B
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int STAGES = 3;
+constexpr int H_SLOTS = 5;
+constexpr int H_COLS = 32;
+constexpr uint32_t H_BYTES = kRows * H_COLS * 2;     // 16 KB
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (kEpiWarps + 3) * 32;       // 352
+constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1, kHWarp = kEpiWarps + 2;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int NUM_BARS = 2 * STAGES + 2 + 3 * H_SLOTS + 2;
+constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * H_BYTES +
+                        8 * NUM_BARS + 16;
+static_assert(SMEM <= 232448, "shared memory budget");
+
+template <int PHASE>
+__global__ void __launch_bounds__(kThreads, 1)
+    proj_gate_wide_kernel(const __grid_constant__ CUtensorMap map_e,
+                          const __grid_constant__ CUtensorMap map_w,
+                          const __grid_constant__ CUtensorMap map_h,
+                          const __grid_constant__ CUtensorMap map_out, GateArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + STAGES * A_BYTES;
+  uint8_t* hbuf = smem + (size_t)STAGES * STAGE_BYTES;
+  const uint32_t sH = smem_u32(hbuf);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(hbuf + (size_t)H_SLOTS * H_BYTES);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES);
+  const uint32_t tempty_bar = tfull_bar + 8u;
+  auto hfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + s); };
+  auto hempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + H_SLOTS + s); };
+  auto hdone_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + 2 * H_SLOTS + s); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 + 3 * H_SLOTS);
+  const uint32_t pair_bar = drain_bar + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = the pair's MMA leader
+  const bool leader = rank == 0;
+  const int R = g.R, d = g.d, M = g.M;
+  const int n_total = PHASE == 0 ? M * d : d;
+  const int num_n = n_total / kCols;
+  const int num_tiles = ((R + 2 * kRows - 1) / (2 * kRows)) * num_n;
+  const int num_kb = (g.d_mem + BK - 1) / BK;
+  const int first_tile = (int)(blockIdx.x >> 1), tile_step = (int)(gridDim.x >> 1);
+  // h sub-tiles per tile: one branch in the key phase, every branch in the
+  // value phase (v is shared across branches, Eq. 6)
+  const int nsub = (kCols / H_COLS) * (PHASE == 0 ? 1 : M);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(tfull_bar, 1);
+    mbar_init(tempty_bar, 2 * kEpiWarps);  // every epilogue warp of the pair
+    for (int s = 0; s < H_SLOTS; ++s) {
+      mbar_init(hfull_bar(s), 1);
+      mbar_init(hempty_bar(s), PHASE == 0 ? kEpiWarps : 1);
+      mbar_init(hdone_bar(s), kEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(pair_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the partner's barriers are initialised before any signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    // ---------------------------------------------------- e / W producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_e) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_w) : "memory");
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
+      const int a_row = m_blk * 2 * kRows + (int)rank * kRows;
+      const int b_row = n_blk * kCols + (int)rank * (kCols / 2);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (lane == 0) ok = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          // the leader's full barrier counts the bytes of both CTAs
+          const uint32_t fb = peer_addr(full_bar(stage), 0);
+          if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          tma_load_2d_pair(sA + stage * A_BYTES, &map_e, fb, kb * BK, a_row);
+          tma_load_2d_pair(sB + stage * B_BYTES, &map_w, fb, kb * BK, b_row);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 100000ull) {
+      }
+    }
+  } else if (warp == kHWarp) {
+    // -------------------------------------------------- h sub-tile producer
+    if (lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_h) : "memory");
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      const int m_blk = tile / num_n, n0 = (tile - m_blk * num_n) * kCols;
+      const int row0 = m_blk * 2 * kRows + (int)rank * kRows;
+      for (int i = 0; i < nsub; ++i) {
+        // h viewed as [R, M*d]: key phase column n0 + 32 i; value phase
+        // branch i % M, column n0 + 32 (i / M)
+        const int x = PHASE == 0 ? n0 + H_COLS * i : (i % M) * d + n0 + H_COLS * (i / M);
+        if (lane == 0) ok = wait_bounded(hempty_bar(slot), phase ^ 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(hfull_bar(slot), H_BYTES);
+          tma_load_2d(sH + slot * H_BYTES, &map_h, hfull_bar(slot), x, row0);
+        }
+        __syncwarp();
+        if (++slot == H_SLOTS) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 100000ull) {
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // --------------------------------------------- MMA issuer (leader only)
+    constexpr uint32_t idesc = idesc_bf16<2 * 128, kCols>();
+    int stage = 0;
+    uint32_t phase = 0, tphase = 0;
+    bool ok = true;
+    if (leader) {
+      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+        if (lane == 0) ok = wait_bounded(tempty_bar, tphase ^ 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (lane == 0) ok = wait_bounded(full_bar(stage), phase, abort_flag, g.err);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t a0 = sw128_desc(sA + stage * A_BYTES);
+            const uint64_t a1 = sw128_desc(sA + stage * A_BYTES + A_BYTES / 2);  // rows 128-255
+            const uint64_t bd = sw128_desc(sB + stage * B_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint32_t accum = (kb | k) != 0;
+              umma_bf16_pair(tmem_base, a0 + 2u * k, bd + 2u * k, idesc, accum);
+              umma_bf16_pair(tmem_base + kCols, a1 + 2u * k, bd + 2u * k, idesc, accum);
+            }
+            umma_commit_pair_both(empty_bar(stage));  // slot free in both CTAs
+          }
+          __syncwarp();
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit_pair_both(tfull_bar);  // tile complete in both CTAs
+        __syncwarp();
+        tphase ^= 1u;
+      }
+      if (lane == 0) {
+        umma_commit_pair_local(drain_bar);  // arrives once every MMA above has finished
+        wait_drain(drain_bar, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = half * 128 + quarter * 32 + lane;  // tile row of this thread
+    int hslot = 0;
+    uint32_t hphase = 0, tphase = 0;
+    bool ok = true;
+    const int tiles_per_branch = d / g.key_tile;
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
+      const int row0 = m_blk * 2 * kRows + (int)rank * kRows;  // first row of this CTA
+      const int row = row0 + r;
+      const bool valid = row < R;
+      const int n0 = n_blk * kCols;
+      float al[kMaxBranches];
+      if (PHASE == 1) {
+        // alpha from the key phase's per-tile partial sums (Eq. 4 / Eq. 6);
+        // computed while the MMAs of this tile run
+#pragma unroll
+        for (int mb = 0; mb < kMaxBranches; ++mb) {
+          al[mb] = 0.f;
+          if (mb < M && valid) {
+            float skk = 0.f, shk = 0.f, shh = 0.f;
+            for (int tb = mb * tiles_per_branch; tb < (mb + 1) * tiles_per_branch; ++tb) {
+              const float4 p = g.partials[(int64_t)tb * R + row];
+              skk += p.x;
+              shk += p.y;
+              shh += p.z;
+            }
+            const float rh = 1.0f / sqrtf(shh / (float)d + g.eps);
+            const float rk = 1.0f / sqrtf(skk / (float)d + g.eps);
+            al[mb] = sigmoid_f(shk * rh * rk * g.inv_sqrt_d);
+            if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
+          }
+        }
+      }
+      if (lane == 0) ok = wait_bounded(tfull_bar, tphase, abort_flag, g.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * kCols);
+      float v[32];
+      if (PHASE == 0) {
+        const int mb = n0 / d, j0 = n0 - mb * d;
+        const float* wrow = g.w_qk + (int64_t)mb * d + j0;
+        float skk = 0.f, shk = 0.f, shh = 0.f;
+#pragma unroll 1
+        for (int q = 0; q < kCols / H_COLS; ++q) {
+          __syncwarp();
+          tmem_ld32(taddr + q * H_COLS, v);
+          if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          const uint8_t* hs = hbuf + hslot * H_BYTES;
+          const float4* wp = reinterpret_cast<const float4*>(wrow + q * H_COLS);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float hf[8];
+            unpack8(*reinterpret_cast<const uint4*>(hs + sw64_off(r, c)), hf);
+            const float4 w0 = __ldg(wp + 2 * c), w1 = __ldg(wp + 2 * c + 1);
+            const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float k = v[c * 8 + i];
+              skk = fmaf(k, k, skk);
+              shh = fmaf(hf[i], hf[i], shh);
+              shk = fmaf(hf[i] * wf[i], k, shk);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(hempty_bar(hslot));
+          if (++hslot == H_SLOTS) {
+            hslot = 0;
+            hphase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
+      } else {
+#pragma unroll 1
+        for (int q = 0; q < kCols / H_COLS; ++q) {
+          __syncwarp();
+          tmem_ld32(taddr + q * H_COLS, v);
+#pragma unroll 1
+          for (int mb = 0; mb < M; ++mb) {
+            if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            uint8_t* hs = hbuf + hslot * H_BYTES;
+            float a = 0.f;
+#pragma unroll
+            for (int b = 0; b < kMaxBranches; ++b)
+              if (b == mb) a = al[b];
+            // out = h + alpha v, written over h in place, then stored by TMA
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint4* p = reinterpret_cast<uint4*>(hs + sw64_off(r, c));
+              float hf[8], o[8];
+              unpack8(*p, hf);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = fmaf(a, v[c * 8 + i], hf[i]);
+              *p = make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]),
+                              pack2(o[6], o[7]));
+            }
+            if (g.delta && valid) {
+              float4* dp = reinterpret_cast<float4*>(g.delta + ((int64_t)row * M + mb) * d + n0 +
+                                                     q * H_COLS);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                dp[c] = make_float4(a * v[4 * c], a * v[4 * c + 1], a * v[4 * c + 2],
+                                    a * v[4 * c + 3]);
+            }
+            fence_async_smem();  // generic-proxy writes -> visible to the TMA store
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hdone_bar(hslot));
+            if (warp == 0) {
+              if (lane == 0) {
+                ok = wait_bounded(hdone_bar(hslot), hphase, abort_flag, g.err);
+                if (ok) {
+                  if (row0 < R) {  // rows past R are clipped; a slot wholly past R stores nothing
+                    tma_store_2d(&map_out, sH + hslot * H_BYTES, mb * d + n0 + q * H_COLS, row0);
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                  }
+                  mbar_arrive(hempty_bar(hslot));
+                }
+              }
+              ok = __shfl_sync(0xffffffffu, ok, 0);
+              if (!ok) break;
+            }
+            if (++hslot == H_SLOTS) {
+              hslot = 0;
+              hphase ^= 1u;
+            }
+          }
+          if (!ok) break;
+        }
+        if (!ok) break;
+      }
+      // accumulators free again: the leader owns the barrier
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+      tphase ^= 1u;
+    }
+    if (PHASE == 1 && warp == 0 && lane == 0)
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // neither CTA leaves while its partner may still read its shared memory (the
+  // leader's MMAs) or signal its barriers (the follower's arrivals)
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(peer_addr(pair_bar, rank ^ 1u));
+    wait_drain(pair_bar, 0);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS));
+}
+
+template <int PHASE>
+cudaError_t launch_wide(const ProjMaps& maps, const GateArgs& g, int grid, cudaStream_t stream) {
+  auto kern = proj_gate_wide_kernel<PHASE>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = SMEM;
+  lc.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, kern, maps.e, maps.w, maps.h, maps.out, g);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
+                                  cudaStream_t stream) {
+  if (g.R == 0) return cudaSuccess;
+  if (grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
+  return phase == 0 ? launch_wide<0>(maps, g, grid, stream) : launch_wide<1>(maps, g, grid, stream);
+}
+
+}  // namespace engram
