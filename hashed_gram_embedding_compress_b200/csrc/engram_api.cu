@@ -653,7 +653,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
       if (!have_wide) {
         if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
         if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
-        if ((rc = make_map(h, &wide.out, out, hcols, R, 256, 32))) return rc;
+        if ((rc = make_map(h, &wide.out, out, hcols, R, 32, 32))) return rc;  // per-warp stores
         have_wide = true;
       }
       wide.w = wmaps[bn_index(128)];  // each CTA of a pair loads 128 of the tile's 256 W rows

@@ -91,7 +91,8 @@ int sm100_stages(int bn);
 // Tensor maps of one launch, all bf16: e [R, d_mem] and W [N, d_mem] with the
 // 128-byte swizzle, h and out viewed as [R, M*d].
 //   single-CTA kernel: e box 64 x 128, W box 64 x BN, h/out box 64 x 128 (128-B swizzle)
-//   CTA-pair kernel:   e box 64 x 256, W box 64 x 128, h/out box 32 x 256 (64-B swizzle)
+//   CTA-pair kernel:   e box 64 x 256, W box 64 x 128, h box 32 x 256, out box 32 x 32
+//                      (h and out with the 64-B swizzle)
 struct ProjMaps {
   CUtensorMap e, w, h, out;
 };

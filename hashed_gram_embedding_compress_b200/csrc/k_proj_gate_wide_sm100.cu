@@ -51,9 +51,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = (kEpiWarps + 3) * 32;       // 352
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1, kHWarp = kEpiWarps + 2;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int NUM_BARS = 2 * STAGES + 2 + 3 * H_SLOTS + 2;
+constexpr uint32_t W_BYTES = kCols * 4;  // the tile's columns of w_q * w_k (fp32)
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 * H_SLOTS + 4;
 constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * H_BYTES +
-                        8 * NUM_BARS + 16;
+                        W_BYTES + 8 * NUM_BARS + 16;
 static_assert(SMEM <= 232448, "shared memory budget");
 
 template <int PHASE>
@@ -69,7 +70,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sB = sA + STAGES * A_BYTES;
   uint8_t* hbuf = smem + (size_t)STAGES * STAGE_BYTES;
   const uint32_t sH = smem_u32(hbuf);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(hbuf + (size_t)H_SLOTS * H_BYTES);
+  const float* wbuf = reinterpret_cast<const float*>(hbuf + (size_t)H_SLOTS * H_BYTES);
+  const uint32_t sW = smem_u32(wbuf);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(hbuf + (size_t)H_SLOTS * H_BYTES + W_BYTES);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -77,9 +80,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tempty_bar = tfull_bar + 8u;
   auto hfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + s); };
   auto hempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + H_SLOTS + s); };
-  auto hdone_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 + 2 * H_SLOTS + s); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 + 3 * H_SLOTS);
-  const uint32_t pair_bar = drain_bar + 8u;
+  const uint32_t wfull_bar = bar0 + 8u * (2 * STAGES + 2 + 2 * H_SLOTS);
+  const uint32_t wempty_bar = wfull_bar + 8u;
+  const uint32_t drain_bar = wfull_bar + 16u;
+  const uint32_t pair_bar = wfull_bar + 24u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -105,9 +109,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(tempty_bar, 2 * kEpiWarps);  // every epilogue warp of the pair
     for (int s = 0; s < H_SLOTS; ++s) {
       mbar_init(hfull_bar(s), 1);
-      mbar_init(hempty_bar(s), PHASE == 0 ? kEpiWarps : 1);
-      mbar_init(hdone_bar(s), kEpiWarps);
+      mbar_init(hempty_bar(s), kEpiWarps);  // every epilogue warp releases its rows
     }
+    mbar_init(wfull_bar, 1);
+    mbar_init(wempty_bar, kEpiWarps);
     mbar_init(drain_bar, 1);
     mbar_init(pair_bar, 1);
     *abort_flag = 0;
@@ -167,9 +172,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
+    uint32_t wphase = 0;
     for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
       const int m_blk = tile / num_n, n0 = (tile - m_blk * num_n) * kCols;
       const int row0 = m_blk * 2 * kRows + (int)rank * kRows;
+      if (PHASE == 0) {
+        // the key epilogue's column weights: w_qk[n0 .. n0+256) of [M*d]
+        if (lane == 0) ok = wait_bounded(wempty_bar, wphase ^ 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(wfull_bar, W_BYTES);
+          bulk_load(sW, g.w_qk + n0, W_BYTES, wfull_bar);
+        }
+        __syncwarp();
+        wphase ^= 1u;
+      }
       for (int i = 0; i < nsub; ++i) {
         // h viewed as [R, M*d]: key phase column n0 + 32 i; value phase
         // branch i % M, column n0 + 32 (i / M)
@@ -242,11 +260,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3, half = warp >> 2;
-    const int r = half * 128 + quarter * 32 + lane;  // tile row of this thread
+    const int wrow0 = half * 128 + quarter * 32;  // first tile row of this warp
+    const int r = wrow0 + lane;                   // tile row of this thread
     int hslot = 0;
-    uint32_t hphase = 0, tphase = 0;
+    uint32_t hphase = 0, tphase = 0, wphase = 0;
     bool ok = true;
     const int tiles_per_branch = d / g.key_tile;
+    constexpr int NQ = kCols / H_COLS;  // 32-column chunks per tile
     for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
       const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
       const int row0 = m_blk * 2 * kRows + (int)rank * kRows;  // first row of this CTA
@@ -281,29 +301,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * kCols);
-      float v[32];
+      // two register sets: chunk q+1 loads from TMEM while chunk q is used
+      static_assert(NQ % 2 == 0, "chunks are processed in pairs");
+      uint32_t va[32], vb[32];
+      __syncwarp();
+      tmem_ld32_async(taddr, va);
       if (PHASE == 0) {
-        const int mb = n0 / d, j0 = n0 - mb * d;
-        const float* wrow = g.w_qk + (int64_t)mb * d + j0;
+        if (lane == 0) ok = wait_bounded(wfull_bar, wphase, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        wphase ^= 1u;
         float skk = 0.f, shk = 0.f, shh = 0.f;
-#pragma unroll 1
-        for (int q = 0; q < kCols / H_COLS; ++q) {
+        // one 32-column chunk: v holds it (loaded), vn receives chunk q+1
+        auto key_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
+          tmem_wait32(v);
           __syncwarp();
-          tmem_ld32(taddr + q * H_COLS, v);
+          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
           if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
+          if (!ok) return;
           const uint8_t* hs = hbuf + hslot * H_BYTES;
-          const float4* wp = reinterpret_cast<const float4*>(wrow + q * H_COLS);
+          const float4* wp = reinterpret_cast<const float4*>(wbuf + q * H_COLS);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             float hf[8];
             unpack8(*reinterpret_cast<const uint4*>(hs + sw64_off(r, c)), hf);
-            const float4 w0 = __ldg(wp + 2 * c), w1 = __ldg(wp + 2 * c + 1);
+            const float4 w0 = wp[2 * c], w1 = wp[2 * c + 1];
             const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float k = v[c * 8 + i];
+              const float k = __uint_as_float(v[c * 8 + i]);
               skk = fmaf(k, k, skk);
               shh = fmaf(hf[i], hf[i], shh);
               shk = fmaf(hf[i] * wf[i], k, shk);
@@ -315,19 +341,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             hslot = 0;
             hphase ^= 1u;
           }
+        };
+#pragma unroll 1
+        for (int q = 0; ok && q < NQ; q += 2) {
+          key_chunk(q, va, vb);
+          if (ok) key_chunk(q + 1, vb, va);
         }
         if (!ok) break;
+        // accumulators and the weight buffer are free again (the pair's leader
+        // owns the accumulator barrier); then the partial sums go out
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+          mbar_arrive(wempty_bar);
+        }
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
       } else {
-#pragma unroll 1
-        for (int q = 0; q < kCols / H_COLS; ++q) {
+        int pending = -1;  // slot whose TMA store may still be reading it
+        auto value_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
+          tmem_wait32(v);
           __syncwarp();
-          tmem_ld32(taddr + q * H_COLS, v);
+          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
             if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
+            if (!ok) return;
             uint8_t* hs = hbuf + hslot * H_BYTES;
             float a = 0.f;
 #pragma unroll
@@ -340,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float hf[8], o[8];
               unpack8(*p, hf);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] = fmaf(a, v[c * 8 + i], hf[i]);
+              for (int i = 0; i < 8; ++i) o[i] = fmaf(a, __uint_as_float(v[c * 8 + i]), hf[i]);
               *p = make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]),
                               pack2(o[6], o[7]));
             }
@@ -349,43 +389,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                      q * H_COLS);
 #pragma unroll
               for (int c = 0; c < 8; ++c)
-                dp[c] = make_float4(a * v[4 * c], a * v[4 * c + 1], a * v[4 * c + 2],
-                                    a * v[4 * c + 3]);
+                dp[c] = make_float4(a * __uint_as_float(v[4 * c]), a * __uint_as_float(v[4 * c + 1]),
+                                    a * __uint_as_float(v[4 * c + 2]),
+                                    a * __uint_as_float(v[4 * c + 3]));
             }
             fence_async_smem();  // generic-proxy writes -> visible to the TMA store
             __syncwarp();
-            if (lane == 0) mbar_arrive(hdone_bar(hslot));
-            if (warp == 0) {
-              if (lane == 0) {
-                ok = wait_bounded(hdone_bar(hslot), hphase, abort_flag, g.err);
-                if (ok) {
-                  if (row0 < R) {  // rows past R are clipped; a slot wholly past R stores nothing
-                    tma_store_2d(&map_out, sH + hslot * H_BYTES, mb * d + n0 + q * H_COLS, row0);
-                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                  }
-                  mbar_arrive(hempty_bar(hslot));
-                }
-              }
-              ok = __shfl_sync(0xffffffffu, ok, 0);
-              if (!ok) break;
+            if (lane == 0) {
+              // this warp's 32 rows of the slot; rows past R are clipped, and a
+              // warp whose rows all lie past R commits an empty group instead
+              if (row0 + wrow0 < R)
+                tma_store_2d(&map_out, sH + hslot * H_BYTES + wrow0 * (H_COLS * 2),
+                             mb * d + n0 + q * H_COLS, row0 + wrow0);
+              else
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+              // release the previous slot once its store has read it
+              asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+              if (pending >= 0) mbar_arrive(hempty_bar(pending));
             }
+            pending = hslot;
             if (++hslot == H_SLOTS) {
               hslot = 0;
               hphase ^= 1u;
             }
           }
-          if (!ok) break;
+        };
+#pragma unroll 1
+        for (int q = 0; ok && q < NQ; q += 2) {
+          value_chunk(q, va, vb);
+          if (ok) value_chunk(q + 1, vb, va);
         }
         if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          if (pending >= 0) mbar_arrive(hempty_bar(pending));
+        }
       }
-      // accumulators free again: the leader owns the barrier
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
       tphase ^= 1u;
     }
-    if (PHASE == 1 && warp == 0 && lane == 0)
-      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (PHASE == 1 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   tc_fence_before();
