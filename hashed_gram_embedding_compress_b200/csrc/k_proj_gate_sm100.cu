@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (lane == 0) ok = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < nsub; ++i) {
         // columns of h viewed as [R, M*d]: key phase n0 + 64q; value phase mb*d + n0 + 64q
         const int x = PHASE == 0 ? n0 + 64 * i : (i % M) * d + n0 + 64 * (i / M);
-        if (lane == 0) ok = wait_bounded(hempty_bar(slot), phase ^ 1u, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(hempty_bar(slot), phase ^ 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
@@ -197,13 +197,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      if (lane == 0) ok = wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, g.err);
+      if (lane == 0) ok = wait_ready(tempty_bar(acc), acc_phase ^ 1u, abort_flag, g.err);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (lane == 0) ok = wait_bounded(full_bar(stage), phase, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(full_bar(stage), phase, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (lane == 0) ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, g.err);
+      if (lane == 0) ok = wait_ready(tfull_bar(acc), acc_phase, abort_flag, g.err);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           tmem_ld32(taddr + q * 64, v);
           tmem_ld32(taddr + q * 64 + 32, v + 32);
-          if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+          if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           const uint8_t* hs = hbuf + hslot * H_BYTES;
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + q * 64 + 32, v + 32);
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
-            if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+            if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             uint8_t* hs = hbuf + hslot * H_BYTES;
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(hdone_bar(hslot));
             if (warp == 0) {
               if (lane == 0) {
-                ok = wait_bounded(hdone_bar(hslot), hphase, abort_flag, g.err);
+                ok = wait_ready(hdone_bar(hslot), hphase, abort_flag, g.err);
                 if (ok) {
                   tma_store_2d(&map_out, sH + hslot * H_BYTES, mb * d + n0 + q * 64, m_blk * BM);
                   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int a_row = m_blk * 2 * kRows + (int)rank * kRows;
       const int b_row = n_blk * kCols + (int)rank * (kCols / 2);
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (lane == 0) ok = wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = m_blk * 2 * kRows + (int)rank * kRows;
       if (PHASE == 0) {
         // the key epilogue's column weights: w_qk[n0 .. n0+256) of [M*d]
-        if (lane == 0) ok = wait_bounded(wempty_bar, wphase ^ 1u, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(wempty_bar, wphase ^ 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // h viewed as [R, M*d]: key phase column n0 + 32 i; value phase
         // branch i % M, column n0 + 32 (i / M)
         const int x = PHASE == 0 ? n0 + H_COLS * i : (i % M) * d + n0 + H_COLS * (i / M);
-        if (lane == 0) ok = wait_bounded(hempty_bar(slot), phase ^ 1u, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(hempty_bar(slot), phase ^ 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
@@ -219,12 +219,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     if (leader) {
       for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
-        if (lane == 0) ok = wait_bounded(tempty_bar, tphase ^ 1u, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(tempty_bar, tphase ^ 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (lane == 0) ok = wait_bounded(full_bar(stage), phase, abort_flag, g.err);
+          if (lane == 0) ok = wait_ready(full_bar(stage), phase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           tc_fence_after();
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (lane == 0) ok = wait_bounded(tfull_bar, tphase, abort_flag, g.err);
+      if (lane == 0) ok = wait_ready(tfull_bar, tphase, abort_flag, g.err);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tmem_ld32_async(taddr, va);
       if (PHASE == 0) {
-        if (lane == 0) ok = wait_bounded(wfull_bar, wphase, abort_flag, g.err);
+        if (lane == 0) ok = wait_ready(wfull_bar, wphase, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         wphase ^= 1u;
         float skk = 0.f, shk = 0.f, shh = 0.f;
@@ -316,25 +316,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait32(v);
           __syncwarp();
           if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
-          if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+          if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) return;
           const uint8_t* hs = hbuf + hslot * H_BYTES;
           const float4* wp = reinterpret_cast<const float4*>(wbuf + q * H_COLS);
+          uint4 hu[4];
+          float4 wv[8];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) hu[c] = *reinterpret_cast<const uint4*>(hs + sw64_off(r, c));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) wv[c] = wp[c];
+          // four independent accumulators per sum: short dependency chains
+          float a_kk[4] = {0.f, 0.f, 0.f, 0.f}, a_hh[4] = {0.f, 0.f, 0.f, 0.f},
+                a_hk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             float hf[8];
-            unpack8(*reinterpret_cast<const uint4*>(hs + sw64_off(r, c)), hf);
-            const float4 w0 = wp[2 * c], w1 = wp[2 * c + 1];
-            const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            unpack8(hu[c], hf);
+            const float wf[8] = {wv[2 * c].x, wv[2 * c].y, wv[2 * c].z, wv[2 * c].w,
+                                 wv[2 * c + 1].x, wv[2 * c + 1].y, wv[2 * c + 1].z,
+                                 wv[2 * c + 1].w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float k = __uint_as_float(v[c * 8 + i]);
-              skk = fmaf(k, k, skk);
-              shh = fmaf(hf[i], hf[i], shh);
-              shk = fmaf(hf[i] * wf[i], k, shk);
+              a_kk[i & 3] = fmaf(k, k, a_kk[i & 3]);
+              a_hh[i & 3] = fmaf(hf[i], hf[i], a_hh[i & 3]);
+              a_hk[i & 3] = fmaf(hf[i] * wf[i], k, a_hk[i & 3]);
             }
           }
+          skk += (a_kk[0] + a_kk[1]) + (a_kk[2] + a_kk[3]);
+          shh += (a_hh[0] + a_hh[1]) + (a_hh[2] + a_hh[3]);
+          shk += (a_hk[0] + a_hk[1]) + (a_hk[2] + a_hk[3]);
           __syncwarp();
           if (lane == 0) mbar_arrive(hempty_bar(hslot));
           if (++hslot == H_SLOTS) {
@@ -365,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
-            if (lane == 0) ok = wait_bounded(hfull_bar(hslot), hphase, abort_flag, g.err);
+            if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) return;
             uint8_t* hs = hbuf + hslot * H_BYTES;

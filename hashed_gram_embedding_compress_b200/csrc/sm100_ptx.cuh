@@ -72,6 +72,25 @@ static __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Non-blocking test of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// wait_bounded with an inlined fast path for a phase that has already completed.
+__device__ __forceinline__ bool wait_ready(uint32_t bar, uint32_t parity,
+                                           volatile int* abort_flag, unsigned* err) {
+  return mbar_test_wait(bar, parity) || wait_bounded(bar, parity, abort_flag, err);
+}
+
 // Same, ignoring the abort flag (used only to drain on the way out).
 static __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
