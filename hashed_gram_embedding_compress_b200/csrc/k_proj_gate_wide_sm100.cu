@@ -327,27 +327,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 4; ++c) hu[c] = *reinterpret_cast<const uint4*>(hs + sw64_off(r, c));
 #pragma unroll
           for (int c = 0; c < 8; ++c) wv[c] = wp[c];
-          // four independent accumulators per sum: short dependency chains
-          float a_kk[4] = {0.f, 0.f, 0.f, 0.f}, a_hh[4] = {0.f, 0.f, 0.f, 0.f},
-                a_hk[4] = {0.f, 0.f, 0.f, 0.f};
+          // packed fp32 pairs, two accumulators per sum: four chains each
+          unsigned long long akk[2] = {0ull, 0ull}, ahh[2] = {0ull, 0ull}, ahk[2] = {0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float hf[8];
-            unpack8(hu[c], hf);
-            const float wf[8] = {wv[2 * c].x, wv[2 * c].y, wv[2 * c].z, wv[2 * c].w,
-                                 wv[2 * c + 1].x, wv[2 * c + 1].y, wv[2 * c + 1].z,
-                                 wv[2 * c + 1].w};
+            const uint32_t hw[4] = {hu[c].x, hu[c].y, hu[c].z, hu[c].w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float k = __uint_as_float(v[c * 8 + i]);
-              a_kk[i & 3] = fmaf(k, k, a_kk[i & 3]);
-              a_hh[i & 3] = fmaf(hf[i], hf[i], a_hh[i & 3]);
-              a_hk[i & 3] = fmaf(hf[i] * wf[i], k, a_hk[i & 3]);
+            for (int j = 0; j < 4; ++j) {
+              const int e = c * 8 + 2 * j;  // elements e, e+1 of the chunk
+              const unsigned long long h2 = bf16x2_to_f2(hw[j]);
+              const unsigned long long k2 = f2_pack(v[e], v[e + 1]);
+              const float4 wq = wv[(c * 8 + 2 * j) / 4];
+              const unsigned long long w2 =
+                  (j & 1) ? f2_pack(__float_as_uint(wq.z), __float_as_uint(wq.w))
+                          : f2_pack(__float_as_uint(wq.x), __float_as_uint(wq.y));
+              akk[j & 1] = f2_fma(k2, k2, akk[j & 1]);
+              ahh[j & 1] = f2_fma(h2, h2, ahh[j & 1]);
+              ahk[j & 1] = f2_fma(f2_mul(h2, w2), k2, ahk[j & 1]);
             }
           }
-          skk += (a_kk[0] + a_kk[1]) + (a_kk[2] + a_kk[3]);
-          shh += (a_hh[0] + a_hh[1]) + (a_hh[2] + a_hh[3]);
-          shk += (a_hk[0] + a_hk[1]) + (a_hk[2] + a_hk[3]);
+          const float2 kk0 = f2_unpack(akk[0]), kk1 = f2_unpack(akk[1]);
+          const float2 hh0 = f2_unpack(ahh[0]), hh1 = f2_unpack(ahh[1]);
+          const float2 hk0 = f2_unpack(ahk[0]), hk1 = f2_unpack(ahk[1]);
+          skk += (kk0.x + kk0.y) + (kk1.x + kk1.y);
+          shh += (hh0.x + hh0.y) + (hh1.x + hh1.y);
+          shk += (hk0.x + hk0.y) + (hk1.x + hk1.y);
           __syncwarp();
           if (lane == 0) mbar_arrive(hempty_bar(hslot));
           if (++hslot == H_SLOTS) {
@@ -387,15 +391,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < kMaxBranches; ++b)
               if (b == mb) a = al[b];
             // out = h + alpha v, written over h in place, then stored by TMA
+            const unsigned long long a2 = f2_pack(__float_as_uint(a), __float_as_uint(a));
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint4* p = reinterpret_cast<uint4*>(hs + sw64_off(r, c));
-              float hf[8], o[8];
-              unpack8(*p, hf);
+              const uint4 hu = *p;
+              const uint32_t hw[4] = {hu.x, hu.y, hu.z, hu.w};
+              uint32_t ow[4];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] = fmaf(a, __uint_as_float(v[c * 8 + i]), hf[i]);
-              *p = make_uint4(pack2(o[0], o[1]), pack2(o[2], o[3]), pack2(o[4], o[5]),
-                              pack2(o[6], o[7]));
+              for (int j = 0; j < 4; ++j) {
+                const int e = c * 8 + 2 * j;
+                const float2 o =
+                    f2_unpack(f2_fma(a2, f2_pack(v[e], v[e + 1]), bf16x2_to_f2(hw[j])));
+                ow[j] = pack2(o.x, o.y);
+              }
+              *p = make_uint4(ow[0], ow[1], ow[2], ow[3]);
             }
             if (g.delta && valid) {
               float4* dp = reinterpret_cast<float4*>(g.delta + ((int64_t)row * M + mb) * d + n0 +

@@ -281,6 +281,38 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE fp32 operations per
+// instruction).  A pair is a 64-bit value {lo, hi}.
+__device__ __forceinline__ unsigned long long f2_pack(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+__device__ __forceinline__ float2 f2_unpack(unsigned long long p) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(p));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// The two bf16 of a packed word as an fp32 pair (exact).
+__device__ __forceinline__ unsigned long long bf16x2_to_f2(uint32_t w) {
+  return f2_pack(w << 16, w & 0xFFFF0000u);
+}
+
 __device__ __forceinline__ float sigmoid_f(float s) { return 1.0f / (1.0f + expf(-s)); }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
