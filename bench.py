@@ -187,11 +187,11 @@ def run_ours(args, rank, world, dist):
     sh, m = P["sh"], P["m"]
     tok_d = P["tokens"].to(device)
     h = P["h"]
-    out = torch.empty_like(h)
     stream = torch.cuda.current_stream()
 
+    # the residual update H <- H + Y in place: out aliases h
     def step():
-        m.forward(tok_d, h, out, stream=stream)
+        m.forward(tok_d, h, h, stream=stream)
 
     clk = ClockSampler(local).__enter__()
     for _ in range(max(3, args.warmup)):
@@ -246,13 +246,12 @@ def run_ours(args, rank, world, dist):
     out_h = torch.empty_like(h_h).pin_memory()
     tok_buf = torch.empty_like(tok_d)
     h_buf = torch.empty_like(h)
-    out_buf = torch.empty_like(h)
 
     def e2e_step():
         tok_buf.copy_(tok_h, non_blocking=True)
         h_buf.copy_(h_h, non_blocking=True)
-        m.forward(tok_buf, h_buf, out_buf, stream=stream)
-        out_h.copy_(out_buf, non_blocking=True)
+        m.forward(tok_buf, h_buf, h_buf, stream=stream)
+        out_h.copy_(h_buf, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -303,6 +302,7 @@ def run_ours(args, rank, world, dist):
             "parallelism": "replicas" if world > 1 else "single",
             "l2": "no flush: inputs larger than L2 (h 168 MB read, out 168 MB written, "
                   "tables 2.7 GB)",
+            "residual": "in place: out aliases h (H <- H + alpha v)",
         },
         "roofline": {
             "kernel": "proj_gate_kernel (tcgen05 key + value launches)",

@@ -659,7 +659,9 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
       wide.w = wmaps[bn_index(128)];  // each CTA of a pair loads 128 of the tile's 256 W rows
       if (phase == 0) g.key_tile = 256;
       const int pairs = (int)(wtiles < h->sms / 2 ? wtiles : h->sms / 2);
-      CK(h, launch_proj_gate_wide(phase, wide, g, 2 * pairs, st));
+      // in place (out aliases h): the value phase adds alpha v into out
+      const int kphase = (phase == 1 && out == hid) ? 2 : phase;
+      CK(h, launch_proj_gate_wide(kphase, wide, g, 2 * pairs, st));
     } else {
       if (!have_single) {
         if ((rc = make_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;

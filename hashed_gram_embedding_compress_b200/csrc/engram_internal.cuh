@@ -99,6 +99,7 @@ struct ProjMaps {
 cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
                                    int grid, cudaStream_t stream);
 // 512 x 256 tiles on CTA pairs (tcgen05 cta_group::2); grid = 2 x pairs.
+// phase 0 keys, 1 values, 2 values added in place (out aliases h).
 cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
                                   cudaStream_t stream);
 

@@ -27,6 +27,11 @@
 //   warp 10     TMA producer of h sub-tiles [256 rows x 32 columns, 64-byte
 //               swizzle], shared by both epilogue warpgroups; in the value
 //               phase out is written over h in the slot and stored by TMA.
+// Phases: 0 = keys (partial sums), 1 = values (out = h + alpha v through the
+// h ring), 2 = values when out aliases h (the residual update in place): the
+// epilogue stages bf16(alpha v) and adds it into out with a TMA reduce-add,
+// so h never passes through shared memory; the sum is rounded once more
+// (RN(h + RN(alpha v)) instead of RN(h + alpha v)).
 // Waits are bounded as in the single-CTA kernel; the pair leaves together
 // through a bounded handshake, then frees TMEM (cta_group::2).
 #include "sm100_ptx.cuh"
@@ -97,8 +102,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_kb = (g.d_mem + BK - 1) / BK;
   const int first_tile = (int)(blockIdx.x >> 1), tile_step = (int)(gridDim.x >> 1);
   // h sub-tiles per tile: one branch in the key phase, every branch in the
-  // value phase (v is shared across branches, Eq. 6)
-  const int nsub = (kCols / H_COLS) * (PHASE == 0 ? 1 : M);
+  // value phase (v is shared across branches, Eq. 6); none when the value
+  // phase adds into h in place
+  const int nsub = PHASE == 2 ? 0 : (kCols / H_COLS) * (PHASE == 0 ? 1 : M);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = row < R;
       const int n0 = n_blk * kCols;
       float al[kMaxBranches];
-      if (PHASE == 1) {
+      if (PHASE >= 1) {
         // alpha from the key phase's per-tile partial sums (Eq. 4 / Eq. 6);
         // computed while the MMAs of this tile run
 #pragma unroll
@@ -374,6 +380,67 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(wempty_bar);
         }
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
+      } else if (PHASE == 2) {
+        // out aliases h: add bf16(alpha v) into it with TMA reduce-add; each
+        // warp stages its 32 rows x 32 columns in one of two 2 KB buffers
+        // (the h ring is unused in this phase)
+        uint8_t* stage0 = hbuf + warp * 4096;
+        int sbuf = 0;
+        auto add_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
+          tmem_wait32(v);
+          __syncwarp();
+          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+#pragma unroll 1
+          for (int mb = 0; mb < M; ++mb) {
+            float a = 0.f;
+#pragma unroll
+            for (int b = 0; b < kMaxBranches; ++b)
+              if (b == mb) a = al[b];
+            const unsigned long long a2 = f2_pack(__float_as_uint(a), __float_as_uint(a));
+            // the buffer's previous reduce has finished reading it
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            __syncwarp();
+            uint8_t* st = stage0 + sbuf * 2048;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t ow[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int e = c * 8 + 2 * j;
+                const float2 o = f2_unpack(f2_mul(a2, f2_pack(v[e], v[e + 1])));
+                ow[j] = pack2(o.x, o.y);
+              }
+              *reinterpret_cast<uint4*>(st + sw64_off(lane, c)) =
+                  make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            }
+            if (g.delta && valid) {
+              float4* dp = reinterpret_cast<float4*>(g.delta + ((int64_t)row * M + mb) * d + n0 +
+                                                     q * H_COLS);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                dp[c] = make_float4(a * __uint_as_float(v[4 * c]), a * __uint_as_float(v[4 * c + 1]),
+                                    a * __uint_as_float(v[4 * c + 2]),
+                                    a * __uint_as_float(v[4 * c + 3]));
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 + wrow0 < R)
+                tma_reduce_add_2d(&map_out, smem_u32(st), mb * d + n0 + q * H_COLS, row0 + wrow0);
+              else
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+            sbuf ^= 1;
+          }
+        };
+#pragma unroll 1
+        for (int q = 0; q < NQ; q += 2) {
+          add_chunk(q, va, vb);
+          add_chunk(q + 1, vb, va);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
       } else {
         int pending = -1;  // slot whose TMA store may still be reading it
         auto value_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
@@ -453,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tphase ^= 1u;
     }
-    if (PHASE == 1 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (PHASE >= 1 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   tc_fence_before();
@@ -500,7 +567,12 @@ cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArg
                                   cudaStream_t stream) {
   if (g.R == 0) return cudaSuccess;
   if (grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
-  return phase == 0 ? launch_wide<0>(maps, g, grid, stream) : launch_wide<1>(maps, g, grid, stream);
+  switch (phase) {
+    case 0: return launch_wide<0>(maps, g, grid, stream);
+    case 1: return launch_wide<1>(maps, g, grid, stream);
+    case 2: return launch_wide<2>(maps, g, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace engram

@@ -103,6 +103,25 @@ def test_prefill_full_size_sampled():
     out1, a1, dl1 = run_forward(p, m1)
     check_rows(p, m1, idx, p.sample_rows(32, seed=1), out1, a1, dl1)
     assert rel_l2(dl1.double(), dl.double()) < 1e-6
+    check_in_place(p, m, out, dl)
+
+
+def check_in_place(p: Problem, m, out, delta):
+    # out aliasing h (the residual update H <- H + Y in place): the value
+    # phase adds bf16(alpha v) into h, one extra rounding of alpha v
+    sh = p.shape
+    h2 = p.h.clone()
+    a2 = torch.empty((sh.rows_out, sh.branches), device="cuda")
+    d2 = torch.empty((sh.rows_out, sh.branches, sh.d_hidden), device="cuda")
+    m.forward(p.tokens.cuda(), h2, h2, t_begin=sh.t_begin, alpha=a2, delta=d2)
+    torch.cuda.synchronize()
+    assert m.check_errors() == 0
+    assert torch.equal(d2, delta)
+    assert rel_l2(h2.double(), out.double()) < 1e-4
+    assert (h2 == out).double().mean().item() > 0.98
+    rows = p.sample_rows(16, seed=2)
+    _, _, _, o_ref = p.oracle_forward(rows)
+    assert out_close(to_oracle(h2[torch.from_numpy(rows).cuda()]), o_ref, "bf16") <= BF16_REL
 
 
 def test_decode_multibranch():
@@ -160,6 +179,13 @@ def test_large_hbm_sampled():
     e = torch.empty((len(rows), p.shape.d_mem), dtype=torch.bfloat16, device="cuda")
     m.gather(idx[rs].contiguous(), e)
     assert np.array_equal(to_oracle(e), e_ref)
+    # in place, four branches
+    h2 = p.h.clone()
+    m.forward(p.tokens.cuda(), h2, h2)
+    torch.cuda.synchronize()
+    assert m.check_errors() == 0
+    assert rel_l2(h2.double(), out.double()) < 1e-4
+    assert out_close(to_oracle(h2[rs]), o_ref, "bf16") <= BF16_REL
 
 
 def test_in_place_update_and_empty_batch():
