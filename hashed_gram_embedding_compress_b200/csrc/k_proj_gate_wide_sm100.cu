@@ -179,9 +179,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     bool ok = true;
     uint32_t wphase = 0;
-    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+    int tix = 0;
+    const int nbox = (kCols / H_COLS) * (PHASE == 0 ? 1 : M);  // h boxes of a tile
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step, ++tix) {
       const int m_blk = tile / num_n, n0 = (tile - m_blk * num_n) * kCols;
       const int row0 = m_blk * 2 * kRows + (int)rank * kRows;
+      // Bring this tile's h into L2 while its MMAs run: the boxes beyond the
+      // smem ring (keys, values) or all of them (values added in place, which
+      // read-modify-write h in L2 from the epilogue).  In place, pace by the
+      // accumulator: prefetch tile i once tile i-1's MMAs are done.
+      if (PHASE == 2 && tix > 0) {
+        if (lane == 0) ok = wait_ready(tfull_bar, (uint32_t)(tix - 1) & 1u, abort_flag, g.err);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+      }
+      if (lane == 0 && row0 < R) {
+        for (int i = PHASE == 2 ? 0 : H_SLOTS; i < nbox; ++i)
+          tma_prefetch_l2_2d(&map_h, PHASE == 0 ? n0 + H_COLS * i
+                                                : (i % M) * d + n0 + H_COLS * (i / M),
+                             row0);
+      }
+      __syncwarp();
       if (PHASE == 0) {
         // the key epilogue's column weights: w_qk[n0 .. n0+256) of [M*d]
         if (lane == 0) ok = wait_ready(wempty_bar, wphase ^ 1u, abort_flag, g.err);
