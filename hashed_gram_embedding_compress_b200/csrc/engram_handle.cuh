@@ -1,0 +1,60 @@
+// The handle behind the C ABI (include/engram.h): configuration, device
+// copies of the hash parameters, borrowed parameters, tensor maps of the
+// weights, scratch and prefetch state.  Internal to libengram.so.
+#pragma once
+
+#include <string>
+
+#include "../../include/engram.h"
+#include "engram_internal.cuh"
+
+struct engram_handle {
+  engram_config cfg{};
+  int device = 0, sms = 148;
+  int S = 0, max_order = 0, d_mem = 0, elt = 4;
+  int64_t primes[engram::kMaxTables] = {};
+  uint64_t mult[engram::kMaxTables * engram::kMaxOrders] = {};
+  std::string last_error;
+
+  // device copies of the configuration
+  int32_t* d_map = nullptr;
+  int64_t* d_primes = nullptr;
+  uint64_t* d_mult = nullptr;
+  unsigned* d_err = nullptr;
+
+  // borrowed parameters
+  bool have_params = false;
+  const void* tables[engram::kMaxTables] = {};
+  const void** d_tables = nullptr;  // device array of S table pointers
+  const void* w_k = nullptr;
+  const void* w_v = nullptr;
+  float* d_wqk = nullptr;           // norm_q * norm_k, [M, d]
+  CUtensorMap map_wk[3], map_wv[3]; // box widths 64, 128, 256
+
+  // scratch, sized for cap_rows emitted positions
+  int64_t cap_rows = 0;
+  int64_t* z = nullptr;
+  void* e = nullptr;
+  float4* partials = nullptr;
+
+  // host-resident tables: prefetch state, double-buffered
+  int64_t pf_cap_rows = 0;
+  uint32_t set_cap = 0;
+  unsigned long long* d_keys = nullptr;
+  int32_t* d_vals = nullptr;
+  unsigned long long* d_count[2] = {nullptr, nullptr};
+  int2* d_uniq = nullptr;
+  int64_t* d_remap[2] = {nullptr, nullptr};
+  void* d_staging[2] = {nullptr, nullptr};
+  const void** d_stage_tables[2] = {nullptr, nullptr};
+  int64_t* d_stage_bound = nullptr;
+  cudaEvent_t ev_ready[2] = {nullptr, nullptr};
+  cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
+  int64_t pf_rows[2] = {0, 0};
+  uint64_t n_prefetch = 0, n_consumed = 0;
+
+  // instrumentation
+  int64_t launches = 0;
+  cudaEvent_t prof[5] = {};
+  bool prof_armed = false;
+};

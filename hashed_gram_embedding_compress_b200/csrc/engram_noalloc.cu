@@ -1,0 +1,196 @@
+// engram_project_gate_noalloc: the projection + gate step for callers that
+// must not have the library allocate device memory.
+//
+// engram_forward keeps its scratch (indices, memory vectors, per-row partial
+// sums) in buffers the handle allocates on demand.  Some callers cannot allow
+// that: code that runs while a CUDA graph is being captured (cudaMalloc is
+// not a capturable operation and fails the capture), and hosts whose device
+// memory must all come from their own allocator or pool budget.  With this
+// entry point such a caller supplies every input and output itself (it can
+// produce e with engram_hash and engram_gather into its own buffers), and the
+// only scratch, the key phase's per-row partial sums, lives in a fixed array
+// in the library's device image.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+#include <string>
+
+#include "engram_handle.cuh"
+
+using namespace engram;
+
+namespace {
+
+// Size of the partial-sum array: 16 bytes per (row, 64-column key tile).
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+
+}  // namespace
+
+// Every GPU that loads the library holds this array until the process exits.
+// All calls on a device share it: calls that overlap on the GPU race.
+static __device__ __align__(256) unsigned char g_noalloc_partials[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+std::mutex g_mu;
+void* g_partials_dev[kMaxDevices] = {};
+
+int fail(engram_handle* h, int code, const std::string& msg) {
+  h->last_error = msg;
+  return code;
+}
+
+// Device address of the array on the current device, looked up once per
+// device with that device current.  In host code the array's name is only a
+// host-side stand-in, never a device address.
+int partials_address(engram_handle* h, float4** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(e));
+  if (dev != h->device) return fail(h, ENGRAM_ERR_INVALID, "the handle's device must be current");
+  if (dev < 0 || dev >= kMaxDevices) return fail(h, ENGRAM_ERR_INVALID, "device id out of range");
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_partials_dev[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess || !p)
+      return fail(h, ENGRAM_ERR_CUDA,
+                  std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    g_partials_dev[dev] = p;
+  }
+  *out = reinterpret_cast<float4*>(g_partials_dev[dev]);
+  return ENGRAM_OK;
+}
+
+int encode_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
+               int box_rows, int box_cols) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapSwizzle sw =
+      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  return ENGRAM_OK;
+}
+
+int map_slot(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int64_t rows,
+                                           const void* hid, void* out, float* alpha,
+                                           void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  const int M = h->cfg.branches, d = h->cfg.d_hidden;
+  const int64_t bytes_per_row = (int64_t)(M * d / 64) * (int64_t)sizeof(float4);
+  const int64_t max_rows = (int64_t)kNoAllocScratchBytes / bytes_per_row;
+  if (rows < 0) return fail(h, ENGRAM_ERR_INVALID, "rows < 0");
+  if (rows > max_rows)
+    return fail(h, ENGRAM_ERR_INVALID,
+                "engram_project_gate_noalloc: " + std::to_string(rows) + " rows exceed the " +
+                    std::to_string(max_rows) + "-row limit of its fixed 4 MiB scratch (" +
+                    std::to_string(bytes_per_row) + " bytes per row); use engram_forward");
+  if (rows == 0) return ENGRAM_OK;
+  if (!e || !hid || !out || !aligned16(e) || !aligned16(hid) || !aligned16(out) ||
+      (alpha && !aligned16(alpha)))
+    return fail(h, ENGRAM_ERR_INVALID, "null or misaligned buffer");
+  float4* partials = nullptr;
+  int rc = partials_address(h, &partials);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int R = (int)rows;
+
+  // Every (row, key tile) entry the value phase reads is written by the key
+  // phase of the same call, so the array needs no clearing between calls.
+  GateArgs g{};
+  g.h = hid;
+  g.out = out;
+  g.w_qk = h->d_wqk;
+  g.partials = partials;
+  g.alpha = alpha;
+  g.delta = nullptr;
+  g.err = h->d_err;
+  g.R = R;
+  g.M = M;
+  g.d = d;
+  g.d_mem = h->d_mem;
+  g.eps = h->cfg.eps;
+  g.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
+  cudaError_t ce;
+  if (h->cfg.dtype == ENGRAM_F32) {
+    g.key_tile = kF32Tile;
+    if ((ce = launch_proj_gate_f32(0, (const float*)e, (const float*)h->w_k, g, st)) ||
+        (ce = launch_proj_gate_f32(1, (const float*)e, (const float*)h->w_v, g, st)))
+      return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
+    h->launches += 2;
+    return ENGRAM_OK;
+  }
+  // the same kernel choice as engram_forward: 512 x 256 CTA-pair tiles when
+  // they fill every pair, else single-CTA 128-row tiles
+  const int64_t hcols = (int64_t)M * d;
+  const bool pairs_ok = !(h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS);
+  ProjMaps single, wide;
+  bool have_single = false, have_wide = false;
+  for (int phase = 0; phase < 2; ++phase) {
+    const int n_total = phase == 0 ? M * d : d;
+    const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
+    const int64_t wtiles = (rows + 511) / 512 * (n_total / 256);
+    if (pairs_ok && n_total % 256 == 0 && wtiles >= h->sms / 2) {
+      if (!have_wide) {
+        if ((rc = encode_map(h, &wide.e, e, h->d_mem, R, 256, 64)) ||
+            (rc = encode_map(h, &wide.h, hid, hcols, R, 256, 32)) ||
+            (rc = encode_map(h, &wide.out, out, hcols, R, 32, 32)))
+          return rc;
+        have_wide = true;
+      }
+      wide.w = wmaps[map_slot(128)];
+      if (phase == 0) g.key_tile = 256;
+      const int pairs = (int)(wtiles < h->sms / 2 ? wtiles : h->sms / 2);
+      const int kphase = (phase == 1 && out == hid) ? 2 : phase;
+      if ((ce = launch_proj_gate_wide(kphase, wide, g, 2 * pairs, st)))
+        return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
+    } else {
+      if (!have_single) {
+        if ((rc = encode_map(h, &single.e, e, h->d_mem, R, 128, 64)) ||
+            (rc = encode_map(h, &single.h, hid, hcols, R, 128, 64)) ||
+            (rc = encode_map(h, &single.out, out, hcols, R, 128, 64)))
+          return rc;
+        have_single = true;
+      }
+      const int64_t mblk = (rows + 127) / 128;
+      int bn = 64;
+      for (int c : {256, 128})
+        if (n_total % c == 0 && mblk * (n_total / c) >= h->sms) {
+          bn = c;
+          break;
+        }
+      const int64_t tiles = mblk * (n_total / bn);
+      single.w = wmaps[map_slot(bn)];
+      if (phase == 0) g.key_tile = bn;
+      if ((ce = launch_proj_gate_sm100(phase, bn, single, g,
+                                       (int)(tiles < h->sms ? tiles : h->sms), st)))
+        return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
+    }
+  }
+  h->launches += 2;
+  return ENGRAM_OK;
+}

@@ -28,7 +28,8 @@ ENGRAM_FLAG_NO_CTA_PAIRS = 1
 EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last_error",
            "engram_set_params", "engram_reserve", "engram_get_hash_params", "engram_hash",
            "engram_gather", "engram_forward", "engram_prefetch", "engram_check_errors",
-           "engram_profile_next_forward", "engram_kernel_launches")
+           "engram_profile_next_forward", "engram_kernel_launches",
+           "engram_project_gate_noalloc")
 
 
 class engram_config(ctypes.Structure):
@@ -72,6 +73,7 @@ def _load():
         "engram_check_errors": ([H, P], ctypes.c_int),
         "engram_profile_next_forward": ([H, P, i32], ctypes.c_int),
         "engram_kernel_launches": ([H], ctypes.c_int64),
+        "engram_project_gate_noalloc": ([H, P, i64, P, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -199,6 +201,11 @@ class Engram:
 
     def kernel_launches(self) -> int:
         return int(lib.engram_kernel_launches(self._h))
+
+    def project_gate_noalloc(self, e, h, out, alpha=None, stream=None):
+        """Projection + gate from caller-supplied memory vectors; allocates nothing."""
+        self._check(lib.engram_project_gate_noalloc(self._h, _ptr(e), e.shape[0], _ptr(h),
+                                                    _ptr(out), _ptr(alpha), _stream_ptr(stream)))
 
     def check_errors(self, stream=None) -> int:
         """Synchronise the stream; return the device error status (0 = none)."""

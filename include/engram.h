@@ -252,6 +252,33 @@ ENGRAM_API int engram_profile_next_forward(engram_handle *h, void *const *events
 /* Number of CUDA kernels this handle has launched since it was created. */
 ENGRAM_API int64_t engram_kernel_launches(const engram_handle *h);
 
+/*
+ * Allocation-free projection + gate (steps 5-7 of engram_forward), for callers
+ * that must not have the library allocate device memory: code that runs while
+ * a CUDA graph is being captured (cudaMalloc cannot be captured and breaks the
+ * capture), and hosts whose device memory must all come from their own
+ * allocator or pool.  This call has no counterpart in the paper; it is the
+ * same computation as engram_forward from the gathered memory vectors on.
+ *  e      device [rows, d_mem] dtype: memory vectors, e.g. from engram_hash +
+ *         engram_gather into the caller's own buffers.
+ *  hid    device [rows, M, d] dtype.
+ *  out    device [rows, M, d] dtype (may alias hid for the in-place update).
+ *  alpha  device fp32 [rows, M] or NULL.
+ * The only scratch, 16 bytes per (row, 64-column key tile) of partial sums, is
+ * a fixed 4 MiB array in the library's device image (every GPU that loads the
+ * library keeps it until the process exits), so rows may not exceed
+ * 4 MiB / (16 * M * d / 64); larger calls fail with ENGRAM_ERR_INVALID and a
+ * message that states the limit.  The first call on a device looks up that
+ * array's device address (cudaGetSymbolAddress) with the handle's device
+ * current; make that first call before any stream capture.  Every call on a
+ * device shares the array and the next call overwrites it: calls whose work
+ * overlaps on the GPU (other streams, other handles) race and must be
+ * serialised by the caller.  Errors: _INVALID, _STATE, _CUDA.
+ */
+ENGRAM_API int engram_project_gate_noalloc(engram_handle *h, const void *e, int64_t rows,
+                                           const void *hid, void *out, float *alpha,
+                                           void *stream);
+
 #ifdef __cplusplus
 }
 #endif

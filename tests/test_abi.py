@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_header_and_binding_agree(eg):
     names = declared_symbols()
-    assert names == set(eg.EXPORTS) and len(names) == 14
+    assert names == set(eg.EXPORTS) and len(names) == 15
 
 
 def test_library_exports_every_declared_symbol(eg):
@@ -88,7 +88,8 @@ def test_null_arguments(eg):
                      ("engram_set_params", (None,) * 6),
                      ("engram_gather", (None, None, 1, None, None)),
                      ("engram_prefetch", (None, None, 1, 1, 0, None, None)),
-                     ("engram_profile_next_forward", (None, None, 5))):
+                     ("engram_profile_next_forward", (None, None, 5)),
+                     ("engram_project_gate_noalloc", (None, None, 1, None, None, None, None))):
         assert getattr(eg.lib, fn)(*args) == eg.ENGRAM_ERR_INVALID, fn
     assert eg.lib.engram_kernel_launches(None) == -1
     eg.lib.engram_destroy(None)
