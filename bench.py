@@ -164,15 +164,16 @@ def algorithmic(sh):
 
 
 def kernel_traffic():
-    """DRAM bytes per launch of the projection kernel from a committed ncu
-    capture, or None when the kernel source changed since the capture."""
+    """DRAM bytes per step of the projection kernel (key + value launches)
+    from a committed ncu capture, or None once its source has changed."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    src = os.path.join(ROOT, "hashed_gram_embedding_compress_b200", "csrc", "k_proj_gate_sm100.cu")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if d.get("source_sha256_16") != h:
+    h = hashlib.sha256()
+    for f in d.get("sources", []):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if d.get("source_sha256_16") != h.hexdigest()[:16]:
         return None
     return d.get("proj_gate_bytes_per_step")
 
@@ -305,7 +306,7 @@ def run_ours(args, rank, world, dist):
             "residual": "in place: out aliases h (H <- H + alpha v)",
         },
         "roofline": {
-            "kernel": "proj_gate_kernel (tcgen05 key + value launches)",
+            "kernel": "proj_gate_wide_kernel: key + in-place value launches per step (tcgen05, CTA pairs)",
             "bound": "tensor",
             "achieved": gemm_tflops,
             "peak": tflops,
