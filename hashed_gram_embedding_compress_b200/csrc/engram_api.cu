@@ -648,6 +648,13 @@ int engram_profile_next_forward(engram_handle* h, void* const* events, int32_t n
 
 int64_t engram_kernel_launches(const engram_handle* h) { return h ? h->launches : -1; }
 
+int engram_selftest_timeout(engram_handle* h, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  CK(h, launch_wait_timeout_selftest(h->d_err, (cudaStream_t)stream));
+  h->launches += 1;
+  return engram_check_errors(h, stream);
+}
+
 int engram_check_errors(engram_handle* h, void* stream) {
   if (!h) return ENGRAM_ERR_INVALID;
   CK(h, cudaStreamSynchronize((cudaStream_t)stream));

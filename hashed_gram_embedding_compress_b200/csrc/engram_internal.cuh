@@ -78,6 +78,7 @@ struct PrefetchArgs {
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
 cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream);
+cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t stream);
 cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);
 
 // fp32 path (SIMT FFMA; 64-column tiles).  phase 0 = key tiles over W_K

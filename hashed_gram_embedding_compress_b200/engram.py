@@ -29,7 +29,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_set_params", "engram_reserve", "engram_get_hash_params", "engram_hash",
            "engram_gather", "engram_forward", "engram_prefetch", "engram_check_errors",
            "engram_profile_next_forward", "engram_kernel_launches",
-           "engram_project_gate_noalloc")
+           "engram_project_gate_noalloc", "engram_selftest_timeout")
 
 
 class engram_config(ctypes.Structure):
@@ -74,6 +74,7 @@ def _load():
         "engram_profile_next_forward": ([H, P, i32], ctypes.c_int),
         "engram_kernel_launches": ([H], ctypes.c_int64),
         "engram_project_gate_noalloc": ([H, P, i64, P, P, P, P], ctypes.c_int),
+        "engram_selftest_timeout": ([H, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -206,6 +207,10 @@ class Engram:
         """Projection + gate from caller-supplied memory vectors; allocates nothing."""
         self._check(lib.engram_project_gate_noalloc(self._h, _ptr(e), e.shape[0], _ptr(h),
                                                     _ptr(out), _ptr(alpha), _stream_ptr(stream)))
+
+    def selftest_timeout(self, stream=None) -> int:
+        """Run the bounded-wait expiry self-test; returns ENGRAM_ERR_TIMEOUT if it works."""
+        return lib.engram_selftest_timeout(self._h, _stream_ptr(stream))
 
     def check_errors(self, stream=None) -> int:
         """Synchronise the stream; return the device error status (0 = none)."""

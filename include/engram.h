@@ -249,6 +249,16 @@ ENGRAM_API int engram_check_errors(engram_handle *h, void *stream);
  */
 ENGRAM_API int engram_profile_next_forward(engram_handle *h, void *const *events, int32_t n_events);
 
+/*
+ * Self-test of device-side failure detection.  Launches on `stream` a one-CTA
+ * kernel that waits on an mbarrier no thread ever arrives at, with the same
+ * bounded wait the tensor-core kernels use (limit 2 s): the wait expires, the
+ * kernel records a timeout in the device error word and returns normally.
+ * Then behaves as engram_check_errors, so it returns ENGRAM_ERR_TIMEOUT when
+ * the mechanism works; the handle and the CUDA context remain usable.
+ */
+ENGRAM_API int engram_selftest_timeout(engram_handle *h, void *stream);
+
 /* Number of CUDA kernels this handle has launched since it was created. */
 ENGRAM_API int64_t engram_kernel_launches(const engram_handle *h);
 

@@ -1,0 +1,86 @@
+"""Host-resident tables: deterministic prefetch over PCIe (section 2.5, Fig. 2b).
+
+The prefetch hashes the tokens ahead, de-duplicates the addressed rows, copies
+each distinct row once from pinned host memory into an HBM staging buffer on a
+side stream, and the forward gathers from there.  Its results must equal the
+device-resident path bit for bit (same rows, same kernels after the gather).
+"""
+import numpy as np
+import pytest
+import torch
+
+from engram_cases import Problem, out_close, rel_l2, to_oracle
+from hashed_gram_embedding_compress_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _pair(shape):
+    host = Problem(shape.replace(table_location="pinned_host"))
+    dev_tables = [t.cuda() for t in host.tables]
+    return host, dev_tables
+
+
+def test_prefetch_then_forward_equals_device_tables():
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=1500, rows_target=1 << 18)
+    p, dev_tables = _pair(sh)
+    assert p.tables[0].is_pinned()
+    m = p.engram()
+    # reference: the same inputs with device-resident tables
+    md = eg.Engram(eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=p.comp_map,
+                                  orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
+                                  d_hidden=sh.d_hidden, branches=sh.branches, dtype=sh.dtype,
+                                  table_rows_target=sh.rows_target, hash_seed=p.hash_seed))
+    md.set_params(dev_tables, p.w_k, p.w_v, p.norm_q, p.norm_k)
+    tok = p.tokens.cuda()
+    ref = torch.empty_like(p.h)
+    a_ref = torch.empty((sh.rows_out, 1), device="cuda")
+    md.forward(tok, p.h, ref, alpha=a_ref)
+
+    side = torch.cuda.Stream()
+    n = m.prefetch(tok, stream=side, want_count=True)
+    # distinct (table, row) pairs among the oracle's indices
+    want = sum(len(np.unique(p.z[:, s])) for s in range(sh.num_tables))
+    assert n == want
+    out = torch.empty_like(p.h)
+    alpha = torch.empty((sh.rows_out, 1), device="cuda")
+    m.forward(tok, p.h, out, alpha=alpha)  # waits for the prefetch on the side stream
+    torch.cuda.synchronize()
+    assert m.check_errors() == 0
+    assert torch.equal(out, ref) and torch.equal(alpha, a_ref)
+    rows = p.sample_rows(24)
+    _, a_o, _, o_o = p.oracle_forward(rows)
+    rs = torch.from_numpy(rows).cuda()
+    assert rel_l2(alpha[rs].double().cpu(), a_o) <= 1e-3
+    assert out_close(to_oracle(out[rs]), o_o, "bf16") <= 1e-3
+
+
+def test_double_buffered_prefetch_and_call_order():
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=300, rows_target=1 << 16, d_hidden=256)
+    p, dev_tables = _pair(sh)
+    m = p.engram()
+    tok_a = p.tokens.cuda()
+    tok_b = torch.flip(p.tokens, dims=[1]).contiguous().cuda()
+    with pytest.raises(eg.EngramError) as ei:
+        m.forward(tok_a, p.h, torch.empty_like(p.h))
+    assert ei.value.code == eg.ENGRAM_ERR_STATE
+    side = torch.cuda.Stream()
+    m.prefetch(tok_a, stream=side)
+    m.prefetch(tok_b, stream=side)
+    with pytest.raises(eg.EngramError) as ei:
+        m.prefetch(tok_a, stream=side)  # a third pending prefetch has no staging slot
+    assert ei.value.code == eg.ENGRAM_ERR_STATE
+    md = eg.Engram(eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=p.comp_map,
+                                  orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
+                                  d_hidden=sh.d_hidden, branches=sh.branches, dtype=sh.dtype,
+                                  table_rows_target=sh.rows_target, hash_seed=p.hash_seed))
+    md.set_params(dev_tables, p.w_k, p.w_v, p.norm_q, p.norm_k)
+    for tok in (tok_a, tok_b):  # consumed in prefetch order
+        out, ref = torch.empty_like(p.h), torch.empty_like(p.h)
+        m.forward(tok, p.h, out)
+        md.forward(tok, p.h, ref)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    assert m.check_errors() == 0

@@ -225,3 +225,17 @@ def test_out_of_range_tokens_are_reported_not_read():
     m.gather(idx, e)
     assert m.check_errors() == eg.ENGRAM_ERR_BOUNDS
     assert torch.all(e[3, 2 * sh.d_head:3 * sh.d_head] == 0)
+
+
+def test_bounded_wait_expiry_is_reported_and_context_survives():
+    # a kernel waits on an mbarrier nothing arrives at: the bounded wait
+    # expires (2 s), the timeout is reported, and the next forward is exact
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["tiny_f32"]
+    p = Problem(sh)
+    m = p.engram()
+    assert m.selftest_timeout() == eg.ENGRAM_ERR_TIMEOUT
+    assert m.check_errors() == 0
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, np.arange(sh.rows_out), out, a, dl)
