@@ -33,6 +33,19 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Engram fwd tokens/s (hash+gather+gate); gather GB/s as % of HBM peak"
 WORKLOAD = "prefill_bf16"
+DESCRIBE = {
+    "prefill_bf16": "prefill_bf16: B=8 x T=4096 tokens, vocab 32768->25231, orders {2,3} x 8 heads, "
+                    "16 tables of primes >= 2^20 rows x 80 bf16 (d_mem 1280), d=2560, M=1, "
+                    "fp32 accumulate",
+    "decode_mb": "decode_mb: B=256 sequences, 1 new token each after a 2-token prefix, tables as "
+                 "prefill_bf16, M=4 branches (own W_K 1280->2560 and RMSNorm weights each, shared "
+                 "W_V), h [256,4,2560] bf16",
+    "large_hbm": "large_hbm: B=4 x T=8192 tokens, vocab 128000->98560, 16 tables of primes >= 2^24 "
+                 "rows x 80 bf16 (43 GB in HBM), d=4096, M=4",
+    "offload": "offload: large_hbm shapes with the tables in pinned host memory, rows prefetched "
+               "over PCIe one step ahead on a side stream, overlapped with a 4096^3 bf16 GEMM "
+               "standing in for the preceding backbone block",
+}
 
 
 def parse():
@@ -45,6 +58,14 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="prefill_bf16",
+                    choices=["prefill_bf16", "decode_mb", "large_hbm", "offload"],
+                    help="prefill_bf16 is the benchmarked line; the others measure the other "
+                         "configurations of the same forward")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step from a captured CUDA graph (launch-bound shapes)")
+    ap.add_argument("--offload-gb", type=float, default=100.0,
+                    help="offload workload: total size of the pinned host tables")
     ap.add_argument("--rows-target", type=int, default=None,
                     help="smaller tables for profiling captures (same kernel shapes); "
                          "not the benchmarked workload")
@@ -121,15 +142,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------ the workload
 
-def setup(rank: int, device, rows_target=None):
+def setup(rank: int, device, rows_target=None, workload=WORKLOAD):
     import torch
     from hashed_gram_embedding_compress_b200 import engram as eg
     from hashed_gram_embedding_compress_b200 import synth
 
-    sh = synth.SHAPES[WORKLOAD]
+    sh = synth.SHAPES[workload]
     if rows_target:
         sh = sh.replace(rows_target=rows_target)
-    seeds = synth.stream_seeds(sh, extra=rank)
+    seeds = rank_seeds(rank, workload)
     tokens = synth.make_tokens(sh, seeds)
     comp_map = synth.make_comp_map(sh, seeds)
     cfg = eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=comp_map, orders=sh.orders,
@@ -178,21 +199,52 @@ def kernel_traffic():
     return d.get("proj_gate_bytes_per_step")
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seeds(rank: int, workload: str = WORKLOAD):
+    """Each rank draws its own batch: independent replicas (weak scaling)."""
+    from hashed_gram_embedding_compress_b200 import synth
+    return synth.stream_seeds(synth.SHAPES[workload], extra=rank)
+
+
 def run_ours(args, rank, world, dist):
     import torch
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    P = setup(rank, device, args.rows_target)
+    P = setup(rank, device, args.rows_target, args.workload)
     sh, m = P["sh"], P["m"]
     tok_d = P["tokens"].to(device)
     h = P["h"]
     stream = torch.cuda.current_stream()
 
     # the residual update H <- H + Y in place: out aliases h
+    def forward_once():
+        m.forward(tok_d, h, h, t_begin=sh.t_begin, stream=torch.cuda.current_stream())
+
+    graph = None
+    if args.graph:
+        forward_once()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            forward_once()
+        torch.cuda.synchronize()
+
     def step():
-        m.forward(tok_d, h, h, stream=stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            forward_once()
 
     clk = ClockSampler(local).__enter__()
     for _ in range(max(3, args.warmup)):
@@ -220,7 +272,8 @@ def run_ours(args, rank, world, dist):
     torch.cuda.synchronize()
     t0.record(stream)
     for k in range(K):
-        m.profile_next_forward(evs[k])
+        if graph is None:
+            m.profile_next_forward(evs[k])
         step()
     t1.record(stream)
     torch.cuda.synchronize()
@@ -230,13 +283,24 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
     launches = m.kernel_launches() - launches0
-    ms = t0.elapsed_time(t1)
-    if dist:
-        tt = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    stage = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)]
-    st_mean = [sum(s[i] for s in stage) / K for i in range(4)]  # hash, gather, key, value (ms)
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, device)
+    if graph is None:
+        stage = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)]
+        st_mean = [sum(s[i] for s in stage) / K for i in range(4)]  # hash, gather, key, value
+    else:
+        # one graph replay per step: no per-kernel events; split by the same
+        # shares would be a guess, so the stages are timed by replaying the
+        # eager forward once more with events
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        for e_ in ev:
+            e_.record(stream)
+        st_mean = [0.0] * 4
+        for _ in range(5):
+            m.profile_next_forward(ev)
+            forward_once()
+            torch.cuda.synchronize()
+            for i in range(4):
+                st_mean[i] += ev[i].elapsed_time(ev[i + 1]) / 5
     if m.check_errors(stream) != 0:
         raise RuntimeError("device error during the timed steps")
 
@@ -251,7 +315,7 @@ def run_ours(args, rank, world, dist):
     def e2e_step():
         tok_buf.copy_(tok_h, non_blocking=True)
         h_buf.copy_(h_h, non_blocking=True)
-        m.forward(tok_buf, h_buf, h_buf, stream=stream)
+        m.forward(tok_buf, h_buf, h_buf, t_begin=sh.t_begin, stream=stream)
         out_h.copy_(h_buf, non_blocking=True)
 
     e2e_step()
@@ -264,11 +328,8 @@ def run_ours(args, rank, world, dist):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     if dist:
-        tt = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         dist.barrier()
     if rank != 0:
         return None
@@ -295,15 +356,15 @@ def run_ours(args, rank, world, dist):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": "prefill_bf16: B=8 x T=4096 tokens, vocab 32768->25231, orders {2,3} x 8 "
-                        "heads, 16 tables of primes >= 2^20 rows x 80 bf16 (d_mem 1280), d=2560, "
-                        "M=1, fp32 accumulate",
+            "workload": DESCRIBE[args.workload],
             "global_batch": tokens_per_step * world,
             "seq_len": sh.T,
             "parallelism": "replicas" if world > 1 else "single",
-            "l2": "no flush: inputs larger than L2 (h 168 MB read, out 168 MB written, "
-                  "tables 2.7 GB)",
+            "l2": "no flush: inputs larger than L2 (h %.0f MB read and written, tables %.1f GB)"
+                  % (h.numel() * h.element_size() / 1e6,
+                     sum(t.numel() * t.element_size() for t in P["tables"]) / 1e9),
             "residual": "in place: out aliases h (H <- H + alpha v)",
+            "cuda_graph": bool(graph is not None),
         },
         "roofline": {
             "kernel": "proj_gate_wide_kernel: key + in-place value launches per step (tcgen05, CTA pairs)",
@@ -336,9 +397,159 @@ def run_ours(args, rank, world, dist):
     }
     if args.rows_target:
         res["config"]["workload"] += " [profiling variant: tables of %d rows]" % args.rows_target
+    if args.workload != "prefill_bf16":
+        res["roofline"]["traffic"] = None  # the committed capture is of the prefill shapes
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(P, args.cpu_seconds)
     return res
+
+
+# ------------------------------------------------------ host-offload leg
+
+def run_offload(args):
+    """Tables in page-locked host memory (section 2.5, Figure 2b).
+
+    Per step: engram_prefetch of the NEXT step's tokens on a side stream (hash,
+    de-duplicate, copy each distinct row once over PCIe into HBM staging),
+    while the main stream runs the backbone stand-in (4096^3 bf16 GEMMs) and
+    the engram forward of the current step from the staged rows."""
+    import torch
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    from hashed_gram_embedding_compress_b200 import synth
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    sh0 = synth.SHAPES["offload"]
+    row_bytes = sh0.d_head * 2
+    sh = sh0.replace(rows_target=int(args.offload_gb * 1e9 / (sh0.num_tables * row_bytes)))
+    seeds = synth.stream_seeds(sh)
+    comp_map = synth.make_comp_map(sh, seeds)
+    hash_seed = synth.make_hash_seed(seeds)
+    m = eg.Engram(eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=comp_map,
+                                 orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
+                                 d_hidden=sh.d_hidden, branches=sh.branches, dtype=sh.dtype,
+                                 table_rows_target=sh.rows_target, hash_seed=hash_seed,
+                                 table_location="pinned_host"))
+    primes, _ = m.hash_params()
+    # pageable buffers, then page-locked and mapped into the device's address space
+    t_setup = time.time()
+    cudart = torch.cuda.cudart()
+    g = torch.Generator(device=dev)
+    g.manual_seed(seeds["tables"])
+    tables = []
+    try:
+        for p in primes.tolist():
+            t = torch.empty((p, sh.d_head), dtype=torch.bfloat16)
+            rc = cudart.cudaHostRegister(t.data_ptr(), t.numel() * 2, 3)  # portable | mapped
+            if int(rc) != 0:
+                raise RuntimeError("cudaHostRegister failed (%s)" % rc)
+            tables.append(t)
+            step = 1 << 22
+            for a in range(0, p, step):
+                b = min(p, a + step)
+                x = torch.randn((b - a, sh.d_head), generator=g, device=dev).mul_(0.02)
+                t[a:b].copy_(x.to(torch.bfloat16))
+        torch.cuda.synchronize()
+        t_setup = time.time() - t_setup
+        w_k, w_v, nq, nk = [x.to(dev) for x in synth.make_weights(sh, seeds)]
+        m.set_params(tables, w_k, w_v, nq, nk)
+        h = synth.make_hidden(sh, seeds, device=dev)
+        K = max(3, args.steps)
+        toks = [synth.make_tokens(sh, synth.stream_seeds(sh, extra=100 + k)).to(dev)
+                for k in range(K + 2)]
+        m.reserve(sh.rows_out)
+        a_ = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
+        b_ = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
+        main = torch.cuda.current_stream()
+        side = torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+
+        def timed(fn, stream, reps):
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            for i in range(reps):
+                fn(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        for _ in range(3):
+            a_ @ b_
+        t_gemm = timed(lambda i: a_ @ b_, main, 20)
+        # prefetch alone (side stream), then the forward from the staged rows
+        uniq, t_pf, t_fw = [], [], []
+        for k in range(K):
+            e0, e1 = ev(), ev()
+            e0.record(side)
+            m.prefetch(toks[k], stream=side)
+            e1.record(side)
+            torch.cuda.synchronize()
+            t_pf.append(e0.elapsed_time(e1))
+            f0, f1 = ev(), ev()
+            f0.record(main)
+            m.forward(toks[k], h, h, stream=main)
+            f1.record(main)
+            torch.cuda.synchronize()
+            t_fw.append(f0.elapsed_time(f1))
+        for k in range(K):
+            uniq.append(m.prefetch(toks[k], stream=side, want_count=True))
+            m.forward(toks[k], h, h, stream=main)
+            torch.cuda.synchronize()
+        t_pf, t_fw = statistics.median(t_pf[1:]), statistics.median(t_fw[1:])
+        n_hide = max(1, int(-(-t_pf // t_gemm)))  # stand-in GEMMs whose time covers a prefetch
+
+        def pipeline(n_gemm):
+            m.prefetch(toks[0], stream=side)
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            e0.record(main)
+            for k in range(K):
+                m.prefetch(toks[k + 1], stream=side)  # next step's rows, overlapped
+                for _ in range(n_gemm):
+                    a_ @ b_
+                m.forward(toks[k], h, h, stream=main)
+            e1.record(main)
+            torch.cuda.synchronize()
+            m.forward(toks[K], h, h, stream=main)  # consume the last pending prefetch
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / K
+
+        t_pipe1 = pipeline(1)
+        t_pipe_n = pipeline(n_hide)
+        if m.check_errors() != 0:
+            raise RuntimeError("device error in the offload run")
+        u = statistics.mean(uniq)
+        pcie_bytes = u * row_bytes
+        total_bytes = sum(t.numel() * 2 for t in tables)
+        return {
+            "metric": METRIC, "value": sh.rows_out / (t_pipe1 / 1e3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": K, "warmup": 1, "ms_per_step": t_pipe1,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": DESCRIBE["offload"], "global_batch": sh.rows_out,
+                       "seq_len": sh.T, "parallelism": "single",
+                       "host_tables_gb": total_bytes / 1e9,
+                       "rows_per_table": primes.tolist()},
+            "offload": {
+                "unique_rows_per_step": u,
+                "unique_fraction": u / (sh.rows_out * sh.num_tables),
+                "pcie_bytes_per_step": pcie_bytes,
+                "prefetch_ms": t_pf,
+                "pcie_gbs": pcie_bytes / (t_pf / 1e3) / 1e9,
+                "forward_from_staging_ms": t_fw,
+                "standin_gemm_ms": t_gemm,
+                "step_ms_1_gemm": t_pipe1,
+                "serial_ms_1_gemm": t_pf + t_gemm + t_fw,
+                "gemms_to_hide_prefetch": n_hide,
+                "step_ms_n_gemm": t_pipe_n,
+                "loss_vs_hidden_prefetch": t_pipe_n / (n_hide * t_gemm + t_fw) - 1.0,
+                "host_setup_s": t_setup,
+            },
+        }
+    finally:
+        torch.cuda.synchronize()
+        for t in tables:
+            cudart.cudaHostUnregister(t.data_ptr())
 
 
 # ----------------------------------------------------------- CPU oracle leg
@@ -359,7 +570,7 @@ def cpu_baseline(P, budget_s: float):
     t0 = time.perf_counter()
     c, z, mult, primes = oracle.forward_indices(tokens, P["comp_map"].numpy(), sh.cvocab,
                                                 sh.orders, sh.heads, P["hash_seed"],
-                                                sh.rows_target)
+                                                sh.rows_target, t_begin=sh.t_begin)
     t_hash = (time.perf_counter() - t0) / sh.rows_out
 
     def to_np(t):
@@ -395,7 +606,7 @@ def run_reference(args, rank, world):
         return None
     import torch
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    P = setup(0, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))))
+    P = setup(0, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))), None, args.workload)
     sh = P["sh"]
     budget = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -407,7 +618,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sh.rows_out / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "prefill_bf16 (as the ours arm)", "global_batch": sh.rows_out,
+        "config": {"workload": DESCRIBE[args.workload], "global_batch": sh.rows_out,
                    "seq_len": sh.T, "parallelism": "single"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": vals[-1]["sample"]},
@@ -430,6 +641,8 @@ def main():
         dist = tdist
     if args.impl == "reference":
         res = run_reference(args, rank, world)
+    elif args.workload == "offload":
+        res = run_offload(args) if rank == 0 else None
     else:
         res = run_ours(args, rank, world, dist)
     if res is not None:
