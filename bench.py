@@ -171,7 +171,7 @@ def setup(rank: int, device, rows_target=None, workload=WORKLOAD):
 
 
 def algorithmic(sh):
-    """Per-step algorithmic work (measurement section)."""
+    """Per-step algorithmic work: bytes of the gather and hash, FLOPs and bytes of the projections."""
     R, S, dm, d, M = sh.rows_out, sh.num_tables, sh.d_mem, sh.d_hidden, sh.branches
     elt = 2 if sh.dtype == "bf16" else 4
     row_bytes = sh.d_head * elt
