@@ -17,14 +17,30 @@ constexpr int kHashThreads = 256;
 // One thread per (row, slot): consecutive threads write consecutive int64, so
 // the index store is coalesced; the three token reads and map lookups per
 // thread hit L1/L2 (the map is at most 512 KB).
+// x mod p for a 64-bit x and 2 <= p < 2^31, by Barrett reduction (P. Barrett,
+// "Implementing the RSA public key encryption algorithm on a standard digital
+// signal processor", CRYPTO 1986): with inv = floor((2^64 - 1) / p), the
+// quotient estimate q = floor(x * inv / 2^64) is floor(x / p) or one less, so
+// x - q p lies in [0, 2p) and one conditional subtraction gives the exact
+// remainder.
+__device__ __forceinline__ uint64_t mod_barrett(uint64_t x, uint64_t p, uint64_t inv) {
+  const uint64_t q = __umul64hi(x, inv);
+  uint64_t r = x - q * p;
+  if (r >= p) r -= p;
+  return r;
+}
+
 __global__ void __launch_bounds__(kHashThreads) hash_kernel(HashArgs a) {
   __shared__ uint64_t s_mult[kMaxTables * kMaxOrders];
   __shared__ uint64_t s_prime[kMaxTables];
+  __shared__ uint64_t s_inv[kMaxTables];
   __shared__ int32_t s_order_of_slot[kMaxTables];
   const int S = a.S;
   for (int i = threadIdx.x; i < S * a.max_order; i += blockDim.x) s_mult[i] = a.mult[i];
   for (int i = threadIdx.x; i < S; i += blockDim.x) {
-    s_prime[i] = (uint64_t)a.primes[i];
+    const uint64_t p = (uint64_t)a.primes[i];
+    s_prime[i] = p;
+    s_inv[i] = 0xFFFFFFFFFFFFFFFFull / p;
     s_order_of_slot[i] = a.orders[i / a.heads];
   }
   __syncthreads();
@@ -53,7 +69,7 @@ __global__ void __launch_bounds__(kHashThreads) hash_kernel(HashArgs a) {
       }
       x ^= (uint64_t)c * s_mult[s * a.max_order + j];
     }
-    a.idx[i] = (int64_t)(x % s_prime[s]);
+    a.idx[i] = (int64_t)mod_barrett(x, s_prime[s], s_inv[s]);
   }
 }
 

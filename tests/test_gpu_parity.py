@@ -98,11 +98,13 @@ def test_prefill_full_size_sampled():
     # without the optional outputs and with caller-supplied indices: same out
     out2, _, _ = run_forward(p, m, idx=idx, alpha=False, delta=False)
     assert torch.equal(out, out2)
-    # single-CTA 128-row tiles: same parity bar, and the same values
-    m1 = p.engram(flags=eg.ENGRAM_FLAG_NO_CTA_PAIRS)
-    out1, a1, dl1 = run_forward(p, m1)
-    check_rows(p, m1, idx, p.sample_rows(32, seed=1), out1, a1, dl1)
-    assert rel_l2(dl1.double(), dl.double()) < 1e-6
+    # the other tilings: CTA pairs without clusters, single CTAs; same bar, same values
+    for flags in (eg.ENGRAM_FLAG_NO_QUAD, eg.ENGRAM_FLAG_NO_CTA_PAIRS):
+        m1 = p.engram(flags=flags)
+        out1, a1, dl1 = run_forward(p, m1)
+        check_rows(p, m1, idx, p.sample_rows(32, seed=1), out1, a1, dl1)
+        assert rel_l2(dl1.double(), dl.double()) < 1e-6
+        check_in_place(p, m1, out1, dl1)
     check_in_place(p, m, out, dl)
 
 
@@ -132,12 +134,14 @@ def test_decode_multibranch():
     check_rows(p, m, idx, p.sample_rows(48), out, a, dl)
 
 
-@pytest.mark.parametrize("R_B,R_T,flags", [(1, 20000, 0), (1, 20000, 1), (1, 10000, 0),
-                                           (1, 2000, 0), (3, 5, 0), (1, 1, 0), (1, 19000, 0)])
+@pytest.mark.parametrize("R_B,R_T,flags", [(1, 20000, 0), (1, 20000, 1), (1, 20000, 2),
+                                           (1, 10000, 0), (1, 2000, 0), (3, 5, 0), (1, 1, 0),
+                                           (1, 19000, 0), (1, 19000, 2)])
 def test_tile_widths_and_ragged_rows(R_B, R_T, flags):
-    # d = 256 lets the launcher pick CTA-pair 256 x 256 tiles, or single-CTA
-    # 256-, 128- and 64-column tiles, by row count (flags=1: no CTA pairs);
-    # 20000 and 19000 rows end in a pair tile whose second CTA has no rows
+    # d = 256 lets the launcher pick 4-CTA clusters, CTA pairs, or single-CTA
+    # 256-, 128- and 64-column tiles, by row count (flags=1: no CTA pairs,
+    # flags=2: no 4-CTA clusters); 20000 and 19000 rows end in a 512-row tile
+    # whose last CTAs have no rows
     sh = synth.SHAPES["prefill_bf16"].replace(B=R_B, T=R_T, rows_target=2053, d_hidden=256,
                                               branches=2)
     p = Problem(sh)
