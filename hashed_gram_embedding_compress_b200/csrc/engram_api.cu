@@ -232,8 +232,7 @@ int engram_create(const engram_config* cfg, engram_handle** out) {
   if (c.table_location != ENGRAM_DEVICE && c.table_location != ENGRAM_PINNED_HOST)
     return fail(nullptr, ENGRAM_ERR_INVALID, "bad table_location");
   if (c.pad_id < -1) return fail(nullptr, ENGRAM_ERR_INVALID, "pad_id must be >= -1");
-  if (c.flags & ~(ENGRAM_FLAG_NO_CTA_PAIRS | ENGRAM_FLAG_NO_QUAD))
-    return fail(nullptr, ENGRAM_ERR_INVALID, "unknown flags");
+  if (c.flags & ~ENGRAM_FLAG_NO_CTA_PAIRS) return fail(nullptr, ENGRAM_ERR_INVALID, "unknown flags");
   const int S = c.num_orders * c.heads;
   const int64_t d_mem = (int64_t)S * c.d_head;
   if (d_mem > (1 << 20)) return fail(nullptr, ENGRAM_ERR_INVALID, "d_mem too large");
@@ -593,31 +592,13 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   // else single-CTA 128-row tiles of the widest N that fills the SMs.
   const int64_t hcols = (int64_t)g.M * g.d;
   const bool pairs_ok = !(h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS);
-  const bool quad_ok = pairs_ok && !(h->cfg.flags & ENGRAM_FLAG_NO_QUAD);
-  if (quad_ok && h->quad_clusters < 0) h->quad_clusters = quad_max_clusters();
-  ProjMaps single, wide, quad;
-  bool have_single = false, have_wide = false, have_quad = false;
+  ProjMaps single, wide;
+  bool have_single = false, have_wide = false;
   for (int phase = 0; phase < 2; ++phase) {
     const int n_total = phase == 0 ? g.M * g.d : g.d;
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
     const int64_t wtiles = (R + 511) / 512 * (n_total / 256);
-    // 512-row tiles waste the rows past R of the last block: use them when
-    // at least 7/8 of the padded rows are real
-    const bool rows_fill = (R + 511) / 512 * 512 * 7 <= R * 8;
-    if (quad_ok && h->quad_clusters > 0 && n_total % 256 == 0 && rows_fill &&
-        wtiles >= h->quad_clusters) {
-      if (!have_quad) {
-        if ((rc = make_map(h, &quad.e, h->e, h->d_mem, R, 128))) return rc;
-        if ((rc = make_map(h, &quad.h, hid, hcols, R, 128, 32))) return rc;
-        if ((rc = make_map(h, &quad.out, out, hcols, R, 32, 32))) return rc;  // per-warp stores
-        have_quad = true;
-      }
-      quad.w = wmaps[bn_index(128)];  // each CTA of a pair holds 128 of the tile's 256 W rows
-      if (phase == 0) g.key_tile = 256;
-      const int clusters = (int)(wtiles < h->quad_clusters ? wtiles : h->quad_clusters);
-      const int kphase = (phase == 1 && out == hid) ? 2 : phase;
-      CK(h, launch_proj_gate_quad(kphase, quad, g, 4 * clusters, st));
-    } else if (pairs_ok && n_total % 256 == 0 && wtiles >= h->sms / 2) {
+    if (pairs_ok && n_total % 256 == 0 && wtiles >= h->sms / 2) {
       if (!have_wide) {
         if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
         if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;

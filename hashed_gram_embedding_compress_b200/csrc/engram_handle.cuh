@@ -11,7 +11,6 @@
 struct engram_handle {
   engram_config cfg{};
   int device = 0, sms = 148;
-  int quad_clusters = -1;  // 4-CTA clusters that fit at once (-1: not queried yet)
   int S = 0, max_order = 0, d_mem = 0, elt = 4;
   int64_t primes[engram::kMaxTables] = {};
   uint64_t mult[engram::kMaxTables * engram::kMaxOrders] = {};

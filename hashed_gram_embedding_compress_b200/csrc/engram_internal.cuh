@@ -94,17 +94,11 @@ int sm100_stages(int bn);
 //   single-CTA kernel: e box 64 x 128, W box 64 x BN, h/out box 64 x 128 (128-B swizzle)
 //   CTA-pair kernel:   e box 64 x 256, W box 64 x 128, h box 32 x 256, out box 32 x 32
 //                      (h and out with the 64-B swizzle)
-//   4-CTA cluster:     e box 64 x 128, W box 64 x 128, h box 32 x 128, out box 32 x 32
 struct ProjMaps {
   CUtensorMap e, w, h, out;
 };
 cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
                                    int grid, cudaStream_t stream);
-// 512 x 256 tiles on clusters of two CTA pairs sharing W over DSMEM; grid =
-// 4 x clusters (at most quad_max_clusters()).
-cudaError_t launch_proj_gate_quad(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
-                                  cudaStream_t stream);
-int quad_max_clusters();
 // 512 x 256 tiles on CTA pairs (tcgen05 cta_group::2); grid = 2 x pairs.
 // phase 0 keys, 1 values, 2 values added in place (out aliases h).
 cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,

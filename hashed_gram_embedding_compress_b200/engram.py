@@ -23,7 +23,6 @@ ENGRAM_OK, ENGRAM_ERR_INVALID, ENGRAM_ERR_BOUNDS, ENGRAM_ERR_CUDA = 0, 1, 2, 3
 ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_UNSUPPORTED, ENGRAM_ERR_STATE = 4, 5, 6, 7
 MAX_ORDERS, MAX_TABLES, MAX_BRANCHES = 4, 64, 4
 ENGRAM_FLAG_NO_CTA_PAIRS = 1
-ENGRAM_FLAG_NO_QUAD = 2
 
 #: every symbol include/engram.h declares
 EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last_error",

@@ -63,8 +63,7 @@ extern "C" {
 #define ENGRAM_PINNED_HOST 1 /* page-locked host memory, read over PCIe */
 
 /* config flags */
-#define ENGRAM_FLAG_NO_CTA_PAIRS 1 /* bf16 projection on single-CTA tiles only          */
-#define ENGRAM_FLAG_NO_QUAD 2      /* no 4-CTA clusters (CTA pairs with 512-row tiles) */
+#define ENGRAM_FLAG_NO_CTA_PAIRS 1 /* bf16 projection on single-CTA tiles only */
 
 /* status codes */
 #define ENGRAM_OK 0
@@ -111,10 +110,8 @@ typedef struct engram_handle engram_handle;
  *  eps             RMSNorm epsilon (the pages give none; 1e-6 is typical).
  *  table_location  ENGRAM_DEVICE or ENGRAM_PINNED_HOST.
  *  flags           0, or ENGRAM_FLAG_NO_CTA_PAIRS to keep the bf16 projection
- *                  on single-CTA 128-row tiles, or ENGRAM_FLAG_NO_QUAD to use
- *                  CTA pairs without 4-CTA clusters.  By default the largest
- *                  tiling whose tiles fill the GPU is used: 4-CTA clusters
- *                  (two CTA pairs sharing W), then CTA pairs, then single CTAs.
+ *                  on single-CTA 128-row tiles (by default 512 x 256 tiles on
+ *                  CTA pairs are used when they fill the GPU).
  */
 typedef struct engram_config {
   int32_t vocab;

@@ -98,8 +98,8 @@ def test_prefill_full_size_sampled():
     # without the optional outputs and with caller-supplied indices: same out
     out2, _, _ = run_forward(p, m, idx=idx, alpha=False, delta=False)
     assert torch.equal(out, out2)
-    # the other tilings: CTA pairs without clusters, single CTAs; same bar, same values
-    for flags in (eg.ENGRAM_FLAG_NO_QUAD, eg.ENGRAM_FLAG_NO_CTA_PAIRS):
+    # single-CTA tiles: same bar, same values
+    for flags in (eg.ENGRAM_FLAG_NO_CTA_PAIRS,):
         m1 = p.engram(flags=flags)
         out1, a1, dl1 = run_forward(p, m1)
         check_rows(p, m1, idx, p.sample_rows(32, seed=1), out1, a1, dl1)
@@ -134,14 +134,12 @@ def test_decode_multibranch():
     check_rows(p, m, idx, p.sample_rows(48), out, a, dl)
 
 
-@pytest.mark.parametrize("R_B,R_T,flags", [(1, 20000, 0), (1, 20000, 1), (1, 20000, 2),
-                                           (1, 10000, 0), (1, 2000, 0), (3, 5, 0), (1, 1, 0),
-                                           (1, 19000, 0), (1, 19000, 2)])
+@pytest.mark.parametrize("R_B,R_T,flags", [(1, 40000, 0), (1, 20000, 0), (1, 20000, 1), (1, 10000, 0),
+                                           (1, 2000, 0), (3, 5, 0), (1, 1, 0), (1, 37900, 0)])
 def test_tile_widths_and_ragged_rows(R_B, R_T, flags):
-    # d = 256 lets the launcher pick 4-CTA clusters, CTA pairs, or single-CTA
-    # 256-, 128- and 64-column tiles, by row count (flags=1: no CTA pairs,
-    # flags=2: no 4-CTA clusters); 20000 and 19000 rows end in a 512-row tile
-    # whose last CTAs have no rows
+    # d = 256, M = 2 lets the launcher pick CTA-pair 512 x 256 tiles or
+    # single-CTA 256-, 128- and 64-column tiles by row count (flags=1: no CTA
+    # pairs); 37900 rows end in a pair tile whose second CTA has no rows
     sh = synth.SHAPES["prefill_bf16"].replace(B=R_B, T=R_T, rows_target=2053, d_hidden=256,
                                               branches=2)
     p = Problem(sh)
