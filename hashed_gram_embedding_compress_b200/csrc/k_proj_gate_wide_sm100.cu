@@ -339,7 +339,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto key_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
           tmem_wait32(v);
           __syncwarp();
-          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          if (q + 1 < NQ) {
+            tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          } else {
+            // every TMEM read of this tile is done: the accumulators are free
+            // for the next tile's MMAs (the leader owns the barrier)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+          }
           if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) return;
@@ -389,14 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) key_chunk(q + 1, vb, va);
         }
         if (!ok) break;
-        // accumulators and the weight buffer are free again (the pair's leader
-        // owns the accumulator barrier); then the partial sums go out
-        tc_fence_before();
+        // the weight buffer is free again; then the partial sums go out
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_cluster(peer_addr(tempty_bar, 0));
-          mbar_arrive(wempty_bar);
-        }
+        if (lane == 0) mbar_arrive(wempty_bar);
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
       } else if (PHASE == 2) {
         // out aliases h: add bf16(alpha v) into it with TMA reduce-add; each
@@ -407,7 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto add_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
           tmem_wait32(v);
           __syncwarp();
-          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          if (q + 1 < NQ) {
+            tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          } else {
+            tc_fence_before();  // last TMEM read done: release the accumulators
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+          }
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
             float a = 0.f;
@@ -456,15 +465,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           add_chunk(q, va, vb);
           add_chunk(q + 1, vb, va);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
       } else {
         int pending = -1;  // slot whose TMA store may still be reading it
         auto value_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
           tmem_wait32(v);
           __syncwarp();
-          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          if (q + 1 < NQ) {
+            tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          } else {
+            tc_fence_before();  // last TMEM read done: release the accumulators
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+          }
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
             if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
@@ -528,10 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) value_chunk(q + 1, vb, va);
         }
         if (!ok) break;
-        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_cluster(peer_addr(tempty_bar, 0));
           asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
           if (pending >= 0) mbar_arrive(hempty_bar(pending));
         }
