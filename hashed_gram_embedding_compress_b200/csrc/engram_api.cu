@@ -107,12 +107,10 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 int ensure_scratch(engram_handle* h, int64_t rows) {
   if (rows <= h->cap_rows) return ENGRAM_OK;
-  free_dev(h->z);
   free_dev(h->e);
   free_dev(h->partials);
   h->cap_rows = 0;
   const int64_t key_tiles = (int64_t)h->cfg.branches * h->cfg.d_hidden / 64;
-  CK(h, cudaMalloc(&h->z, (size_t)rows * h->S * sizeof(int64_t)));
   CK(h, cudaMalloc(&h->e, (size_t)rows * h->d_mem * h->elt));
   CK(h, cudaMalloc(&h->partials, (size_t)rows * key_tiles * sizeof(float4)));
   h->cap_rows = rows;
@@ -124,7 +122,9 @@ int check_shape(engram_handle* h, int32_t B, int32_t T, int32_t t_begin) {
   if (B > 0 && T > 0 && (t_begin < 0 || t_begin >= T))
     return fail(h, ENGRAM_ERR_INVALID, "t_begin must lie in [0, T)");
   const int64_t rows = (int64_t)B * (T - t_begin);
-  if (rows > (int64_t)1 << 31) return fail(h, ENGRAM_ERR_INVALID, "too many rows");
+  const int64_t per_row = (int64_t)h->S * ((h->cfg.d_head * h->elt) >> 4);  // gather chunks per row
+  if (rows * per_row >= ((int64_t)1 << 31))
+    return fail(h, ENGRAM_ERR_INVALID, "too many rows for one call (rows x tables x row chunks >= 2^31)");
   return ENGRAM_OK;
 }
 
@@ -135,6 +135,7 @@ HashArgs hash_args(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T
   a.map = h->d_map;
   a.mult = h->d_mult;
   a.primes = h->d_primes;
+  a.barrett = h->d_barrett;
   a.idx = idx;
   a.err = h->d_err;
   a.V = h->cfg.vocab;
@@ -289,6 +290,10 @@ int engram_create(const engram_config* cfg, engram_handle** out) {
                           cudaMemcpyHostToDevice));
          CK(h, cudaMalloc(&h->d_primes, S * sizeof(int64_t)));
          CK(h, cudaMemcpy(h->d_primes, h->primes, S * sizeof(int64_t), cudaMemcpyHostToDevice));
+         uint64_t barrett[ENGRAM_MAX_TABLES];
+         for (int i = 0; i < S; ++i) barrett[i] = ~0ull / (uint64_t)h->primes[i];
+         CK(h, cudaMalloc(&h->d_barrett, S * sizeof(uint64_t)));
+         CK(h, cudaMemcpy(h->d_barrett, barrett, S * sizeof(uint64_t), cudaMemcpyHostToDevice));
          CK(h, cudaMalloc(&h->d_mult, (size_t)S * h->max_order * sizeof(uint64_t)));
          CK(h, cudaMemcpy(h->d_mult, h->mult, (size_t)S * h->max_order * sizeof(uint64_t),
                           cudaMemcpyHostToDevice));
@@ -315,11 +320,11 @@ void engram_destroy(engram_handle* h) {
   cudaDeviceSynchronize();
   free_dev(h->d_map);
   free_dev(h->d_primes);
+  free_dev(h->d_barrett);
   free_dev(h->d_mult);
   free_dev(h->d_err);
   free_dev(h->d_tables);
   free_dev(h->d_wqk);
-  free_dev(h->z);
   free_dev(h->e);
   free_dev(h->partials);
   free_dev(h->d_keys);
@@ -424,6 +429,8 @@ int engram_gather(engram_handle* h, const int64_t* idx, int64_t rows, void* e, v
     return fail(h, ENGRAM_ERR_UNSUPPORTED, "engram_gather reads device-resident tables only");
   if (rows < 0) return fail(h, ENGRAM_ERR_INVALID, "rows < 0");
   if (rows == 0) return ENGRAM_OK;
+  if (rows * h->S * ((h->cfg.d_head * h->elt) >> 4) >= ((int64_t)1 << 31))
+    return fail(h, ENGRAM_ERR_INVALID, "too many rows for one call");
   if (!idx || !e || !aligned16(e)) return fail(h, ENGRAM_ERR_INVALID, "null or misaligned buffer");
   GatherArgs g{};
   g.tables = h->d_tables;
@@ -545,17 +552,24 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     ga.primes = h->d_stage_bound;
     ga.idx = h->d_remap[slot];
   } else {
-    if (!idx) {
-      CK(h, launch_hash(hash_args(h, tokens, B, T, t_begin, h->z), st));
-      h->launches += 1;
-      idx = h->z;
-    }
     ga.tables = h->d_tables;
     ga.primes = h->d_primes;
     ga.idx = idx;
   }
-  CK(h, mark(1));
-  CK(h, launch_gather(ga, st));
+  if (!host_tables && !idx) {
+    // indices computed and consumed on chip: one kernel for steps 1-4 (the
+    // hash stage of a profiled forward is then empty)
+    HashGatherArgs hg{};
+    hg.hash = hash_args(h, tokens, B, T, t_begin, nullptr);
+    hg.tables = h->d_tables;
+    hg.e = h->e;
+    hg.row_bytes = ga.row_bytes;
+    CK(h, mark(1));
+    CK(h, launch_hash_gather(hg, st));
+  } else {
+    CK(h, mark(1));
+    CK(h, launch_gather(ga, st));
+  }
   h->launches += 1;
   CK(h, mark(2));
   if (host_tables) {

@@ -19,6 +19,7 @@ struct engram_handle {
   // device copies of the configuration
   int32_t* d_map = nullptr;
   int64_t* d_primes = nullptr;
+  uint64_t* d_barrett = nullptr;  // floor((2^64 - 1) / p) per table, for x mod p
   uint64_t* d_mult = nullptr;
   unsigned* d_err = nullptr;
 
@@ -33,7 +34,6 @@ struct engram_handle {
 
   // scratch, sized for cap_rows emitted positions
   int64_t cap_rows = 0;
-  int64_t* z = nullptr;
   void* e = nullptr;
   float4* partials = nullptr;
 

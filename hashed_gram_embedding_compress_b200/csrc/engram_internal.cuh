@@ -23,6 +23,7 @@ struct HashArgs {
   const int32_t* map;      // [V] compression map
   const uint64_t* mult;    // [S, max_order] odd multipliers
   const int64_t* primes;   // [S]
+  const uint64_t* barrett; // [S] floor((2^64 - 1) / primes[s])
   int64_t* idx;            // [B*(T-t_begin), S]
   unsigned* err;
   int32_t V, pad, B, T, t_begin, S, heads, num_orders, max_order;
@@ -38,6 +39,14 @@ struct GatherArgs {
   unsigned* err;
   int64_t rows;
   int32_t S;
+  int32_t row_bytes;          // d_head * element size, a multiple of 16
+};
+
+// Hash and gather in one pass (Eq. 1 then Eq. 2), for device-resident tables.
+struct HashGatherArgs {
+  HashArgs hash;              // idx is unused: the indices stay on chip
+  const void* const* tables;  // device array [S] of table base pointers
+  void* e;                    // [rows, S*d_head]
   int32_t row_bytes;          // d_head * element size, a multiple of 16
 };
 
@@ -77,6 +86,7 @@ struct PrefetchArgs {
 // Launchers (all asynchronous on `stream`; return the launch error).
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
+cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream);
 cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t stream);
 cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);

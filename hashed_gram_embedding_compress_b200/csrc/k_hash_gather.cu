@@ -19,7 +19,8 @@ constexpr int kHashThreads = 256;
 // thread hit L1/L2 (the map is at most 512 KB).
 // x mod p for a 64-bit x and 2 <= p < 2^31, by Barrett reduction (P. Barrett,
 // "Implementing the RSA public key encryption algorithm on a standard digital
-// signal processor", CRYPTO 1986): with inv = floor((2^64 - 1) / p), the
+// signal processor", CRYPTO 1986): with inv = floor((2^64 - 1) / p) (computed
+// once on the host when the tables are set), the
 // quotient estimate q = floor(x * inv / 2^64) is floor(x / p) or one less, so
 // x - q p lies in [0, 2p) and one conditional subtraction gives the exact
 // remainder.
@@ -28,6 +29,35 @@ __device__ __forceinline__ uint64_t mod_barrett(uint64_t x, uint64_t p, uint64_t
   uint64_t r = x - q * p;
   if (r >= p) r -= p;
   return r;
+}
+
+// phi_{n,k} of the n-gram ending at position t of one sequence, for table
+// slot s: all token loads are issued before the map lookups, and all map
+// lookups before the products, so a thread waits on two memory round trips.
+__device__ __forceinline__ uint64_t hash_slot(const HashArgs& a, const int32_t* seq, int t, int n,
+                                              const uint64_t* mult, uint64_t p, uint64_t inv) {
+  int32_t tok[kMaxOrders];
+#pragma unroll
+  for (int j = 0; j < kMaxOrders; ++j)
+    tok[j] = (j < n && t - j >= 0) ? __ldg(seq + t - j) : 0;
+  uint32_t c[kMaxOrders];
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < kMaxOrders; ++j) {
+    c[j] = (uint32_t)a.pad;  // positions before the sequence start
+    if (j < n && t - j >= 0) {
+      if (tok[j] >= 0 && tok[j] < a.V)
+        c[j] = (uint32_t)__ldg(a.map + tok[j]);
+      else
+        bad = true;
+    }
+  }
+  if (bad) atomicOr(a.err, kDevErrToken);
+  uint64_t x = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxOrders; ++j)
+    if (j < n) x ^= (uint64_t)c[j] * mult[j];
+  return mod_barrett(x, p, inv);
 }
 
 __global__ void __launch_bounds__(kHashThreads) hash_kernel(HashArgs a) {
@@ -40,36 +70,22 @@ __global__ void __launch_bounds__(kHashThreads) hash_kernel(HashArgs a) {
   for (int i = threadIdx.x; i < S; i += blockDim.x) {
     const uint64_t p = (uint64_t)a.primes[i];
     s_prime[i] = p;
-    s_inv[i] = 0xFFFFFFFFFFFFFFFFull / p;
+    s_inv[i] = a.barrett[i];
     s_order_of_slot[i] = a.orders[i / a.heads];
   }
   __syncthreads();
 
-  const int Tout = a.T - a.t_begin;
-  const int64_t total = (int64_t)a.B * Tout * S;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / S;
-    const int s = (int)(i - row * S);
+  // 32-bit index arithmetic (the launcher keeps B * (T - t_begin) * S < 2^31):
+  // 64-bit division is a long software sequence on the GPU
+  const uint32_t Tout = (uint32_t)(a.T - a.t_begin);
+  const uint32_t total = (uint32_t)a.B * Tout * (uint32_t)S;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t row = i / (uint32_t)S;
+    const int s = (int)(i - row * (uint32_t)S);
     const int b = (int)(row / Tout);
-    const int t = a.t_begin + (int)(row - (int64_t)b * Tout);
-    const int n = s_order_of_slot[s];
-    const int32_t* seq = a.tokens + (int64_t)b * a.T;
-    uint64_t x = 0;
-    for (int j = 0; j < n; ++j) {
-      const int pos = t - j;
-      uint32_t c = (uint32_t)a.pad;
-      if (pos >= 0) {
-        const int32_t tok = __ldg(seq + pos);
-        if (tok >= 0 && tok < a.V) {
-          c = (uint32_t)__ldg(a.map + tok);
-        } else {
-          atomicOr(a.err, kDevErrToken);
-        }
-      }
-      x ^= (uint64_t)c * s_mult[s * a.max_order + j];
-    }
-    a.idx[i] = (int64_t)mod_barrett(x, s_prime[s], s_inv[s]);
+    const int t = a.t_begin + (int)(row - (uint32_t)b * Tout);
+    a.idx[i] = (int64_t)hash_slot(a, a.tokens + (int64_t)b * a.T, t, s_order_of_slot[s],
+                                  s_mult + s * a.max_order, s_prime[s], s_inv[s]);
   }
 }
 
@@ -94,14 +110,15 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
     s_prime[i] = a.primes[i];
   }
   __syncthreads();
-  const int cpr = a.row_bytes >> 4;  // chunks per table row
-  const int64_t total = a.rows * a.S * cpr;
+  const uint32_t cpr = (uint32_t)(a.row_bytes >> 4);  // chunks per table row
+  const uint32_t S = (uint32_t)a.S;
+  // 32-bit index arithmetic (the launcher keeps rows * S * cpr < 2^31)
+  const uint32_t total = (uint32_t)a.rows * S * cpr;
   char* e = (char*)a.e;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t rs = i / cpr;
-    const int c = (int)(i - rs * cpr);
-    const int s = (int)(rs % a.S);
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t rs = i / cpr;
+    const uint32_t c = i - rs * cpr;
+    const uint32_t s = rs % S;
     const int64_t z = __ldg(a.idx + rs);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (z >= 0 && z < s_prime[s]) {
@@ -109,7 +126,74 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
     } else if (c == 0) {
       atomicOr(a.err, kDevErrIndex);
     }
-    *reinterpret_cast<uint4*>(e + rs * a.row_bytes + c * 16) = v;
+    *reinterpret_cast<uint4*>(e + (int64_t)rs * a.row_bytes + c * 16) = v;
+  }
+}
+
+// Hash and gather fused: a block owns 256 / S consecutive output rows.  Its
+// threads first compute the rows' S indices each (one per thread, as in
+// hash_kernel) and keep the source row addresses in shared memory; then they
+// copy the rows' table rows into e, 16 bytes per thread and load, four loads
+// in flight per thread.  The block's part of e is one contiguous run, so the
+// stores are coalesced, and the indices never travel through HBM.
+constexpr int kFusedThreads = 256;
+
+__global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherArgs g) {
+  const HashArgs& a = g.hash;
+  __shared__ uint64_t s_mult[kMaxTables * kMaxOrders];
+  __shared__ uint64_t s_prime[kMaxTables];
+  __shared__ uint64_t s_inv[kMaxTables];
+  __shared__ int32_t s_order_of_slot[kMaxTables];
+  __shared__ const char* s_tab[kMaxTables];
+  __shared__ const char* s_src[kFusedThreads];  // source row of (row, slot)
+  const int S = a.S;
+  for (int i = threadIdx.x; i < S * a.max_order; i += blockDim.x) s_mult[i] = a.mult[i];
+  for (int i = threadIdx.x; i < S; i += blockDim.x) {
+    s_prime[i] = (uint64_t)a.primes[i];
+    s_inv[i] = a.barrett[i];
+    s_order_of_slot[i] = a.orders[i / a.heads];
+    s_tab[i] = (const char*)g.tables[i];
+  }
+  __syncthreads();
+
+  const uint32_t Tout = (uint32_t)(a.T - a.t_begin);
+  const uint32_t rows = (uint32_t)a.B * Tout;
+  const uint32_t rb = kFusedThreads / (uint32_t)S;  // rows per block
+  const uint32_t row0 = blockIdx.x * rb;
+  const uint32_t nrows = min(rb, rows - row0);
+  const uint32_t nslots = nrows * (uint32_t)S;
+  if (threadIdx.x < nslots) {
+    const uint32_t rl = threadIdx.x / (uint32_t)S;
+    const int s = (int)(threadIdx.x - rl * (uint32_t)S);
+    const uint32_t row = row0 + rl;
+    const int b = (int)(row / Tout);
+    const int t = a.t_begin + (int)(row - (uint32_t)b * Tout);
+    const uint64_t z = hash_slot(a, a.tokens + (int64_t)b * a.T, t, s_order_of_slot[s],
+                                 s_mult + s * a.max_order, s_prime[s], s_inv[s]);
+    s_src[threadIdx.x] = s_tab[s] + z * (uint64_t)g.row_bytes;
+  }
+  __syncthreads();
+
+  const uint32_t cpr = (uint32_t)(g.row_bytes >> 4);
+  const uint32_t nchunks = nslots * cpr;
+  // row0 * S * row_bytes < 2^31 * 16 by the launcher's bound
+  uint4* dst = reinterpret_cast<uint4*>((char*)g.e + (int64_t)row0 * S * g.row_bytes);
+  constexpr int kInFlight = 4;
+  for (uint32_t i0 = threadIdx.x; i0 < nchunks; i0 += kInFlight * kFusedThreads) {
+    uint4 v[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const uint32_t i = i0 + k * kFusedThreads;
+      if (i < nchunks) {
+        const uint32_t rs = i / cpr;
+        v[k] = ld_stream_16(s_src[rs] + (i - rs * cpr) * 16);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const uint32_t i = i0 + k * kFusedThreads;
+      if (i < nchunks) dst[i] = v[k];
+    }
   }
 }
 
@@ -134,6 +218,7 @@ int grid_for(int64_t work, int threads) {
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream) {
   const int64_t total = (int64_t)a.B * (a.T - a.t_begin) * a.S;
   if (total == 0) return cudaSuccess;
+  if (total >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
   hash_kernel<<<grid_for(total, kHashThreads), kHashThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
@@ -141,7 +226,18 @@ cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream) {
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream) {
   const int64_t total = a.rows * a.S * (a.row_bytes >> 4);
   if (total == 0) return cudaSuccess;
+  if (total >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
   gather_kernel<<<grid_for(total, kGatherThreads), kGatherThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream) {
+  const int64_t rows = (int64_t)a.hash.B * (a.hash.T - a.hash.t_begin);
+  if (rows == 0) return cudaSuccess;
+  if (a.hash.S < 1 || a.hash.S > kMaxTables) return cudaErrorInvalidValue;
+  if (rows * a.hash.S * (a.row_bytes >> 4) >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+  const int64_t rb = kFusedThreads / a.hash.S;
+  hash_gather_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

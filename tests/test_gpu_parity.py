@@ -126,6 +126,26 @@ def check_in_place(p: Problem, m, out, delta):
     assert out_close(to_oracle(h2[torch.from_numpy(rows).cuda()]), o_ref, "bf16") <= BF16_REL
 
 
+@pytest.mark.parametrize("shape", [
+    synth.SHAPES["tiny_f32"],                                            # S = 8: 32 rows per block
+    synth.SHAPES["decode_mb"],                                           # blocks span sequences
+    synth.SHAPES["tiny_f32"].replace(orders=(2, 3, 4), heads=5, T=37),    # S = 15: 17 rows per block
+    synth.SHAPES["prefill_bf16"].replace(B=3, T=171, heads=3, rows_target=4099, d_hidden=256),
+])
+def test_fused_hash_gather_matches_separate_kernels(shape):
+    # forward from tokens computes the indices on chip (one hash + gather
+    # kernel); from caller-supplied indices it runs the gather kernel alone.
+    # Equal memory vectors give bit-identical outputs.
+    p = Problem(shape)
+    m = p.engram()
+    idx = check_indices(p, m)
+    out1, a1, d1 = run_forward(p, m)
+    out2, a2, d2 = run_forward(p, m, idx=idx)
+    assert torch.equal(out1, out2) and torch.equal(a1, a2) and torch.equal(d1, d2)
+    rows = np.arange(min(shape.rows_out, 64))
+    check_rows(p, m, idx, rows, out1, a1, d1)
+
+
 def test_decode_multibranch():
     p = Problem(synth.SHAPES["decode_mb"])
     m = p.engram()
