@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // for the next tile's MMAs (the leader owns the barrier)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+            if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
           }
           if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tc_fence_before();  // last TMEM read done: release the accumulators
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+            if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
           }
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tc_fence_before();  // last TMEM read done: release the accumulators
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(peer_addr(tempty_bar, 0));
+            if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
           }
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
