@@ -94,15 +94,6 @@ int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, i
 
 int bn_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
 
-// Widest tile (fewest B re-reads) that still gives every SM a tile; else 64.
-int choose_bn(int64_t R, int n_total, int sms) {
-  const int64_t mblk = (R + 127) / 128;
-  for (int bn : {256, 128}) {
-    if (n_total % bn == 0 && mblk * (n_total / bn) >= sms) return bn;
-  }
-  return 64;
-}
-
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 int ensure_scratch(engram_handle* h, int64_t rows) {
@@ -601,30 +592,27 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     h->launches += 2;
     return ENGRAM_OK;
   }
-  // Tensor maps are built for whichever kernel each phase uses: 512 x 256
-  // tiles on CTA pairs when the tile count fills every pair at least once,
-  // else single-CTA 128-row tiles of the widest N that fills the SMs.
+  // Tensor maps are built for whichever kernel each phase uses (choose_proj):
+  // 512 x 256 tiles on CTA pairs when the tile count fills every pair at least
+  // once, else single-CTA 128-row tiles of the widest N that fills the SMs.
   const int64_t hcols = (int64_t)g.M * g.d;
-  const bool pairs_ok = !(h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS);
   ProjMaps single, wide;
   bool have_single = false, have_wide = false;
   for (int phase = 0; phase < 2; ++phase) {
-    const int n_total = phase == 0 ? g.M * g.d : g.d;
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
-    const int64_t wtiles = (R + 511) / 512 * (n_total / 256);
-    if (pairs_ok && n_total % 256 == 0 && wtiles >= h->sms / 2) {
+    const ProjChoice pc = choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags);
+    if (phase == 0) g.key_tile = pc.key_tile;
+    // in place (out aliases h): the value phase adds alpha v into out
+    const int kphase = (phase == 1 && out == hid) ? 2 : phase;
+    if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
         if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
-        if ((rc = make_map(h, &wide.out, out, hcols, R, 32, 32))) return rc;  // per-warp stores
+        if ((rc = make_map(h, &wide.out, out, hcols, R, 32, 32))) return rc;
         have_wide = true;
       }
-      wide.w = wmaps[bn_index(128)];  // each CTA of a pair loads 128 of the tile's 256 W rows
-      if (phase == 0) g.key_tile = 256;
-      const int pairs = (int)(wtiles < h->sms / 2 ? wtiles : h->sms / 2);
-      // in place (out aliases h): the value phase adds alpha v into out
-      const int kphase = (phase == 1 && out == hid) ? 2 : phase;
-      CK(h, launch_proj_gate_wide(kphase, wide, g, 2 * pairs, st));
+      wide.w = wmaps[bn_index(pc.bn)];
+      CK(h, launch_proj_gate_wide(kphase, wide, g, pc.grid, st));
     } else {
       if (!have_single) {
         if ((rc = make_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;
@@ -632,12 +620,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
         if ((rc = make_map(h, &single.out, out, hcols, R, 128))) return rc;
         have_single = true;
       }
-      const int bn = choose_bn(R, n_total, h->sms);
-      const int64_t tiles = (R + 127) / 128 * (n_total / bn);
-      single.w = wmaps[bn_index(bn)];
-      if (phase == 0) g.key_tile = bn;
-      CK(h, launch_proj_gate_sm100(phase, bn, single, g, (int)(tiles < h->sms ? tiles : h->sms),
-                                   st));
+      single.w = wmaps[bn_index(pc.bn)];
+      CK(h, launch_proj_gate_sm100(phase, pc.bn, single, g, pc.grid, st));
     }
     CK(h, mark(3 + phase));
   }

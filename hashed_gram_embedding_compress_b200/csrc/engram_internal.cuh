@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/engram.h"
+
 namespace engram {
 
 // Bits of the handle's device error word.
@@ -113,5 +115,33 @@ cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, cons
 // phase 0 keys, 1 values, 2 values added in place (out aliases h).
 cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
                                   cudaStream_t stream);
+
+// The bf16 projection kernel of one phase (0 keys, 1 values) for R rows.
+enum class ProjKernel { Wide, Single };
+struct ProjChoice {
+  ProjKernel kind;
+  int bn;        // W rows per TMA box (the tensor map of W to use)
+  int grid;      // CTAs
+  int key_tile;  // columns per partial-sum tile (phase 0)
+};
+// 512 x 256 CTA-pair tiles whenever there are enough of them for every pair,
+// else single-CTA 128-row tiles of the widest N that still gives every SM a
+// tile.  Key tiles must not straddle branches, so their width divides d.
+inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int flags) {
+  const int n_total = phase == 0 ? M * d : d;
+  const int pairs = sms / 2;
+  if (!(flags & ENGRAM_FLAG_NO_CTA_PAIRS) && n_total % 256 == 0 && d % 256 == 0 &&
+      (R + 511) / 512 * (n_total / 256) >= pairs)
+    return {ProjKernel::Wide, 128, 2 * pairs, 256};
+  const int64_t mblk = (R + 127) / 128;
+  int bn = 64;
+  for (int c : {256, 128})
+    if (n_total % c == 0 && d % c == 0 && mblk * (n_total / c) >= sms) {
+      bn = c;
+      break;
+    }
+  const int64_t tiles = mblk * (n_total / bn);
+  return {ProjKernel::Single, bn, (int)(tiles < sms ? tiles : sms), bn};
+}
 
 }  // namespace engram

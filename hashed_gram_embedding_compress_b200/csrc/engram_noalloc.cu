@@ -144,17 +144,16 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
     h->launches += 2;
     return ENGRAM_OK;
   }
-  // the same kernel choice as engram_forward: 512 x 256 CTA-pair tiles when
-  // they fill every pair, else single-CTA 128-row tiles
+  // the same kernel choice as engram_forward (choose_proj)
   const int64_t hcols = (int64_t)M * d;
-  const bool pairs_ok = !(h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS);
   ProjMaps single, wide;
   bool have_single = false, have_wide = false;
   for (int phase = 0; phase < 2; ++phase) {
-    const int n_total = phase == 0 ? M * d : d;
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
-    const int64_t wtiles = (rows + 511) / 512 * (n_total / 256);
-    if (pairs_ok && n_total % 256 == 0 && wtiles >= h->sms / 2) {
+    const ProjChoice pc = choose_proj(phase, rows, M, d, h->sms, h->cfg.flags);
+    if (phase == 0) g.key_tile = pc.key_tile;
+    const int kphase = (phase == 1 && out == hid) ? 2 : phase;
+    if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if ((rc = encode_map(h, &wide.e, e, h->d_mem, R, 256, 64)) ||
             (rc = encode_map(h, &wide.h, hid, hcols, R, 256, 32)) ||
@@ -162,11 +161,8 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
           return rc;
         have_wide = true;
       }
-      wide.w = wmaps[map_slot(128)];
-      if (phase == 0) g.key_tile = 256;
-      const int pairs = (int)(wtiles < h->sms / 2 ? wtiles : h->sms / 2);
-      const int kphase = (phase == 1 && out == hid) ? 2 : phase;
-      if ((ce = launch_proj_gate_wide(kphase, wide, g, 2 * pairs, st)))
+      wide.w = wmaps[map_slot(pc.bn)];
+      if ((ce = launch_proj_gate_wide(kphase, wide, g, pc.grid, st)))
         return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
     } else {
       if (!have_single) {
@@ -176,18 +172,8 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
           return rc;
         have_single = true;
       }
-      const int64_t mblk = (rows + 127) / 128;
-      int bn = 64;
-      for (int c : {256, 128})
-        if (n_total % c == 0 && mblk * (n_total / c) >= h->sms) {
-          bn = c;
-          break;
-        }
-      const int64_t tiles = mblk * (n_total / bn);
-      single.w = wmaps[map_slot(bn)];
-      if (phase == 0) g.key_tile = bn;
-      if ((ce = launch_proj_gate_sm100(phase, bn, single, g,
-                                       (int)(tiles < h->sms ? tiles : h->sms), st)))
+      single.w = wmaps[map_slot(pc.bn)];
+      if ((ce = launch_proj_gate_sm100(phase, pc.bn, single, g, pc.grid, st)))
         return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
     }
   }

@@ -111,7 +111,8 @@ typedef struct engram_handle engram_handle;
  *  table_location  ENGRAM_DEVICE or ENGRAM_PINNED_HOST.
  *  flags           0, or ENGRAM_FLAG_NO_CTA_PAIRS to keep the bf16 projection
  *                  on single-CTA 128-row tiles (by default 512 x 256 tiles on
- *                  CTA pairs are used when they fill the GPU).
+ *                  CTA pairs are used when they fill the GPU).  Both give the
+ *                  same results up to fp32 summation order.
  */
 typedef struct engram_config {
   int32_t vocab;

@@ -169,6 +169,20 @@ def test_tile_widths_and_ragged_rows(R_B, R_T, flags):
     check_rows(p, m, idx, p.sample_rows(64), out, a, dl)
 
 
+@pytest.mark.parametrize("flags", [0, 1])
+def test_key_tiles_do_not_straddle_branches(flags):
+    # d = 384, M = 2: the key phase spans M d = 768 columns, a multiple of 256,
+    # but 256-column partial-sum tiles would straddle the two branches; every
+    # kernel choice must use key tiles whose width divides d
+    sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=9000, rows_target=2053, d_hidden=384,
+                                              branches=2)
+    p = Problem(sh)
+    m = p.engram(flags=flags)
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, p.sample_rows(64), out, a, dl)
+
+
 def test_hidden_not_multiple_of_128_and_three_branches():
     sh = synth.SHAPES["decode_mb"].replace(B=37, T=9, t_begin=4, rows_target=1031, d_hidden=192,
                                            branches=3)
