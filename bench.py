@@ -73,11 +73,16 @@ def parse():
 
 
 def load_peaks():
+    """HBM GB/s and the dense bf16 TFLOP/s of this GPU.  The projection
+    kernels are timed inside seconds of back-to-back steps under the power
+    cap, so the sustained GEMM figure is their denominator (the burst figure
+    is reported beside it)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d["hbm_gbs"], d["bf16_tflops"], "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (d["hbm_gbs"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), d["bf16_tflops"],
+                "measured" if "bf16_tflops_sustained" in d else "measured burst")
+    return 6650.0, 1400.0, 1590.0, "fallback"
 
 
 # ------------------------------------------------------------------ clocks
@@ -339,7 +344,7 @@ def run_ours(args, rank, world, dist):
     if rank != 0:
         return None
 
-    hbm, tflops, peak_kind = load_peaks()
+    hbm, tflops, tflops_burst, peak_kind = load_peaks()
     A = algorithmic(sh)
     tokens_per_step = sh.rows_out
     value = tokens_per_step * world * K / (ms / 1e3)
@@ -380,7 +385,9 @@ def run_ours(args, rank, world, dist):
             "unit": "TFLOP/s",
             "frac": gemm_tflops / tflops,
             "traffic": traffic,
-            "peak_source": "%s bf16 burst" % peak_kind,
+            "peak_source": "%s bf16 sustained (cuBLAS back to back under the power cap)" % peak_kind
+                           if peak_kind == "measured" else peak_kind,
+            "frac_of_burst": gemm_tflops / tflops_burst,
         },
         "gather": {
             "kernel": "hash_gather_kernel" if fused else "gather_kernel",

@@ -36,7 +36,7 @@ import torch
 BASE_SEED = 20261202
 
 #: names of the independent sub-streams of one problem
-STREAMS = ("tokens", "map", "hash", "tables", "weights", "hidden", "norms")
+STREAMS = ("tokens", "map", "hash", "tables", "weights", "hidden", "norms", "conv")
 
 
 @dataclass(frozen=True)
@@ -178,6 +178,19 @@ def make_weights(shape: EngramShape, seeds: dict):
     norm_q = 1.0 + 0.1 * torch.randn((M, d), generator=gn)
     norm_k = 1.0 + 0.1 * torch.randn((M, d), generator=gn)
     return w_k, w_v, norm_q.float(), norm_k.float()
+
+
+def make_conv_weights(shape: EngramShape, seeds: dict, kernel_size: int = 4):
+    """ShortConv weights (Eq. 5): conv_w [d, W] (tap i multiplies position
+    t - i * dilation) with N(0, 0.5^2) entries, so the conv output is O(1) and
+    SiLU is exercised on both sides of zero (the paper initialises them to
+    zero, which makes the conv the identity); norm_w [d] = 1 + 0.1 N(0, 1).
+    Both fp32."""
+    g = _gen(seeds["conv"])
+    d = shape.d_hidden
+    conv_w = 0.5 * torch.randn((d, kernel_size), generator=g)
+    norm_w = 1.0 + 0.1 * torch.randn((d,), generator=g)
+    return conv_w.float(), norm_w.float()
 
 
 def make_hidden(shape: EngramShape, seeds: dict, device="cpu", rows: Optional[int] = None,

@@ -65,6 +65,12 @@ def lib():
         L.eo_project_gate.argtypes = [P, i32, i64, i32, P, P, P, P, i32, i32, f64, P,
                                       P, P, P, P, P, P]
         L.eo_project_gate.restype = None
+        L.eo_short_conv_at.argtypes = [P, P, i32, i32, P, P, f64, P, P]
+        L.eo_short_conv_at.restype = None
+        L.eo_short_conv.argtypes = [P, i32, i32, P, i32, i32, P, f64, P, P, P, P]
+        L.eo_short_conv.restype = None
+        L.eo_add_round.argtypes = [P, i32, i64, P, P]
+        L.eo_add_round.restype = None
         _lib = L
     return _lib
 
@@ -192,6 +198,54 @@ def project_gate(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: bool = 
                           _p(h), _p(alpha), _p(delta) if delta is not None else None, _p(out),
                           _p(kb), _p(vb), _p(hb))
     return alpha, delta, out
+
+
+# ---------------------------------------------------------------- short conv
+
+def short_conv(vt: np.ndarray, conv_w: np.ndarray, norm_w: np.ndarray, dil: int,
+               eps: float) -> np.ndarray:
+    """Y = SiLU(Conv1D(RMSNorm(V~))) + V~ over one sequence (Eq. 5).
+
+    vt [n_pos, d] gated values of one branch; conv_w [d, W] (tap i multiplies
+    position t - i*dil); norm_w [d].  Returns Y [n_pos, d] in double."""
+    vt = np.ascontiguousarray(vt, dtype=np.float64)
+    n_pos, d = vt.shape
+    cw = np.ascontiguousarray(conv_w, dtype=np.float32)
+    nw = np.ascontiguousarray(norm_w, dtype=np.float32)
+    W = cw.shape[1]
+    assert cw.shape == (d, W) and nw.shape == (d,)
+    y = np.empty_like(vt)
+    taps = np.empty(W * d, dtype=np.float64)
+    have = np.empty(W, dtype=np.int32)
+    norm = np.empty(d, dtype=np.float64)
+    lib().eo_short_conv(_p(vt), n_pos, d, _p(cw), W, dil, _p(nw), eps, _p(y), _p(taps),
+                        _p(have), _p(norm))
+    return y
+
+
+def short_conv_at(taps: np.ndarray, have: np.ndarray, conv_w: np.ndarray, norm_w: np.ndarray,
+                  eps: float) -> np.ndarray:
+    """Y at one position (Eq. 5) from V~ at positions t - i*dil (taps [W, d];
+    have[i] = 0 where the position precedes the sequence)."""
+    taps = np.ascontiguousarray(taps, dtype=np.float64)
+    W, d = taps.shape
+    have = np.ascontiguousarray(have, dtype=np.int32)
+    cw = np.ascontiguousarray(conv_w, dtype=np.float32)
+    nw = np.ascontiguousarray(norm_w, dtype=np.float32)
+    y = np.empty(d, dtype=np.float64)
+    norm = np.empty(d, dtype=np.float64)
+    lib().eo_short_conv_at(_p(taps), _p(have), W, d, _p(cw), _p(nw), eps, _p(y), _p(norm))
+    return y
+
+
+def add_round(h: np.ndarray, y: np.ndarray) -> np.ndarray:
+    """h + y rounded to h's dtype (fp32, or bf16 bits as uint16)."""
+    h = np.ascontiguousarray(h)
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    assert y.size == h.size
+    out = np.empty_like(h)
+    lib().eo_add_round(_p(h), F32 if h.dtype == np.float32 else BF16, h.size, _p(y), _p(out))
+    return out
 
 
 # ------------------------------------------------------------------ pipeline

@@ -40,6 +40,19 @@
  *    the projection (Eq. 4), the scale is 1/sqrt(d) with d the hidden size.
  *  - ShortConv (Eq. 5) is zero-initialised in the paper (Table 5), so at
  *    initialisation its output equals the gated value and out = h + alpha v.
+ *    With trained (non-zero) weights it is the last step below.
+ *
+ *   short conv Y = SiLU(Conv1D(RMSNorm(V~))) + V~,  H <- H + Y
+ *                                                     section 2.3, Eq. (5)
+ *
+ *  - Conv1D is depthwise and causal over the positions of one sequence, with
+ *    kernel size W and dilation delta (the paper sets W = 4 and delta to the
+ *    largest n-gram order): tap i of channel c multiplies channel c of the
+ *    normalised gated value at position t - i*delta; positions before the
+ *    sequence start contribute zero.  No bias.  RMSNorm has its own weight
+ *    per channel and the same epsilon as the gate.  In the multi-branch form
+ *    one set of conv and norm weights is applied to each branch's sequence
+ *    u^(m) = alpha^(m) v separately.
  *
  * Floating point: every sum is accumulated in double over the exact values of
  * the fp32 or bf16 inputs.  bf16 outputs are rounded to nearest-even
@@ -267,5 +280,65 @@ void eo_project_gate(const void *e, int32_t dtype, int64_t rows, int32_t d_mem,
                 else ((uint16_t *)out)[base + i] = eo_bf16_rne(o);
             }
         }
+    }
+}
+
+/* -------------------------------------------------------------- short conv */
+
+static double eo_silu(double x) { return x / (1.0 + exp(-x)); }
+
+/*
+ * Y at one position t of one sequence and branch (Eq. 5):
+ *   Y_t = SiLU( sum_i cw[c][i] * RMSNorm(V~_{t - i*dil})[c] ) + V~_t[c]
+ *   taps  [W][d] double: V~ at positions t, t - dil, ..., t - (W-1) dil
+ *   have  [W]    int:    0 where that position lies before the sequence start
+ *   cw    [d][W] float, nw [d] float (RMSNorm weight), y [d] double (out).
+ * Scratch: norm [d] doubles supplied by the caller.
+ */
+void eo_short_conv_at(const double *taps, const int32_t *have, int32_t W, int32_t d,
+                      const float *cw, const float *nw, double eps, double *y, double *norm)
+{
+    int32_t i, c;
+    for (c = 0; c < d; ++c) y[c] = 0.0;
+    for (i = 0; i < W; ++i) {
+        const double *x = taps + (int64_t)i * d;
+        double ss = 0.0, r;
+        if (!have[i]) continue;
+        for (c = 0; c < d; ++c) ss += x[c] * x[c];
+        r = 1.0 / sqrt(ss / d + eps);
+        for (c = 0; c < d; ++c) norm[c] = x[c] * r * (double)nw[c];
+        for (c = 0; c < d; ++c) y[c] += (double)cw[(int64_t)c * W + i] * norm[c];
+    }
+    for (c = 0; c < d; ++c) y[c] = eo_silu(y[c]) + taps[c];
+}
+
+/*
+ * Y for every position of one sequence and branch: vt [n_pos, d] double
+ * (V~ at positions 0 .. n_pos-1), y [n_pos, d] double (out).
+ * Scratch: taps [W * d], norm [d] doubles, have [W] ints.
+ */
+void eo_short_conv(const double *vt, int32_t n_pos, int32_t d, const float *cw, int32_t W,
+                   int32_t dil, const float *nw, double eps, double *y,
+                   double *taps, int32_t *have, double *norm)
+{
+    int32_t t, i, c;
+    for (t = 0; t < n_pos; ++t) {
+        for (i = 0; i < W; ++i) {
+            const int32_t p = t - i * dil;
+            have[i] = p >= 0;
+            for (c = 0; c < d; ++c) taps[(int64_t)i * d + c] = p >= 0 ? vt[(int64_t)p * d + c] : 0.0;
+        }
+        eo_short_conv_at(taps, have, W, d, cw, nw, eps, y + (int64_t)t * d, norm);
+    }
+}
+
+/* out = h + Y rounded to the h dtype, for n values. */
+void eo_add_round(const void *h, int32_t dtype, int64_t n, const double *y, void *out)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i) {
+        double o = eo_load(h, dtype, i) + y[i];
+        if (dtype == EO_F32) ((float *)out)[i] = (float)o;
+        else ((uint16_t *)out)[i] = eo_bf16_rne(o);
     }
 }

@@ -254,3 +254,70 @@ def test_project_gate_shared_value_per_branch():
     alpha, delta, _ = oracle.project_gate(e, wk, wv, nq, nk, h, 1e-6)
     assert np.array_equal(alpha[:, 0], alpha[:, 1])
     assert np.array_equal(delta[:, 0], delta[:, 1])
+
+
+# ------------------------------------------------------------ ShortConv (Eq. 5)
+
+def _conv_case(seed, n_pos=41, d=24, W=4):
+    rng = np.random.default_rng(seed)
+    vt = rng.normal(size=(n_pos, d)) * rng.uniform(0.1, 3.0, size=(n_pos, 1))
+    cw = rng.normal(size=(d, W)).astype(np.float32)
+    nw = (1 + 0.1 * rng.normal(size=d)).astype(np.float32)
+    return vt, cw, nw
+
+
+@pytest.mark.parametrize("dil,W", [(3, 4), (2, 4), (1, 3), (4, 2)])
+def test_short_conv_matches_library_routines(dil, W):
+    # RMSNorm, a causal dilated depthwise conv1d and SiLU from torch, in fp64:
+    # torch's conv1d is a cross-correlation, so its kernel is the oracle's
+    # taps reversed, and left padding of (W-1) dil makes it causal
+    vt, cw, nw = _conv_case(dil * 10 + W, W=W)
+    eps = 1e-6
+    y = oracle.short_conv(vt, cw, nw, dil, eps)
+    x = torch.from_numpy(vt)
+    n = torch.nn.functional.rms_norm(x, (x.shape[1],), weight=torch.from_numpy(nw).double(), eps=eps)
+    k = torch.from_numpy(cw).double().flip(1).unsqueeze(1)           # [d, 1, W]
+    xin = torch.nn.functional.pad(n.T.unsqueeze(0), ((W - 1) * dil, 0))
+    conv = torch.nn.functional.conv1d(xin, k, groups=x.shape[1], dilation=dil)[0].T
+    ref = torch.nn.functional.silu(conv) + x
+    assert np.abs(y - ref.numpy()).max() < 1e-12
+
+
+def test_short_conv_zero_weights_is_identity():
+    # the paper's zero initialisation: SiLU(0) = 0, so Y = V~ exactly
+    vt, cw, nw = _conv_case(1)
+    y = oracle.short_conv(vt, np.zeros_like(cw), nw, 3, 1e-6)
+    assert np.array_equal(y, vt)
+
+
+def test_short_conv_causal_dilated_support():
+    # a change of V~ at position p moves Y exactly at p, p+dil, ..., p+(W-1)dil
+    vt, cw, nw = _conv_case(2, n_pos=40)
+    y0 = oracle.short_conv(vt, cw, nw, 3, 1e-6)
+    for p in (0, 5, 33):
+        v2 = vt.copy()
+        v2[p] *= 1.7
+        v2[p, 3] += 0.5
+        y1 = oracle.short_conv(v2, cw, nw, 3, 1e-6)
+        changed = set(np.nonzero(np.abs(y1 - y0).max(axis=1) > 0)[0].tolist())
+        assert changed == {q for q in (p, p + 3, p + 6, p + 9) if q < 40}
+
+
+def test_short_conv_at_equals_sequence_form():
+    vt, cw, nw = _conv_case(3)
+    y = oracle.short_conv(vt, cw, nw, 3, 1e-6)
+    for t in (0, 2, 3, 8, 9, 40):
+        taps = np.stack([vt[t - 3 * i] if t - 3 * i >= 0 else np.zeros(vt.shape[1]) for i in range(4)])
+        have = np.array([t - 3 * i >= 0 for i in range(4)], dtype=np.int32)
+        assert np.array_equal(oracle.short_conv_at(taps, have, cw, nw, 1e-6), y[t])
+
+
+def test_add_round_matches_torch_rounding():
+    rng = np.random.default_rng(4)
+    hb = torch.randn(4096, dtype=torch.float64).to(torch.bfloat16)
+    y = rng.normal(size=4096) * 0.01
+    out = oracle.add_round(hb.view(torch.int16).numpy().view(np.uint16), y)
+    ref = (hb.double() + torch.from_numpy(y)).float().to(torch.bfloat16)
+    assert np.array_equal(out, ref.view(torch.int16).numpy().view(np.uint16))
+    hf = rng.normal(size=100).astype(np.float32)
+    assert np.array_equal(oracle.add_round(hf, y[:100]), (hf.astype(np.float64) + y[:100]).astype(np.float32))
