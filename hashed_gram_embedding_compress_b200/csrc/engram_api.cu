@@ -108,6 +108,20 @@ int ensure_scratch(engram_handle* h, int64_t rows) {
   return ENGRAM_OK;
 }
 
+int ensure_conv_scratch(engram_handle* h, int64_t rows) {
+  if (rows <= h->conv_cap_rows) return ENGRAM_OK;
+  free_dev(h->conv_v);
+  free_dev(h->conv_vv);
+  free_dev(h->conv_alpha);
+  h->conv_cap_rows = 0;
+  const int d = h->cfg.d_hidden;
+  CK(h, cudaMalloc(&h->conv_v, (size_t)rows * d * sizeof(float)));
+  CK(h, cudaMalloc(&h->conv_vv, (size_t)rows * (d / 64) * sizeof(float)));
+  CK(h, cudaMalloc(&h->conv_alpha, (size_t)rows * h->cfg.branches * sizeof(float)));
+  h->conv_cap_rows = rows;
+  return ENGRAM_OK;
+}
+
 int check_shape(engram_handle* h, int32_t B, int32_t T, int32_t t_begin) {
   if (B < 0 || T < 0) return fail(h, ENGRAM_ERR_INVALID, "B and T must be >= 0");
   if (B > 0 && T > 0 && (t_begin < 0 || t_begin >= T))
@@ -318,6 +332,11 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->d_wqk);
   free_dev(h->e);
   free_dev(h->partials);
+  free_dev(h->d_conv_w);
+  free_dev(h->d_conv_nw);
+  free_dev(h->conv_v);
+  free_dev(h->conv_vv);
+  free_dev(h->conv_alpha);
   free_dev(h->d_keys);
   free_dev(h->d_vals);
   free_dev(h->d_uniq);
@@ -384,12 +403,43 @@ int engram_set_params(engram_handle* h, const void* const* tables, const void* w
   return ENGRAM_OK;
 }
 
+int engram_set_short_conv(engram_handle* h, const float* conv_w, const float* norm_w,
+                          int32_t kernel_size, int32_t dilation, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (kernel_size == 0) {
+    h->conv_W = 0;
+    return ENGRAM_OK;
+  }
+  if (kernel_size < 1 || kernel_size > 4)
+    return fail(h, ENGRAM_ERR_INVALID, "kernel_size must be 0 (off) or 1..4");
+  if (dilation < 1 || dilation > 4) return fail(h, ENGRAM_ERR_INVALID, "dilation must be 1..4");
+  if (!conv_w || !norm_w) return fail(h, ENGRAM_ERR_INVALID, "null conv_w or norm_w");
+  const int d = h->cfg.d_hidden;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!h->d_conv_w) {
+    CK(h, cudaMalloc(&h->d_conv_w, (size_t)d * 4 * sizeof(float)));
+    CK(h, cudaMalloc(&h->d_conv_nw, (size_t)d * sizeof(float)));
+  }
+  // [d][kernel_size] -> [d][4] with the unused taps zero
+  CK(h, cudaMemsetAsync(h->d_conv_w, 0, (size_t)d * 4 * sizeof(float), st));
+  CK(h, cudaMemcpy2DAsync(h->d_conv_w, 4 * sizeof(float), conv_w, kernel_size * sizeof(float),
+                          kernel_size * sizeof(float), d, cudaMemcpyDeviceToDevice, st));
+  CK(h, cudaMemcpyAsync(h->d_conv_nw, norm_w, (size_t)d * sizeof(float), cudaMemcpyDeviceToDevice,
+                        st));
+  CK(h, cudaStreamSynchronize(st));
+  h->conv_W = kernel_size;
+  h->conv_dil = dilation;
+  return ENGRAM_OK;
+}
+
 int engram_reserve(engram_handle* h, int64_t max_rows) {
   if (!h) return ENGRAM_ERR_INVALID;
   if (max_rows < 0 || max_rows > ((int64_t)1 << 31))
     return fail(h, ENGRAM_ERR_INVALID, "max_rows out of range");
   int rc = ensure_scratch(h, max_rows);
   if (rc) return rc;
+  if (h->conv_W > 0 && (rc = ensure_conv_scratch(h, max_rows))) return rc;
   if (h->cfg.table_location == ENGRAM_PINNED_HOST) return ensure_prefetch_scratch(h, max_rows);
   return ENGRAM_OK;
 }
@@ -526,8 +576,15 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   const bool prof = h->prof_armed;
   h->prof_armed = false;
   auto mark = [&](int i) -> cudaError_t {
-    return prof ? cudaEventRecord(h->prof[i], st) : cudaSuccess;
+    return prof && i < h->n_prof ? cudaEventRecord(h->prof[i], st) : cudaSuccess;
   };
+  // with the short convolution on: the value phase leaves v, its sums of
+  // squares and alpha, and one more kernel forms out = h + Y (Eq. 5)
+  const bool conv = h->conv_W > 0;
+  if (conv && t_begin != 0)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED,
+                "the short convolution needs every position of each sequence (t_begin = 0)");
+  if (conv && (rc = ensure_conv_scratch(h, R))) return rc;
   CK(h, mark(0));
 
   // steps 1-4: indices, then the gathered memory vectors e
@@ -583,13 +640,44 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   g.d_mem = h->d_mem;
   g.eps = h->cfg.eps;
   g.inv_sqrt_d = (float)(1.0 / std::sqrt((double)h->cfg.d_hidden));
+  if (conv) {
+    g.vals = h->conv_v;
+    g.vv = h->conv_vv;
+    if (!g.alpha) g.alpha = h->conv_alpha;
+  }
+  // step 7 with the short convolution (Eq. 5), after the value phase left v,
+  // its sums of squares per value tile and alpha
+  auto short_conv = [&](int value_tile) -> int {
+    ConvArgs ca{};
+    ca.vals = h->conv_v;
+    ca.vv = h->conv_vv;
+    ca.alpha = g.alpha;
+    ca.h = hid;
+    ca.out = out;
+    ca.delta = delta;
+    ca.conv_w = h->d_conv_w;
+    ca.norm_w = h->d_conv_nw;
+    ca.B = B;
+    ca.T = T;
+    ca.M = g.M;
+    ca.d = g.d;
+    ca.n_vtiles = g.d / value_tile;
+    ca.bf16 = h->cfg.dtype == ENGRAM_BF16;
+    ca.eps = g.eps;
+    CK(h, launch_short_conv(ca, h->conv_dil, st));
+    h->launches += 1;
+    CK(h, mark(5));
+    return ENGRAM_OK;
+  };
   if (h->cfg.dtype == ENGRAM_F32) {
     g.key_tile = kF32Tile;
     CK(h, launch_proj_gate_f32(0, (const float*)h->e, (const float*)h->w_k, g, st));
     CK(h, mark(3));
-    CK(h, launch_proj_gate_f32(1, (const float*)h->e, (const float*)h->w_v, g, st));
+    CK(h, launch_proj_gate_f32(conv ? 3 : 1, (const float*)h->e, (const float*)h->w_v, g, st));
     CK(h, mark(4));
     h->launches += 2;
+    if (conv) return short_conv(kF32Tile);
+    CK(h, mark(5));
     return ENGRAM_OK;
   }
   // Tensor maps are built for whichever kernel each phase uses (choose_proj):
@@ -598,12 +686,15 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   const int64_t hcols = (int64_t)g.M * g.d;
   ProjMaps single, wide;
   bool have_single = false, have_wide = false;
+  int value_tile = 0;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
     const ProjChoice pc = choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags);
     if (phase == 0) g.key_tile = pc.key_tile;
-    // in place (out aliases h): the value phase adds alpha v into out
-    const int kphase = (phase == 1 && out == hid) ? 2 : phase;
+    if (phase == 1) value_tile = pc.key_tile;
+    // values: 3 = v for the short convolution; 2 = in place (out aliases h,
+    // alpha v is added into out); 1 = out = h + alpha v
+    const int kphase = phase == 0 ? 0 : conv ? 3 : out == hid ? 2 : 1;
     if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
@@ -621,11 +712,13 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
         have_single = true;
       }
       single.w = wmaps[bn_index(pc.bn)];
-      CK(h, launch_proj_gate_sm100(phase, pc.bn, single, g, pc.grid, st));
+      CK(h, launch_proj_gate_sm100(kphase == 3 ? 3 : phase, pc.bn, single, g, pc.grid, st));
     }
     CK(h, mark(3 + phase));
   }
   h->launches += 2;
+  if (conv) return short_conv(value_tile);
+  CK(h, mark(5));
   return ENGRAM_OK;
 }
 
@@ -635,11 +728,12 @@ int engram_profile_next_forward(engram_handle* h, void* const* events, int32_t n
     h->prof_armed = false;
     return ENGRAM_OK;
   }
-  if (n_events != 5) return fail(h, ENGRAM_ERR_INVALID, "n_events must be 5");
-  for (int i = 0; i < 5; ++i) {
+  if (n_events != 5 && n_events != 6) return fail(h, ENGRAM_ERR_INVALID, "n_events must be 5 or 6");
+  for (int i = 0; i < n_events; ++i) {
     if (!events[i]) return fail(h, ENGRAM_ERR_INVALID, "null event");
     h->prof[i] = (cudaEvent_t)events[i];
   }
+  h->n_prof = n_events;
   h->prof_armed = true;
   return ENGRAM_OK;
 }

@@ -32,10 +32,20 @@ struct engram_handle {
   float* d_wqk = nullptr;           // norm_q * norm_k, [M, d]
   CUtensorMap map_wk[3], map_wv[3]; // box widths 64, 128, 256
 
+  // short convolution (Eq. 5): off while conv_W == 0
+  int conv_W = 0, conv_dil = 0;
+  float* d_conv_w = nullptr;   // [d][4], taps >= conv_W zero
+  float* d_conv_nw = nullptr;  // [d]
+
   // scratch, sized for cap_rows emitted positions
   int64_t cap_rows = 0;
   void* e = nullptr;
   float4* partials = nullptr;
+  // short-convolution scratch, sized for conv_cap_rows
+  int64_t conv_cap_rows = 0;
+  float* conv_v = nullptr;      // [rows, d] v = W_V e
+  float* conv_vv = nullptr;     // [d / 64][rows] sums of v^2 per value tile
+  float* conv_alpha = nullptr;  // [rows, M] when the caller passes none
 
   // host-resident tables: prefetch state, double-buffered
   int64_t pf_cap_rows = 0;
@@ -55,6 +65,7 @@ struct engram_handle {
 
   // instrumentation
   int64_t launches = 0;
-  cudaEvent_t prof[5] = {};
+  cudaEvent_t prof[6] = {};
+  int n_prof = 0;
   bool prof_armed = false;
 };

@@ -60,11 +60,27 @@ struct GateArgs {
   float4* partials;     // [num key tiles][R]: (sum k^2, sum h w_q w_k k, sum h^2, 0)
   float* alpha;         // [R, M] or null
   float* delta;         // [R, M, d] or null
+  float* vals;          // phase 3: v = W_V e, fp32 [R, d]
+  float* vv;            // phase 3: sum of v^2 per value tile and row, [d / value tile][R]
   unsigned* err;
   int32_t R, M, d, d_mem;
   int32_t key_tile;     // width of the key-phase tiles that wrote `partials`
   float eps;
   float inv_sqrt_d;
+};
+
+// Short convolution and residual (Eq. 5) over B sequences of T positions.
+struct ConvArgs {
+  const float* vals;    // [B*T, d] v = W_V e (fp32)
+  const float* vv;      // [n_vtiles][B*T] sums of v^2 per value tile
+  const float* alpha;   // [B*T, M]
+  const void* h;        // [B*T, M, d] fp32 or bf16
+  void* out;            // [B*T, M, d], may alias h
+  float* delta;         // [B*T, M, d] the increment Y, or null
+  const float* conv_w;  // [d][4]: tap i multiplies position t - i * dilation
+  const float* norm_w;  // [d]
+  int32_t B, T, M, d, n_vtiles, bf16;
+  float eps;
 };
 
 // Prefetch of host-resident rows into an HBM staging buffer (section 2.5).
@@ -89,6 +105,8 @@ struct PrefetchArgs {
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
 cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream);
+// dilation 1..4; the grid covers B * ceil(T / 64) position tiles.
+cudaError_t launch_short_conv(const ConvArgs& a, int dilation, cudaStream_t stream);
 cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t stream);
 cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);

@@ -100,6 +100,9 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
                                            void* stream) {
   if (!h) return ENGRAM_ERR_INVALID;
   if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (h->conv_W > 0)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED,
+                "engram_project_gate_noalloc: the short convolution needs scratch; use engram_forward");
   const int M = h->cfg.branches, d = h->cfg.d_hidden;
   const int64_t bytes_per_row = (int64_t)(M * d / 64) * (int64_t)sizeof(float4);
   const int64_t max_rows = (int64_t)kNoAllocScratchBytes / bytes_per_row;

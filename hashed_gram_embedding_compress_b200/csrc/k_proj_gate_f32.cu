@@ -10,7 +10,9 @@
 //            sums (sum k^2, sum h (w_q w_k) k, sum h^2) of the RMSNorm-ed dot;
 //   phase 1: value tiles v = e W_V^T; the epilogue finishes alpha from the
 //            partials of every key tile of the branch and writes
-//            out = h + alpha v (plus alpha and alpha v when requested).
+//            out = h + alpha v (plus alpha and alpha v when requested);
+//   phase 3: value tiles for the short convolution (Eq. 5): alpha, v and the
+//            per-row sum of v^2 of the tile; h is not read.
 #include "engram_internal.cuh"
 
 namespace engram {
@@ -87,6 +89,35 @@ __global__ void __launch_bounds__(256) proj_gate_f32_kernel(const float* __restr
       if (tx == 0 && row < R)
         g.partials[(int64_t)blockIdx.x * R + row] = make_float4(skk, shk, shh, 0.f);
     }
+  } else if (PHASE == 3) {
+    const int tiles_per_branch = d / g.key_tile;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = m0 + ty * 4 + i;
+      float svv = 0.f;
+      if (row < R) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) svv = fmaf(acc[i][j], acc[i][j], svv);
+        *reinterpret_cast<float4*>(g.vals + (int64_t)row * d + n0 + tx * 4) =
+            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        if (blockIdx.x == 0 && tx == 0)
+          for (int mb = 0; mb < M; ++mb) {
+            float skk = 0.f, shk = 0.f, shh = 0.f;
+            for (int tb = mb * tiles_per_branch; tb < (mb + 1) * tiles_per_branch; ++tb) {
+              const float4 p = g.partials[(int64_t)tb * R + row];
+              skk += p.x;
+              shk += p.y;
+              shh += p.z;
+            }
+            const float rh = 1.0f / sqrtf(shh / (float)d + g.eps);
+            const float rk = 1.0f / sqrtf(skk / (float)d + g.eps);
+            g.alpha[(int64_t)row * M + mb] = sigmoid_f(shk * rh * rk * g.inv_sqrt_d);
+          }
+      }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) svv += __shfl_xor_sync(0xffffffffu, svv, off);
+      if (tx == 0 && row < R) g.vv[(int64_t)blockIdx.x * R + row] = svv;
+    }
   } else {
     const int tiles_per_branch = d / g.key_tile;
     float* out = (float*)g.out;
@@ -127,6 +158,8 @@ cudaError_t launch_proj_gate_f32(int phase, const float* e, const float* w, cons
   dim3 grid(n_total / BN, (g.R + BM - 1) / BM);
   if (phase == 0)
     proj_gate_f32_kernel<0><<<grid, 256, 0, stream>>>(e, w, n_total, g);
+  else if (phase == 3)
+    proj_gate_f32_kernel<3><<<grid, 256, 0, stream>>>(e, w, n_total, g);
   else
     proj_gate_f32_kernel<1><<<grid, 256, 0, stream>>>(e, w, n_total, g);
   return cudaGetLastError();

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_kb = (g.d_mem + BK - 1) / BK;
   // h sub-tiles per output tile: the key phase reads one branch, the value
   // phase every branch (v is shared, Eq. 6)
-  const int nsub = (BN / 64) * (PHASE == 0 ? 1 : M);
+  const int nsub = PHASE == 3 ? 0 : (BN / 64) * (PHASE == 0 ? 1 : M);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = row < R;
       const int n0 = n_blk * BN;
       float al[kMaxBranches];
-      if (PHASE == 1) {
+      if (PHASE >= 1) {
         // alpha from the key phase's per-tile partial sums (Eq. 4 / Eq. 6)
 #pragma unroll
         for (int mb = 0; mb < kMaxBranches; ++mb) {
@@ -312,6 +312,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
+      } else if (PHASE == 3) {
+        // values for the short convolution (Eq. 5): v in fp32 and the row's
+        // sum of v^2 over this tile
+        float svv = 0.f;
+#pragma unroll 1
+        for (int q = 0; q < BN / 64; ++q) {
+          __syncwarp();
+          tmem_ld32(taddr + q * 64, v);
+          tmem_ld32(taddr + q * 64 + 32, v + 32);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) svv = fmaf(v[i], v[i], svv);
+          if (valid) {
+            float4* vp = reinterpret_cast<float4*>(g.vals + (int64_t)row * d + n0 + q * 64);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              vp[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          }
+        }
+        if (valid) g.vv[(int64_t)n_blk * R + row] = svv;
       } else {
 #pragma unroll 1
         for (int q = 0; q < BN / 64; ++q) {
@@ -418,6 +437,9 @@ cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, cons
     case 257: return launch_bn<128, 1>(maps, g, grid, stream);
     case 128: return launch_bn<64, 0>(maps, g, grid, stream);
     case 129: return launch_bn<64, 1>(maps, g, grid, stream);
+    case 515: return launch_bn<256, 3>(maps, g, grid, stream);
+    case 259: return launch_bn<128, 3>(maps, g, grid, stream);
+    case 131: return launch_bn<64, 3>(maps, g, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -31,7 +31,9 @@
 // h ring), 2 = values when out aliases h (the residual update in place): the
 // epilogue stages bf16(alpha v) and adds it into out with a TMA reduce-add,
 // so h never passes through shared memory; the sum is rounded once more
-// (RN(h + RN(alpha v)) instead of RN(h + alpha v)).
+// (RN(h + RN(alpha v)) instead of RN(h + alpha v)); 3 = values for the short
+// convolution (Eq. 5): v in fp32 and its sum of squares per row and tile,
+// plus alpha; h is not read.
 // Waits are bounded as in the single-CTA kernel; the pair leaves together
 // through a bounded handshake, then frees TMEM (cta_group::2).
 #include "sm100_ptx.cuh"
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // h sub-tiles per tile: one branch in the key phase, every branch in the
   // value phase (v is shared across branches, Eq. 6); none when the value
   // phase adds into h in place
-  const int nsub = PHASE == 2 ? 0 : (kCols / H_COLS) * (PHASE == 0 ? 1 : M);
+  const int nsub = PHASE >= 2 ? 0 : (kCols / H_COLS) * (PHASE == 0 ? 1 : M);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
       }
-      if (lane == 0 && row0 < R) {
+      if (PHASE != 3 && lane == 0 && row0 < R) {
         for (int i = PHASE == 2 ? 0 : H_SLOTS; i < nbox; ++i)
           tma_prefetch_l2_2d(&map_h, PHASE == 0 ? n0 + H_COLS * i
                                                 : (i % M) * d + n0 + H_COLS * (i / M),
@@ -401,6 +403,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(wempty_bar);
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
+      } else if (PHASE == 3) {
+        // values for the short convolution (Eq. 5): v in fp32 and the row's
+        // sum of v^2 over this tile; the conv kernel forms alpha v from them
+        float svv = 0.f;
+        auto vals_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
+          tmem_wait32(v);
+          __syncwarp();
+          if (q + 1 < NQ) {
+            tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+          } else {
+            tc_fence_before();  // last TMEM read done: release the accumulators
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
+          }
+          unsigned long long s2[2] = {0ull, 0ull};
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const unsigned long long v2 = f2_pack(v[e], v[e + 1]);
+            s2[(e >> 1) & 1] = f2_fma(v2, v2, s2[(e >> 1) & 1]);
+          }
+          const float2 s0 = f2_unpack(s2[0]), s1 = f2_unpack(s2[1]);
+          svv += (s0.x + s0.y) + (s1.x + s1.y);
+          if (valid) {
+            float4* vp = reinterpret_cast<float4*>(g.vals + (int64_t)row * d + n0 + q * H_COLS);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              vp[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                  __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+          }
+        };
+#pragma unroll 1
+        for (int q = 0; q < NQ; q += 2) {
+          vals_chunk(q, va, vb);
+          vals_chunk(q + 1, vb, va);
+        }
+        if (valid) g.vv[(int64_t)n_blk * R + row] = svv;
       } else if (PHASE == 2) {
         // out aliases h: add bf16(alpha v) into it with TMA reduce-add; each
         // warp stages its 32 rows x 32 columns in one of two 2 KB buffers
@@ -599,6 +637,7 @@ cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArg
     case 0: return launch_wide<0>(maps, g, grid, stream);
     case 1: return launch_wide<1>(maps, g, grid, stream);
     case 2: return launch_wide<2>(maps, g, grid, stream);
+    case 3: return launch_wide<3>(maps, g, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -29,7 +29,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_set_params", "engram_reserve", "engram_get_hash_params", "engram_hash",
            "engram_gather", "engram_forward", "engram_prefetch", "engram_check_errors",
            "engram_profile_next_forward", "engram_kernel_launches",
-           "engram_project_gate_noalloc", "engram_selftest_timeout")
+           "engram_project_gate_noalloc", "engram_selftest_timeout", "engram_set_short_conv")
 
 
 class engram_config(ctypes.Structure):
@@ -65,6 +65,7 @@ def _load():
         "engram_last_error": ([H], ctypes.c_char_p),
         "engram_set_params": ([H, P, P, P, P, P], ctypes.c_int),
         "engram_reserve": ([H, i64], ctypes.c_int),
+        "engram_set_short_conv": ([H, P, P, i32, i32, P], ctypes.c_int),
         "engram_get_hash_params": ([H, P, P], ctypes.c_int),
         "engram_hash": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
@@ -170,6 +171,13 @@ class Engram:
                                           _ptr(w_v), _ptr(norm_q), _ptr(norm_k)))
         self._params = (list(tables), w_k, w_v, norm_q, norm_k)  # borrowed: keep alive
 
+    def set_short_conv(self, conv_w, norm_w, kernel_size: int = 4, dilation: int = 3,
+                       stream=None):
+        """Switch on the short convolution of Eq. (5) with conv_w [d, kernel_size]
+        and norm_w [d] (fp32, device; copied); kernel_size 0 switches it off."""
+        self._check(lib.engram_set_short_conv(self._h, _ptr(conv_w), _ptr(norm_w), kernel_size,
+                                              dilation, _stream_ptr(stream)))
+
     def reserve(self, max_rows: int):
         self._check(lib.engram_reserve(self._h, max_rows))
 
@@ -195,10 +203,11 @@ class Engram:
         return n.value if want_count else None
 
     def profile_next_forward(self, events):
-        """Record 5 CUDA events inside the next forward (stage boundaries)."""
+        """Record 5 or 6 CUDA events inside the next forward (stage boundaries)."""
         self._prof_keep = list(events)
-        arr = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
-        self._check(lib.engram_profile_next_forward(self._h, ctypes.cast(arr, ctypes.c_void_p), 5))
+        n = len(events)
+        arr = (ctypes.c_void_p * n)(*[e.cuda_event for e in events])
+        self._check(lib.engram_profile_next_forward(self._h, ctypes.cast(arr, ctypes.c_void_p), n))
 
     def kernel_launches(self) -> int:
         return int(lib.engram_kernel_launches(self._h))

@@ -167,6 +167,29 @@ ENGRAM_API int engram_set_params(engram_handle *h, const void *const *tables, co
                       const void *w_v, const float *norm_q, const float *norm_k);
 
 /*
+ * The short convolution of the module output (section 2.3, Eq. 5):
+ *   Y = SiLU(Conv1D(RMSNorm(V~))) + V~,  out = h + Y,  V~ = alpha * v,
+ * Conv1D depthwise and causal over the positions of each sequence (zero
+ * before its start, no bias), kernel size W, dilation delta: tap i of channel
+ * c multiplies position t - i * delta.  The paper uses W = 4, delta = the
+ * largest n-gram order, zero-initialised weights (then Y = V~ exactly).  In
+ * the multi-branch form the same weights act on each branch's gated values.
+ *  conv_w  device fp32 [d, kernel_size] (row c holds the taps of channel c).
+ *  norm_w  device fp32 [d]: RMSNorm weight (the handle's eps is used).
+ *  kernel_size 1..4, or 0 to switch the convolution off again (pointers
+ *          ignored); dilation 1..4.
+ * The weights are copied (on `stream`, which is synchronised before the call
+ * returns).  While it is on, engram_forward needs t_begin = 0 (every position
+ * of each sequence is an input of the convolution) and returns
+ * ENGRAM_ERR_UNSUPPORTED otherwise; its delta output receives Y; and
+ * engram_project_gate_noalloc returns ENGRAM_ERR_UNSUPPORTED.  Extra scratch
+ * per row: 4 d bytes of v and 4 (d / 64 + M) bytes.
+ * Errors: _INVALID, _STATE (engram_set_params first), _OOM, _CUDA.
+ */
+ENGRAM_API int engram_set_short_conv(engram_handle *h, const float *conv_w, const float *norm_w,
+                                     int32_t kernel_size, int32_t dilation, void *stream);
+
+/*
  * Pre-allocate the handle's device scratch for calls of up to `max_rows`
  * emitted positions (rows = B * (T - t_begin)).  Calls with more rows grow the
  * scratch themselves; reserving first keeps allocation out of timed or
@@ -202,14 +225,16 @@ ENGRAM_API int engram_gather(engram_handle *h, const int64_t *idx, int64_t rows,
  * The whole forward (steps 1-7): out = h + alpha * (W_V e) per branch, with
  * alpha = sigmoid(RMSNorm_q(h) . RMSNorm_k(W_K e) / sqrt(d)) (Eq. 3, 4, 6).
  * At the paper's zero-initialised ShortConv (Eq. 5, Table 5) this equals the
- * module output added to the residual stream.
+ * module output added to the residual stream; with engram_set_short_conv the
+ * convolution is applied (out = h + Y, Eq. 5).
  *  tokens  device int32 [B, T].
  *  idx     device int64 [rows, S] precomputed by engram_hash, or NULL to hash
  *          inside this call.
  *  hid     device [rows, M, d] dtype, rows = B*(T-t_begin).
  *  out     device [rows, M, d] dtype (may alias hid for an in-place update).
  *  alpha   device fp32 [rows, M] or NULL.
- *  delta   device fp32 [rows, M, d] or NULL: alpha * v before the residual add.
+ *  delta   device fp32 [rows, M, d] or NULL: what is added to h (alpha * v,
+ *          or Y with the short convolution).
  * With ENGRAM_PINNED_HOST tables, the rows must have been staged by
  * engram_prefetch for the same tokens; the call waits (on the stream) for
  * that prefetch.  Errors: _INVALID, _STATE, _OOM, _CUDA.
@@ -242,11 +267,13 @@ ENGRAM_API int engram_check_errors(engram_handle *h, void *stream);
 
 /*
  * Stage timing for the NEXT engram_forward on this handle (one-shot).
- * `events` holds 5 cudaEvent_t (as void*), created by the caller with timing
- * enabled.  That forward records them on its stream at: start, after hashing,
- * after the gather, after the key-projection kernel, after the value-
- * projection kernel (consecutive events coincide for a stage that does not
- * run, e.g. hashing when idx is given).  n_events must be 5; NULL clears.
+ * `events` holds 5 or 6 cudaEvent_t (as void*), created by the caller with
+ * timing enabled.  That forward records them on its stream at: start, after
+ * hashing, after the gather, after the key-projection kernel, after the
+ * value-projection kernel, and (6th) after the short convolution
+ * (consecutive events coincide for a stage that does not run, e.g. hashing
+ * when idx is given or when it is fused into the gather).  With 5 events the
+ * convolution counts in the value stage.  NULL clears.
  */
 ENGRAM_API int engram_profile_next_forward(engram_handle *h, void *const *events, int32_t n_events);
 

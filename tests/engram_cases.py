@@ -99,6 +99,40 @@ class Problem:
                                                 self.nq_cpu.numpy(), self.nk_cpu.numpy(), h, eps)
         return e, alpha, delta, out
 
+    def conv_weights(self, kernel_size: int = 4):
+        """Seeded ShortConv weights (conv_w [d, W], norm_w [d], fp32 on the CPU)."""
+        return synth.make_conv_weights(self.shape, self.seeds, kernel_size)
+
+    def oracle_forward_conv(self, rows: np.ndarray, conv_w, norm_w, dilation: int,
+                            eps: float = 1e-6):
+        """Y [n, M, d] (double) and out [n, M, d] (h's dtype) of Eq. (5) at `rows`
+        (t_begin = 0, row = b T + t): the gated values alpha v are formed by
+        the oracle at the positions the taps read, t - i * dilation."""
+        sh = self.shape
+        assert sh.t_begin == 0
+        W = conv_w.shape[1]
+        T = sh.T
+        need = sorted({int(r) - i * dilation for r in rows for i in range(W)
+                       if (int(r) % T) - i * dilation >= 0})
+        need = np.array(need, dtype=np.int64)
+        _, _, vt, _ = self.oracle_forward(need, eps)          # delta = alpha v [n, M, d]
+        pos = {int(r): j for j, r in enumerate(need)}
+        M, d = sh.branches, sh.d_hidden
+        cw, nw = conv_w.numpy(), norm_w.numpy()
+        Y = np.empty((len(rows), M, d))
+        for j, r in enumerate(rows):
+            r = int(r)
+            have = np.array([(r % T) - i * dilation >= 0 for i in range(W)], dtype=np.int32)
+            for m in range(M):
+                taps = np.zeros((W, d))
+                for i in range(W):
+                    if have[i]:
+                        taps[i] = vt[pos[r - i * dilation], m]
+                Y[j, m] = oracle.short_conv_at(taps, have, cw, nw, eps)
+        h = to_oracle(self.h[torch.from_numpy(np.asarray(rows)).to(self.h.device)])
+        out = oracle.add_round(h, Y.reshape(h.shape))
+        return Y, out
+
     def sample_rows(self, n: int, seed: int = 0) -> np.ndarray:
         """Every sequence's first three and last emitted positions, plus random rows."""
         sh = self.shape
