@@ -62,6 +62,9 @@ def parse():
                     choices=["prefill_bf16", "decode_mb", "large_hbm", "offload"],
                     help="prefill_bf16 is the benchmarked line; the others measure the other "
                          "configurations of the same forward")
+    ap.add_argument("--short-conv", action="store_true",
+                    help="with the short convolution of Eq. 5 (W = 4, dilation = the largest "
+                         "n-gram order, seeded non-zero weights); prefill-type workloads")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a captured CUDA graph (launch-bound shapes)")
     ap.add_argument("--offload-gb", type=float, default=100.0,
@@ -147,7 +150,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------ the workload
 
-def setup(rank: int, device, rows_target=None, workload=WORKLOAD):
+def setup(rank: int, device, rows_target=None, workload=WORKLOAD, short_conv=False):
     import torch
     from hashed_gram_embedding_compress_b200 import engram as eg
     from hashed_gram_embedding_compress_b200 import synth
@@ -169,10 +172,15 @@ def setup(rank: int, device, rows_target=None, workload=WORKLOAD):
     w_k, w_v, nq, nk = w_k.to(device), w_v.to(device), nq.to(device), nk.to(device)
     m.set_params(tables, w_k, w_v, nq, nk)
     h = synth.make_hidden(sh, seeds, device=device)
+    conv = None
+    if short_conv:
+        cw, nw = synth.make_conv_weights(sh, seeds, 4)
+        conv = (cw.to(device), nw.to(device), 4, max(sh.orders))
+        m.set_short_conv(*conv)
     m.reserve(sh.rows_out)
     return dict(sh=sh, m=m, tokens=tokens, comp_map=comp_map, tables=tables, w_k=w_k, w_v=w_v,
                 nq=nq, nk=nk, h=h, seeds=seeds, hash_seed=synth.make_hash_seed(seeds),
-                primes=primes)
+                primes=primes, conv=conv)
 
 
 def algorithmic(sh):
@@ -190,7 +198,11 @@ def algorithmic(sh):
     gemm_flops = 2.0 * R * dm * (M * d + d)          # [W_K^(1..M); W_V] e
     # key kernel: e read, W_K read, h read; value kernel: e, W_V, h read, out written
     gemm_bytes = (2 * R * dm * elt + (M * d + d) * dm * elt + 3 * R * M * d * elt)
+    # short conv: v (fp32) read once, h read and out written per branch, plus
+    # alpha and the per-tile sums of v^2
+    conv_bytes = R * d * 4 + 2 * R * M * d * elt + R * (M + d // 256) * 4
     return dict(gather_bytes=gather_bytes, hash_bytes=hash_bytes, gemm_flops=gemm_flops,
+                conv_bytes=conv_bytes,
                 gemm_bytes=gemm_bytes)
 
 
@@ -231,8 +243,9 @@ def run_ours(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    P = setup(rank, device, args.rows_target, args.workload)
+    P = setup(rank, device, args.rows_target, args.workload, args.short_conv)
     sh, m = P["sh"], P["m"]
+    NEV = 6 if args.short_conv else 5  # stage events per forward
     tok_d = P["tokens"].to(device)
     h = P["h"]
     stream = torch.cuda.current_stream()
@@ -271,7 +284,7 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NEV)] for _ in range(K)]
     for row in evs:  # torch creates the CUDA event at its first record
         for ev in row:
             ev.record(stream)
@@ -295,21 +308,22 @@ def run_ours(args, rank, world, dist):
     launches = m.kernel_launches() - launches0
     ms = max_over_ranks(t0.elapsed_time(t1), dist, device)
     if graph is None:
-        stage = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)]
-        st_mean = [sum(s[i] for s in stage) / K for i in range(4)]  # hash, gather, key, value
+        stage = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(NEV - 1)] for k in range(K)]
+        # hash, gather, key, value (, short conv)
+        st_mean = [sum(s[i] for s in stage) / K for i in range(NEV - 1)]
     else:
         # one graph replay per step: no per-kernel events; split by the same
         # shares would be a guess, so the stages are timed by replaying the
         # eager forward once more with events
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(NEV)]
         for e_ in ev:
             e_.record(stream)
-        st_mean = [0.0] * 4
+        st_mean = [0.0] * (NEV - 1)
         for _ in range(5):
             m.profile_next_forward(ev)
             forward_once()
             torch.cuda.synchronize()
-            for i in range(4):
+            for i in range(NEV - 1):
                 st_mean[i] += ev[i].elapsed_time(ev[i + 1]) / 5
     if m.check_errors(stream) != 0:
         raise RuntimeError("device error during the timed steps")
@@ -398,7 +412,8 @@ def run_ours(args, rank, world, dist):
         },
         "stages_ms": ({"hash_gather": st_mean[0] + st_mean[1]} if fused else
                       {"hash": st_mean[0], "gather": st_mean[1]}) |
-                     {"key_proj_gate": st_mean[2], "value_proj_gate": st_mean[3]},
+                     {"key_proj_gate": st_mean[2], "value_proj_gate": st_mean[3]} |
+                     ({"short_conv": st_mean[4]} if args.short_conv else {}),
         "e2e": {
             "value": tokens_per_step * world * E / (e2e_ms / 1e3),
             "unit": "tokens/s",
@@ -410,6 +425,19 @@ def run_ours(args, rank, world, dist):
         "clocks": dict(clk.summary(t_load + 0.5, t_end + 0.15),
                        window="last 1 s of back-to-back warm-up steps and the timed steps"),
     }
+    if args.short_conv:
+        res["config"]["workload"] += (" + ShortConv (Eq. 5: W=4, dilation %d, RMSNorm, SiLU, "
+                                      "seeded non-zero weights)" % max(sh.orders))
+        res["config"]["residual"] = "in place: out aliases h (H <- H + Y, Eq. 5)"
+        res["short_conv"] = {
+            "kernel": "short_conv_kernel",
+            "bound": "hbm",
+            "achieved_gbs": A["conv_bytes"] / (st_mean[4] / 1e3) / 1e9,
+            "peak_gbs": hbm,
+            "frac": A["conv_bytes"] / (st_mean[4] / 1e3) / 1e9 / hbm,
+            "bytes_per_step": A["conv_bytes"],
+        }
+        res["roofline"]["traffic"] = None  # the committed capture is of the conv-less value phase
     if args.rows_target:
         res["config"]["workload"] += " [profiling variant: tables of %d rows]" % args.rows_target
     if args.workload != "prefill_bf16":
@@ -603,7 +631,13 @@ def cpu_baseline(P, budget_s: float):
         hr = to_np(P["h"][torch.from_numpy(rows).to(P["h"].device)])
         t0 = time.perf_counter()
         e = oracle.gather(mini, zz)
-        oracle.project_gate(e, wk, wv, nq, nk, hr, 1e-6, want_delta=False)
+        _, delta, _ = oracle.project_gate(e, wk, wv, nq, nk, hr, 1e-6, want_delta=P["conv"] is not None)
+        if P["conv"] is not None:
+            # Eq. 5 over the sample's positions (consecutive rows of one sequence)
+            cw, nw, W, dil = P["conv"]
+            for mb in range(sh.branches):
+                y = oracle.short_conv(delta[:, mb], cw.cpu().numpy(), nw.cpu().numpy(), dil, 1e-6)
+                oracle.add_round(np.ascontiguousarray(hr[:, mb]), y)
         dt = time.perf_counter() - t0
         total_rows += len(rows)
         total_t += dt
@@ -611,9 +645,10 @@ def cpu_baseline(P, budget_s: float):
         n *= 2
     per_row = t_hash + total_t / total_rows
     return {"value": 1.0 / per_row, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "compress+hash on all %d positions; gather+projection+gate on the first "
-                      "%d rows (%.1f s); single-threaded C, fp64" % (sh.rows_out, total_rows,
-                                                                    total_t)}
+            "sample": "compress+hash on all %d positions; gather+projection+gate%s on the first "
+                      "%d rows (%.1f s); single-threaded C, fp64" % (
+                          sh.rows_out, "+short conv" if P["conv"] is not None else "",
+                          total_rows, total_t)}
 
 
 def run_reference(args, rank, world):
@@ -621,7 +656,8 @@ def run_reference(args, rank, world):
         return None
     import torch
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    P = setup(0, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))), None, args.workload)
+    P = setup(0, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))), None, args.workload,
+              args.short_conv)
     sh = P["sh"]
     budget = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):

@@ -75,18 +75,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D bf16 tensor map: `rows` rows of `cols` elements, box box_cols x box_rows;
 // the swizzle width is the box row width (64 columns = 128 B, 32 columns = 64 B).
+// 2-D row-major tensor map; the swizzle follows the box's row bytes (128-byte
+// rows: 128-byte swizzle, 64-byte rows: 64-byte swizzle).  bf16 unless f32.
 int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
-             int box_rows, int box_cols = 64) {
+             int box_rows, int box_cols = 64, bool f32 = false) {
   auto fn = encode_fn();
   if (!fn) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const int esz = f32 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * esz};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
   const CUtensorMapSwizzle sw =
-      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+      box_cols * esz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   return ENGRAM_OK;
@@ -113,11 +116,13 @@ int ensure_conv_scratch(engram_handle* h, int64_t rows) {
   free_dev(h->conv_v);
   free_dev(h->conv_vv);
   free_dev(h->conv_alpha);
+  free_dev(h->conv_scale);
   h->conv_cap_rows = 0;
   const int d = h->cfg.d_hidden;
   CK(h, cudaMalloc(&h->conv_v, (size_t)rows * d * sizeof(float)));
   CK(h, cudaMalloc(&h->conv_vv, (size_t)rows * (d / 64) * sizeof(float)));
   CK(h, cudaMalloc(&h->conv_alpha, (size_t)rows * h->cfg.branches * sizeof(float)));
+  CK(h, cudaMalloc(&h->conv_scale, (size_t)rows * h->cfg.branches * sizeof(float)));
   h->conv_cap_rows = rows;
   return ENGRAM_OK;
 }
@@ -334,9 +339,11 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->partials);
   free_dev(h->d_conv_w);
   free_dev(h->d_conv_nw);
+  free_dev(h->d_conv_taps);
   free_dev(h->conv_v);
   free_dev(h->conv_vv);
   free_dev(h->conv_alpha);
+  free_dev(h->conv_scale);
   free_dev(h->d_keys);
   free_dev(h->d_vals);
   free_dev(h->d_uniq);
@@ -420,6 +427,7 @@ int engram_set_short_conv(engram_handle* h, const float* conv_w, const float* no
   if (!h->d_conv_w) {
     CK(h, cudaMalloc(&h->d_conv_w, (size_t)d * 4 * sizeof(float)));
     CK(h, cudaMalloc(&h->d_conv_nw, (size_t)d * sizeof(float)));
+    CK(h, cudaMalloc(&h->d_conv_taps, (size_t)d * 4 * sizeof(float)));
   }
   // [d][kernel_size] -> [d][4] with the unused taps zero
   CK(h, cudaMemsetAsync(h->d_conv_w, 0, (size_t)d * 4 * sizeof(float), st));
@@ -427,6 +435,8 @@ int engram_set_short_conv(engram_handle* h, const float* conv_w, const float* no
                           kernel_size * sizeof(float), d, cudaMemcpyDeviceToDevice, st));
   CK(h, cudaMemcpyAsync(h->d_conv_nw, norm_w, (size_t)d * sizeof(float), cudaMemcpyDeviceToDevice,
                         st));
+  CK(h, launch_conv_taps(h->d_conv_w, h->d_conv_nw, d, h->d_conv_taps, st));
+  h->launches += 1;
   CK(h, cudaStreamSynchronize(st));
   h->conv_W = kernel_size;
   h->conv_dil = dilation;
@@ -584,6 +594,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   if (conv && t_begin != 0)
     return fail(h, ENGRAM_ERR_UNSUPPORTED,
                 "the short convolution needs every position of each sequence (t_begin = 0)");
+  if (conv && R * (h->cfg.d_hidden / 4) >= ((int64_t)1 << 31))
+    return fail(h, ENGRAM_ERR_INVALID, "too many rows for the short convolution in one call");
   if (conv && (rc = ensure_conv_scratch(h, R))) return rc;
   CK(h, mark(0));
 
@@ -655,8 +667,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     ca.h = hid;
     ca.out = out;
     ca.delta = delta;
-    ca.conv_w = h->d_conv_w;
-    ca.norm_w = h->d_conv_nw;
+    ca.taps = h->d_conv_taps;
     ca.B = B;
     ca.T = T;
     ca.M = g.M;
@@ -664,8 +675,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     ca.n_vtiles = g.d / value_tile;
     ca.bf16 = h->cfg.dtype == ENGRAM_BF16;
     ca.eps = g.eps;
-    CK(h, launch_short_conv(ca, h->conv_dil, st));
-    h->launches += 1;
+    CK(h, launch_short_conv(ca, h->conv_dil, h->conv_scale, st));
+    h->launches += 2;
     CK(h, mark(5));
     return ENGRAM_OK;
   };
@@ -703,7 +714,14 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
         have_wide = true;
       }
       wide.w = wmaps[bn_index(pc.bn)];
-      CK(h, launch_proj_gate_wide(kphase, wide, g, pc.grid, st));
+      if (kphase == 3) {
+        // v leaves through per-warp TMA stores of 32 x 32 fp32 boxes
+        ProjMaps wv = wide;
+        if ((rc = make_map(h, &wv.out, h->conv_v, g.d, R, 32, 32, true))) return rc;
+        CK(h, launch_proj_gate_wide(kphase, wv, g, pc.grid, st));
+      } else {
+        CK(h, launch_proj_gate_wide(kphase, wide, g, pc.grid, st));
+      }
     } else {
       if (!have_single) {
         if ((rc = make_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;

@@ -36,6 +36,7 @@ struct engram_handle {
   int conv_W = 0, conv_dil = 0;
   float* d_conv_w = nullptr;   // [d][4], taps >= conv_W zero
   float* d_conv_nw = nullptr;  // [d]
+  float* d_conv_taps = nullptr;  // [4][d]: conv_w times norm_w, tap-major
 
   // scratch, sized for cap_rows emitted positions
   int64_t cap_rows = 0;
@@ -46,6 +47,7 @@ struct engram_handle {
   float* conv_v = nullptr;      // [rows, d] v = W_V e
   float* conv_vv = nullptr;     // [d / 64][rows] sums of v^2 per value tile
   float* conv_alpha = nullptr;  // [rows, M] when the caller passes none
+  float* conv_scale = nullptr;  // [rows, M] alpha / sqrt(alpha^2 mean(v^2) + eps)
 
   // host-resident tables: prefetch state, double-buffered
   int64_t pf_cap_rows = 0;

@@ -77,8 +77,8 @@ struct ConvArgs {
   const void* h;        // [B*T, M, d] fp32 or bf16
   void* out;            // [B*T, M, d], may alias h
   float* delta;         // [B*T, M, d] the increment Y, or null
-  const float* conv_w;  // [d][4]: tap i multiplies position t - i * dilation
-  const float* norm_w;  // [d]
+  const float* taps;    // [4][d]: tap i of channel c (it multiplies position
+                        // t - i * dilation) times the RMSNorm weight of c
   int32_t B, T, M, d, n_vtiles, bf16;
   float eps;
 };
@@ -105,8 +105,12 @@ struct PrefetchArgs {
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
 cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream);
-// dilation 1..4; the grid covers B * ceil(T / 64) position tiles.
-cudaError_t launch_short_conv(const ConvArgs& a, int dilation, cudaStream_t stream);
+// taps[i][c] = conv_w[c][i] * norm_w[c] for the [d][4] conv weights.
+cudaError_t launch_conv_taps(const float* conv_w, const float* norm_w, int d, float* taps,
+                             cudaStream_t stream);
+// dilation 1..4; scale is scratch [B*T, M] fp32.  Two launches: the RMS
+// scale per (position, branch), then the convolution and residual.
+cudaError_t launch_short_conv(const ConvArgs& a, int dilation, float* scale, cudaStream_t stream);
 cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t stream);
 cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);

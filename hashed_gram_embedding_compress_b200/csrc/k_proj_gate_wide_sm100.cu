@@ -63,6 +63,7 @@ constexpr int NUM_BARS = 2 * STAGES + 2 + 2 * H_SLOTS + 4;
 constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * H_BYTES +
                         W_BYTES + 8 * NUM_BARS + 16;
 static_assert(SMEM <= 232448, "shared memory budget");
+static_assert(kEpiWarps * 8192 <= H_SLOTS * H_BYTES, "per-warp store staging fits in the h ring");
 
 template <int PHASE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -405,8 +406,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
       } else if (PHASE == 3) {
         // values for the short convolution (Eq. 5): v in fp32 and the row's
-        // sum of v^2 over this tile; the conv kernel forms alpha v from them
+        // sum of v^2 over this tile; the conv kernel forms alpha v from them.
+        // Each warp stages its 32 rows x 32 columns (4 KB, 128-byte swizzle)
+        // in one of two buffers and stores them by TMA (map_out covers v).
         float svv = 0.f;
+        uint8_t* stage0 = hbuf + warp * 8192;
+        int sbuf = 0;
         auto vals_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
           tmem_wait32(v);
           __syncwarp();
@@ -425,13 +430,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float2 s0 = f2_unpack(s2[0]), s1 = f2_unpack(s2[1]);
           svv += (s0.x + s0.y) + (s1.x + s1.y);
-          if (valid) {
-            float4* vp = reinterpret_cast<float4*>(g.vals + (int64_t)row * d + n0 + q * H_COLS);
+          // the buffer's previous store has finished reading it
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
+          uint8_t* st = stage0 + sbuf * 4096;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              vp[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
-                                  __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(st + sw128_off(lane, c)) =
+                make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 + wrow0 < R)
+              tma_store_2d(&map_out, smem_u32(st), n0 + q * H_COLS, row0 + wrow0);
+            else
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           }
+          sbuf ^= 1;
         };
 #pragma unroll 1
         for (int q = 0; q < NQ; q += 2) {

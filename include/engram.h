@@ -183,7 +183,7 @@ ENGRAM_API int engram_set_params(engram_handle *h, const void *const *tables, co
  * of each sequence is an input of the convolution) and returns
  * ENGRAM_ERR_UNSUPPORTED otherwise; its delta output receives Y; and
  * engram_project_gate_noalloc returns ENGRAM_ERR_UNSUPPORTED.  Extra scratch
- * per row: 4 d bytes of v and 4 (d / 64 + M) bytes.
+ * per row: 4 d bytes of v and 4 (d / 64 + 2 M) bytes.
  * Errors: _INVALID, _STATE (engram_set_params first), _OOM, _CUDA.
  */
 ENGRAM_API int engram_set_short_conv(engram_handle *h, const float *conv_w, const float *norm_w,
