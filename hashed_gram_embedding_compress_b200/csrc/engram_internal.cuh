@@ -147,8 +147,11 @@ struct ProjChoice {
   int key_tile;  // columns per partial-sum tile (phase 0)
 };
 // 512 x 256 CTA-pair tiles whenever there are enough of them for every pair,
-// else single-CTA 128-row tiles of the widest N that still gives every SM a
-// tile.  Key tiles must not straddle branches, so their width divides d.
+// else single-CTA 128-row tiles of the N that minimises rounds of tiles per
+// SM x operand bytes per tile (128 + N rows of K): the mainloop streams its
+// operands from L2 at a fixed rate per SM, so a second, partly filled round
+// of narrow tiles costs more than one round of wide ones.  Key tiles must not
+// straddle branches, so their width divides d.
 inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int flags) {
   const int n_total = phase == 0 ? M * d : d;
   const int pairs = sms / 2;
@@ -157,11 +160,16 @@ inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int f
     return {ProjKernel::Wide, 128, 2 * pairs, 256};
   const int64_t mblk = (R + 127) / 128;
   int bn = 64;
-  for (int c : {256, 128})
-    if (n_total % c == 0 && d % c == 0 && mblk * (n_total / c) >= sms) {
+  int64_t best = -1;
+  for (int c : {256, 128, 64}) {
+    if (n_total % c != 0 || d % c != 0) continue;
+    const int64_t rounds = (mblk * (n_total / c) + sms - 1) / sms;
+    const int64_t cost = rounds * (128 + c);
+    if (best < 0 || cost < best) {
+      best = cost;
       bn = c;
-      break;
     }
+  }
   const int64_t tiles = mblk * (n_total / bn);
   return {ProjKernel::Single, bn, (int)(tiles < sms ? tiles : sms), bn};
 }

@@ -24,7 +24,7 @@
 //   warp 5      TMEM allocator and MMA issuer: tcgen05.mma.cta_group::1
 //               kind::f16 (bf16 in, fp32 accumulate), M=128, N=BN, K=16,
 //               accumulators double-buffered in TMEM (2*BN columns);
-//   warp 6      TMA producer of h sub-tiles [128 x 64] into a 2-slot ring;
+//   warp 6      TMA producer of h sub-tiles [128 x 64] into a 2- or 4-slot ring;
 //   warps 0-3   epilogue: tcgen05.ld 32 columns at a time (warp w owns TMEM
 //               lanes 32w..32w+31, i.e. rows of the tile), fused gate math
 //               against h in shared memory; the value phase writes out over h
@@ -44,14 +44,18 @@ constexpr int BM = 128;
 constexpr int BK = 64;                     // 64 bf16 = one 128-byte swizzle row
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int kThreads = 224;              // 7 warps
-constexpr int H_SLOTS = 2;                 // ring of h / out sub-tiles
 constexpr uint32_t H_BYTES = BM * 64 * 2;  // one sub-tile: 128 rows x 64 bf16, 128-B swizzle
 
 template <int BN>
 struct Cfg {
+  // ring of h / out sub-tiles: with 64-column tiles there is room to hold a
+  // chunk's sub-tiles of up to four branches while the mainloop runs
+  static constexpr int H_SLOTS = BN == 64 ? 4 : 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int STAGES = ((229376 - H_SLOTS * H_BYTES) / STAGE_BYTES) > 8
+                                    ? 8
+                                    : ((229376 - H_SLOTS * H_BYTES) / STAGE_BYTES);
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr int NUM_BARS = 2 * STAGES + 4 + 3 * H_SLOTS + 1;
   static constexpr uint32_t BAR_BYTES = 8 * NUM_BARS + 16;
@@ -68,6 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap map_out, GateArgs g) {
   using C = Cfg<BN>;
   constexpr int STAGES = C::STAGES;
+  constexpr int H_SLOTS = C::H_SLOTS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -239,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Thread (warp w, lane l) owns tile row r = 32w + l: TMEM lane r and
     // row r of every h sub-tile in shared memory.
     const int r = warp * 32 + lane;
+    int pending = -1;  // value phase, warp 0: slot whose TMA store may still read it
     int acc = 0, hslot = 0;
     uint32_t acc_phase = 0, hphase = 0;
     bool ok = true;
@@ -374,8 +380,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_ready(hdone_bar(hslot), hphase, abort_flag, g.err);
                 if (ok) {
                   tma_store_2d(&map_out, sH + hslot * H_BYTES, mb * d + n0 + q * 64, m_blk * BM);
-                  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                  mbar_arrive(hempty_bar(hslot));
+                  // hand back the previous slot once its store has read it;
+                  // this one stays with its store in flight
+                  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                  if (pending >= 0) mbar_arrive(hempty_bar(pending));
+                  pending = hslot;
                 }
               }
               ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -398,8 +407,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
-    if (PHASE == 1 && warp == 0 && lane == 0)
+    if (PHASE == 1 && warp == 0 && lane == 0) {
       asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      if (pending >= 0 && ok) mbar_arrive(hempty_bar(pending));
+    }
   }
 
   tc_fence_before();
