@@ -50,6 +50,7 @@ struct HashGatherArgs {
   const void* const* tables;  // device array [S] of table base pointers
   void* e;                    // [rows, S*d_head]
   int32_t row_bytes;          // d_head * element size, a multiple of 16
+  int32_t rows_per_block;     // set by the launcher
 };
 
 // Projection + gate epilogue arguments (Eq. 3, 4, 6).

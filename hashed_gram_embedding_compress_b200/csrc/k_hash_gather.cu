@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
   }
 }
 
-// Hash and gather fused: a block owns 256 / S consecutive output rows.  Its
+// Hash and gather fused: a block owns up to 256 / S consecutive output rows.  Its
 // threads first compute the rows' S indices each (one per thread, as in
 // hash_kernel) and keep the source row addresses in shared memory; then they
 // copy the rows' table rows into e, 16 bytes per thread and load, four loads
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
 
   const uint32_t Tout = (uint32_t)(a.T - a.t_begin);
   const uint32_t rows = (uint32_t)a.B * Tout;
-  const uint32_t rb = kFusedThreads / (uint32_t)S;  // rows per block
+  const uint32_t rb = (uint32_t)g.rows_per_block;  // <= 256 / S
   const uint32_t row0 = blockIdx.x * rb;
   const uint32_t nrows = min(rb, rows - row0);
   const uint32_t nslots = nrows * (uint32_t)S;
@@ -236,8 +236,17 @@ cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   if (a.hash.S < 1 || a.hash.S > kMaxTables) return cudaErrorInvalidValue;
   if (rows * a.hash.S * (a.row_bytes >> 4) >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
-  const int64_t rb = kFusedThreads / a.hash.S;
-  hash_gather_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(a);
+  // 256 / S rows per block, fewer when that leaves SMs idle (short calls,
+  // e.g. decode): the copies of a block then take a single round
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t rb = kFusedThreads / a.hash.S;
+  const int64_t fill = (rows + 2 * (int64_t)sms - 1) / (2 * (int64_t)sms);
+  if (fill < rb) rb = fill < 1 ? 1 : fill;
+  HashGatherArgs b = a;
+  b.rows_per_block = (int32_t)rb;
+  hash_gather_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(b);
   return cudaGetLastError();
 }
 

@@ -127,10 +127,12 @@ def check_in_place(p: Problem, m, out, delta):
 
 
 @pytest.mark.parametrize("shape", [
-    synth.SHAPES["tiny_f32"],                                            # S = 8: 32 rows per block
-    synth.SHAPES["decode_mb"],                                           # blocks span sequences
+    synth.SHAPES["tiny_f32"],                                            # S = 8
+    synth.SHAPES["decode_mb"],                                           # one row per block
     synth.SHAPES["tiny_f32"].replace(orders=(2, 3, 4), heads=5, T=37),    # S = 15: 17 rows per block
     synth.SHAPES["prefill_bf16"].replace(B=3, T=171, heads=3, rows_target=4099, d_hidden=256),
+    # 3000 rows: 11 rows per block, so blocks straddle the sequence starts
+    synth.SHAPES["prefill_bf16"].replace(B=3, T=1000, heads=3, rows_target=4099, d_hidden=256),
 ])
 def test_fused_hash_gather_matches_separate_kernels(shape):
     # forward from tokens computes the indices on chip (one hash + gather
