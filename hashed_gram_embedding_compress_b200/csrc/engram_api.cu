@@ -714,7 +714,12 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
         have_wide = true;
       }
       wide.w = wmaps[bn_index(pc.bn)];
-      if (kphase == 3) {
+      if (kphase == 2) {
+        // in place: per-warp reduce-adds of 32 rows x 64 columns
+        ProjMaps wr = wide;
+        if ((rc = make_map(h, &wr.out, out, hcols, R, 32, 64))) return rc;
+        CK(h, launch_proj_gate_wide(kphase, wr, g, pc.grid, st));
+      } else if (kphase == 3) {
         // v leaves through per-warp TMA stores of 32 x 32 fp32 boxes
         ProjMaps wv = wide;
         if ((rc = make_map(h, &wv.out, h->conv_v, g.d, R, 32, 32, true))) return rc;

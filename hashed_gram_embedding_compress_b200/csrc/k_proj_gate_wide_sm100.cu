@@ -29,8 +29,8 @@
 //               phase out is written over h in the slot and stored by TMA.
 // Phases: 0 = keys (partial sums), 1 = values (out = h + alpha v through the
 // h ring), 2 = values when out aliases h (the residual update in place): the
-// epilogue stages bf16(alpha v) and adds it into out with a TMA reduce-add,
-// so h never passes through shared memory; the sum is rounded once more
+// epilogue stages bf16(alpha v) for 64 columns at a time and adds it into out
+// with a TMA reduce-add, so h never passes through shared memory; the sum is rounded once more
 // (RN(h + RN(alpha v)) instead of RN(h + alpha v)); 3 = values for the short
 // convolution (Eq. 5): v in fp32 and its sum of squares per row and tile,
 // plus alpha; h is not read.
@@ -455,17 +455,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (valid) g.vv[(int64_t)n_blk * R + row] = svv;
       } else if (PHASE == 2) {
-        // out aliases h: add bf16(alpha v) into it with TMA reduce-add; each
-        // warp stages its 32 rows x 32 columns in one of two 2 KB buffers
-        // (the h ring is unused in this phase)
-        uint8_t* stage0 = hbuf + warp * 4096;
+        // out aliases h: add bf16(alpha v) into it with TMA reduce-add, two
+        // 32-column chunks per operation (32 rows x 64 columns, 4 KB,
+        // 128-byte swizzle); each warp stages in one of two buffers (the h
+        // ring is unused in this phase)
+        uint8_t* stage0 = hbuf + warp * 8192;
         int sbuf = 0;
-        auto add_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
-          tmem_wait32(v);
+        __syncwarp();
+        tmem_ld32_async(taddr + H_COLS, vb);  // chunk 1 (chunk 0 is on its way into va)
+#pragma unroll 1
+        for (int q = 0; q < NQ; q += 2) {
+          tmem_wait32(va);
+          tmem_wait32(vb);
           __syncwarp();
-          if (q + 1 < NQ) {
-            tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
-          } else {
+          if (q + 2 >= NQ) {
             tc_fence_before();  // last TMEM read done: release the accumulators
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
@@ -480,27 +483,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the buffer's previous reduce has finished reading it
             if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
             __syncwarp();
-            uint8_t* st = stage0 + sbuf * 2048;
+            uint8_t* st = stage0 + sbuf * 4096;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* v = c < 4 ? va : vb;
               uint32_t ow[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const int e = c * 8 + 2 * j;
+                const int e = (c & 3) * 8 + 2 * j;
                 const float2 o = f2_unpack(f2_mul(a2, f2_pack(v[e], v[e + 1])));
                 ow[j] = pack2(o.x, o.y);
               }
-              *reinterpret_cast<uint4*>(st + sw64_off(lane, c)) =
+              *reinterpret_cast<uint4*>(st + sw128_off(lane, c)) =
                   make_uint4(ow[0], ow[1], ow[2], ow[3]);
             }
             if (g.delta && valid) {
               float4* dp = reinterpret_cast<float4*>(g.delta + ((int64_t)row * M + mb) * d + n0 +
                                                      q * H_COLS);
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                dp[c] = make_float4(a * __uint_as_float(v[4 * c]), a * __uint_as_float(v[4 * c + 1]),
-                                    a * __uint_as_float(v[4 * c + 2]),
-                                    a * __uint_as_float(v[4 * c + 3]));
+              for (int c = 0; c < 16; ++c) {
+                const uint32_t* v = c < 8 ? va : vb;
+                const int e = (c & 7) * 4;
+                dp[c] = make_float4(a * __uint_as_float(v[e]), a * __uint_as_float(v[e + 1]),
+                                    a * __uint_as_float(v[e + 2]), a * __uint_as_float(v[e + 3]));
+              }
+            }
+            if (mb == M - 1 && q + 2 < NQ) {
+              // both register sets are staged: fetch the next two chunks now
+              __syncwarp();
+              tmem_ld32_async(taddr + (q + 2) * H_COLS, va);
+              tmem_ld32_async(taddr + (q + 3) * H_COLS, vb);
             }
             fence_async_smem();
             __syncwarp();
@@ -512,11 +524,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             sbuf ^= 1;
           }
-        };
-#pragma unroll 1
-        for (int q = 0; q < NQ; q += 2) {
-          add_chunk(q, va, vb);
-          add_chunk(q + 1, vb, va);
         }
       } else {
         int pending = -1;  // slot whose TMA store may still be reading it
