@@ -693,20 +693,29 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   }
   // Tensor maps are built for whichever kernel each phase uses (choose_proj):
   // 512 x 256 tiles on CTA pairs when the tile count fills every pair at least
-  // once, else single-CTA 128-row tiles of the widest N that fills the SMs.
+  // once, else 256 x 256 pair tiles or single-CTA 128-row tiles by cost.
   const int64_t hcols = (int64_t)g.M * g.d;
-  ProjMaps single, wide;
-  bool have_single = false, have_wide = false;
+  ProjMaps single, wide, pair;
+  bool have_single = false, have_wide = false, have_pair = false;
   int value_tile = 0;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
-    const ProjChoice pc = choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags);
+    const ProjChoice pc = choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv);
     if (phase == 0) g.key_tile = pc.key_tile;
     if (phase == 1) value_tile = pc.key_tile;
     // values: 3 = v for the short convolution; 2 = in place (out aliases h,
     // alpha v is added into out); 1 = out = h + alpha v
     const int kphase = phase == 0 ? 0 : conv ? 3 : out == hid ? 2 : 1;
-    if (pc.kind == ProjKernel::Wide) {
+    if (pc.kind == ProjKernel::Pair) {
+      if (!have_pair) {
+        if ((rc = make_map(h, &pair.e, h->e, h->d_mem, R, 128))) return rc;
+        if ((rc = make_map(h, &pair.h, hid, hcols, R, 128, 32))) return rc;
+        if ((rc = make_map(h, &pair.out, out, hcols, R, 32, 32))) return rc;  // per-warp boxes
+        have_pair = true;
+      }
+      pair.w = wmaps[bn_index(pc.bn)];  // each CTA of a pair loads 128 of the tile's 256 W rows
+      CK(h, launch_proj_gate_pair(kphase, pair, g, pc.grid, st));
+    } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
         if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;

@@ -139,40 +139,62 @@ cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, cons
 cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
                                   cudaStream_t stream);
 
+// 256 x 256 tiles on CTA pairs with two TMEM accumulators (few rows, many
+// columns); grid = 2 x pairs; key tiles of 128 columns (g.key_tile must be
+// 128 in phase 0).  Phases 0-2 as above.
+cudaError_t launch_proj_gate_pair(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
+                                  cudaStream_t stream);
+
 // The bf16 projection kernel of one phase (0 keys, 1 values) for R rows.
-enum class ProjKernel { Wide, Single };
+enum class ProjKernel { Wide, Pair, Single };
 struct ProjChoice {
   ProjKernel kind;
   int bn;        // W rows per TMA box (the tensor map of W to use)
   int grid;      // CTAs
   int key_tile;  // columns per partial-sum tile (phase 0)
 };
-// 512 x 256 CTA-pair tiles whenever there are enough of them for every pair,
-// else single-CTA 128-row tiles of the N that minimises rounds of tiles per
-// SM x operand bytes per tile (128 + N rows of K): the mainloop streams its
-// operands from L2 at a fixed rate per SM, so a second, partly filled round
-// of narrow tiles costs more than one round of wide ones.  Key tiles must not
-// straddle branches, so their width divides d.
-inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int flags) {
+// The kernel with the least estimated time: rounds of tiles per SM (or per
+// CTA pair) x the time of one tile.  A tile's mainloop streams its operands
+// from L2 at a fixed rate per SM, so its time is about the rows of K it
+// streams per CTA: 512 x 256 pair tiles 256 + 128, 256 x 256 pair tiles
+// 128 + 128, single-CTA 128 x N tiles 128 + N; the 512 x 256 tile holds its
+// accumulators through the gate epilogue (one TMEM buffer), which adds about
+// 30 % per tile, while the other two overlap it with the next tile (measured
+// on B200: 13.2 us mainloop + 3.1-4.3 us epilogue per 512 x 256 tile).  Key
+// tiles must not straddle branches, so their width divides d.  The value
+// phase of the short convolution (phase 3) has no 256 x 256 pair variant.
+inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int flags,
+                              bool conv = false) {
   const int n_total = phase == 0 ? M * d : d;
   const int pairs = sms / 2;
-  if (!(flags & ENGRAM_FLAG_NO_CTA_PAIRS) && n_total % 256 == 0 && d % 256 == 0 &&
-      (R + 511) / 512 * (n_total / 256) >= pairs)
-    return {ProjKernel::Wide, 128, 2 * pairs, 256};
+  const bool pairs_ok = !(flags & ENGRAM_FLAG_NO_CTA_PAIRS) && n_total % 256 == 0;
   const int64_t mblk = (R + 127) / 128;
-  int bn = 64;
-  int64_t best = -1;
+  ProjChoice best{ProjKernel::Single, 64, 1, 64};
+  int64_t best_cost = -1;
   for (int c : {256, 128, 64}) {
     if (n_total % c != 0 || d % c != 0) continue;
-    const int64_t rounds = (mblk * (n_total / c) + sms - 1) / sms;
-    const int64_t cost = rounds * (128 + c);
-    if (best < 0 || cost < best) {
-      best = cost;
-      bn = c;
+    const int64_t tiles = mblk * (n_total / c);
+    const int64_t cost = (tiles + sms - 1) / sms * (128 + c) * 10;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = {ProjKernel::Single, c, (int)(tiles < sms ? tiles : sms), c};
     }
   }
-  const int64_t tiles = mblk * (n_total / bn);
-  return {ProjKernel::Single, bn, (int)(tiles < sms ? tiles : sms), bn};
+  if (pairs_ok && d % 128 == 0 && !(phase == 1 && conv)) {
+    const int64_t tiles = (R + 255) / 256 * (n_total / 256);
+    const int64_t cost = (tiles + pairs - 1) / pairs * 256 * 10;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = {ProjKernel::Pair, 128, 2 * (int)(tiles < pairs ? tiles : pairs), 128};
+    }
+  }
+  if (pairs_ok && d % 256 == 0) {
+    const int64_t tiles = (R + 511) / 512 * (n_total / 256);
+    const int64_t cost = (tiles + pairs - 1) / pairs * 384 * 13;
+    if (cost <= best_cost)
+      best = {ProjKernel::Wide, 128, 2 * (int)(tiles < pairs ? tiles : pairs), 256};
+  }
+  return best;
 }
 
 }  // namespace engram

@@ -149,14 +149,25 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
   }
   // the same kernel choice as engram_forward (choose_proj)
   const int64_t hcols = (int64_t)M * d;
-  ProjMaps single, wide;
-  bool have_single = false, have_wide = false;
+  ProjMaps single, wide, pair;
+  bool have_single = false, have_wide = false, have_pair = false;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
     const ProjChoice pc = choose_proj(phase, rows, M, d, h->sms, h->cfg.flags);
     if (phase == 0) g.key_tile = pc.key_tile;
     const int kphase = (phase == 1 && out == hid) ? 2 : phase;
-    if (pc.kind == ProjKernel::Wide) {
+    if (pc.kind == ProjKernel::Pair) {
+      if (!have_pair) {
+        if ((rc = encode_map(h, &pair.e, e, h->d_mem, R, 128, 64)) ||
+            (rc = encode_map(h, &pair.h, hid, hcols, R, 128, 32)) ||
+            (rc = encode_map(h, &pair.out, out, hcols, R, 32, 32)))
+          return rc;
+        have_pair = true;
+      }
+      pair.w = wmaps[map_slot(pc.bn)];
+      if ((ce = launch_proj_gate_pair(kphase, pair, g, pc.grid, st)))
+        return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
+    } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if ((rc = encode_map(h, &wide.e, e, h->d_mem, R, 256, 64)) ||
             (rc = encode_map(h, &wide.h, hid, hcols, R, 256, 32)) ||

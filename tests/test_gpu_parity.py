@@ -159,9 +159,10 @@ def test_decode_multibranch():
 @pytest.mark.parametrize("R_B,R_T,flags", [(1, 40000, 0), (1, 20000, 0), (1, 20000, 1), (1, 10000, 0),
                                            (1, 2000, 0), (3, 5, 0), (1, 1, 0), (1, 37900, 0)])
 def test_tile_widths_and_ragged_rows(R_B, R_T, flags):
-    # d = 256, M = 2 lets the launcher pick CTA-pair 512 x 256 tiles or
-    # single-CTA 256-, 128- and 64-column tiles by row count (flags=1: no CTA
-    # pairs); 37900 rows end in a pair tile whose second CTA has no rows
+    # d = 256, M = 2 lets the launcher pick CTA-pair 512 x 256 tiles (40000,
+    # 37900 rows), CTA-pair 256 x 256 tiles (10000; values of 20000) or
+    # single-CTA tiles (2000 and fewer; flags=1: no CTA pairs) by cost;
+    # 37900 rows end in a 512-row tile whose second CTA has no rows
     sh = synth.SHAPES["prefill_bf16"].replace(B=R_B, T=R_T, rows_target=2053, d_hidden=256,
                                               branches=2)
     p = Problem(sh)
@@ -169,6 +170,19 @@ def test_tile_widths_and_ragged_rows(R_B, R_T, flags):
     idx = check_indices(p, m)
     out, a, dl = run_forward(p, m)
     check_rows(p, m, idx, p.sample_rows(64), out, a, dl)
+
+
+def test_pair_tiles_in_place():
+    # 10000 rows, d = 256, M = 2: keys and values on 256 x 256 CTA-pair tiles
+    # (two TMEM accumulators); in place the values are added by TMA reduce-add
+    sh = synth.SHAPES["prefill_bf16"].replace(B=1, T=10000, rows_target=2053, d_hidden=256,
+                                              branches=2)
+    p = Problem(sh)
+    m = p.engram()
+    idx = check_indices(p, m)
+    out, a, dl = run_forward(p, m)
+    check_rows(p, m, idx, p.sample_rows(48), out, a, dl)
+    check_in_place(p, m, out, dl)
 
 
 @pytest.mark.parametrize("flags", [0, 1])
