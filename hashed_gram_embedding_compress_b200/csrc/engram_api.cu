@@ -714,7 +714,10 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
         have_pair = true;
       }
       pair.w = wmaps[bn_index(pc.bn)];  // each CTA of a pair loads 128 of the tile's 256 W rows
-      CK(h, launch_proj_gate_pair(kphase, pair, g, pc.grid, st));
+      ProjMaps pm = pair;
+      // in place: per-warp reduce-adds of 32 rows x 64 columns
+      if (kphase == 2 && (rc = make_map(h, &pm.out, out, hcols, R, 32, 64))) return rc;
+      CK(h, launch_proj_gate_pair(kphase, pm, g, pc.grid, st));
     } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;

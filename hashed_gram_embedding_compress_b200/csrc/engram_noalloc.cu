@@ -165,7 +165,10 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
         have_pair = true;
       }
       pair.w = wmaps[map_slot(pc.bn)];
-      if ((ce = launch_proj_gate_pair(kphase, pair, g, pc.grid, st)))
+      ProjMaps pm = pair;
+      // in place: per-warp reduce-adds of 32 rows x 64 columns
+      if (kphase == 2 && (rc = encode_map(h, &pm.out, out, hcols, R, 32, 64))) return rc;
+      if ((ce = launch_proj_gate_pair(kphase, pm, g, pc.grid, st)))
         return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
     } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {

@@ -25,8 +25,9 @@
 //               column weights w_q * w_k (double-buffered with the tiles).
 // Phases: 0 = keys (partial sums per 128-column half tile), 1 = values
 // (out = h + alpha v, written over h in its ring slot and stored by TMA),
-// 2 = values when out aliases h (bf16(alpha v) staged per warp and added into
-// out with a TMA reduce-add: RN(h + RN(alpha v)) instead of RN(h + alpha v)).
+// 2 = values when out aliases h (bf16(alpha v) staged per warp, 32 x 64 at a
+// time, and added into out with a TMA reduce-add: RN(h + RN(alpha v))
+// instead of RN(h + alpha v)).
 // Every wait is bounded (kWaitLimitNs); on expiry the CTA raises its abort
 // flag and kDevErrTimeout, every role leaves its loop, and the pair leaves
 // together through a bounded handshake before TMEM is freed (cta_group::2).
@@ -60,7 +61,7 @@ constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * H_SLOTS + 4 + 2;
 constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * H_BYTES +
                         2 * W_BYTES + 8 * NUM_BARS + 16;
 static_assert(SMEM <= 232448, "shared memory budget");
-static_assert(kEpiWarps * 4096 <= H_SLOTS * H_BYTES, "in-place staging fits in the h ring");
+static_assert(kEpiWarps * 8192 <= H_SLOTS * H_BYTES, "in-place staging fits in the h ring");
 static_assert(NQ % 2 == 0, "chunks are processed in pairs");
 
 // Column offset, within the [R, M*d] view of h, of ring entry i of a tile
@@ -427,12 +428,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (valid)
           g.partials[(int64_t)(n_blk * 2 + colhalf) * R + row] = make_float4(skk, shk, shh, 0.f);
       } else if (PHASE == 2) {
-        // out aliases h: add bf16(alpha v) into it with TMA reduce-add; each
-        // warp stages its 32 rows x 32 columns in one of two 2 KB buffers
-        // (the h ring is unused in this phase)
-        uint8_t* stage0 = hbuf + warp * 4096;
-        auto add_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
-          next_chunk(q, v, vn);
+        // out aliases h: add bf16(alpha v) into it with TMA reduce-add, two
+        // 32-column chunks per operation (32 rows x 64 columns, 4 KB,
+        // 128-byte swizzle); each warp stages in one of two buffers (the h
+        // ring is unused in this phase)
+        uint8_t* stage0 = hbuf + warp * 8192;
+        __syncwarp();
+        tmem_ld32_async(taddr + H_COLS, vb);  // chunk 1 (chunk 0 is on its way into va)
+#pragma unroll 1
+        for (int q = 0; q < NQ; q += 2) {
+          tmem_wait32(va);
+          tmem_wait32(vb);
+          __syncwarp();
+          if (q + 2 >= NQ) {
+            tc_fence_before();  // last TMEM read done: release the accumulators
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar(b), 0));
+          }
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
             float a = 0.f;
@@ -443,27 +455,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the buffer's previous reduce has finished reading it
             if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
             __syncwarp();
-            uint8_t* st = stage0 + sbuf * 2048;
+            uint8_t* st = stage0 + sbuf * 4096;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* v = c < 4 ? va : vb;
               uint32_t ow[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const int e = c * 8 + 2 * j;
+                const int e = (c & 3) * 8 + 2 * j;
                 const float2 o = f2_unpack(f2_mul(a2, f2_pack(v[e], v[e + 1])));
                 ow[j] = pack2(o.x, o.y);
               }
-              *reinterpret_cast<uint4*>(st + sw64_off(lane, c)) =
+              *reinterpret_cast<uint4*>(st + sw128_off(lane, c)) =
                   make_uint4(ow[0], ow[1], ow[2], ow[3]);
             }
             if (g.delta && valid) {
               float4* dp = reinterpret_cast<float4*>(g.delta + ((int64_t)row * M + mb) * d + c0 +
                                                      q * H_COLS);
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                dp[c] = make_float4(a * __uint_as_float(v[4 * c]), a * __uint_as_float(v[4 * c + 1]),
-                                    a * __uint_as_float(v[4 * c + 2]),
-                                    a * __uint_as_float(v[4 * c + 3]));
+              for (int c = 0; c < 16; ++c) {
+                const uint32_t* v = c < 8 ? va : vb;
+                const int e = (c & 7) * 4;
+                dp[c] = make_float4(a * __uint_as_float(v[e]), a * __uint_as_float(v[e + 1]),
+                                    a * __uint_as_float(v[e + 2]), a * __uint_as_float(v[e + 3]));
+              }
+            }
+            if (mb == M - 1 && q + 2 < NQ) {
+              // both register sets are staged: fetch the next two chunks now
+              __syncwarp();
+              tmem_ld32_async(taddr + (q + 2) * H_COLS, va);
+              tmem_ld32_async(taddr + (q + 3) * H_COLS, vb);
             }
             fence_async_smem();
             __syncwarp();
@@ -476,11 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             sbuf ^= 1;
           }
-        };
-#pragma unroll 1
-        for (int q = 0; q < NQ; q += 2) {
-          add_chunk(q, va, vb);
-          add_chunk(q + 1, vb, va);
         }
       } else {
         auto value_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
