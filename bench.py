@@ -14,7 +14,7 @@ With N > 1 (torchrun), every rank runs its own replica on its own seeded batch
 (the forward has no cross-rank exchange); the time is the max over ranks.
 
 --impl reference times the CPU oracle (plain single-threaded C, fp64) on a
-bounded sample of the same workload: the reference arm of this build.
+bounded sample of the same workload: the reference arm.
 """
 from __future__ import annotations
 

@@ -72,7 +72,7 @@ extern "C" {
 #define ENGRAM_ERR_CUDA 3        /* a CUDA runtime call failed                     */
 #define ENGRAM_ERR_OOM 4         /* device or pinned allocation failed             */
 #define ENGRAM_ERR_TIMEOUT 5     /* a bounded device-side or prefetch wait expired */
-#define ENGRAM_ERR_UNSUPPORTED 6 /* valid request this build does not implement   */
+#define ENGRAM_ERR_UNSUPPORTED 6 /* valid request the library does not implement */
 #define ENGRAM_ERR_STATE 7       /* call out of order (e.g. forward before params) */
 
 typedef struct engram_handle engram_handle;
