@@ -69,6 +69,9 @@ def parse():
                     help="replay each step from a captured CUDA graph (launch-bound shapes)")
     ap.add_argument("--offload-gb", type=float, default=100.0,
                     help="offload workload: total size of the pinned host tables")
+    ap.add_argument("--hot-rows", type=int, default=0,
+                    help="offload workload: rows of the HBM hot-row cache in front of the host "
+                         "tables, chosen from 4 calibration batches of other tokens (0: none)")
     ap.add_argument("--rows-target", type=int, default=None,
                     help="smaller tables for profiling captures (same kernel shapes); "
                          "not the benchmarked workload")
@@ -505,6 +508,15 @@ def run_offload(args):
         toks = [synth.make_tokens(sh, synth.stream_seeds(sh, extra=100 + k)).to(dev)
                 for k in range(K + 2)]
         m.reserve(sh.rows_out)
+        t_hot = 0.0
+        if args.hot_rows > 0:
+            # calibration: the rows four other batches of the same token
+            # distribution address most often
+            calib = torch.cat([synth.make_tokens(sh, synth.stream_seeds(sh, extra=1000 + c))
+                               for c in range(4)]).to(dev)
+            t0 = time.time()
+            m.build_hot_cache(calib, args.hot_rows)
+            t_hot = time.time() - t0
         a_ = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
         b_ = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
         main = torch.cuda.current_stream()
@@ -538,8 +550,10 @@ def run_offload(args):
             f1.record(main)
             torch.cuda.synchronize()
             t_fw.append(f0.elapsed_time(f1))
+        hits = []
         for k in range(K):
             uniq.append(m.prefetch(toks[k], stream=side, want_count=True))
+            hits.append(m.prefetch_hot_hits())
             m.forward(toks[k], h, h, stream=main)
             torch.cuda.synchronize()
         t_pf, t_fw = statistics.median(t_pf[1:]), statistics.median(t_fw[1:])
@@ -566,7 +580,8 @@ def run_offload(args):
         if m.check_errors() != 0:
             raise RuntimeError("device error in the offload run")
         u = statistics.mean(uniq)
-        pcie_bytes = u * row_bytes
+        hot = statistics.mean(hits)
+        pcie_bytes = (u - hot) * row_bytes
         total_bytes = sum(t.numel() * 2 for t in tables)
         return {
             "metric": METRIC, "value": sh.rows_out / (t_pipe1 / 1e3), "unit": "tokens/s",
@@ -591,6 +606,13 @@ def run_offload(args):
                 "step_ms_n_gemm": t_pipe_n,
                 "loss_vs_hidden_prefetch": t_pipe_n / (n_hide * t_gemm + t_fw) - 1.0,
                 "host_setup_s": t_setup,
+                "hot_cache": {
+                    "rows": args.hot_rows,
+                    "gb": args.hot_rows * row_bytes / 1e9,
+                    "hits_per_step": hot,
+                    "hit_fraction": hot / u if u else 0.0,
+                    "build_s": t_hot,
+                },
             },
         }
     finally:

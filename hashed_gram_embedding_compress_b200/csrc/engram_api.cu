@@ -3,11 +3,14 @@
 // Engram forward ("Conditional Memory via Scalable Lookup", section 2).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <new>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "engram_handle.cuh"
 
@@ -190,6 +193,10 @@ int ensure_prefetch_scratch(engram_handle* h, int64_t rows) {
   for (int s = 0; s < h->S; ++s) bound[s] = entries;
   CK(h, cudaMemcpy(h->d_stage_bound, bound, h->S * sizeof(int64_t), cudaMemcpyHostToDevice));
   for (int i = 0; i < 2; ++i) {
+    if (!h->d_hot_hits[i]) {
+      CK(h, cudaMalloc(&h->d_hot_hits[i], sizeof(unsigned long long)));
+      CK(h, cudaMemset(h->d_hot_hits[i], 0, sizeof(unsigned long long)));
+    }
     CK(h, cudaMalloc(&h->d_count[i], sizeof(unsigned long long)));
     CK(h, cudaMalloc(&h->d_remap[i], (size_t)entries * sizeof(int64_t)));
     CK(h, cudaMalloc(&h->d_staging[i], (size_t)entries * row_bytes));
@@ -348,6 +355,10 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->d_vals);
   free_dev(h->d_uniq);
   free_dev(h->d_stage_bound);
+  free_dev(h->d_hot_keys);
+  free_dev(h->d_hot_slots);
+  free_dev(h->d_hot_rows);
+  for (int i = 0; i < 2; ++i) free_dev(h->d_hot_hits[i]);
   for (int i = 0; i < 2; ++i) {
     free_dev(h->d_count[i]);
     free_dev(h->d_remap[i]);
@@ -497,6 +508,107 @@ int engram_gather(engram_handle* h, const int64_t* idx, int64_t rows, void* e, v
   return ENGRAM_OK;
 }
 
+int engram_build_hot_cache(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T,
+                           int32_t t_begin, int64_t max_rows, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (h->cfg.table_location != ENGRAM_PINNED_HOST)
+    return fail(h, ENGRAM_ERR_STATE, "the hot-row cache fronts ENGRAM_PINNED_HOST tables");
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (max_rows < 0) return fail(h, ENGRAM_ERR_INVALID, "max_rows < 0");
+  int rc = check_shape(h, B, T, t_begin);
+  if (rc) return rc;
+  const int64_t rows = (int64_t)B * (T - t_begin);
+  if (rows > 0 && !tokens) return fail(h, ENGRAM_ERR_INVALID, "null tokens");
+  cudaStream_t st = (cudaStream_t)stream;
+  // no prefetch may still read the old cache
+  CK(h, cudaDeviceSynchronize());
+  free_dev(h->d_hot_keys);
+  free_dev(h->d_hot_slots);
+  free_dev(h->d_hot_rows);
+  h->n_hot = 0;
+  h->hot_cap = 0;
+  const int64_t entries = rows * h->S;
+  if (max_rows == 0 || entries == 0) return ENGRAM_OK;
+  uint64_t cap = 1;
+  while (cap < (uint64_t)(2 * entries)) cap <<= 1;
+  if (cap > (1ull << 31)) return fail(h, ENGRAM_ERR_INVALID, "calibration batch too large");
+  // 1. indices of the calibration tokens, 2. how often each row is addressed
+  int64_t* d_idx = nullptr;
+  unsigned long long *d_keys = nullptr, *d_counts = nullptr, *d_list = nullptr;
+  auto release = [&]() {
+    free_dev(d_idx);
+    free_dev(d_keys);
+    free_dev(d_counts);
+    free_dev(d_list);
+  };
+  auto body = [&]() -> int {
+    CK(h, cudaMalloc(&d_idx, (size_t)entries * sizeof(int64_t)));
+    CK(h, cudaMalloc(&d_keys, cap * sizeof(unsigned long long)));
+    CK(h, cudaMalloc(&d_counts, cap * sizeof(unsigned long long)));
+    CK(h, launch_hash(hash_args(h, tokens, B, T, t_begin, d_idx), st));
+    CK(h, launch_count_rows(d_idx, entries, h->S, d_keys, d_counts, (uint32_t)cap, h->sms, st));
+    h->launches += 3;
+    std::vector<unsigned long long> keys(cap), counts(cap);
+    CK(h, cudaMemcpyAsync(keys.data(), d_keys, cap * sizeof(unsigned long long),
+                          cudaMemcpyDeviceToHost, st));
+    CK(h, cudaMemcpyAsync(counts.data(), d_counts, cap * sizeof(unsigned long long),
+                          cudaMemcpyDeviceToHost, st));
+    CK(h, cudaStreamSynchronize(st));
+    // 3. the max_rows most frequent rows; ties go to the lower (table, row)
+    std::vector<std::pair<unsigned long long, unsigned long long>> seen;  // (count, key)
+    for (uint64_t i = 0; i < cap; ++i)
+      if (keys[i] != ~0ull) seen.emplace_back(counts[i], keys[i]);
+    const int64_t n = std::min<int64_t>(max_rows, (int64_t)seen.size());
+    auto more_frequent = [](const std::pair<unsigned long long, unsigned long long>& x,
+                            const std::pair<unsigned long long, unsigned long long>& y) {
+      return x.first != y.first ? x.first > y.first : x.second < y.second;
+    };
+    std::partial_sort(seen.begin(), seen.begin() + n, seen.end(), more_frequent);
+    std::vector<unsigned long long> list((size_t)n);
+    for (int64_t i = 0; i < n; ++i) list[i] = seen[i].second;
+    // 4. the cache: a lookup table (slot = rank) and the rows, copied once
+    uint64_t hcap = 1;
+    while (hcap < (uint64_t)(2 * n)) hcap <<= 1;
+    const size_t row_bytes = (size_t)h->cfg.d_head * h->elt;
+    CK(h, cudaMalloc(&d_list, (size_t)n * sizeof(unsigned long long)));
+    CK(h, cudaMemcpyAsync(d_list, list.data(), (size_t)n * sizeof(unsigned long long),
+                          cudaMemcpyHostToDevice, st));
+    CK(h, cudaMalloc(&h->d_hot_keys, hcap * sizeof(unsigned long long)));
+    CK(h, cudaMalloc(&h->d_hot_slots, hcap * sizeof(int32_t)));
+    CK(h, cudaMalloc(&h->d_hot_rows, (size_t)n * row_bytes));
+    CK(h, launch_fill_hot_cache(d_list, n, h->d_hot_keys, h->d_hot_slots, (uint32_t)hcap,
+                                (const void* const*)h->d_tables, (int32_t)row_bytes,
+                                h->d_hot_rows, h->sms, st));
+    h->launches += 3;
+    CK(h, cudaStreamSynchronize(st));
+    h->n_hot = n;
+    h->hot_cap = (uint32_t)hcap;
+    return ENGRAM_OK;
+  };
+  rc = body();
+  release();
+  if (rc != ENGRAM_OK) {
+    free_dev(h->d_hot_keys);
+    free_dev(h->d_hot_slots);
+    free_dev(h->d_hot_rows);
+    h->n_hot = 0;
+    h->hot_cap = 0;
+  }
+  return rc;
+}
+
+int engram_prefetch_hot_hits(engram_handle* h, int64_t* hits) {
+  if (!h || !hits) return ENGRAM_ERR_INVALID;
+  *hits = 0;
+  if (h->n_prefetch == 0 || !h->d_hot_hits[(h->n_prefetch - 1) & 1]) return ENGRAM_OK;
+  CK(h, cudaDeviceSynchronize());
+  unsigned long long v = 0;
+  CK(h, cudaMemcpy(&v, h->d_hot_hits[(h->n_prefetch - 1) & 1], sizeof(v),
+                   cudaMemcpyDeviceToHost));
+  *hits = (int64_t)v;
+  return ENGRAM_OK;
+}
+
 int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T, int32_t t_begin,
                     void* side_stream, int64_t* unique_rows) {
   if (!h) return ENGRAM_ERR_INVALID;
@@ -535,6 +647,13 @@ int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t 
   a.staging = h->d_staging[slot];
   a.sms = h->sms;
   a.fetch_blocks = h->sms * 8;
+  if (h->n_hot > 0) {
+    a.hot_keys = h->d_hot_keys;
+    a.hot_slots = h->d_hot_slots;
+    a.hot_cap = h->hot_cap;
+    a.hot_rows = h->d_hot_rows;
+  }
+  a.hot_hits = h->d_hot_hits[slot];
   CK(h, launch_prefetch(a, st));
   h->launches += rows > 0 ? 5 : 1;
   CK(h, cudaEventRecord(h->ev_ready[slot], st));

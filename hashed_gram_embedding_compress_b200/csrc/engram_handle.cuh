@@ -64,6 +64,14 @@ struct engram_handle {
   cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
   int64_t pf_rows[2] = {0, 0};
   uint64_t n_prefetch = 0, n_consumed = 0;
+  unsigned long long* d_hot_hits[2] = {nullptr, nullptr};  // per prefetch slot
+
+  // hot-row cache in HBM in front of the host tables (engram_build_hot_cache)
+  int64_t n_hot = 0;
+  uint32_t hot_cap = 0;
+  unsigned long long* d_hot_keys = nullptr;  // [hot_cap] set of (s << 40 | z)
+  int32_t* d_hot_slots = nullptr;            // [hot_cap] cache slot per bucket
+  void* d_hot_rows = nullptr;                // [n_hot, row_bytes]
 
   // instrumentation
   int64_t launches = 0;

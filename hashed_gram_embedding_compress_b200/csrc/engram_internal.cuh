@@ -100,7 +100,28 @@ struct PrefetchArgs {
   void* staging;                // [rows*S, row_bytes] device
   int sms;
   int fetch_blocks;             // grid cap of the PCIe copy kernel
+  // hot-row cache in HBM (null hot_keys: none): rows found there are copied
+  // from HBM instead of over PCIe
+  const unsigned long long* hot_keys;  // [hot_cap] open-addressing set of (s << 40 | z)
+  const int32_t* hot_slots;     // [hot_cap] cache slot of each occupied bucket
+  uint32_t hot_cap;             // power of two
+  const void* hot_rows;         // [cached rows, row_bytes]
+  unsigned long long* hot_hits; // distinct rows of this prefetch served from the cache
 };
+
+// Hot-row cache building blocks (host-resident tables).
+// Count how often each (s, z) of idx [n / S, S] is addressed: keys/counts are
+// an open-addressing table of cap (a power of two >= 2 n) buckets.
+cudaError_t launch_count_rows(const int64_t* idx, int64_t n, int32_t S, unsigned long long* keys,
+                              unsigned long long* counts, uint32_t cap, int sms,
+                              cudaStream_t stream);
+// Insert the n chosen keys (cache slot = list position) into the cache's
+// lookup table (hot_cap buckets) and copy their rows from the host tables
+// into rows [n, row_bytes].
+cudaError_t launch_fill_hot_cache(const unsigned long long* list, int64_t n,
+                                  unsigned long long* hot_keys, int32_t* hot_slots,
+                                  uint32_t hot_cap, const void* const* tables, int32_t row_bytes,
+                                  void* rows, int sms, cudaStream_t stream);
 
 // Launchers (all asynchronous on `stream`; return the launch error).
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);

@@ -18,6 +18,12 @@
 //      over PCIe, 16 bytes per thread, whole rows per run of threads) into
 //      the HBM staging buffer.
 // The forward then gathers from the staging buffer with the remapped indices.
+//
+// Hot-row cache (the paper's cache hierarchy over a Zipfian access pattern,
+// section 2.5): engram_build_hot_cache counts the rows calibration tokens
+// address (count_kernel), keeps the most frequent ones in HBM
+// (hot_insert_kernel, hot_copy_kernel), and step 5 then copies a cached row
+// from HBM instead of over PCIe.
 #include "engram_internal.cuh"
 
 namespace engram {
@@ -39,9 +45,9 @@ __global__ void clear_kernel(unsigned long long* keys, int32_t* vals, uint32_t c
                              unsigned long long* count) {
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < cap; i += gridDim.x * blockDim.x) {
     keys[i] = kEmpty;
-    vals[i] = -1;
+    if (vals) vals[i] = -1;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *count = 0;
+  if (count && blockIdx.x == 0 && threadIdx.x == 0) *count = 0;
 }
 
 // Linear probing; the set holds at least twice as many buckets as inserted
@@ -102,19 +108,96 @@ __device__ __forceinline__ uint4 ld_host_16(const void* p) {
   return v;
 }
 
+// Cache slot of key in the hot-row table, or -1.
+__device__ __forceinline__ int32_t hot_lookup(const unsigned long long* keys, const int32_t* slots,
+                                              uint32_t mask, unsigned long long key) {
+  uint32_t b = mix_bucket(key, mask);
+  for (uint32_t probe = 0; probe <= mask; ++probe) {
+    const unsigned long long k = keys[b];
+    if (k == key) return slots[b];
+    if (k == kEmpty) return -1;
+    b = (b + 1) & mask;
+  }
+  return -1;
+}
+
 // One thread per 16-byte chunk of a distinct row; threads past the distinct
-// count (known only on the device) return at once.
-__global__ void fetch_kernel(const void* const* tables, const int2* uniq,
-                             const unsigned long long* count, int32_t row_bytes, char* staging) {
-  const int cpr = row_bytes >> 4;
-  const int64_t total = (int64_t)(*count) * cpr;
+// count (known only on the device) return at once.  A row held in the hot
+// cache is copied from HBM, any other over PCIe.
+__global__ void fetch_kernel(PrefetchArgs a) {
+  const int cpr = a.row_bytes >> 4;
+  const int64_t total = (int64_t)(*a.count) * cpr;
+  char* staging = (char*)a.staging;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t u = i / cpr;
     const int c = (int)(i - u * cpr);
-    const int2 sz = uniq[u];
-    const char* src = (const char*)tables[sz.x] + (int64_t)sz.y * row_bytes + c * 16;
-    *reinterpret_cast<uint4*>(staging + u * row_bytes + c * 16) = ld_host_16(src);
+    const int2 sz = a.uniq[u];
+    int32_t hot = -1;
+    if (a.hot_keys) {
+      const unsigned long long key = ((unsigned long long)sz.x << 40) | (unsigned long long)sz.y;
+      hot = hot_lookup(a.hot_keys, a.hot_slots, a.hot_cap - 1, key);
+      if (hot >= 0 && c == 0) atomicAdd(a.hot_hits, 1ull);
+    }
+    uint4 v;
+    if (hot >= 0)
+      v = __ldg(reinterpret_cast<const uint4*>((const char*)a.hot_rows +
+                                               (int64_t)hot * a.row_bytes + c * 16));
+    else
+      v = ld_host_16((const char*)a.tables[sz.x] + (int64_t)sz.y * a.row_bytes + c * 16);
+    *reinterpret_cast<uint4*>(staging + u * a.row_bytes + c * 16) = v;
+  }
+}
+
+// Frequency count for the hot-row cache: insert like insert_kernel, then
+// count the key's bucket.
+__global__ void count_kernel(const int64_t* idx, int64_t n, int32_t S, unsigned long long* keys,
+                             unsigned long long* counts, uint32_t mask) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int s = (int)(i % S);
+    const unsigned long long key = ((unsigned long long)s << 40) | (unsigned long long)idx[i];
+    uint32_t b = mix_bucket(key, mask);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+      const unsigned long long prev = atomicCAS(keys + b, kEmpty, key);
+      if (prev == kEmpty || prev == key) {
+        atomicAdd(counts + b, 1ull);
+        break;
+      }
+      b = (b + 1) & mask;
+    }
+  }
+}
+
+__global__ void hot_insert_kernel(const unsigned long long* list, int64_t n,
+                                  unsigned long long* keys, int32_t* slots, uint32_t mask) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const unsigned long long key = list[i];
+    uint32_t b = mix_bucket(key, mask);
+    for (uint32_t probe = 0; probe <= mask; ++probe) {
+      const unsigned long long prev = atomicCAS(keys + b, kEmpty, key);
+      if (prev == kEmpty || prev == key) {
+        slots[b] = (int32_t)i;
+        break;
+      }
+      b = (b + 1) & mask;
+    }
+  }
+}
+
+__global__ void hot_copy_kernel(const unsigned long long* list, int64_t n,
+                                const void* const* tables, int32_t row_bytes, char* rows) {
+  const int cpr = row_bytes >> 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n * cpr;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = i / cpr;
+    const int c = (int)(i - u * cpr);
+    const unsigned long long key = list[u];
+    const int s = (int)(key >> 40);
+    const int64_t z = (int64_t)(key & 0xFFFFFFFFFFull);
+    *reinterpret_cast<uint4*>(rows + u * row_bytes + c * 16) =
+        ld_host_16((const char*)tables[s] + z * row_bytes + c * 16);
   }
 }
 
@@ -131,6 +214,10 @@ cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream) {
   const int cap_blocks = a.sms * 16;
   const int64_t entries = a.rows * a.S;
   clear_kernel<<<blocks_for(a.cap, n, cap_blocks), n, 0, stream>>>(a.keys, a.vals, a.cap, a.count);
+  if (a.hot_hits) {
+    cudaError_t e = cudaMemsetAsync(a.hot_hits, 0, sizeof(unsigned long long), stream);
+    if (e != cudaSuccess) return e;
+  }
   if (entries > 0) {
     insert_kernel<<<blocks_for(entries, n, cap_blocks), n, 0, stream>>>(a.idx, entries, a.S,
                                                                        a.keys, a.cap - 1);
@@ -139,8 +226,34 @@ cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream) {
     remap_kernel<<<blocks_for(entries, n, cap_blocks), n, 0, stream>>>(
         a.idx, entries, a.S, a.keys, a.vals, a.cap - 1, a.remapped);
     // at most `entries` distinct rows
-    fetch_kernel<<<blocks_for(entries * (a.row_bytes >> 4), n, a.fetch_blocks), n, 0, stream>>>(
-        a.tables, a.uniq, a.count, a.row_bytes, (char*)a.staging);
+    fetch_kernel<<<blocks_for(entries * (a.row_bytes >> 4), n, a.fetch_blocks), n, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_count_rows(const int64_t* idx, int64_t n, int32_t S, unsigned long long* keys,
+                              unsigned long long* counts, uint32_t cap, int sms,
+                              cudaStream_t stream) {
+  const int t = 256;
+  clear_kernel<<<blocks_for(cap, t, sms * 16), t, 0, stream>>>(keys, nullptr, cap, nullptr);
+  cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)cap * sizeof(unsigned long long), stream);
+  if (e != cudaSuccess) return e;
+  if (n > 0) count_kernel<<<blocks_for(n, t, sms * 16), t, 0, stream>>>(idx, n, S, keys, counts, cap - 1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_hot_cache(const unsigned long long* list, int64_t n,
+                                  unsigned long long* hot_keys, int32_t* hot_slots,
+                                  uint32_t hot_cap, const void* const* tables, int32_t row_bytes,
+                                  void* rows, int sms, cudaStream_t stream) {
+  const int t = 256;
+  clear_kernel<<<blocks_for(hot_cap, t, sms * 16), t, 0, stream>>>(hot_keys, hot_slots, hot_cap,
+                                                                 nullptr);
+  if (n > 0) {
+    hot_insert_kernel<<<blocks_for(n, t, sms * 16), t, 0, stream>>>(list, n, hot_keys, hot_slots,
+                                                                   hot_cap - 1);
+    hot_copy_kernel<<<blocks_for(n * (row_bytes >> 4), t, sms * 8), t, 0, stream>>>(
+        list, n, tables, row_bytes, (char*)rows);
   }
   return cudaGetLastError();
 }

@@ -29,7 +29,8 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_set_params", "engram_reserve", "engram_get_hash_params", "engram_hash",
            "engram_gather", "engram_forward", "engram_prefetch", "engram_check_errors",
            "engram_profile_next_forward", "engram_kernel_launches",
-           "engram_project_gate_noalloc", "engram_selftest_timeout", "engram_set_short_conv")
+           "engram_project_gate_noalloc", "engram_selftest_timeout", "engram_set_short_conv",
+           "engram_build_hot_cache", "engram_prefetch_hot_hits")
 
 
 class engram_config(ctypes.Structure):
@@ -66,6 +67,8 @@ def _load():
         "engram_set_params": ([H, P, P, P, P, P], ctypes.c_int),
         "engram_reserve": ([H, i64], ctypes.c_int),
         "engram_set_short_conv": ([H, P, P, i32, i32, P], ctypes.c_int),
+        "engram_build_hot_cache": ([H, P, i32, i32, i32, i64, P], ctypes.c_int),
+        "engram_prefetch_hot_hits": ([H, P], ctypes.c_int),
         "engram_get_hash_params": ([H, P, P], ctypes.c_int),
         "engram_hash": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
@@ -201,6 +204,18 @@ class Engram:
         self._check(lib.engram_prefetch(self._h, _ptr(tokens), B, T, t_begin, _stream_ptr(stream),
                                         ctypes.byref(n) if want_count else None))
         return n.value if want_count else None
+
+    def build_hot_cache(self, tokens, max_rows: int, t_begin=0, stream=None):
+        """Keep the max_rows rows the calibration tokens address most often in HBM."""
+        B, T = tokens.shape
+        self._check(lib.engram_build_hot_cache(self._h, _ptr(tokens), B, T, t_begin, max_rows,
+                                               _stream_ptr(stream)))
+
+    def prefetch_hot_hits(self) -> int:
+        """Distinct rows of the last prefetch served from the hot-row cache."""
+        n = ctypes.c_int64(0)
+        self._check(lib.engram_prefetch_hot_hits(self._h, ctypes.byref(n)))
+        return n.value
 
     def profile_next_forward(self, events):
         """Record 5 or 6 CUDA events inside the next forward (stage boundaries)."""

@@ -258,6 +258,29 @@ ENGRAM_API int engram_prefetch(engram_handle *h, const int32_t *tokens, int32_t 
                     int32_t t_begin, void *side_stream, int64_t *unique_rows);
 
 /*
+ * Hot-row cache for host-resident tables (section 2.5: the accesses follow
+ * the Zipfian n-gram statistics, so a small set of rows carries much of the
+ * traffic).  Hashes the calibration tokens on `stream`, counts how often each
+ * (table, row) is addressed, and copies the max_rows most frequent rows (ties:
+ * lower table slot, then lower row) once from the host tables into HBM.
+ * Every later engram_prefetch copies the distinct rows it needs from this
+ * cache when they are there and over PCIe otherwise; results are unchanged.
+ * max_rows = 0 drops the cache.  Waits for all device work first (no prefetch
+ * may read the old cache) and synchronises `stream` before returning.
+ * HBM used: max_rows x d_head x element size, plus 12 bytes x 2 max_rows of
+ * lookup table, plus a temporary 16 bytes x 2 B (T - t_begin) S.
+ * ENGRAM_PINNED_HOST handles only.  Errors: _INVALID, _STATE, _OOM, _CUDA.
+ */
+ENGRAM_API int engram_build_hot_cache(engram_handle *h, const int32_t *tokens, int32_t B,
+                                      int32_t T, int32_t t_begin, int64_t max_rows, void *stream);
+
+/*
+ * Distinct rows of the most recent engram_prefetch that were copied from the
+ * hot-row cache instead of over PCIe (host int64).  Waits for all device work.
+ */
+ENGRAM_API int engram_prefetch_hot_hits(engram_handle *h, int64_t *hits);
+
+/*
  * Synchronise `stream`, then read and clear the handle's device error word.
  * Returns ENGRAM_OK, ENGRAM_ERR_BOUNDS (a token or index out of range was
  * replaced) or ENGRAM_ERR_TIMEOUT (a kernel's bounded wait expired and the

@@ -84,3 +84,55 @@ def test_double_buffered_prefetch_and_call_order():
         torch.cuda.synchronize()
         assert torch.equal(out, ref)
     assert m.check_errors() == 0
+
+
+def _expected_hits(p, calib_z, step_z, max_rows):
+    """Hot rows: the max_rows (table, row) keys the calibration indices address
+    most often (ties: lower table, then lower row); hits: the step's distinct
+    keys among them.  Computed from the oracle's indices alone."""
+    S = calib_z.shape[1]
+    keys = (np.arange(S, dtype=np.int64)[None, :] << 40) | calib_z
+    uk, cnt = np.unique(keys.ravel(), return_counts=True)
+    order = np.lexsort((uk, -cnt))  # count descending, then key ascending
+    hot = set(uk[order[:max_rows]].tolist())
+    step = np.unique(((np.arange(S, dtype=np.int64)[None, :] << 40) | step_z).ravel())
+    return sum(1 for k in step.tolist() if k in hot)
+
+
+@pytest.mark.parametrize("max_rows", [1000, 10 ** 7])
+def test_hot_row_cache_serves_rows_and_keeps_results(max_rows):
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    import oracle
+    sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=1200, rows_target=1 << 17, d_hidden=256)
+    p, _ = _pair(sh)
+    m0 = p.engram()
+    m1 = p.engram()
+    side = torch.cuda.Stream()
+    # calibrate on other tokens of the same distribution (the step's own
+    # indices would overstate the hits)
+    calib = synth.make_tokens(sh, synth.stream_seeds(sh, extra=7))
+    m1.build_hot_cache(calib.cuda(), max_rows)
+    tok = p.tokens.cuda()
+    outs = []
+    for m in (m0, m1):
+        m.prefetch(tok, stream=side)
+        out = torch.empty_like(p.h)
+        m.forward(tok, p.h, out)
+        torch.cuda.synchronize()
+        assert m.check_errors() == 0
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1])  # the cached rows are the same bytes
+    _, calib_z, _, _ = oracle.forward_indices(calib.numpy(), p.comp_map.numpy(), sh.cvocab,
+                                              sh.orders, sh.heads, p.hash_seed, sh.rows_target)
+    want = _expected_hits(p, calib_z, p.z, max_rows)
+    assert m1.prefetch_hot_hits() == want and want > 0
+    assert m0.prefetch_hot_hits() == 0
+
+
+def test_hot_row_cache_needs_host_tables():
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    p = Problem(synth.SHAPES["tiny_f32"])
+    m = p.engram()
+    with pytest.raises(eg.EngramError) as ei:
+        m.build_hot_cache(p.tokens.cuda(), 10)
+    assert ei.value.code == eg.ENGRAM_ERR_STATE
