@@ -23,7 +23,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "engram_oracle.c")
 _LIB = os.path.join(_HERE, "_engram_oracle.so")
 
-F32, BF16 = 0, 1
+F32, BF16, F64 = 0, 1, 2
 _lib = None
 
 
@@ -71,6 +71,19 @@ def lib():
         L.eo_short_conv.restype = None
         L.eo_add_round.argtypes = [P, i32, i64, P, P]
         L.eo_add_round.restype = None
+        L.eo_project_gate_mixed.argtypes = [P, i32, i64, i32, P, P, P, P, i32, i32, f64, P,
+                                            i32, P, P, P, P, P, P]
+        L.eo_project_gate_mixed.restype = None
+        L.eo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.eo_e4m3_decode.restype = f64
+        L.eo_e4m3_encode.argtypes = [f64]
+        L.eo_e4m3_encode.restype = ctypes.c_uint8
+        L.eo_e4m3_scale_exp.argtypes = [f64]
+        L.eo_e4m3_scale_exp.restype = i32
+        L.eo_quantize_e4m3_rows.argtypes = [P, i32, i64, i32, P, P]
+        L.eo_quantize_e4m3_rows.restype = None
+        L.eo_dequantize_e4m3_rows.argtypes = [P, P, i64, i32, P]
+        L.eo_dequantize_e4m3_rows.restype = None
         _lib = L
     return _lib
 
@@ -198,6 +211,94 @@ def project_gate(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: bool = 
                           _p(h), _p(alpha), _p(delta) if delta is not None else None, _p(out),
                           _p(kb), _p(vb), _p(hb))
     return alpha, delta, out
+
+
+# ------------------------------------------------------------ FP8 projection
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Values (double) of E4M3 codes (NaN for S.1111.111)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    L = lib()
+    return np.array([L.eo_e4m3_decode(int(v)) for v in c.ravel()]).reshape(c.shape)
+
+
+def e4m3_encode(y: np.ndarray) -> np.ndarray:
+    """E4M3 codes of y: nearest, ties to even, saturating at +-448."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    L = lib()
+    return np.array([L.eo_e4m3_encode(float(v)) for v in y.ravel()],
+                    dtype=np.uint8).reshape(y.shape)
+
+
+def e4m3_scale_exp(amax: float) -> int:
+    """Smallest E with amax <= 448 * 2^E (0 for amax = 0)."""
+    return int(lib().eo_e4m3_scale_exp(float(amax)))
+
+
+def quantize_e4m3_rows(x: np.ndarray):
+    """(codes uint8 [rows, cols], scales float32 [rows]) of x [rows, cols]
+    (float32, or uint16 bf16 bit patterns): one power-of-two scale per row."""
+    x = np.ascontiguousarray(x)
+    dtype = F32 if x.dtype == np.float32 else BF16
+    assert x.dtype in (np.float32, np.uint16) and x.ndim == 2
+    rows, cols = x.shape
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    scales = np.empty(rows, dtype=np.float32)
+    lib().eo_quantize_e4m3_rows(_p(x), dtype, rows, cols, _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequantize_e4m3_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    rows, cols = codes.shape
+    y = np.empty((rows, cols), dtype=np.float64)
+    lib().eo_dequantize_e4m3_rows(_p(codes), _p(scales), rows, cols, _p(y))
+    return y
+
+
+def project_gate_mixed(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: bool = True):
+    """project_gate with e, w_k, w_v in double and h in its own dtype."""
+    e = np.ascontiguousarray(e, dtype=np.float64)
+    rows, dm = e.shape
+    M, d, dm2 = w_k.shape
+    assert dm2 == dm and w_v.shape == (d, dm) and h.shape == (rows, M, d)
+    w_k = np.ascontiguousarray(w_k, dtype=np.float64)
+    w_v = np.ascontiguousarray(w_v, dtype=np.float64)
+    h = np.ascontiguousarray(h)
+    hdtype = F32 if h.dtype == np.float32 else BF16
+    nq = np.ascontiguousarray(norm_q, dtype=np.float32)
+    nk = np.ascontiguousarray(norm_k, dtype=np.float32)
+    alpha = np.empty((rows, M), dtype=np.float64)
+    delta = np.empty((rows, M, d), dtype=np.float64) if want_delta else None
+    out = np.empty_like(h)
+    kb = np.empty(M * d, dtype=np.float64)
+    vb = np.empty(d, dtype=np.float64)
+    hb = np.empty(d, dtype=np.float64)
+    lib().eo_project_gate_mixed(_p(e), F64, rows, dm, _p(w_k), _p(w_v), _p(nq), _p(nk), M, d,
+                                eps, _p(h), hdtype, _p(alpha),
+                                _p(delta) if delta is not None else None, _p(out),
+                                _p(kb), _p(vb), _p(hb))
+    return alpha, delta, out
+
+
+def quantize_weights_e4m3(w_k: np.ndarray, w_v: np.ndarray):
+    """Dequantised W_K [M, d, d_mem] and W_V [d, d_mem]: one scale per output
+    channel (row of W)."""
+    M, d, dm = w_k.shape
+    wk = dequantize_e4m3_rows(*quantize_e4m3_rows(np.ascontiguousarray(w_k).reshape(M * d, dm)))
+    wv = dequantize_e4m3_rows(*quantize_e4m3_rows(np.ascontiguousarray(w_v)))
+    return wk.reshape(M, d, dm), wv
+
+
+def project_gate_fp8(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: bool = True,
+                     weights=None):
+    """The FP8 form of project_gate (section 2.4): e quantised per row, W per
+    output channel, then Eq. (3)-(4)/(6) on the dequantised operands.
+    `weights` may hold quantize_weights_e4m3's result to skip recomputing it."""
+    ehat = dequantize_e4m3_rows(*quantize_e4m3_rows(e))
+    wk, wv = weights if weights is not None else quantize_weights_e4m3(w_k, w_v)
+    return project_gate_mixed(ehat, wk, wv, norm_q, norm_k, h, eps, want_delta)
 
 
 # ---------------------------------------------------------------- short conv

@@ -38,6 +38,9 @@
  *  - RMSNorm(x) = x / sqrt(mean(x^2) + eps) * w, with a learnable weight w
  *    per branch for the query and for the key; the key is normalised after
  *    the projection (Eq. 4), the scale is 1/sqrt(d) with d the hidden size.
+ *  - the FP8 form of the projection (section 2.4) quantises e and W to E4M3
+ *    with a power-of-two scale per row; its reading is stated beside
+ *    eo_e4m3_encode below.
  *  - ShortConv (Eq. 5) is zero-initialised in the paper (Table 5), so at
  *    initialisation its output equals the gated value and out = h + alpha v.
  *    With trained (non-zero) weights it is the last step below.
@@ -64,6 +67,7 @@
 
 #define EO_F32 0
 #define EO_BF16 1
+#define EO_F64 2 /* double operands: the dequantised FP8 values below */
 
 /* ---------------------------------------------------------------- SplitMix64 */
 
@@ -180,6 +184,7 @@ void eo_gather(const void *const *tables, int32_t elem_bytes, int32_t d_head,
 
 static double eo_load(const void *p, int32_t dtype, int64_t i)
 {
+    if (dtype == EO_F64) return ((const double *)p)[i];
     if (dtype == EO_F32) return (double)((const float *)p)[i];
     {
         uint32_t u = (uint32_t)((const uint16_t *)p)[i] << 16;
@@ -187,6 +192,11 @@ static double eo_load(const void *p, int32_t dtype, int64_t i)
         memcpy(&f, &u, 4);
         return (double)f;
     }
+}
+
+static size_t eo_elem_bytes(int32_t dtype)
+{
+    return dtype == EO_F64 ? 8 : dtype == EO_F32 ? 4 : 2;
 }
 
 static uint16_t eo_bf16_rne(double v)
@@ -244,43 +254,149 @@ double eo_gate(const double *h, const double *k, const float *wq, const float *w
 /*
  * Projection, gate and output for `rows` rows whose memory vectors e are given
  * (Eq. 3, Eq. 4 / Eq. 6, gated residual).
- *   e     [rows, d_mem]          dtype
- *   w_k   [M, d, d_mem]          dtype   (one key projection per branch)
- *   w_v   [d, d_mem]             dtype   (shared value projection)
+ *   e     [rows, d_mem]          wdtype
+ *   w_k   [M, d, d_mem]          wdtype  (one key projection per branch)
+ *   w_v   [d, d_mem]             wdtype  (shared value projection)
  *   wq,wk [M, d]                 float   (RMSNorm weights of query and key)
- *   h     [rows, M, d]           dtype
+ *   h     [rows, M, d]           hdtype  (fp32 or bf16)
  *   alpha [rows, M]              double  (out)
  *   delta [rows, M, d]           double  (out; alpha * v; may be NULL)
- *   out   [rows, M, d]           dtype   (out; h + alpha * v rounded to dtype)
+ *   out   [rows, M, d]           hdtype  (out; h + alpha * v rounded to hdtype)
  * Scratch: kbuf [M * d], vbuf [d], hbuf [d] doubles supplied by the caller.
  */
-void eo_project_gate(const void *e, int32_t dtype, int64_t rows, int32_t d_mem,
-                     const void *w_k, const void *w_v, const float *wq, const float *wk,
-                     int32_t M, int32_t d, double eps, const void *h,
-                     double *alpha, double *delta, void *out,
-                     double *kbuf, double *vbuf, double *hbuf)
+void eo_project_gate_mixed(const void *e, int32_t wdtype, int64_t rows, int32_t d_mem,
+                           const void *w_k, const void *w_v, const float *wq, const float *wk,
+                           int32_t M, int32_t d, double eps, const void *h, int32_t hdtype,
+                           double *alpha, double *delta, void *out,
+                           double *kbuf, double *vbuf, double *hbuf)
 {
     int64_t r;
     int32_t m, i;
     for (r = 0; r < rows; ++r) {
-        const char *er = (const char *)e + (size_t)r * d_mem * (dtype == EO_F32 ? 4 : 2);
-        eo_project(er, dtype, 1, d_mem, w_k, M * d, kbuf);
-        eo_project(er, dtype, 1, d_mem, w_v, d, vbuf);
+        const char *er = (const char *)e + (size_t)r * d_mem * eo_elem_bytes(wdtype);
+        eo_project(er, wdtype, 1, d_mem, w_k, M * d, kbuf);
+        eo_project(er, wdtype, 1, d_mem, w_v, d, vbuf);
         for (m = 0; m < M; ++m) {
             int64_t base = (r * M + m) * (int64_t)d;
             double a;
-            for (i = 0; i < d; ++i) hbuf[i] = eo_load(h, dtype, base + i);
+            for (i = 0; i < d; ++i) hbuf[i] = eo_load(h, hdtype, base + i);
             a = eo_gate(hbuf, kbuf + (int64_t)m * d, wq + (int64_t)m * d, wk + (int64_t)m * d, d, eps);
             alpha[r * M + m] = a;
             for (i = 0; i < d; ++i) {
                 double dl = a * vbuf[i];
                 double o = hbuf[i] + dl;
                 if (delta) delta[base + i] = dl;
-                if (dtype == EO_F32) ((float *)out)[base + i] = (float)o;
+                if (hdtype == EO_F32) ((float *)out)[base + i] = (float)o;
                 else ((uint16_t *)out)[base + i] = eo_bf16_rne(o);
             }
         }
     }
+}
+
+/* The same with one dtype for every operand. */
+void eo_project_gate(const void *e, int32_t dtype, int64_t rows, int32_t d_mem,
+                     const void *w_k, const void *w_v, const float *wq, const float *wk,
+                     int32_t M, int32_t d, double eps, const void *h,
+                     double *alpha, double *delta, void *out,
+                     double *kbuf, double *vbuf, double *hbuf)
+{
+    eo_project_gate_mixed(e, dtype, rows, d_mem, w_k, w_v, wq, wk, M, d, eps, h, dtype,
+                          alpha, delta, out, kbuf, vbuf, hbuf);
+}
+
+/* ------------------------------------------------------- FP8 projection */
+
+/*
+ * Section 2.4 fuses W_V and the M key projections W_K into one dense FP8
+ * matmul.  The pages name neither the FP8 format nor how values are scaled
+ * into it; the reading taken here:
+ *  - the operands e and W are E4M3 (1 sign bit, 4 exponent bits with bias 7,
+ *    3 mantissa bits; exponent field 0 holds the subnormals m * 2^-9; no
+ *    infinities; S.1111.111 is NaN; the largest finite magnitude is 448);
+ *  - one scale per row of e (per position) and one per row of W (per output
+ *    channel), each a power of two 2^E, E the smallest integer for which the
+ *    row's largest magnitude is at most 448 * 2^E (E = 0 for an all-zero row);
+ *  - code = E4M3(x * 2^-E), rounded to nearest with ties to even, saturating
+ *    at +-448, the sign kept for values that round to zero; the dequantised
+ *    value is E4M3value(code) * 2^E.
+ * Both scales factor out of every dot product of Eq. (3), so k and v are the
+ * projections of the dequantised operands, and the gate and output follow
+ * unchanged (eo_project_gate_mixed with EO_F64 operands).
+ */
+
+/* The value of an E4M3 code (NaN for S.1111.111). */
+double eo_e4m3_decode(uint8_t code)
+{
+    const int sign = code >> 7, ex = (code >> 3) & 15, man = code & 7;
+    double v;
+    if (ex == 15 && man == 7) return NAN;
+    v = ex == 0 ? ldexp((double)man, -9) : ldexp(8.0 + man, ex - 10); /* (1 + m/8) 2^(ex-7) */
+    return sign ? -v : v;
+}
+
+/* E4M3 code of y: round to nearest, ties to even, saturate at +-448. */
+uint8_t eo_e4m3_encode(double y)
+{
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    const double a = fabs(y);
+    double step, v;
+    int ex;
+    if (isnan(y)) return 0x7F;
+    if (a >= 448.0) return sign | 0x7E;
+    /* spacing of the representable values around a: 2^-9 below the smallest
+       normal 2^-6, else 2^(floor(log2 a) - 3) */
+    if (a < ldexp(1.0, -6)) {
+        step = ldexp(1.0, -9);
+    } else {
+        frexp(a, &ex); /* a = f 2^ex, 0.5 <= f < 1: floor(log2 a) = ex - 1 */
+        step = ldexp(1.0, ex - 4);
+    }
+    v = nearbyint(a / step) * step; /* a / step is exact; ties to even */
+    if (v == 0.0) return sign;
+    if (v < ldexp(1.0, -6)) return sign | (uint8_t)(v / ldexp(1.0, -9));
+    frexp(v, &ex);
+    return sign | (uint8_t)((ex - 1 + 7) << 3) | (uint8_t)(ldexp(v, 4 - ex) - 8.0);
+}
+
+/* E of the power-of-two scale 2^E for a row whose largest magnitude is amax. */
+int32_t eo_e4m3_scale_exp(double amax)
+{
+    int ex;
+    double f;
+    if (!(amax > 0.0)) return 0;
+    f = frexp(amax, &ex); /* amax = f 2^ex; 448 = 0.875 2^9 */
+    return f <= 0.875 ? ex - 9 : ex - 8;
+}
+
+/* codes [rows, cols] and scales [rows] (2^E as float) of x [rows, cols]. */
+void eo_quantize_e4m3_rows(const void *x, int32_t dtype, int64_t rows, int32_t cols,
+                           uint8_t *code, float *scale)
+{
+    int64_t r;
+    int32_t j;
+    for (r = 0; r < rows; ++r) {
+        double amax = 0.0;
+        int32_t E;
+        for (j = 0; j < cols; ++j) {
+            const double a = fabs(eo_load(x, dtype, r * cols + j));
+            if (a > amax) amax = a;
+        }
+        E = eo_e4m3_scale_exp(amax);
+        for (j = 0; j < cols; ++j)
+            code[r * cols + j] = eo_e4m3_encode(ldexp(eo_load(x, dtype, r * cols + j), -E));
+        scale[r] = (float)ldexp(1.0, E);
+    }
+}
+
+/* y [rows, cols] = E4M3value(code) * scale[row]. */
+void eo_dequantize_e4m3_rows(const uint8_t *code, const float *scale, int64_t rows, int32_t cols,
+                             double *y)
+{
+    int64_t r;
+    int32_t j;
+    for (r = 0; r < rows; ++r)
+        for (j = 0; j < cols; ++j)
+            y[r * cols + j] = eo_e4m3_decode(code[r * cols + j]) * (double)scale[r];
 }
 
 /* -------------------------------------------------------------- short conv */

@@ -321,3 +321,153 @@ def test_add_round_matches_torch_rounding():
     assert np.array_equal(out, ref.view(torch.int16).numpy().view(np.uint16))
     hf = rng.normal(size=100).astype(np.float32)
     assert np.array_equal(oracle.add_round(hf, y[:100]), (hf.astype(np.float64) + y[:100]).astype(np.float32))
+
+
+# ------------------------------------------------- FP8 projection (section 2.4)
+
+def _torch_e4m3(x32: np.ndarray) -> np.ndarray:
+    """E4M3 codes from torch's own float -> float8_e4m3fn conversion."""
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    v = oracle.e4m3_decode(codes)
+    t = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(v), np.isnan(t)) and np.isnan(v).sum() == 2
+    assert np.array_equal(v[~np.isnan(v)], t[~np.isnan(t)])
+    # the format's fixed points: largest finite 448, smallest subnormal 2^-9, smallest normal 2^-6
+    assert v[0x7E] == 448.0 and v[0x01] == 2.0 ** -9 and v[0x08] == 2.0 ** -6
+    assert np.array_equal(v[0x80:0xFE], -v[0x00:0x7E])
+
+
+def test_e4m3_encode_matches_torch_rounding():
+    rng = np.random.default_rng(7)
+    grid = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8))  # 0 .. 448
+    mids = (grid[:-1] + grid[1:]) / 2                              # ties: to even
+    vals = [grid, mids, np.nextafter(mids.astype(np.float32), np.float32(0)),
+            np.nextafter(mids.astype(np.float32), np.float32(500)),
+            rng.uniform(0, 448, 20000) * np.exp2(rng.integers(-14, 1, 20000)),
+            rng.uniform(0, 2.0 ** -6, 5000), np.array([0.0, 2.0 ** -11, 3 * 2.0 ** -11])]
+    x = np.concatenate([v.astype(np.float32) for v in vals])
+    x = np.concatenate([x, -x])
+    assert np.array_equal(oracle.e4m3_encode(x.astype(np.float64)), _torch_e4m3(x))
+
+
+def test_e4m3_encode_saturates_and_keeps_zero_sign():
+    c = oracle.e4m3_encode(np.array([448.0, 460.0, 480.0, 1e30, np.inf, -1e9, -0.0, -2.0 ** -12]))
+    assert c.tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x80, 0x80]
+    assert oracle.e4m3_encode(np.array([np.nan]))[0] & 0x7F == 0x7F
+
+
+def test_e4m3_scale_exp_is_the_smallest_power_of_two():
+    rng = np.random.default_rng(3)
+    amaxes = list(rng.uniform(0, 1, 2000) * np.exp2(rng.integers(-40, 40, 2000)))
+    amaxes += [448.0 * 2.0 ** k for k in range(-20, 20)]
+    amaxes += [math.nextafter(448.0 * 2.0 ** k, math.inf) for k in range(-5, 5)]
+    amaxes += [2.0 ** k for k in range(-30, 30)]
+    for a in amaxes:
+        E = oracle.e4m3_scale_exp(a)
+        assert a <= math.ldexp(448.0, E) and a > math.ldexp(448.0, E - 1), (a, E)
+    assert oracle.e4m3_scale_exp(0.0) == 0
+
+
+def _bf16_rows(rows, cols, seed, scale=0.02):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(rows, cols, generator=g) * scale).bfloat16()
+    x[1] = 0                        # an all-zero row
+    x[2] *= 1e4                     # a wide row
+    x[3, 5] = -3.0                  # one large element: most of the row in subnormals
+    return x
+
+
+def test_quantize_rows_match_torch_conversion():
+    x = _bf16_rows(16, 96, seed=11)
+    codes, scales = oracle.quantize_e4m3_rows(_bf16_bits(x))
+    xd = x.double().numpy()
+    for r in range(x.shape[0]):
+        amax = np.abs(xd[r]).max()
+        f, ex = math.frexp(amax) if amax > 0 else (0.5, 0)
+        E = 0 if amax == 0 else (ex - 9 if f <= 0.875 else ex - 8)
+        assert scales[r] == math.ldexp(1.0, E)
+        assert np.array_equal(codes[r], _torch_e4m3(np.ldexp(xd[r], -E)))
+    y = oracle.dequantize_e4m3_rows(codes, scales)
+    mx = np.abs(y).max(1) / scales
+    nz = np.abs(xd).max(1) > 0
+    # amax / scale lies in (224, 448]; rounding may bring it down to 224
+    assert ((mx[nz] >= 224) & (mx[nz] <= 448)).all()
+    # round to nearest with 3 mantissa bits: |error| <= 2^-4 |x| in the normal
+    # range, <= half the subnormal spacing 2^-10 (times the scale) below it
+    err = np.abs(y - xd)
+    normal = np.abs(xd) >= scales[:, None] * 2.0 ** -6
+    assert (err[normal] <= 2.0 ** -4 * np.abs(xd[normal])).all()
+    assert (err[~normal] <= (scales[:, None] * 2.0 ** -10 * np.ones_like(xd))[~normal]).all()
+
+
+def _fp8_grid_rows(rows, cols, seed):
+    """Rows whose values are already E4M3 values times the row's scale, with
+    the row's largest magnitude hitting a code of (224, 448]: quantisation is
+    then lossless."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 0x7F, (rows, cols)).astype(np.uint8) | (
+        rng.integers(0, 2, (rows, cols)).astype(np.uint8) << 7)
+    codes[:, 0] = 0x7A                                   # 320
+    E = rng.integers(-14, -4, rows)
+    v = oracle.e4m3_decode(codes) * np.exp2(E)[:, None]
+    return torch.from_numpy(v).bfloat16()
+
+
+def test_project_gate_fp8_equals_plain_on_representable_operands():
+    rows, M, d, dm = 5, 2, 32, 64
+    e = _fp8_grid_rows(rows, dm, 1)
+    wk = _fp8_grid_rows(M * d, dm, 2).reshape(M, d, dm)
+    wv = _fp8_grid_rows(d, dm, 3)
+    g = torch.Generator().manual_seed(4)
+    h = torch.randn(rows, M, d, generator=g).bfloat16()
+    nq = (1 + 0.1 * torch.randn(M, d, generator=g)).numpy()
+    nk = (1 + 0.1 * torch.randn(M, d, generator=g)).numpy()
+    args = [_bf16_bits(t) for t in (e, wk, wv)]
+    a0, d0, o0 = oracle.project_gate(args[0], args[1], args[2], nq, nk, _bf16_bits(h), 1e-6)
+    a1, d1, o1 = oracle.project_gate_fp8(args[0], args[1], args[2], nq, nk, _bf16_bits(h), 1e-6)
+    assert np.array_equal(a0, a1) and np.array_equal(d0, d1) and np.array_equal(o0, o1)
+
+
+def test_project_gate_fp8_against_torch_fp64():
+    rows, M, d, dm = 6, 2, 64, 96
+    g = torch.Generator().manual_seed(9)
+    e = (torch.randn(rows, dm, generator=g) * 0.02).bfloat16()
+    wk = (torch.randn(M, d, dm, generator=g) / math.sqrt(dm)).bfloat16()
+    wv = (torch.randn(d, dm, generator=g) / math.sqrt(dm)).bfloat16()
+    h = torch.randn(rows, M, d, generator=g).bfloat16()
+    nq = (1 + 0.1 * torch.randn(M, d, generator=g)).numpy()
+    nk = (1 + 0.1 * torch.randn(M, d, generator=g)).numpy()
+    alpha, delta, out = oracle.project_gate_fp8(_bf16_bits(e), _bf16_bits(wk), _bf16_bits(wv),
+                                                nq, nk, _bf16_bits(h), 1e-6)
+
+    def deq(x):  # per row: power-of-two scale from frexp, codes by torch's conversion
+        x = x.double().reshape(-1, x.shape[-1])
+        amax = x.abs().amax(1)
+        out = torch.empty_like(x)
+        for r in range(x.shape[0]):
+            f, ex = math.frexp(float(amax[r]))
+            E = 0 if amax[r] == 0 else (ex - 9 if f <= 0.875 else ex - 8)
+            q = torch.from_numpy(np.ldexp(x[r].numpy(), -E)).float().to(torch.float8_e4m3fn)
+            out[r] = q.double() * 2.0 ** E
+        return out
+
+    E8, WV8 = deq(e), deq(wv)
+    WK8 = deq(wk).reshape(M, d, dm)
+    H = h.double()
+    k = torch.einsum("rj,mij->rmi", E8, WK8)
+    v = E8 @ WV8.T
+    qn = H / torch.sqrt(H.pow(2).mean(-1, keepdim=True) + 1e-6) * torch.from_numpy(nq).double()
+    kn = k / torch.sqrt(k.pow(2).mean(-1, keepdim=True) + 1e-6) * torch.from_numpy(nk).double()
+    a_ref = torch.sigmoid((qn * kn).sum(-1) / math.sqrt(d))
+    assert np.allclose(alpha, a_ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(delta, (a_ref[..., None] * v[:, None, :]).numpy(), rtol=1e-12, atol=1e-12)
+    # and it differs from the bf16 projection by quantisation error only
+    a0, d0, _ = oracle.project_gate(_bf16_bits(e), _bf16_bits(wk), _bf16_bits(wv), nq, nk,
+                                    _bf16_bits(h), 1e-6)
+    rel = np.linalg.norm(delta - d0) / np.linalg.norm(d0)
+    assert 1e-4 < rel < 0.1
