@@ -65,6 +65,9 @@ def parse():
     ap.add_argument("--short-conv", action="store_true",
                     help="with the short convolution of Eq. 5 (W = 4, dilation = the largest "
                          "n-gram order, seeded non-zero weights); prefill-type workloads")
+    ap.add_argument("--fp8", action="store_true",
+                    help="projections on E4M3 operands (section 2.4's FP8 matmul): e quantised "
+                         "per row inside the gather, W per output channel; prefill-type workloads")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a captured CUDA graph (launch-bound shapes)")
     ap.add_argument("--offload-gb", type=float, default=100.0,
@@ -153,7 +156,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------ the workload
 
-def setup(rank: int, device, rows_target=None, workload=WORKLOAD, short_conv=False):
+def setup(rank: int, device, rows_target=None, workload=WORKLOAD, short_conv=False, fp8=False):
     import torch
     from hashed_gram_embedding_compress_b200 import engram as eg
     from hashed_gram_embedding_compress_b200 import synth
@@ -180,27 +183,33 @@ def setup(rank: int, device, rows_target=None, workload=WORKLOAD, short_conv=Fal
         cw, nw = synth.make_conv_weights(sh, seeds, 4)
         conv = (cw.to(device), nw.to(device), 4, max(sh.orders))
         m.set_short_conv(*conv)
+    if fp8:
+        m.set_fp8(True)
     m.reserve(sh.rows_out)
     return dict(sh=sh, m=m, tokens=tokens, comp_map=comp_map, tables=tables, w_k=w_k, w_v=w_v,
                 nq=nq, nk=nk, h=h, seeds=seeds, hash_seed=synth.make_hash_seed(seeds),
-                primes=primes, conv=conv)
+                primes=primes, conv=conv, fp8=fp8)
 
 
-def algorithmic(sh):
-    """Per-step algorithmic work: bytes of the gather and hash, FLOPs and bytes of the projections."""
+def algorithmic(sh, fp8=False):
+    """Per-step algorithmic work: bytes of the gather and hash, FLOPs and bytes of the projections.
+    fp8: e is written as one E4M3 byte per element plus a 4-byte scale per row."""
     R, S, dm, d, M = sh.rows_out, sh.num_tables, sh.d_mem, sh.d_hidden, sh.branches
     elt = 2 if sh.dtype == "bf16" else 4
     row_bytes = sh.d_head * elt
     if sh.table_location == "device":
         # hash fused into the gather: tokens read, table rows read, e written
         gather_bytes = R * S * row_bytes * 2 + sh.B * sh.T * 4
+        if fp8:
+            gather_bytes = R * S * row_bytes + R * (dm + 4) + sh.B * sh.T * 4
         hash_bytes = 0
     else:
         gather_bytes = R * S * (row_bytes * 2 + 8)   # rows read, e written, indices read
         hash_bytes = R * S * 8 + sh.B * sh.T * 4     # indices written, tokens read
     gemm_flops = 2.0 * R * dm * (M * d + d)          # [W_K^(1..M); W_V] e
     # key kernel: e read, W_K read, h read; value kernel: e, W_V, h read, out written
-    gemm_bytes = (2 * R * dm * elt + (M * d + d) * dm * elt + 3 * R * M * d * elt)
+    op = 1 if fp8 else elt                           # bytes per operand element of the matmul
+    gemm_bytes = (2 * R * dm * op + (M * d + d) * dm * op + 3 * R * M * d * elt)
     # short conv: v (fp32) read once, h read and out written per branch, plus
     # alpha and the per-tile sums of v^2
     conv_bytes = R * d * 4 + 2 * R * M * d * elt + R * (M + d // 256) * 4
@@ -209,10 +218,10 @@ def algorithmic(sh):
                 gemm_bytes=gemm_bytes)
 
 
-def kernel_traffic():
+def kernel_traffic(name="traffic.json"):
     """DRAM bytes per step of the projection kernel (key + value launches)
     from a committed ncu capture, or None once its source has changed."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
@@ -246,7 +255,7 @@ def run_ours(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    P = setup(rank, device, args.rows_target, args.workload, args.short_conv)
+    P = setup(rank, device, args.rows_target, args.workload, args.short_conv, args.fp8)
     sh, m = P["sh"], P["m"]
     NEV = 6 if args.short_conv else 5  # stage events per forward
     tok_d = P["tokens"].to(device)
@@ -366,14 +375,18 @@ def run_ours(args, rank, world, dist):
         return None
 
     hbm, tflops, tflops_burst, peak_kind = load_peaks()
-    A = algorithmic(sh)
+    A = algorithmic(sh, args.fp8)
+    if args.fp8:
+        # E4M3 operands: the nominal dense FP8 rate is twice the bf16 one (4.5 vs 2.25
+        # PFLOP/s), applied to the measured bf16 figures
+        tflops, tflops_burst = 2 * tflops, 2 * tflops_burst
     tokens_per_step = sh.rows_out
     value = tokens_per_step * world * K / (ms / 1e3)
     gemm_s = (st_mean[2] + st_mean[3]) / 1e3
     gemm_tflops = A["gemm_flops"] / gemm_s / 1e12
     fused = sh.table_location == "device"  # one hash + gather kernel: its time is stage 1
     gather_gbs = A["gather_bytes"] / ((st_mean[0] + st_mean[1] if fused else st_mean[1]) / 1e3) / 1e9
-    traffic = kernel_traffic()
+    traffic = None if args.fp8 else kernel_traffic()
     res = {
         "metric": METRIC,
         "value": value,
@@ -385,7 +398,7 @@ def run_ours(args, rank, world, dist):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3" if args.fp8 else "bf16",
         "data": "synthetic",
         "config": {
             "workload": DESCRIBE[args.workload],
@@ -406,12 +419,14 @@ def run_ours(args, rank, world, dist):
             "unit": "TFLOP/s",
             "frac": gemm_tflops / tflops,
             "traffic": traffic,
-            "peak_source": "%s bf16 sustained (cuBLAS back to back under the power cap)" % peak_kind
-                           if peak_kind == "measured" else peak_kind,
+            "peak_source": ("%s bf16 sustained (cuBLAS back to back under the power cap)" % peak_kind
+                            if peak_kind == "measured" else peak_kind) +
+                           (" x 2, the nominal FP8 / bf16 ratio" if args.fp8 else ""),
             "frac_of_burst": gemm_tflops / tflops_burst,
         },
         "gather": {
-            "kernel": "hash_gather_kernel" if fused else "gather_kernel",
+            "kernel": ("hash_gather_e4m3_kernel" if args.fp8 else "hash_gather_kernel")
+                      if fused else "gather_kernel",
             "achieved_gbs": gather_gbs,
             "frac_of_hbm": gather_gbs / hbm,
             "peak_gbs": hbm,
@@ -445,6 +460,11 @@ def run_ours(args, rank, world, dist):
             "bytes_per_step": A["conv_bytes"],
         }
         res["roofline"]["traffic"] = None  # the committed capture is of the conv-less value phase
+    if args.fp8:
+        res["config"]["workload"] += (" + FP8 projections (E4M3 e and W, power-of-two scales per "
+                                      "row and output channel, fp32 accumulation)")
+        res["roofline"]["kernel"] = res["roofline"]["kernel"].replace("(tcgen05", "(tcgen05 kind::f8f6f4")
+        res["roofline"]["traffic"] = kernel_traffic("traffic_fp8.json")
     if args.rows_target:
         res["config"]["workload"] += " [profiling variant: tables of %d rows]" % args.rows_target
     if args.workload != "prefill_bf16":
@@ -648,6 +668,8 @@ def cpu_baseline(P, budget_s: float):
 
     wk, wv = to_np(P["w_k"]), to_np(P["w_v"])
     nq, nk = P["nq"].cpu().numpy(), P["nk"].cpu().numpy()
+    # FP8 projections: W quantised once, as the library does when they are switched on
+    w8 = oracle.quantize_weights_e4m3(wk, wv) if P.get("fp8") else None
     n, spent, total_rows, total_t = 8, 0.0, 0, 0.0
     while spent < budget_s and total_rows < sh.rows_out:
         rows = np.arange(total_rows, min(sh.rows_out, total_rows + n))
@@ -657,7 +679,12 @@ def cpu_baseline(P, budget_s: float):
         hr = to_np(P["h"][torch.from_numpy(rows).to(P["h"].device)])
         t0 = time.perf_counter()
         e = oracle.gather(mini, zz)
-        _, delta, _ = oracle.project_gate(e, wk, wv, nq, nk, hr, 1e-6, want_delta=P["conv"] is not None)
+        want = P["conv"] is not None
+        if w8 is not None:
+            _, delta, _ = oracle.project_gate_fp8(e, wk, wv, nq, nk, hr, 1e-6, want_delta=want,
+                                                  weights=w8)
+        else:
+            _, delta, _ = oracle.project_gate(e, wk, wv, nq, nk, hr, 1e-6, want_delta=want)
         if P["conv"] is not None:
             # Eq. 5 over the sample's positions (consecutive rows of one sequence)
             cw, nw, W, dil = P["conv"]
@@ -671,10 +698,10 @@ def cpu_baseline(P, budget_s: float):
         n *= 2
     per_row = t_hash + total_t / total_rows
     return {"value": 1.0 / per_row, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "compress+hash on all %d positions; gather+projection+gate%s on the first "
+            "sample": "compress+hash on all %d positions; gather+%sprojection+gate%s on the first "
                       "%d rows (%.1f s); single-threaded C, fp64" % (
-                          sh.rows_out, "+short conv" if P["conv"] is not None else "",
-                          total_rows, total_t)}
+                          sh.rows_out, "E4M3 quantisation+" if w8 is not None else "",
+                          "+short conv" if P["conv"] is not None else "", total_rows, total_t)}
 
 
 def run_reference(args, rank, world):
@@ -683,7 +710,7 @@ def run_reference(args, rank, world):
     import torch
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     P = setup(0, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))), None, args.workload,
-              args.short_conv)
+              args.short_conv, args.fp8)
     sh = P["sh"]
     budget = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):

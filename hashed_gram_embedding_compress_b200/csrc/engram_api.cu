@@ -76,22 +76,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `rows` rows of `cols` elements, box box_cols x box_rows;
-// the swizzle width is the box row width (64 columns = 128 B, 32 columns = 64 B).
-// 2-D row-major tensor map; the swizzle follows the box's row bytes (128-byte
-// rows: 128-byte swizzle, 64-byte rows: 64-byte swizzle).  bf16 unless f32.
+// 2-D row-major tensor map: `rows` rows of `cols` elements of esz bytes (2:
+// bf16, 4: fp32, 1: E4M3 codes), box box_cols x box_rows; the swizzle follows
+// the box's row bytes (128-byte rows: 128-byte swizzle, 64-byte rows: 64-byte
+// swizzle).
 int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
-             int box_rows, int box_cols = 64, bool f32 = false) {
+             int box_rows, int box_cols = 64, int esz = 2) {
   auto fn = encode_fn();
   if (!fn) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const int esz = f32 ? 4 : 2;
+  const CUtensorMapDataType dt = esz == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                            : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * esz};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
   const CUtensorMapSwizzle sw =
       box_cols * esz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUresult r = fn(m, dt, 2,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
@@ -112,6 +114,34 @@ int ensure_scratch(engram_handle* h, int64_t rows) {
   CK(h, cudaMalloc(&h->partials, (size_t)rows * key_tiles * sizeof(float4)));
   h->cap_rows = rows;
   return ENGRAM_OK;
+}
+
+int ensure_fp8_scratch(engram_handle* h, int64_t rows) {
+  if (rows <= h->fp8_cap_rows) return ENGRAM_OK;
+  free_dev(h->e8);
+  free_dev(h->se8);
+  h->fp8_cap_rows = 0;
+  CK(h, cudaMalloc(&h->e8, (size_t)rows * h->d_mem));
+  CK(h, cudaMalloc(&h->se8, (size_t)rows * sizeof(float)));
+  h->fp8_cap_rows = rows;
+  return ENGRAM_OK;
+}
+
+// E4M3 copy of [W_K; W_V] (one scale per row) and its tensor maps (boxes of
+// 128 rows x 128 codes for the CTA-pair kernel); synchronises the device.
+int quantize_weights(engram_handle* h, cudaStream_t st) {
+  const int64_t M = h->cfg.branches, d = h->cfg.d_hidden, dm = h->d_mem;
+  if (!h->d_w8) {
+    CK(h, cudaMalloc(&h->d_w8, (size_t)(M + 1) * d * dm));
+    CK(h, cudaMalloc(&h->d_sw8, (size_t)(M + 1) * d * sizeof(float)));
+  }
+  CK(h, launch_quantize_e4m3(h->w_k, M * d, (int)dm, h->d_w8, h->d_sw8, st));
+  CK(h, launch_quantize_e4m3(h->w_v, d, (int)dm, h->d_w8 + M * d * dm, h->d_sw8 + M * d, st));
+  h->launches += 2;
+  CK(h, cudaDeviceSynchronize());
+  int rc = make_map(h, &h->map_wk8, h->d_w8, dm, M * d, 128, 128, 1);
+  if (rc) return rc;
+  return make_map(h, &h->map_wv8, h->d_w8 + M * d * dm, dm, d, 128, 128, 1);
 }
 
 int ensure_conv_scratch(engram_handle* h, int64_t rows) {
@@ -344,6 +374,10 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->d_wqk);
   free_dev(h->e);
   free_dev(h->partials);
+  free_dev(h->d_w8);
+  free_dev(h->d_sw8);
+  free_dev(h->e8);
+  free_dev(h->se8);
   free_dev(h->d_conv_w);
   free_dev(h->d_conv_nw);
   free_dev(h->d_conv_taps);
@@ -418,6 +452,42 @@ int engram_set_params(engram_handle* h, const void* const* tables, const void* w
     }
   }
   h->have_params = true;
+  if (h->fp8) return quantize_weights(h, 0);  // the new weights' E4M3 copy
+  return ENGRAM_OK;
+}
+
+int engram_set_fp8(engram_handle* h, int32_t enable, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (enable != 0 && enable != 1) return fail(h, ENGRAM_ERR_INVALID, "enable must be 0 or 1");
+  if (!enable) {
+    h->fp8 = false;
+    return ENGRAM_OK;
+  }
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (h->cfg.dtype != ENGRAM_BF16)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED, "FP8 projections need bf16 tables, weights and h");
+  if (h->cfg.d_hidden % 256 || h->d_mem % 128 || h->d_mem > 2048)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED,
+                "FP8 projections need d a multiple of 256 and d_mem a multiple of 128, <= 2048");
+  if (h->cfg.flags & ENGRAM_FLAG_NO_CTA_PAIRS)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED, "FP8 projections run on CTA pairs only");
+  int rc = quantize_weights(h, (cudaStream_t)stream);
+  if (rc) return rc;
+  h->fp8 = true;
+  return ENGRAM_OK;
+}
+
+int engram_quantize_e4m3(engram_handle* h, const void* x, int64_t rows, int32_t cols, uint8_t* q,
+                         float* scale, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (rows < 0 || rows > ((int64_t)1 << 31)) return fail(h, ENGRAM_ERR_INVALID, "rows out of range");
+  if (cols < 16 || cols > 2048 || cols % 16)
+    return fail(h, ENGRAM_ERR_INVALID, "cols must be a multiple of 16 in [16, 2048]");
+  if (rows == 0) return ENGRAM_OK;
+  if (!x || !q || !scale || !aligned16(x) || !aligned16(q) || ((uintptr_t)scale & 3u))
+    return fail(h, ENGRAM_ERR_INVALID, "x and q must be 16-byte aligned, scale 4-byte aligned");
+  CK(h, launch_quantize_e4m3(x, rows, cols, q, scale, (cudaStream_t)stream));
+  h->launches += 1;
   return ENGRAM_OK;
 }
 
@@ -461,6 +531,7 @@ int engram_reserve(engram_handle* h, int64_t max_rows) {
   int rc = ensure_scratch(h, max_rows);
   if (rc) return rc;
   if (h->conv_W > 0 && (rc = ensure_conv_scratch(h, max_rows))) return rc;
+  if (h->fp8 && (rc = ensure_fp8_scratch(h, max_rows))) return rc;
   if (h->cfg.table_location == ENGRAM_PINNED_HOST) return ensure_prefetch_scratch(h, max_rows);
   return ENGRAM_OK;
 }
@@ -702,6 +773,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   if (R > (int64_t)65535 * 64 && h->cfg.dtype == ENGRAM_F32)
     return fail(h, ENGRAM_ERR_INVALID, "fp32 path limited to 4194240 rows per call");
   if ((rc = ensure_scratch(h, R))) return rc;
+  const bool fp8 = h->fp8;  // E4M3 operands for the projections (bf16 handles only)
+  if (fp8 && (rc = ensure_fp8_scratch(h, R))) return rc;
   const bool prof = h->prof_armed;
   h->prof_armed = false;
   auto mark = [&](int i) -> cudaError_t {
@@ -742,12 +815,19 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     hg.hash = hash_args(h, tokens, B, T, t_begin, nullptr);
     hg.tables = h->d_tables;
     hg.e = h->e;
+    hg.q = h->e8;
+    hg.scale = h->se8;
     hg.row_bytes = ga.row_bytes;
     CK(h, mark(1));
-    CK(h, launch_hash_gather(hg, st));
+    // FP8: e leaves the gather as E4M3 codes and row scales
+    CK(h, fp8 ? launch_hash_gather_e4m3(hg, st) : launch_hash_gather(hg, st));
   } else {
     CK(h, mark(1));
     CK(h, launch_gather(ga, st));
+    if (fp8) {
+      CK(h, launch_quantize_e4m3(h->e, R, h->d_mem, h->e8, h->se8, st));
+      h->launches += 1;
+    }
   }
   h->launches += 1;
   CK(h, mark(2));
@@ -817,9 +897,13 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   ProjMaps single, wide, pair;
   bool have_single = false, have_wide = false, have_pair = false;
   int value_tile = 0;
+  if (fp8) g.s_row = h->se8;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
-    const ProjChoice pc = choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv);
+    // the E4M3 operands run on the 512 x 256 CTA-pair kernel only
+    const ProjChoice pc = fp8 ? wide_proj(phase, R, g.M, g.d, h->sms)
+                              : choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv);
+    if (fp8) g.s_col = h->d_sw8 + (phase == 0 ? 0 : (int64_t)g.M * g.d);
     if (phase == 0) g.key_tile = pc.key_tile;
     if (phase == 1) value_tile = pc.key_tile;
     // values: 3 = v for the short convolution; 2 = in place (out aliases h,
@@ -839,24 +923,28 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
       CK(h, launch_proj_gate_pair(kphase, pm, g, pc.grid, st));
     } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
-        if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) return rc;
+        if (fp8) {
+          if ((rc = make_map(h, &wide.e, h->e8, h->d_mem, R, 256, 128, 1))) return rc;
+        } else if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) {
+          return rc;
+        }
         if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
         if ((rc = make_map(h, &wide.out, out, hcols, R, 32, 32))) return rc;
         have_wide = true;
       }
-      wide.w = wmaps[bn_index(pc.bn)];
+      wide.w = fp8 ? (phase == 0 ? h->map_wk8 : h->map_wv8) : wmaps[bn_index(pc.bn)];
       if (kphase == 2) {
         // in place: per-warp reduce-adds of 32 rows x 64 columns
         ProjMaps wr = wide;
         if ((rc = make_map(h, &wr.out, out, hcols, R, 32, 64))) return rc;
-        CK(h, launch_proj_gate_wide(kphase, wr, g, pc.grid, st));
+        CK(h, launch_proj_gate_wide(kphase, wr, g, pc.grid, st, fp8));
       } else if (kphase == 3) {
         // v leaves through per-warp TMA stores of 32 x 32 fp32 boxes
         ProjMaps wv = wide;
-        if ((rc = make_map(h, &wv.out, h->conv_v, g.d, R, 32, 32, true))) return rc;
-        CK(h, launch_proj_gate_wide(kphase, wv, g, pc.grid, st));
+        if ((rc = make_map(h, &wv.out, h->conv_v, g.d, R, 32, 32, 4))) return rc;
+        CK(h, launch_proj_gate_wide(kphase, wv, g, pc.grid, st, fp8));
       } else {
-        CK(h, launch_proj_gate_wide(kphase, wide, g, pc.grid, st));
+        CK(h, launch_proj_gate_wide(kphase, wide, g, pc.grid, st, fp8));
       }
     } else {
       if (!have_single) {

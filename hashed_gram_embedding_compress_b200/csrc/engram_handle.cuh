@@ -38,6 +38,16 @@ struct engram_handle {
   float* d_conv_nw = nullptr;  // [d]
   float* d_conv_taps = nullptr;  // [4][d]: conv_w times norm_w, tap-major
 
+  // FP8 projections (engram_set_fp8): E4M3 copy of [W_K; W_V] with one scale
+  // per row, and per-row E4M3 scratch of e
+  bool fp8 = false;
+  uint8_t* d_w8 = nullptr;     // [(M + 1) d, d_mem]: the M d rows of W_K, then W_V
+  float* d_sw8 = nullptr;      // [(M + 1) d]
+  CUtensorMap map_wk8, map_wv8;
+  int64_t fp8_cap_rows = 0;
+  uint8_t* e8 = nullptr;       // [rows, d_mem] codes of e
+  float* se8 = nullptr;        // [rows] scales of e
+
   // scratch, sized for cap_rows emitted positions
   int64_t cap_rows = 0;
   void* e = nullptr;

@@ -49,6 +49,8 @@ struct HashGatherArgs {
   HashArgs hash;              // idx is unused: the indices stay on chip
   const void* const* tables;  // device array [S] of table base pointers
   void* e;                    // [rows, S*d_head]
+  uint8_t* q;                 // E4M3 form: codes [rows, S*d_head] (bf16 tables)
+  float* scale;               // E4M3 form: power-of-two scale per row
   int32_t row_bytes;          // d_head * element size, a multiple of 16
   int32_t rows_per_block;     // set by the launcher
 };
@@ -65,6 +67,8 @@ struct GateArgs {
   float* vv;            // phase 3: sum of v^2 per value tile and row, [d / value tile][R]
   unsigned* err;
   int32_t R, M, d, d_mem;
+  const float* s_row;   // FP8 operands: scale of each row of e [R] (else null)
+  const float* s_col;   // FP8 operands: scale of each W row of this phase's columns
   int32_t key_tile;     // width of the key-phase tiles that wrote `partials`
   float eps;
   float inv_sqrt_d;
@@ -127,6 +131,13 @@ cudaError_t launch_fill_hot_cache(const unsigned long long* list, int64_t n,
 cudaError_t launch_hash(const HashArgs& a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs& a, cudaStream_t stream);
 cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream);
+// Hash + gather + E4M3 quantisation of each row of e (FP8 projections): writes
+// a.q and a.scale instead of a.e; bf16 tables, S * d_head <= 2048.
+cudaError_t launch_hash_gather_e4m3(const HashGatherArgs& a, cudaStream_t stream);
+// E4M3 codes q [rows, cols] and power-of-two scales [rows] of bf16 x [rows,
+// cols]; 16 <= cols <= 2048, cols a multiple of 16.
+cudaError_t launch_quantize_e4m3(const void* x, int64_t rows, int cols, uint8_t* q, float* scale,
+                                 cudaStream_t stream);
 // taps[i][c] = conv_w[c][i] * norm_w[c] for the [d][4] conv weights.
 cudaError_t launch_conv_taps(const float* conv_w, const float* norm_w, int d, float* taps,
                              cudaStream_t stream);
@@ -156,9 +167,11 @@ struct ProjMaps {
 cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
                                    int grid, cudaStream_t stream);
 // 512 x 256 tiles on CTA pairs (tcgen05 cta_group::2); grid = 2 x pairs.
-// phase 0 keys, 1 values, 2 values added in place (out aliases h).
+// phase 0 keys, 1 values, 2 values added in place (out aliases h), 3 values
+// for the short convolution.  f8: e and W are E4M3 codes (maps of uint8 with
+// 128-column boxes) with the scales g.s_row and g.s_col.
 cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, bool f8 = false);
 
 // 256 x 256 tiles on CTA pairs with two TMEM accumulators (few rows, many
 // columns); grid = 2 x pairs; key tiles of 128 columns (g.key_tile must be
@@ -184,6 +197,15 @@ struct ProjChoice {
 // on B200: 13.2 us mainloop + 3.1-4.3 us epilogue per 512 x 256 tile).  Key
 // tiles must not straddle branches, so their width divides d.  The value
 // phase of the short convolution (phase 3) has no 256 x 256 pair variant.
+// The 512 x 256 CTA-pair kernel (the only one with E4M3 operands): one CTA
+// pair per tile up to every pair of SMs.  d a multiple of 256.
+inline ProjChoice wide_proj(int phase, int64_t R, int M, int d, int sms) {
+  const int n_total = phase == 0 ? M * d : d;
+  const int pairs = sms / 2;
+  const int64_t tiles = (R + 511) / 512 * (n_total / 256);
+  return {ProjKernel::Wide, 128, 2 * (int)(tiles < pairs ? tiles : pairs), 256};
+}
+
 inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int flags,
                               bool conv = false) {
   const int n_total = phase == 0 ? M * d : d;
@@ -212,8 +234,7 @@ inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int f
   if (pairs_ok && d % 256 == 0) {
     const int64_t tiles = (R + 511) / 512 * (n_total / 256);
     const int64_t cost = (tiles + pairs - 1) / pairs * 384 * 13;
-    if (cost <= best_cost)
-      best = {ProjKernel::Wide, 128, 2 * (int)(tiles < pairs ? tiles : pairs), 256};
+    if (cost <= best_cost) best = wide_proj(phase, R, M, d, sms);
   }
   return best;
 }

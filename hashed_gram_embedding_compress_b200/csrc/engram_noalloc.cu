@@ -100,6 +100,9 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
                                            void* stream) {
   if (!h) return ENGRAM_ERR_INVALID;
   if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (h->fp8)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED,
+                "engram_project_gate_noalloc: FP8 projections are on; use engram_forward");
   if (h->conv_W > 0)
     return fail(h, ENGRAM_ERR_UNSUPPORTED,
                 "engram_project_gate_noalloc: the short convolution needs scratch; use engram_forward");

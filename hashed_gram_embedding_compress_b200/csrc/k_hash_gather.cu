@@ -6,6 +6,7 @@
 //
 // phi is the multiplicative-XOR form fixed by this library (see engram.h):
 // x = XOR_j c[t-j] * m[s][j] in wrapping 64-bit arithmetic, z = x mod p[s].
+#include "e4m3.cuh"
 #include "engram_internal.cuh"
 
 namespace engram {
@@ -197,6 +198,76 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
   }
 }
 
+// Hash, gather and E4M3 quantisation fused (the FP8 projections): the hash
+// stage is hash_gather_kernel's; then each warp takes whole rows of the block,
+// loads the row's S table rows (each lane up to 8 chunks of 16 bytes, all in
+// flight together), reduces the row's largest magnitude over the warp and
+// writes the row's codes (half the bytes of e) and its scale.
+__global__ void __launch_bounds__(kFusedThreads) hash_gather_e4m3_kernel(HashGatherArgs g) {
+  const HashArgs& a = g.hash;
+  __shared__ uint64_t s_mult[kMaxTables * kMaxOrders];
+  __shared__ uint64_t s_prime[kMaxTables];
+  __shared__ uint64_t s_inv[kMaxTables];
+  __shared__ int32_t s_order_of_slot[kMaxTables];
+  __shared__ const char* s_tab[kMaxTables];
+  __shared__ const char* s_src[kFusedThreads];  // source row of (row, slot)
+  const int S = a.S;
+  for (int i = threadIdx.x; i < S * a.max_order; i += blockDim.x) s_mult[i] = a.mult[i];
+  for (int i = threadIdx.x; i < S; i += blockDim.x) {
+    s_prime[i] = (uint64_t)a.primes[i];
+    s_inv[i] = a.barrett[i];
+    s_order_of_slot[i] = a.orders[i / a.heads];
+    s_tab[i] = (const char*)g.tables[i];
+  }
+  __syncthreads();
+
+  const uint32_t Tout = (uint32_t)(a.T - a.t_begin);
+  const uint32_t rows = (uint32_t)a.B * Tout;
+  const uint32_t rb = (uint32_t)g.rows_per_block;  // <= 256 / S
+  const uint32_t row0 = blockIdx.x * rb;
+  const uint32_t nrows = min(rb, rows - row0);
+  const uint32_t nslots = nrows * (uint32_t)S;
+  if (threadIdx.x < nslots) {
+    const uint32_t rl = threadIdx.x / (uint32_t)S;
+    const int s = (int)(threadIdx.x - rl * (uint32_t)S);
+    const uint32_t row = row0 + rl;
+    const int b = (int)(row / Tout);
+    const int t = a.t_begin + (int)(row - (uint32_t)b * Tout);
+    const uint64_t z = hash_slot(a, a.tokens + (int64_t)b * a.T, t, s_order_of_slot[s],
+                                 s_mult + s * a.max_order, s_prime[s], s_inv[s]);
+    s_src[threadIdx.x] = s_tab[s] + z * (uint64_t)g.row_bytes;
+  }
+  __syncthreads();
+
+  const int cpr = g.row_bytes >> 4;  // chunks per table row
+  const int C = S * cpr;             // chunks per row of e (<= 32 * kQuantMaxChunks)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (uint32_t rl = warp; rl < nrows; rl += kFusedThreads / 32) {
+    const char* const* src = s_src + rl * S;
+    auto chunk = [&](int c) {
+      const int s = c / cpr;
+      return ld_stream_16(src[s] + (c - s * cpr) * 16);
+    };
+    quant_row_warp(chunk, C, g.q + (int64_t)(row0 + rl) * C * 8, g.scale + row0 + rl, lane);
+  }
+}
+
+// E4M3 codes and scales of bf16 rows (the quantiser on its own: for W when
+// the FP8 projections are switched on, and for e gathered by gather_kernel).
+// One warp per row.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* x, int64_t rows,
+                                                            int cols, uint8_t* q, float* scale) {
+  const int lane = threadIdx.x & 31;
+  const int C = cols / 8;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows;
+       r += nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + r * cols);
+    auto chunk = [&](int c) { return ld_stream_16(src + c); };
+    quant_row_warp(chunk, C, q + r * cols, scale + r, lane);
+  }
+}
+
 __global__ void mul_kernel(const float* x, const float* y, float* out, int64_t n) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
@@ -247,6 +318,35 @@ cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream) {
   HashGatherArgs b = a;
   b.rows_per_block = (int32_t)rb;
   hash_gather_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hash_gather_e4m3(const HashGatherArgs& a, cudaStream_t stream) {
+  const int64_t rows = (int64_t)a.hash.B * (a.hash.T - a.hash.t_begin);
+  if (rows == 0) return cudaSuccess;
+  if (a.hash.S < 1 || a.hash.S > kMaxTables) return cudaErrorInvalidValue;
+  const int64_t chunks = (int64_t)a.hash.S * (a.row_bytes >> 4);
+  if (chunks > 32 * kQuantMaxChunks || rows * chunks >= ((int64_t)1 << 31))
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t rb = kFusedThreads / a.hash.S;
+  const int64_t fill = (rows + 2 * (int64_t)sms - 1) / (2 * (int64_t)sms);
+  if (fill < rb) rb = fill < 1 ? 1 : fill;
+  HashGatherArgs b = a;
+  b.rows_per_block = (int32_t)rb;
+  hash_gather_e4m3_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_e4m3(const void* x, int64_t rows, int cols, uint8_t* q, float* scale,
+                                 cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  if (cols < 16 || cols % 16 || cols > 8 * 32 * kQuantMaxChunks) return cudaErrorInvalidValue;
+  // a warp per row, eight rows per block, at most 16 blocks per SM (grid-stride)
+  quantize_rows_kernel<<<grid_for(rows * 32, 256), 256, 0, stream>>>(static_cast<const uint16_t*>(x), rows, cols, q,
+                                                  scale);
   return cudaGetLastError();
 }
 

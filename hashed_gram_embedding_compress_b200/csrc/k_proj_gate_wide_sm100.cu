@@ -34,6 +34,12 @@
 // (RN(h + RN(alpha v)) instead of RN(h + alpha v)); 3 = values for the short
 // convolution (Eq. 5): v in fp32 and its sum of squares per row and tile,
 // plus alpha; h is not read.
+// FP8 form (section 2.4, the projections as one dense FP8 matmul): e and W
+// arrive as E4M3 codes, 128 per 128-byte row of a stage (K = 32 per MMA,
+// tcgen05.mma kind::f8f6f4, fp32 accumulation), and every accumulator chunk
+// is multiplied by W's per-column scale as it leaves TMEM; e's per-row scale
+// multiplies the row's key sums (keys) or alpha (values), or v itself (phase
+// 3).  Both scales are powers of two.
 // Waits are bounded as in the single-CTA kernel; the pair leaves together
 // through a bounded handshake, then frees TMEM (cta_group::2).
 #include "sm100_ptx.cuh"
@@ -46,9 +52,10 @@ using namespace sm100;
 
 constexpr int kRows = 256;                           // tile rows per CTA
 constexpr int kCols = 256;                           // tile columns
-constexpr int BK = 64;
-constexpr uint32_t A_BYTES = kRows * BK * 2;         // 32 KB
-constexpr uint32_t B_BYTES = (kCols / 2) * BK * 2;   // 16 KB: this CTA's half of B
+constexpr int ROW_BYTES = 128;                       // of K per row and stage: 64 bf16 or 128 E4M3
+constexpr int kMmaPerStage = ROW_BYTES / 32;         // K = 16 bf16 or 32 E4M3 per MMA
+constexpr uint32_t A_BYTES = kRows * ROW_BYTES;      // 32 KB
+constexpr uint32_t B_BYTES = (kCols / 2) * ROW_BYTES;  // 16 KB: this CTA's half of B
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int STAGES = 3;
 constexpr int H_SLOTS = 5;
@@ -65,7 +72,32 @@ constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * 
 static_assert(SMEM <= 232448, "shared memory budget");
 static_assert(kEpiWarps * 8192 <= H_SLOTS * H_BYTES, "per-warp store staging fits in the h ring");
 
-template <int PHASE>
+// v[0..31] (fp32 bits, one accumulator chunk of 32 columns) *= sc[0..31]
+// (times rs when ROW): the E4M3 operands' scales.
+template <bool ROW>
+__device__ __forceinline__ void dequant_chunk(uint32_t (&v)[32], const float* sc, float rs) {
+  const float4* sp = reinterpret_cast<const float4*>(sc);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float4 s4 = __ldg(sp + c);
+    if (ROW) {
+      s4.x *= rs;
+      s4.y *= rs;
+      s4.z *= rs;
+      s4.w *= rs;
+    }
+    const float2 a = f2_unpack(
+        f2_mul(f2_pack(v[4 * c], v[4 * c + 1]), f2_pack(__float_as_uint(s4.x), __float_as_uint(s4.y))));
+    const float2 b = f2_unpack(f2_mul(f2_pack(v[4 * c + 2], v[4 * c + 3]),
+                                      f2_pack(__float_as_uint(s4.z), __float_as_uint(s4.w))));
+    v[4 * c] = __float_as_uint(a.x);
+    v[4 * c + 1] = __float_as_uint(a.y);
+    v[4 * c + 2] = __float_as_uint(b.x);
+    v[4 * c + 3] = __float_as_uint(b.y);
+  }
+}
+
+template <int PHASE, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     proj_gate_wide_kernel(const __grid_constant__ CUtensorMap map_e,
                           const __grid_constant__ CUtensorMap map_w,
@@ -102,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_total = PHASE == 0 ? M * d : d;
   const int num_n = n_total / kCols;
   const int num_tiles = ((R + 2 * kRows - 1) / (2 * kRows)) * num_n;
+  constexpr int BK = F8 ? ROW_BYTES : ROW_BYTES / 2;  // K elements per stage
   const int num_kb = (g.d_mem + BK - 1) / BK;
   const int first_tile = (int)(blockIdx.x >> 1), tile_step = (int)(gridDim.x >> 1);
   // h sub-tiles per tile: one branch in the key phase, every branch in the
@@ -240,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // --------------------------------------------- MMA issuer (leader only)
-    constexpr uint32_t idesc = idesc_bf16<2 * 128, kCols>();
+    constexpr uint32_t idesc = F8 ? idesc_e4m3<2 * 128, kCols>() : idesc_bf16<2 * 128, kCols>();
     int stage = 0;
     uint32_t phase = 0, tphase = 0;
     bool ok = true;
@@ -260,10 +293,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t a1 = sw128_desc(sA + stage * A_BYTES + A_BYTES / 2);  // rows 128-255
             const uint64_t bd = sw128_desc(sB + stage * B_BYTES);
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
+            for (int k = 0; k < kMmaPerStage; ++k) {
+              // 32 bytes of K per MMA: +2 in the descriptor's 16-byte address units
               const uint32_t accum = (kb | k) != 0;
-              umma_bf16_pair(tmem_base, a0 + 2u * k, bd + 2u * k, idesc, accum);
-              umma_bf16_pair(tmem_base + kCols, a1 + 2u * k, bd + 2u * k, idesc, accum);
+              if (F8) {
+                umma_e4m3_pair(tmem_base, a0 + 2u * k, bd + 2u * k, idesc, accum);
+                umma_e4m3_pair(tmem_base + kCols, a1 + 2u * k, bd + 2u * k, idesc, accum);
+              } else {
+                umma_bf16_pair(tmem_base, a0 + 2u * k, bd + 2u * k, idesc, accum);
+                umma_bf16_pair(tmem_base + kCols, a1 + 2u * k, bd + 2u * k, idesc, accum);
+              }
             }
             umma_commit_pair_both(empty_bar(stage));  // slot free in both CTAs
           }
@@ -300,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = row0 + r;
       const bool valid = row < R;
       const int n0 = n_blk * kCols;
+      const float se = F8 && valid ? __ldg(g.s_row + row) : 1.f;  // e's row scale
       float al[kMaxBranches];
       if (PHASE >= 1) {
         // alpha from the key phase's per-tile partial sums (Eq. 4 / Eq. 6);
@@ -351,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
           }
+          if (F8) dequant_chunk<false>(v, g.s_col + n0 + q * H_COLS, 0.f);
           if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) return;
@@ -403,6 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the weight buffer is free again; then the partial sums go out
         __syncwarp();
         if (lane == 0) mbar_arrive(wempty_bar);
+        if (F8) {  // k = se * (the column-scaled accumulator)
+          skk *= se * se;
+          shk *= se;
+        }
         if (valid) g.partials[(int64_t)n_blk * R + row] = make_float4(skk, shk, shh, 0.f);
       } else if (PHASE == 3) {
         // values for the short convolution (Eq. 5): v in fp32 and the row's
@@ -422,6 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
           }
+          if (F8) dequant_chunk<true>(v, g.s_col + n0 + q * H_COLS, se);
           unsigned long long s2[2] = {0ull, 0ull};
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -468,6 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait32(va);
           tmem_wait32(vb);
           __syncwarp();
+          if (F8) {
+            dequant_chunk<false>(va, g.s_col + n0 + q * H_COLS, 0.f);
+            dequant_chunk<false>(vb, g.s_col + n0 + (q + 1) * H_COLS, 0.f);
+          }
           if (q + 2 >= NQ) {
             tc_fence_before();  // last TMEM read done: release the accumulators
             __syncwarp();
@@ -479,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int b = 0; b < kMaxBranches; ++b)
               if (b == mb) a = al[b];
+            if (F8) a *= se;  // alpha v = (alpha se) (the column-scaled accumulator)
             const unsigned long long a2 = f2_pack(__float_as_uint(a), __float_as_uint(a));
             // the buffer's previous reduce has finished reading it
             if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
@@ -537,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
           }
+          if (F8) dequant_chunk<false>(v, g.s_col + n0 + q * H_COLS, 0.f);
 #pragma unroll 1
           for (int mb = 0; mb < M; ++mb) {
             if (lane == 0) ok = wait_ready(hfull_bar(hslot), hphase, abort_flag, g.err);
@@ -547,6 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int b = 0; b < kMaxBranches; ++b)
               if (b == mb) a = al[b];
+            if (F8) a *= se;  // alpha v = (alpha se) (the column-scaled accumulator)
             // out = h + alpha v, written over h in place, then stored by TMA
             const unsigned long long a2 = f2_pack(__float_as_uint(a), __float_as_uint(a));
 #pragma unroll
@@ -626,9 +679,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                  "r"(TMEM_COLS));
 }
 
-template <int PHASE>
+template <int PHASE, bool F8>
 cudaError_t launch_wide(const ProjMaps& maps, const GateArgs& g, int grid, cudaStream_t stream) {
-  auto kern = proj_gate_wide_kernel<PHASE>;
+  auto kern = proj_gate_wide_kernel<PHASE, F8>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
   if (e != cudaSuccess) return e;
@@ -652,14 +705,19 @@ cudaError_t launch_wide(const ProjMaps& maps, const GateArgs& g, int grid, cudaS
 }  // namespace
 
 cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, bool f8) {
   if (g.R == 0) return cudaSuccess;
   if (grid < 2 || (grid & 1)) return cudaErrorInvalidValue;
-  switch (phase) {
-    case 0: return launch_wide<0>(maps, g, grid, stream);
-    case 1: return launch_wide<1>(maps, g, grid, stream);
-    case 2: return launch_wide<2>(maps, g, grid, stream);
-    case 3: return launch_wide<3>(maps, g, grid, stream);
+  if (f8 && (!g.s_row || !g.s_col)) return cudaErrorInvalidValue;
+  switch (phase * 2 + (f8 ? 1 : 0)) {
+    case 0: return launch_wide<0, false>(maps, g, grid, stream);
+    case 1: return launch_wide<0, true>(maps, g, grid, stream);
+    case 2: return launch_wide<1, false>(maps, g, grid, stream);
+    case 3: return launch_wide<1, true>(maps, g, grid, stream);
+    case 4: return launch_wide<2, false>(maps, g, grid, stream);
+    case 5: return launch_wide<2, true>(maps, g, grid, stream);
+    case 6: return launch_wide<3, false>(maps, g, grid, stream);
+    case 7: return launch_wide<3, true>(maps, g, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -30,7 +30,8 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_gather", "engram_forward", "engram_prefetch", "engram_check_errors",
            "engram_profile_next_forward", "engram_kernel_launches",
            "engram_project_gate_noalloc", "engram_selftest_timeout", "engram_set_short_conv",
-           "engram_build_hot_cache", "engram_prefetch_hot_hits")
+           "engram_build_hot_cache", "engram_prefetch_hot_hits", "engram_set_fp8",
+           "engram_quantize_e4m3")
 
 
 class engram_config(ctypes.Structure):
@@ -69,6 +70,8 @@ def _load():
         "engram_set_short_conv": ([H, P, P, i32, i32, P], ctypes.c_int),
         "engram_build_hot_cache": ([H, P, i32, i32, i32, i64, P], ctypes.c_int),
         "engram_prefetch_hot_hits": ([H, P], ctypes.c_int),
+        "engram_set_fp8": ([H, i32, P], ctypes.c_int),
+        "engram_quantize_e4m3": ([H, P, i64, i32, P, P, P], ctypes.c_int),
         "engram_get_hash_params": ([H, P, P], ctypes.c_int),
         "engram_hash": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
@@ -180,6 +183,17 @@ class Engram:
         and norm_w [d] (fp32, device; copied); kernel_size 0 switches it off."""
         self._check(lib.engram_set_short_conv(self._h, _ptr(conv_w), _ptr(norm_w), kernel_size,
                                               dilation, _stream_ptr(stream)))
+
+    def set_fp8(self, enable: bool = True, stream=None):
+        """Projections on E4M3 operands (section 2.4), or back to bf16."""
+        self._check(lib.engram_set_fp8(self._h, 1 if enable else 0, _stream_ptr(stream)))
+
+    def quantize_e4m3(self, x, q, scale, stream=None):
+        """E4M3 codes q (uint8 [rows, cols]) and power-of-two row scales
+        (fp32 [rows]) of bf16 x [rows, cols], all on the device."""
+        rows, cols = x.shape
+        self._check(lib.engram_quantize_e4m3(self._h, _ptr(x), rows, cols, _ptr(q), _ptr(scale),
+                                             _stream_ptr(stream)))
 
     def reserve(self, max_rows: int):
         self._check(lib.engram_reserve(self._h, max_rows))

@@ -190,6 +190,43 @@ ENGRAM_API int engram_set_short_conv(engram_handle *h, const float *conv_w, cons
                                      int32_t kernel_size, int32_t dilation, void *stream);
 
 /*
+ * FP8 projections (section 2.4: the value projection and the M key
+ * projections computed as one dense FP8 matmul).  enable = 1: every later
+ * engram_forward multiplies an E4M3 form of e by an E4M3 copy of [W_K; W_V]
+ * with fp32 accumulation (tcgen05.mma kind::f8f6f4); enable = 0 returns to
+ * bf16 operands.  The pages give neither the format nor the scaling; here
+ * each row of e (position) and each row of W (output channel) is quantised
+ * as engram_quantize_e4m3 describes, and both scales multiply the fp32
+ * products in the epilogue; the gate and output are unchanged.  The copy of
+ * W is made now (on `stream`, then the device is synchronised) and again by
+ * every engram_set_params while FP8 is on.  Needs a bf16 handle, d a multiple
+ * of 256, d_mem a multiple of 128 and at most 2048, and CTA pairs (no
+ * ENGRAM_FLAG_NO_CTA_PAIRS); otherwise ENGRAM_ERR_UNSUPPORTED.  While it is
+ * on, engram_project_gate_noalloc returns ENGRAM_ERR_UNSUPPORTED.  Device
+ * memory: (M + 1) d (d_mem + 4) bytes for W, and d_mem + 4 bytes of scratch
+ * per row.  Errors: _INVALID (enable not 0 or 1), _STATE (engram_set_params
+ * first), _UNSUPPORTED, _OOM, _CUDA.
+ */
+ENGRAM_API int engram_set_fp8(engram_handle *h, int32_t enable, void *stream);
+
+/*
+ * The quantiser of the FP8 projections, one row at a time: with amax the
+ * largest magnitude in row r of x and E the smallest integer for which
+ * amax <= 448 * 2^E (E = 0 when amax = 0), scale[r] = 2^E and
+ * q[r, j] = E4M3(x[r, j] * 2^-E), rounded to the nearest E4M3 value with ties
+ * to even and saturated at +-448 (E4M3: 1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits, no infinities, S.1111.111 NaN; zero keeps its sign).
+ * x * 2^-E is exact, so the codes are a function of x alone.
+ *  x      device bf16 [rows, cols], finite values, 16-byte aligned.
+ *  q      device uint8 [rows, cols] E4M3 codes, 16-byte aligned.
+ *  scale  device fp32 [rows], 4-byte aligned.
+ * 16 <= cols <= 2048, cols a multiple of 16.  Enqueued on `stream`.
+ * Errors: _INVALID, _CUDA.
+ */
+ENGRAM_API int engram_quantize_e4m3(engram_handle *h, const void *x, int64_t rows, int32_t cols,
+                                    uint8_t *q, float *scale, void *stream);
+
+/*
  * Pre-allocate the handle's device scratch for calls of up to `max_rows`
  * emitted positions (rows = B * (T - t_begin)).  Calls with more rows grow the
  * scratch themselves; reserving first keeps allocation out of timed or

@@ -91,12 +91,20 @@ class Problem:
             zz[:, s] = np.arange(len(rows))
         return mini, zz
 
-    def oracle_forward(self, rows: np.ndarray, eps: float = 1e-6):
+    def oracle_forward(self, rows: np.ndarray, eps: float = 1e-6, fp8: bool = False):
+        """e, alpha, delta, out at `rows`; fp8: the projections on E4M3 operands
+        (section 2.4), e quantised per row and W per output channel."""
         mini, zz = self.table_rows(rows)
         e = oracle.gather(mini, zz)
         h = to_oracle(self.h[torch.from_numpy(rows).to(self.h.device)])
-        alpha, delta, out = oracle.project_gate(e, to_oracle(self.w_k_cpu), to_oracle(self.w_v_cpu),
-                                                self.nq_cpu.numpy(), self.nk_cpu.numpy(), h, eps)
+        args = (e, to_oracle(self.w_k_cpu), to_oracle(self.w_v_cpu), self.nq_cpu.numpy(),
+                self.nk_cpu.numpy(), h, eps)
+        if fp8:
+            if getattr(self, "_w8", None) is None:
+                self._w8 = oracle.quantize_weights_e4m3(args[1], args[2])
+            alpha, delta, out = oracle.project_gate_fp8(*args, weights=self._w8)
+        else:
+            alpha, delta, out = oracle.project_gate(*args)
         return e, alpha, delta, out
 
     def conv_weights(self, kernel_size: int = 4):
@@ -104,7 +112,7 @@ class Problem:
         return synth.make_conv_weights(self.shape, self.seeds, kernel_size)
 
     def oracle_forward_conv(self, rows: np.ndarray, conv_w, norm_w, dilation: int,
-                            eps: float = 1e-6):
+                            eps: float = 1e-6, fp8: bool = False):
         """Y [n, M, d] (double) and out [n, M, d] (h's dtype) of Eq. (5) at `rows`
         (t_begin = 0, row = b T + t): the gated values alpha v are formed by
         the oracle at the positions the taps read, t - i * dilation."""
@@ -115,7 +123,7 @@ class Problem:
         need = sorted({int(r) - i * dilation for r in rows for i in range(W)
                        if (int(r) % T) - i * dilation >= 0})
         need = np.array(need, dtype=np.int64)
-        _, _, vt, _ = self.oracle_forward(need, eps)          # delta = alpha v [n, M, d]
+        _, _, vt, _ = self.oracle_forward(need, eps, fp8)     # delta = alpha v [n, M, d]
         pos = {int(r): j for j, r in enumerate(need)}
         M, d = sh.branches, sh.d_hidden
         cw, nw = conv_w.numpy(), norm_w.numpy()

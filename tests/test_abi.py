@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_header_and_binding_agree(eg):
     names = declared_symbols()
-    assert names == set(eg.EXPORTS) and len(names) == 19
+    assert names == set(eg.EXPORTS) and len(names) == 21
 
 
 def test_library_exports_every_declared_symbol(eg):
@@ -94,7 +94,9 @@ def test_null_arguments(eg):
                      ("engram_selftest_timeout", (None, None)),
                      ("engram_set_short_conv", (None, None, None, 4, 3, None)),
                      ("engram_build_hot_cache", (None, None, 1, 1, 0, 1, None)),
-                     ("engram_prefetch_hot_hits", (None, None))):
+                     ("engram_prefetch_hot_hits", (None, None)),
+                     ("engram_set_fp8", (None, 1, None)),
+                     ("engram_quantize_e4m3", (None, None, 1, 16, None, None, None))):
         assert getattr(eg.lib, fn)(*args) == eg.ENGRAM_ERR_INVALID, fn
     assert eg.lib.engram_kernel_launches(None) == -1
     eg.lib.engram_destroy(None)
