@@ -84,8 +84,18 @@ def lib():
         L.eo_quantize_e4m3_rows.restype = None
         L.eo_dequantize_e4m3_rows.argtypes = [P, P, i64, i32, P]
         L.eo_dequantize_e4m3_rows.restype = None
+        L.eo_backward.argtypes = [P, i32, i64, i32, P, P, P, P, i32, i32, f64, P, i32, P, i32,
+                                  P, P, P, P, P, P, P, P, P]
+        L.eo_backward.restype = None
+        L.eo_table_grad.argtypes = [P, P, i64, i32, i32, P]
+        L.eo_table_grad.restype = None
         _lib = L
     return _lib
+
+
+def _dtype_of(a: np.ndarray) -> int:
+    return {np.dtype(np.float64): F64, np.dtype(np.float32): F32,
+            np.dtype(np.uint16): BF16}[a.dtype]
 
 
 def _p(a: np.ndarray):
@@ -258,7 +268,8 @@ def dequantize_e4m3_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 
 def project_gate_mixed(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: bool = True):
-    """project_gate with e, w_k, w_v in double and h in its own dtype."""
+    """project_gate with e, w_k, w_v in double and h in its own dtype (float64,
+    float32 or uint16 bf16 bits; out in the same)."""
     e = np.ascontiguousarray(e, dtype=np.float64)
     rows, dm = e.shape
     M, d, dm2 = w_k.shape
@@ -266,7 +277,7 @@ def project_gate_mixed(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: b
     w_k = np.ascontiguousarray(w_k, dtype=np.float64)
     w_v = np.ascontiguousarray(w_v, dtype=np.float64)
     h = np.ascontiguousarray(h)
-    hdtype = F32 if h.dtype == np.float32 else BF16
+    hdtype = _dtype_of(h)
     nq = np.ascontiguousarray(norm_q, dtype=np.float32)
     nk = np.ascontiguousarray(norm_k, dtype=np.float32)
     alpha = np.empty((rows, M), dtype=np.float64)
@@ -299,6 +310,56 @@ def project_gate_fp8(e, w_k, w_v, norm_q, norm_k, h, eps: float, want_delta: boo
     ehat = dequantize_e4m3_rows(*quantize_e4m3_rows(e))
     wk, wv = weights if weights is not None else quantize_weights_e4m3(w_k, w_v)
     return project_gate_mixed(ehat, wk, wv, norm_q, norm_k, h, eps, want_delta)
+
+
+# ------------------------------------------------------------------ backward
+
+def backward(e, w_k, w_v, norm_q, norm_k, h, dout, eps: float, round_dkv: bool = False):
+    """Gradients of project_gate's out for the upstream gradient dout [rows, M, d].
+
+    e, w_k, w_v share one dtype (float64, float32 or uint16 bf16 bits); h has
+    its own.  Returns dict(dh [rows, M, d], dkv [rows, (M+1) d] (dk of each
+    branch, then dv; bf16-rounded when round_dkv), dw_k [M, d, d_mem],
+    dw_v [d, d_mem], dnorm_q [M, d], dnorm_k [M, d], de [rows, d_mem]), all
+    double."""
+    e = np.ascontiguousarray(e)
+    rows, dm = e.shape
+    M, d, dm2 = w_k.shape
+    assert dm2 == dm and w_v.shape == (d, dm) and h.shape == (rows, M, d)
+    w_k = np.ascontiguousarray(w_k, dtype=e.dtype)
+    w_v = np.ascontiguousarray(w_v, dtype=e.dtype)
+    h = np.ascontiguousarray(h)
+    g = np.ascontiguousarray(dout, dtype=np.float64)
+    assert g.shape == h.shape
+    nq = np.ascontiguousarray(norm_q, dtype=np.float32)
+    nk = np.ascontiguousarray(norm_k, dtype=np.float32)
+    dh = np.empty((rows, M, d))
+    dkv = np.empty((rows, (M + 1) * d))
+    dw = np.zeros(((M + 1) * d, dm))
+    dwq = np.zeros((M, d))
+    dwk = np.zeros((M, d))
+    de = np.empty((rows, dm))
+    kb, vb, hb = np.empty(M * d), np.empty(d), np.empty(d)
+    lib().eo_backward(_p(e), _dtype_of(e), rows, dm, _p(w_k), _p(w_v), _p(nq), _p(nk), M, d,
+                      eps, _p(h), _dtype_of(h), _p(g), 1 if round_dkv else 0, _p(dh), _p(dkv),
+                      _p(dw), _p(dwq), _p(dwk), _p(de), _p(kb), _p(vb), _p(hb))
+    return dict(dh=dh, dkv=dkv, dw_k=dw[:M * d].reshape(M, d, dm), dw_v=dw[M * d:],
+                dnorm_q=dwq, dnorm_k=dwk, de=de)
+
+
+def table_grad(de: np.ndarray, z: np.ndarray, table_rows: Sequence[int], d_head: int):
+    """dE_s [p_s, d_h] (double) += the slot-s slices of de at rows z[:, s] (Eq. 2
+    transposed); returns the list of S arrays."""
+    de = np.ascontiguousarray(de, dtype=np.float64)
+    z = np.ascontiguousarray(z, dtype=np.int64)
+    rows, S = z.shape
+    assert de.shape == (rows, S * d_head) and len(table_rows) == S
+    if z.size:
+        assert (z >= 0).all() and (z < np.asarray(table_rows)[None, :]).all()
+    out = [np.zeros((int(p), d_head)) for p in table_rows]
+    ptrs = (ctypes.c_void_p * S)(*[t.ctypes.data for t in out])
+    lib().eo_table_grad(_p(de), _p(z), rows, S, d_head, ptrs)
+    return out
 
 
 # ---------------------------------------------------------------- short conv

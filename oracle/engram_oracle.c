@@ -286,7 +286,8 @@ void eo_project_gate_mixed(const void *e, int32_t wdtype, int64_t rows, int32_t 
                 double dl = a * vbuf[i];
                 double o = hbuf[i] + dl;
                 if (delta) delta[base + i] = dl;
-                if (hdtype == EO_F32) ((float *)out)[base + i] = (float)o;
+                if (hdtype == EO_F64) ((double *)out)[base + i] = o;
+                else if (hdtype == EO_F32) ((float *)out)[base + i] = (float)o;
                 else ((uint16_t *)out)[base + i] = eo_bf16_rne(o);
             }
         }
@@ -457,4 +458,132 @@ void eo_add_round(const void *h, int32_t dtype, int64_t n, const double *y, void
         if (dtype == EO_F32) ((float *)out)[i] = (float)o;
         else ((uint16_t *)out)[i] = eo_bf16_rne(o);
     }
+}
+
+/* ---------------------------------------------------------------- backward */
+
+/*
+ * Gradients of the forward above (Eq. 3, Eq. 4 / Eq. 6 and the gated
+ * residual) for a scalar loss whose gradient with respect to out is dout.
+ * The pages give only the forward; the backward is its exact derivative,
+ * written out per row r and branch m (all in double):
+ *
+ *   k = W_K^(m) e, v = W_V e, rh = (mean(h^2) + eps)^-1/2, rk likewise for k,
+ *   qn = h rh w_q, kn = k rk w_k, s = qn . kn / sqrt(d), alpha = sigmoid(s),
+ *   out = h + alpha v.
+ *
+ *   dalpha = dout . v                  dv   += alpha dout
+ *   ds     = dalpha alpha (1 - alpha)
+ *   dqn    = ds kn / sqrt(d)           dkn   = ds qn / sqrt(d)
+ *   dw_q  += dqn h rh                  dw_k += dkn k rk
+ *   RMSNorm x^ = x r: with u = dqn w_q (resp. dkn w_k),
+ *     dx = r u - r^3 / d x (u . x)
+ *   dh     = dout + rh u_q - rh^3 / d h (u_q . h)
+ *   dk     = rk u_k - rk^3 / d k (u_k . k)
+ *   dW_K^(m) += dk e^T,  dW_V += dv e^T,
+ *   de     = sum_m W_K^(m)T dk + W_V^T dv,
+ *   dE_s[z_s] += the slot-s slice of de (slot_rows_grad below).
+ *
+ * round_dkv != 0: dk and dv are rounded to bf16 (nearest-even, through
+ * float) before they multiply e and W, as a bf16 training step feeds them to
+ * its tensor-core GEMMs; the gradients are then exact functions of those
+ * rounded values.  dh is returned in double.
+ *   e     [rows, d_mem] wdtype;  w_k [M, d, d_mem], w_v [d, d_mem] wdtype
+ *   h     [rows, M, d] hdtype;   dout [rows, M, d] double
+ *   dh    [rows, M, d] double (out)
+ *   dkv   [rows, (M + 1) d] double (out): dk of each branch, then dv, as used
+ *         by the weight GEMMs (rounded when round_dkv)
+ *   dw    [(M + 1) d, d_mem] double, accumulated: dW_K rows, then dW_V
+ *   dwq, dwk [M, d] double, accumulated
+ *   de    [rows, d_mem] double (out)
+ * Scratch: kbuf [M d], vbuf [d], hbuf [d] doubles.
+ */
+void eo_backward(const void *e, int32_t wdtype, int64_t rows, int32_t d_mem,
+                 const void *w_k, const void *w_v, const float *wq, const float *wk,
+                 int32_t M, int32_t d, double eps, const void *h, int32_t hdtype,
+                 const double *dout, int32_t round_dkv, double *dh, double *dkv, double *dw,
+                 double *dwq, double *dwk, double *de,
+                 double *kbuf, double *vbuf, double *hbuf)
+{
+    const int64_t nkv = (int64_t)(M + 1) * d;
+    const double isd = 1.0 / sqrt((double)d);
+    int64_t r, o;
+    int32_t m, i, j;
+    for (r = 0; r < rows; ++r) {
+        const char *er = (const char *)e + (size_t)r * d_mem * eo_elem_bytes(wdtype);
+        double *gkv = dkv + r * nkv;
+        double *dv = gkv + (int64_t)M * d;
+        eo_project(er, wdtype, 1, d_mem, w_k, M * d, kbuf);
+        eo_project(er, wdtype, 1, d_mem, w_v, d, vbuf);
+        for (i = 0; i < d; ++i) dv[i] = 0.0;
+        for (m = 0; m < M; ++m) {
+            const int64_t base = (r * M + m) * (int64_t)d;
+            const double *k = kbuf + (int64_t)m * d;
+            const float *wqm = wq + (int64_t)m * d, *wkm = wk + (int64_t)m * d;
+            const double *g = dout + base;
+            double sh = 0.0, sk = 0.0, s = 0.0, da = 0.0, uh = 0.0, uk = 0.0;
+            double rh, rk, a, ds;
+            for (i = 0; i < d; ++i) hbuf[i] = eo_load(h, hdtype, base + i);
+            for (i = 0; i < d; ++i) { sh += hbuf[i] * hbuf[i]; sk += k[i] * k[i]; }
+            rh = 1.0 / sqrt(sh / d + eps);
+            rk = 1.0 / sqrt(sk / d + eps);
+            for (i = 0; i < d; ++i) s += (hbuf[i] * rh * wqm[i]) * (k[i] * rk * wkm[i]);
+            a = 1.0 / (1.0 + exp(-s * isd));
+            for (i = 0; i < d; ++i) { da += g[i] * vbuf[i]; dv[i] += a * g[i]; }
+            ds = da * a * (1.0 - a);
+            /* u_q = dqn w_q, u_k = dkn w_k, with dqn = ds kn / sqrt(d), dkn = ds qn / sqrt(d) */
+            for (i = 0; i < d; ++i) {
+                const double qn = hbuf[i] * rh * wqm[i], kn = k[i] * rk * wkm[i];
+                const double dqn = ds * kn * isd, dkn = ds * qn * isd;
+                dwq[(int64_t)m * d + i] += dqn * hbuf[i] * rh;
+                dwk[(int64_t)m * d + i] += dkn * k[i] * rk;
+                uh += dqn * wqm[i] * hbuf[i];
+                uk += dkn * wkm[i] * k[i];
+            }
+            for (i = 0; i < d; ++i) {
+                const double qn = hbuf[i] * rh * wqm[i], kn = k[i] * rk * wkm[i];
+                const double dqn = ds * kn * isd, dkn = ds * qn * isd;
+                dh[base + i] = g[i] + rh * dqn * wqm[i] - rh * rh * rh / d * hbuf[i] * uh;
+                gkv[(int64_t)m * d + i] = rk * dkn * wkm[i] - rk * rk * rk / d * k[i] * uk;
+            }
+        }
+        if (round_dkv)
+            for (o = 0; o < nkv; ++o) {
+                const uint16_t b = eo_bf16_rne(gkv[o]);
+                uint32_t u = (uint32_t)b << 16;
+                float f;
+                memcpy(&f, &u, 4);
+                gkv[o] = (double)f;
+            }
+        /* weight gradients and de (Eq. 3 transposed) */
+        for (o = 0; o < nkv; ++o)
+            for (j = 0; j < d_mem; ++j)
+                dw[o * d_mem + j] += gkv[o] * eo_load(e, wdtype, r * d_mem + j);
+        for (j = 0; j < d_mem; ++j) {
+            double acc = 0.0;
+            for (o = 0; o < nkv; ++o) {
+                const void *w = o < (int64_t)M * d ? w_k : w_v;
+                const int64_t wo = o < (int64_t)M * d ? o : o - (int64_t)M * d;
+                acc += gkv[o] * eo_load(w, wdtype, wo * d_mem + j);
+            }
+            de[r * d_mem + j] = acc;
+        }
+    }
+}
+
+/*
+ * Table gradients (Eq. 2 transposed): for every row r and slot s,
+ * dtab[s][z[r][s]][i] += de[r][s d_h + i].  dtab is an array of S pointers to
+ * double [p_s, d_h]; z [rows, S] the indices of the forward.
+ */
+void eo_table_grad(const double *de, const int64_t *z, int64_t rows, int32_t S, int32_t d_head,
+                   double *const *dtab)
+{
+    int64_t r;
+    int32_t s, i;
+    for (r = 0; r < rows; ++r)
+        for (s = 0; s < S; ++s) {
+            double *row = dtab[s] + z[r * S + s] * d_head;
+            for (i = 0; i < d_head; ++i) row[i] += de[r * (int64_t)S * d_head + (int64_t)s * d_head + i];
+        }
 }

@@ -471,3 +471,99 @@ def test_project_gate_fp8_against_torch_fp64():
                                     _bf16_bits(h), 1e-6)
     rel = np.linalg.norm(delta - d0) / np.linalg.norm(d0)
     assert 1e-4 < rel < 0.1
+
+
+# ------------------------------------------------------- backward (row f4)
+
+def _bw_problem(R=3, M=2, d=8, dm=12, seed=0):
+    rng = np.random.default_rng(seed)
+    e = rng.normal(size=(R, dm))
+    wk = rng.normal(size=(M, d, dm)) / 3
+    wv = rng.normal(size=(d, dm)) / 3
+    h = rng.normal(size=(R, M, d))
+    g = rng.normal(size=(R, M, d))
+    nq = (1 + 0.1 * rng.normal(size=(M, d))).astype(np.float32)
+    nk = (1 + 0.1 * rng.normal(size=(M, d))).astype(np.float32)
+    return e, wk, wv, nq, nk, h, g
+
+
+def _loss(e, wk, wv, nq, nk, h, g):
+    _, delta, _ = oracle.project_gate_mixed(e, wk, wv, nq, nk, h, 1e-6)
+    return float(np.sum(g * (h + delta)))
+
+
+def test_backward_matches_finite_differences():
+    e, wk, wv, nq, nk, h, g = _bw_problem()
+    b = oracle.backward(e, wk, wv, nq, nk, h, g, 1e-6)
+    step = 1e-6
+    for name, arr, grad in (("e", e, b["de"]), ("w_k", wk, b["dw_k"]), ("w_v", wv, b["dw_v"]),
+                            ("h", h, b["dh"])):
+        rng = np.random.default_rng(len(name))
+        for flat in rng.choice(arr.size, size=min(arr.size, 12), replace=False):
+            idx = np.unravel_index(flat, arr.shape)
+            orig = arr[idx]
+            arr[idx] = orig + step
+            lp = _loss(e, wk, wv, nq, nk, h, g)
+            arr[idx] = orig - step
+            lm = _loss(e, wk, wv, nq, nk, h, g)
+            arr[idx] = orig
+            fd = (lp - lm) / (2 * step)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_backward_matches_torch_autograd():
+    e, wk, wv, nq, nk, h, g = _bw_problem(R=4, M=3, d=16, dm=24, seed=5)
+    b = oracle.backward(e, wk, wv, nq, nk, h, g, 1e-6)
+    E, WK, WV, H = [torch.tensor(x, requires_grad=True) for x in (e, wk, wv, h)]
+    NQ = torch.tensor(nq.astype(np.float64), requires_grad=True)
+    NK = torch.tensor(nk.astype(np.float64), requires_grad=True)
+    k = torch.einsum("rj,mij->rmi", E, WK)
+    v = E @ WV.T
+    qn = torch.nn.functional.rms_norm(H, (16,), eps=1e-6) * NQ
+    kn = torch.nn.functional.rms_norm(k, (16,), eps=1e-6) * NK
+    a = torch.sigmoid((qn * kn).sum(-1) / 4.0)
+    out = H + a[..., None] * v[:, None, :]
+    (out * torch.tensor(g)).sum().backward()
+    for mine, ref in ((b["de"], E.grad), (b["dw_k"], WK.grad), (b["dw_v"], WV.grad),
+                      (b["dh"], H.grad), (b["dnorm_q"], NQ.grad), (b["dnorm_k"], NK.grad)):
+        assert np.allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_special_cases():
+    e, wk, wv, nq, nk, h, g = _bw_problem(seed=2)
+    z = oracle.backward(e, wk, wv, nq, nk, h, np.zeros_like(g), 1e-6)
+    assert all((v == 0).all() for k, v in z.items() if k != "dh") and (z["dh"] == 0).all()
+    # W_V = 0: alpha multiplies nothing, so dalpha = 0 and only the residual and dv remain
+    b = oracle.backward(e, wk, np.zeros_like(wv), nq, nk, h, g, 1e-6)
+    assert np.array_equal(b["dh"], g) and (b["dw_k"] == 0).all() and (b["dnorm_q"] == 0).all()
+    alpha, _, _ = oracle.project_gate_mixed(e, wk, np.zeros_like(wv), nq, nk, h, 1e-6)
+    dv = np.einsum("rm,rmi->ri", alpha, g)
+    assert np.allclose(b["dw_v"], dv.T @ e, rtol=1e-12, atol=1e-14)
+
+
+def test_backward_bf16_rounding_of_gemm_operands():
+    e, wk, wv, nq, nk, h, g = _bw_problem(R=5, M=2, d=16, dm=24, seed=7)
+    exact = oracle.backward(e, wk, wv, nq, nk, h, g, 1e-6)
+    b = oracle.backward(e, wk, wv, nq, nk, h, g, 1e-6, round_dkv=True)
+    want = torch.tensor(exact["dkv"]).float().bfloat16().double().numpy()
+    assert np.array_equal(b["dkv"], want)
+    assert np.array_equal(b["dh"], exact["dh"]) and np.array_equal(b["dnorm_q"], exact["dnorm_q"])
+    M, d, dm = wk.shape
+    dw = torch.tensor(want).T @ torch.tensor(e)
+    assert np.allclose(np.concatenate([b["dw_k"].reshape(M * d, dm), b["dw_v"]]), dw.numpy(),
+                       rtol=1e-12, atol=1e-14)
+    W = np.concatenate([wk.reshape(M * d, dm), wv])
+    assert np.allclose(b["de"], want @ W, rtol=1e-12, atol=1e-14)
+
+
+def test_table_grad_matches_numpy_scatter_add():
+    rng = np.random.default_rng(4)
+    rows, S, dh = 50, 3, 4
+    sizes = [7, 11, 13]
+    z = np.stack([rng.integers(0, p, rows) for p in sizes], 1)   # repeats: rows collide
+    de = rng.normal(size=(rows, S * dh))
+    got = oracle.table_grad(de, z, sizes, dh)
+    for s, p in enumerate(sizes):
+        want = np.zeros((p, dh))
+        np.add.at(want, z[:, s], de[:, s * dh:(s + 1) * dh])
+        assert np.allclose(got[s], want, rtol=1e-14, atol=1e-15)
