@@ -68,6 +68,9 @@ def parse():
     ap.add_argument("--fp8", action="store_true",
                     help="projections on E4M3 operands (section 2.4's FP8 matmul): e quantised "
                          "per row inside the gather, W per output channel; prefill-type workloads")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward (training) step instead of the forward: gradients "
+                         "of h, W_K, W_V, the RMSNorm weights and the tables for a seeded dL/dout")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a captured CUDA graph (launch-bound shapes)")
     ap.add_argument("--offload-gb", type=float, default=100.0,
@@ -474,6 +477,130 @@ def run_ours(args, rank, world, dist):
     return res
 
 
+# ---------------------------------------------------------- backward leg
+
+def run_backward_bench(args, rank, world, dist):
+    """The backward step on the same workload: dh, dW_K, dW_V, dnorm_q,
+    dnorm_k and the fp32 table gradients (accumulated) for a seeded dL/dout."""
+    import torch
+    from hashed_gram_embedding_compress_b200 import synth
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    P = setup(rank, device, args.rows_target, args.workload)
+    sh, m, h = P["sh"], P["m"], P["h"]
+    R, M, d, dm = sh.rows_out, sh.branches, sh.d_hidden, sh.d_mem
+    tok_d = P["tokens"].to(device)
+    dout = synth.make_grad_out(sh, P["seeds"], device=device)
+    dh = torch.empty_like(h)
+    g = dict(dw_k=torch.zeros((M, d, dm), device=device), dw_v=torch.zeros((d, dm), device=device),
+             dnorm_q=torch.zeros((M, d), device=device), dnorm_k=torch.zeros((M, d), device=device),
+             dtables=[torch.zeros((int(p), sh.d_head), device=device) for p in P["primes"]])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        m.backward(tok_d, h, dout, dh, t_begin=sh.t_begin, stream=stream, **g)
+
+    clk = ClockSampler(local).__enter__()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if m.check_errors(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    t_load = time.monotonic()
+    while time.monotonic() - t_load < 1.5:
+        for _ in range(5):
+            step()
+        torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    for row in evs:
+        for ev in row:
+            ev.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = m.kernel_launches()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(K):
+        m.profile_next_backward(evs[k])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    t_end = time.monotonic()
+    time.sleep(0.3)
+    clk.__exit__(None, None, None)
+    if dist:
+        dist.barrier()
+    launches = m.kernel_launches() - launches0
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, device)
+    st = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)) / K for i in range(5)]
+    if m.check_errors(stream) != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    # e2e: h and dL/dout in from pinned host memory, dh back, every step
+    E = max(1, args.e2e_steps)
+    h_h, g_h = h.cpu().pin_memory(), dout.cpu().pin_memory()
+    dh_h = torch.empty_like(h_h).pin_memory()
+    tok_h = P["tokens"].pin_memory()
+    tok_b, h_b, g_b = torch.empty_like(tok_d), torch.empty_like(h), torch.empty_like(dout)
+
+    def e2e_step():
+        tok_b.copy_(tok_h, non_blocking=True)
+        h_b.copy_(h_h, non_blocking=True)
+        g_b.copy_(g_h, non_blocking=True)
+        m.backward(tok_b, h_b, g_b, dh, t_begin=sh.t_begin, stream=stream, **g)
+        dh_h.copy_(dh, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    if rank != 0:
+        return None
+
+    hbm, tflops, tflops_burst, peak_kind = load_peaks()
+    A = algorithmic(sh)
+    gemm_flops = 3 * A["gemm_flops"]       # k, v recomputed; weight gradients; de
+    gemm_s = (st[1] + st[3] + st[4]) / 1e3
+    elt = 2 if sh.dtype == "bf16" else 4
+    # gate backward: h, dout, k and v (fp32) read; dh and [dk dv] written
+    gate_bytes = R * (2 * M * d * elt + 4 * (M + 1) * d + M * d * elt + (M + 1) * d * elt)
+    return {
+        "metric": "Engram backward tokens/s (gradients of h, W_K, W_V, RMSNorm weights, tables)",
+        "value": R * world * K / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype, "data": "synthetic",
+        "config": {"workload": DESCRIBE[args.workload] + " [backward step, dL/dout ~ N(0, 1)]",
+                   "global_batch": R * world, "seq_len": sh.T,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "no flush: inputs larger than L2"},
+        "roofline": {"kernel": "cuBLAS GEMMs (k, v recomputed; dW; de) of the backward",
+                     "bound": "tensor", "achieved": gemm_flops / gemm_s / 1e12, "peak": tflops,
+                     "unit": "TFLOP/s", "frac": gemm_flops / gemm_s / 1e12 / tflops,
+                     "traffic": None, "frac_of_burst": gemm_flops / gemm_s / 1e12 / tflops_burst},
+        "gate_backward": {"kernel": "gate_backward_kernel + dnorm_reduce_kernel", "bound": "hbm",
+                          "achieved_gbs": gate_bytes / (st[2] / 1e3) / 1e9, "peak_gbs": hbm,
+                          "frac": gate_bytes / (st[2] / 1e3) / 1e9 / hbm,
+                          "bytes_per_step": gate_bytes},
+        "stages_ms": {"hash_gather": st[0], "kv_recompute": st[1], "gate_backward": st[2],
+                      "weight_grads": st[3], "de_and_table_grads": st[4]},
+        "e2e": {"value": R * world * E / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": tok_h.numel() * 4 + 2 * h_h.numel() * h_h.element_size(),
+                "d2h_bytes_per_step": dh_h.numel() * dh_h.element_size(), "steps": E},
+        "gpu_launches": launches,
+        "clocks": dict(clk.summary(t_load + 0.5, t_end + 0.15),
+                       window="last 1 s of back-to-back warm-up steps and the timed steps"),
+    }
+
+
 # ------------------------------------------------------ host-offload leg
 
 def run_offload(args):
@@ -747,6 +874,8 @@ def main():
         res = run_reference(args, rank, world)
     elif args.workload == "offload":
         res = run_offload(args) if rank == 0 else None
+    elif args.backward:
+        res = run_backward_bench(args, rank, world, dist)
     else:
         res = run_ours(args, rank, world, dist)
     if res is not None:

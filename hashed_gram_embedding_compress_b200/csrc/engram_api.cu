@@ -376,6 +376,12 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->partials);
   free_dev(h->d_w8);
   free_dev(h->d_sw8);
+  free_dev(h->bw_idx);
+  free_dev(h->bw_kv);
+  free_dev(h->bw_dkv);
+  free_dev(h->bw_de);
+  free_dev(h->bw_partials);
+  if (h->blas) cublasDestroy(h->blas);
   free_dev(h->e8);
   free_dev(h->se8);
   free_dev(h->d_conv_w);
@@ -442,6 +448,8 @@ int engram_set_params(engram_handle* h, const void* const* tables, const void* w
   CK(h, cudaDeviceSynchronize());
   h->w_k = w_k;
   h->w_v = w_v;
+  h->norm_q = norm_q;
+  h->norm_k = norm_k;
   if (h->cfg.dtype == ENGRAM_BF16) {
     for (int bn : {64, 128, 256}) {
       if (d % bn) continue;
@@ -961,6 +969,194 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   h->launches += 2;
   if (conv) return short_conv(value_tile);
   CK(h, mark(5));
+  return ENGRAM_OK;
+}
+
+namespace {
+
+int ensure_bw_scratch(engram_handle* h, int64_t rows, int grid) {
+  const int64_t M = h->cfg.branches, d = h->cfg.d_hidden;
+  if (rows > h->bw_cap_rows) {
+    free_dev(h->bw_idx);
+    free_dev(h->bw_kv);
+    free_dev(h->bw_dkv);
+    free_dev(h->bw_de);
+    h->bw_cap_rows = 0;
+    CK(h, cudaMalloc(&h->bw_idx, (size_t)rows * h->S * sizeof(int64_t)));
+    CK(h, cudaMalloc(&h->bw_kv, (size_t)rows * (M + 1) * d * sizeof(float)));
+    CK(h, cudaMalloc(&h->bw_dkv, (size_t)rows * (M + 1) * d * h->elt));
+    CK(h, cudaMalloc(&h->bw_de, (size_t)rows * h->d_mem * sizeof(float)));
+    h->bw_cap_rows = rows;
+  }
+  if (grid > h->bw_part_blocks) {
+    free_dev(h->bw_partials);
+    h->bw_part_blocks = 0;
+    CK(h, cudaMalloc(&h->bw_partials, (size_t)grid * 2 * M * d * sizeof(float)));
+    h->bw_part_blocks = grid;
+  }
+  if (!h->blas) {
+    if (cublasCreate(&h->blas) != CUBLAS_STATUS_SUCCESS) {
+      h->blas = nullptr;
+      return fail(h, ENGRAM_ERR_CUDA, "cublasCreate failed");
+    }
+  }
+  return ENGRAM_OK;
+}
+
+// Column-major C[m x n] = alpha op(A) op(B) + beta C with A, B in the handle's
+// dtype and C fp32, fp32 accumulation (no TF32 for fp32 operands).
+int gemm(engram_handle* h, bool ta, bool tb, int m, int n, int k, const void* A, int lda,
+         const void* B, int ldb, float beta, float* C, int ldc) {
+  const float alpha = 1.f;
+  const bool bf16 = h->cfg.dtype == ENGRAM_BF16;
+  const cudaDataType_t t = bf16 ? CUDA_R_16BF : CUDA_R_32F;
+  const cublasStatus_t st = cublasGemmEx(
+      h->blas, ta ? CUBLAS_OP_T : CUBLAS_OP_N, tb ? CUBLAS_OP_T : CUBLAS_OP_N, m, n, k, &alpha, A,
+      t, lda, B, t, ldb, &beta, C, CUDA_R_32F, ldc,
+      bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC, CUBLAS_GEMM_DEFAULT);
+  if (st != CUBLAS_STATUS_SUCCESS)
+    return fail(h, ENGRAM_ERR_CUDA, "cublasGemmEx failed (status " + std::to_string((int)st) + ")");
+  return ENGRAM_OK;
+}
+
+}  // namespace
+
+int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx, int32_t B,
+                    int32_t T, int32_t t_begin, const void* hid, const void* dout, void* dhid,
+                    float* dw_k, float* dw_v, float* dnorm_q, float* dnorm_k,
+                    float* const* dtables, void* stream) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  int rc = check_shape(h, B, T, t_begin);
+  if (rc) return rc;
+  if (h->cfg.table_location == ENGRAM_PINNED_HOST)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED, "engram_backward: device-resident tables only");
+  if (h->fp8 || h->conv_W > 0)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED,
+                "engram_backward: the FP8 projections and the short convolution have no backward");
+  const int M = h->cfg.branches, d = h->cfg.d_hidden, dm = h->d_mem, S = h->S;
+  if (d > 4096 || gate_bw_smem(M, d) > 232448)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED, "engram_backward: d must be <= 4096");
+  const int64_t R = (int64_t)B * (T - t_begin);
+  if (R == 0) return ENGRAM_OK;
+  if (R > INT32_MAX / std::max(M + 1, 1) / std::max(d, 1) || R * dm > INT32_MAX)
+    return fail(h, ENGRAM_ERR_INVALID, "engram_backward: too many rows for one call");
+  if (!hid || !dout || !dhid || !aligned16(hid) || !aligned16(dout) || !aligned16(dhid))
+    return fail(h, ENGRAM_ERR_INVALID, "h, dout and dh must be non-null and 16-byte aligned");
+  if (!idx && !tokens) return fail(h, ENGRAM_ERR_INVALID, "need tokens or idx");
+  if (dtables)
+    for (int s = 0; s < S; ++s)
+      if (!dtables[s]) return fail(h, ENGRAM_ERR_INVALID, "null table-gradient pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int grid = gate_bw_grid(M, d, R);
+  if ((rc = ensure_scratch(h, R))) return rc;
+  if ((rc = ensure_bw_scratch(h, R, grid))) return rc;
+  if (cublasSetStream(h->blas, st) != CUBLAS_STATUS_SUCCESS)
+    return fail(h, ENGRAM_ERR_CUDA, "cublasSetStream failed");
+  const bool prof = h->bprof_armed;
+  h->bprof_armed = false;
+  auto mark = [&](int i) -> cudaError_t {
+    return prof ? cudaEventRecord(h->bprof[i], st) : cudaSuccess;
+  };
+  CK(h, mark(0));
+
+  // steps 1-4 again: indices (kept for the table gradients) and e
+  const int64_t* z = idx;
+  if (!idx) {
+    CK(h, launch_hash(hash_args(h, tokens, B, T, t_begin, h->bw_idx), st));
+    h->launches += 1;
+    z = h->bw_idx;
+  }
+  GatherArgs ga{};
+  ga.tables = h->d_tables;
+  ga.primes = h->d_primes;
+  ga.idx = z;
+  ga.e = h->e;
+  ga.err = h->d_err;
+  ga.rows = R;
+  ga.S = S;
+  ga.row_bytes = h->cfg.d_head * h->elt;
+  CK(h, launch_gather(ga, st));
+  h->launches += 1;
+  CK(h, mark(1));
+
+  // k and v recomputed (Eq. 3): kv [R, (M+1) d] = e [W_K; W_V]^T
+  const int nkv = (M + 1) * d;
+  const char* dkv = static_cast<const char*>(h->bw_dkv);
+  if ((rc = gemm(h, true, false, M * d, (int)R, dm, h->w_k, dm, h->e, dm, 0.f, h->bw_kv, nkv)))
+    return rc;
+  if ((rc = gemm(h, true, false, d, (int)R, dm, h->w_v, dm, h->e, dm, 0.f,
+                 h->bw_kv + (int64_t)M * d, nkv)))
+    return rc;
+  CK(h, mark(2));
+
+  // gate and residual backward: dh, dk, dv, RMSNorm weight gradients
+  GateBwArgs a{};
+  a.h = hid;
+  a.dout = dout;
+  a.kv = h->bw_kv;
+  a.w_q = h->norm_q;
+  a.w_k = h->norm_k;
+  a.dh = dhid;
+  a.dkv = h->bw_dkv;
+  a.partials = h->bw_partials;
+  a.R = R;
+  a.M = M;
+  a.d = d;
+  a.bf16 = h->cfg.dtype == ENGRAM_BF16;
+  a.eps = h->cfg.eps;
+  a.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
+  CK(h, launch_gate_backward(a, grid, st));
+  h->launches += 1;
+  if (dnorm_q || dnorm_k) {
+    CK(h, launch_dnorm_reduce(h->bw_partials, grid, (int64_t)M * d, dnorm_q, dnorm_k, st));
+    h->launches += 1;
+  }
+  CK(h, mark(3));
+
+  // weight gradients (Eq. 3 transposed): dW_K += dk^T e, dW_V += dv^T e
+  if (dw_k && (rc = gemm(h, false, true, dm, M * d, (int)R, h->e, dm, dkv, nkv, 1.f, dw_k, dm)))
+    return rc;
+  if (dw_v && (rc = gemm(h, false, true, dm, d, (int)R, h->e, dm,
+                         dkv + (int64_t)M * d * h->elt, nkv, 1.f, dw_v, dm)))
+    return rc;
+  CK(h, mark(4));
+
+  // memory-vector gradient de = [dk dv] [W_K; W_V], then the table rows (Eq. 2 transposed)
+  if (dtables) {
+    if ((rc = gemm(h, false, false, dm, (int)R, M * d, h->w_k, dm, dkv, nkv, 0.f, h->bw_de, dm)))
+      return rc;
+    if ((rc = gemm(h, false, false, dm, (int)R, d, h->w_v, dm, dkv + (int64_t)M * d * h->elt, nkv,
+                   1.f, h->bw_de, dm)))
+      return rc;
+    TableGradArgs tg{};
+    tg.de = h->bw_de;
+    tg.idx = z;
+    tg.primes = h->d_primes;
+    for (int s = 0; s < S; ++s) tg.dtables[s] = dtables[s];
+    tg.err = h->d_err;
+    tg.rows = R;
+    tg.S = S;
+    tg.d_head = h->cfg.d_head;
+    CK(h, launch_table_grad(tg, st));
+    h->launches += 1;
+  }
+  CK(h, mark(5));
+  return ENGRAM_OK;
+}
+
+int engram_profile_next_backward(engram_handle* h, void* const* events, int32_t n_events) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!events) {
+    h->bprof_armed = false;
+    return ENGRAM_OK;
+  }
+  if (n_events != 6) return fail(h, ENGRAM_ERR_INVALID, "n_events must be 6");
+  for (int i = 0; i < n_events; ++i) {
+    if (!events[i]) return fail(h, ENGRAM_ERR_INVALID, "null event");
+    h->bprof[i] = (cudaEvent_t)events[i];
+  }
+  h->bprof_armed = true;
   return ENGRAM_OK;
 }
 

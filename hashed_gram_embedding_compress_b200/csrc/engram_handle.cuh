@@ -3,6 +3,8 @@
 // weights, scratch and prefetch state.  Internal to libengram.so.
 #pragma once
 
+#include <cublas_v2.h>
+
 #include <string>
 
 #include "../../include/engram.h"
@@ -30,6 +32,8 @@ struct engram_handle {
   const void* w_k = nullptr;
   const void* w_v = nullptr;
   float* d_wqk = nullptr;           // norm_q * norm_k, [M, d]
+  const float* norm_q = nullptr;    // [M, d] (borrowed; the backward needs both factors)
+  const float* norm_k = nullptr;
   CUtensorMap map_wk[3], map_wv[3]; // box widths 64, 128, 256
 
   // short convolution (Eq. 5): off while conv_W == 0
@@ -83,9 +87,22 @@ struct engram_handle {
   int32_t* d_hot_slots = nullptr;            // [hot_cap] cache slot per bucket
   void* d_hot_rows = nullptr;                // [n_hot, row_bytes]
 
+  // backward (engram_backward): scratch sized for bw_cap_rows, cuBLAS for its
+  // dense GEMMs (k and v recomputed, weight and memory-vector gradients)
+  int64_t bw_cap_rows = 0;
+  int64_t* bw_idx = nullptr;       // [rows, S]
+  float* bw_kv = nullptr;          // [rows, (M + 1) d]
+  void* bw_dkv = nullptr;          // [rows, (M + 1) d] dtype
+  float* bw_de = nullptr;          // [rows, d_mem]
+  float* bw_partials = nullptr;    // [bw_part_blocks][2][M][d]
+  int bw_part_blocks = 0;
+  cublasHandle_t blas = nullptr;
+
   // instrumentation
   int64_t launches = 0;
   cudaEvent_t prof[6] = {};
   int n_prof = 0;
   bool prof_armed = false;
+  cudaEvent_t bprof[6] = {};  // stages of the next engram_backward
+  bool bprof_armed = false;
 };

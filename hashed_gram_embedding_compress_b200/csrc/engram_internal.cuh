@@ -88,6 +88,43 @@ struct ConvArgs {
   float eps;
 };
 
+// Backward of the gate and residual (training): see k_backward.cu.
+struct GateBwArgs {
+  const void* h;        // [R, M, d] fp32 or bf16
+  const void* dout;     // [R, M, d] gradient of out, same dtype
+  const float* kv;      // [R, (M + 1) d]: k of each branch, then v (recomputed, fp32)
+  const float* w_q;     // [M, d] RMSNorm weight of the query
+  const float* w_k;     // [M, d] RMSNorm weight of the key
+  void* dh;             // [R, M, d] gradient of h, same dtype
+  void* dkv;            // [R, (M + 1) d] dk of each branch, then dv, same dtype
+  float* partials;      // [grid][2][M][d] per-CTA sums for the RMSNorm weight gradients
+  int64_t R;
+  int32_t M, d;
+  bool bf16;
+  float eps, inv_sqrt_d;
+};
+
+// Table gradients: dtables[s][idx[r][s]] += the slot-s slice of de[r].
+struct TableGradArgs {
+  const float* de;               // [rows, S * d_head]
+  const int64_t* idx;            // [rows, S]
+  const int64_t* primes;         // [S] (indices outside a table are skipped and flagged)
+  float* dtables[kMaxTables];    // fp32 [primes[s], d_head] each
+  unsigned* err;
+  int64_t rows;
+  int32_t S, d_head;
+};
+
+size_t gate_bw_smem(int M, int d);
+int gate_bw_grid(int M, int d, int64_t R);
+// d <= 4096 and gate_bw_smem(M, d) within the per-CTA shared memory limit.
+cudaError_t launch_gate_backward(const GateBwArgs& a, int grid, cudaStream_t stream);
+// dnorm_q[i] += sum_b partials[b][0][i], dnorm_k[i] += sum_b partials[b][1][i]
+// over the nblocks CTAs in order (n = M d; either output may be null).
+cudaError_t launch_dnorm_reduce(const float* partials, int nblocks, int64_t n, float* dnorm_q,
+                                float* dnorm_k, cudaStream_t stream);
+cudaError_t launch_table_grad(const TableGradArgs& a, cudaStream_t stream);
+
 // Prefetch of host-resident rows into an HBM staging buffer (section 2.5).
 struct PrefetchArgs {
   const int64_t* idx;           // [rows, S] table indices of the upcoming step

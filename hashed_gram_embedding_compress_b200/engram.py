@@ -31,7 +31,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_profile_next_forward", "engram_kernel_launches",
            "engram_project_gate_noalloc", "engram_selftest_timeout", "engram_set_short_conv",
            "engram_build_hot_cache", "engram_prefetch_hot_hits", "engram_set_fp8",
-           "engram_quantize_e4m3")
+           "engram_quantize_e4m3", "engram_backward", "engram_profile_next_backward")
 
 
 class engram_config(ctypes.Structure):
@@ -72,6 +72,7 @@ def _load():
         "engram_prefetch_hot_hits": ([H, P], ctypes.c_int),
         "engram_set_fp8": ([H, i32, P], ctypes.c_int),
         "engram_quantize_e4m3": ([H, P, i64, i32, P, P, P], ctypes.c_int),
+        "engram_backward": ([H, P, P, i32, i32, i32, P, P, P, P, P, P, P, P, P], ctypes.c_int),
         "engram_get_hash_params": ([H, P, P], ctypes.c_int),
         "engram_hash": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
@@ -79,6 +80,7 @@ def _load():
         "engram_prefetch": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_check_errors": ([H, P], ctypes.c_int),
         "engram_profile_next_forward": ([H, P, i32], ctypes.c_int),
+        "engram_profile_next_backward": ([H, P, i32], ctypes.c_int),
         "engram_kernel_launches": ([H], ctypes.c_int64),
         "engram_project_gate_noalloc": ([H, P, i64, P, P, P, P], ctypes.c_int),
         "engram_selftest_timeout": ([H, P], ctypes.c_int),
@@ -212,6 +214,19 @@ class Engram:
         self._check(lib.engram_forward(self._h, _ptr(tokens), _ptr(idx), B, T, t_begin, _ptr(h),
                                        _ptr(out), _ptr(alpha), _ptr(delta), _stream_ptr(stream)))
 
+    def backward(self, tokens, h, dout, dh, dw_k=None, dw_v=None, dnorm_q=None, dnorm_k=None,
+                 dtables=None, idx=None, t_begin=0, stream=None):
+        """Gradients of the forward for dL/dout = dout: dh written; dw_k, dw_v,
+        dnorm_q, dnorm_k and the S fp32 table gradients accumulated (any may be None)."""
+        B, T = tokens.shape
+        arr = None
+        if dtables is not None:
+            arr = ctypes.cast((ctypes.c_void_p * self.S)(*[t.data_ptr() for t in dtables]),
+                              ctypes.c_void_p)
+        self._check(lib.engram_backward(self._h, _ptr(tokens), _ptr(idx), B, T, t_begin, _ptr(h),
+                                        _ptr(dout), _ptr(dh), _ptr(dw_k), _ptr(dw_v),
+                                        _ptr(dnorm_q), _ptr(dnorm_k), arr, _stream_ptr(stream)))
+
     def prefetch(self, tokens, t_begin=0, stream=None, want_count=False):
         B, T = tokens.shape
         n = ctypes.c_int64(0)
@@ -237,6 +252,13 @@ class Engram:
         n = len(events)
         arr = (ctypes.c_void_p * n)(*[e.cuda_event for e in events])
         self._check(lib.engram_profile_next_forward(self._h, ctypes.cast(arr, ctypes.c_void_p), n))
+
+    def profile_next_backward(self, events):
+        """Record 6 CUDA events inside the next backward (stage boundaries)."""
+        self._bprof_keep = list(events)
+        arr = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events])
+        self._check(lib.engram_profile_next_backward(self._h, ctypes.cast(arr, ctypes.c_void_p),
+                                                     len(events)))
 
     def kernel_launches(self) -> int:
         return int(lib.engram_kernel_launches(self._h))

@@ -36,7 +36,8 @@ import torch
 BASE_SEED = 20261202
 
 #: names of the independent sub-streams of one problem
-STREAMS = ("tokens", "map", "hash", "tables", "weights", "hidden", "norms", "conv")
+# appended streams keep the seeds of the earlier ones (SeedSequence children by index)
+STREAMS = ("tokens", "map", "hash", "tables", "weights", "hidden", "norms", "conv", "dout")
 
 
 @dataclass(frozen=True)
@@ -194,12 +195,12 @@ def make_conv_weights(shape: EngramShape, seeds: dict, kernel_size: int = 4):
 
 
 def make_hidden(shape: EngramShape, seeds: dict, device="cpu", rows: Optional[int] = None,
-                chunk_elems: int = 1 << 26) -> torch.Tensor:
+                chunk_elems: int = 1 << 26, stream: str = "hidden") -> torch.Tensor:
     """h [rows_out, M, d] ~ N(0, 1) in shape.dtype."""
     dt = torch_dtype(shape.dtype)
     n = shape.rows_out if rows is None else rows
     per = shape.branches * shape.d_hidden
-    g = _gen(seeds["hidden"], device)
+    g = _gen(seeds[stream], device)
     h = torch.empty((n, shape.branches, shape.d_hidden), dtype=dt, device=device)
     step = max(1, chunk_elems // per)
     for a in range(0, n, step):
@@ -207,3 +208,8 @@ def make_hidden(shape: EngramShape, seeds: dict, device="cpu", rows: Optional[in
         h[a:b].copy_(torch.randn((b - a, shape.branches, shape.d_hidden), generator=g,
                                  device=device, dtype=torch.float32).to(dt))
     return h
+
+
+def make_grad_out(shape: EngramShape, seeds: dict, device="cpu") -> torch.Tensor:
+    """dL/dout [rows_out, M, d] ~ N(0, 1) in shape.dtype, for the backward."""
+    return make_hidden(shape, seeds, device=device, stream="dout")

@@ -281,6 +281,41 @@ ENGRAM_API int engram_forward(engram_handle *h, const int32_t *tokens, const int
                    float *delta, void *stream);
 
 /*
+ * Backward of engram_forward (training): the exact derivative of
+ * out = h + alpha v (Eq. 3, 4, 6) for a loss whose gradient with respect to
+ * out is dout, for the same tokens (or idx) and h.  The pages give only the
+ * forward; per row and branch, with qn = RMSNorm_q(h), kn = RMSNorm_k(k):
+ *   dalpha = dout . v, dv = sum over branches of alpha dout,
+ *   ds = dalpha alpha (1 - alpha), dqn = ds kn / sqrt(d), dkn = ds qn / sqrt(d),
+ *   dh = dout + (RMSNorm backward of dqn), dk = (RMSNorm backward of dkn),
+ *   dW_K += dk e^T, dW_V += dv e^T, de = W_K^T dk + W_V^T dv,
+ *   dtable_s[z_s] += the slot-s slice of de.
+ * k and v are recomputed (the forward keeps neither).  bf16 handles round dk
+ * and dv to bf16 for the GEMMs (fp32 accumulation), as bf16 training does;
+ * fp32 handles keep fp32 throughout.
+ *  tokens, idx  as engram_forward (idx NULL: hashed here).
+ *  hid     device [rows, M, d] dtype: the forward's h.
+ *  dout    device [rows, M, d] dtype.
+ *  dhid    device [rows, M, d] dtype: written with dL/dh.
+ *  dw_k    device fp32 [M, d, d_mem] or NULL, accumulated (+=).
+ *  dw_v    device fp32 [d, d_mem] or NULL, accumulated.
+ *  dnorm_q, dnorm_k  device fp32 [M, d] or NULL, accumulated.
+ *  dtables host array of S device pointers to fp32 [primes[s], d_head]
+ *          table gradients, accumulated (atomic adds: the order of additions
+ *          into one row varies between runs); or NULL.
+ * Device-resident tables, d <= 4096; not with the FP8 projections or the
+ * short convolution on (ENGRAM_ERR_UNSUPPORTED).  Scratch per row: S int64,
+ * (M + 1) d (4 + element size) bytes and 4 d_mem bytes, plus the forward's.
+ * The dense contractions run through cuBLAS on `stream`.
+ * Errors: _INVALID, _STATE, _UNSUPPORTED, _OOM, _CUDA.
+ */
+ENGRAM_API int engram_backward(engram_handle *h, const int32_t *tokens, const int64_t *idx,
+                               int32_t B, int32_t T, int32_t t_begin, const void *hid,
+                               const void *dout, void *dhid, float *dw_k, float *dw_v,
+                               float *dnorm_q, float *dnorm_k, float *const *dtables,
+                               void *stream);
+
+/*
  * Deterministic prefetch for host-resident tables (section 2.5, Figure 2b):
  * hash the tokens of an upcoming step, de-duplicate the addressed rows per
  * table, and copy each distinct row once from pinned host memory over PCIe
@@ -336,6 +371,17 @@ ENGRAM_API int engram_check_errors(engram_handle *h, void *stream);
  * convolution counts in the value stage.  NULL clears.
  */
 ENGRAM_API int engram_profile_next_forward(engram_handle *h, void *const *events, int32_t n_events);
+
+/*
+ * Stage timing for the NEXT engram_backward on this handle (one-shot).
+ * `events` holds 6 cudaEvent_t (as void*) created with timing enabled; that
+ * call records them on its stream at: start, after hashing and the gather,
+ * after k and v are recomputed, after the gate backward (and the RMSNorm
+ * weight-gradient reduction), after the weight-gradient GEMMs, and after the
+ * memory-vector GEMMs and the table-gradient scatter.  NULL clears.
+ */
+ENGRAM_API int engram_profile_next_backward(engram_handle *h, void *const *events,
+                                            int32_t n_events);
 
 /*
  * Self-test of device-side failure detection.  Launches on `stream` a one-CTA

@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_header_and_binding_agree(eg):
     names = declared_symbols()
-    assert names == set(eg.EXPORTS) and len(names) == 21
+    assert names == set(eg.EXPORTS) and len(names) == 23
 
 
 def test_library_exports_every_declared_symbol(eg):
@@ -96,7 +96,9 @@ def test_null_arguments(eg):
                      ("engram_build_hot_cache", (None, None, 1, 1, 0, 1, None)),
                      ("engram_prefetch_hot_hits", (None, None)),
                      ("engram_set_fp8", (None, 1, None)),
-                     ("engram_quantize_e4m3", (None, None, 1, 16, None, None, None))):
+                     ("engram_quantize_e4m3", (None, None, 1, 16, None, None, None)),
+                     ("engram_backward", (None, None, None, 1, 1, 0) + (None,) * 9),
+                     ("engram_profile_next_backward", (None, None, 6))):
         assert getattr(eg.lib, fn)(*args) == eg.ENGRAM_ERR_INVALID, fn
     assert eg.lib.engram_kernel_launches(None) == -1
     eg.lib.engram_destroy(None)
