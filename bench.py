@@ -499,8 +499,13 @@ def run_backward_bench(args, rank, world, dist):
              dtables=[torch.zeros((int(p), sh.d_head), device=device) for p in P["primes"]])
     stream = torch.cuda.current_stream()
 
+    from hashed_gram_embedding_compress_b200 import dp
+
     def step():
         m.backward(tok_d, h, dout, dh, t_begin=sh.t_begin, stream=stream, **g)
+        if dist:
+            # data-parallel replicas: the dense gradients are summed over the ranks
+            dp.all_reduce_dense([g["dw_k"], g["dw_v"], g["dnorm_q"], g["dnorm_k"]])
 
     clk = ClockSampler(local).__enter__()
     for _ in range(max(3, args.warmup)):
@@ -552,6 +557,8 @@ def run_backward_bench(args, rank, world, dist):
         h_b.copy_(h_h, non_blocking=True)
         g_b.copy_(g_h, non_blocking=True)
         m.backward(tok_b, h_b, g_b, dh, t_begin=sh.t_begin, stream=stream, **g)
+        if dist:
+            dp.all_reduce_dense([g["dw_k"], g["dw_v"], g["dnorm_q"], g["dnorm_k"]])
         dh_h.copy_(dh, non_blocking=True)
 
     e2e_step()
