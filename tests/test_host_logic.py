@@ -1,0 +1,93 @@
+"""Host-side logic that needs no GPU: the projection-kernel choice of the
+library (compiled from its header as plain C++) and the benchmark's
+algorithmic work per step.
+"""
+import itertools
+import os
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "hashed_gram_embedding_compress_b200", "csrc")
+
+_PROBE = r"""
+#include "engram_internal.cuh"
+#include <cstdio>
+int main() {
+  long long R;
+  int phase, M, d, sms, flags, conv, wide;
+  while (scanf("%d %lld %d %d %d %d %d %d", &phase, &R, &M, &d, &sms, &flags, &conv, &wide) == 8) {
+    const engram::ProjChoice c = wide ? engram::wide_proj(phase, R, M, d, sms)
+                                      : engram::choose_proj(phase, R, M, d, sms, flags, conv != 0);
+    printf("%d %d %d %d\n", (int)c.kind, c.bn, c.grid, c.key_tile);
+  }
+  return 0;
+}
+"""
+WIDE, PAIR, SINGLE = 0, 1, 2
+
+
+@pytest.fixture(scope="module")
+def choose(tmp_path_factory):
+    d = tmp_path_factory.mktemp("choose")
+    src, exe = d / "probe.cpp", d / "probe"
+    src.write_text(_PROBE)
+    subprocess.check_call(["g++", "-std=c++17", "-I", "/usr/local/cuda/include", "-I", CSRC,
+                           str(src), "-o", str(exe)])
+
+    def run(cases):
+        inp = "".join("%d %d %d %d %d %d %d %d\n" % c for c in cases)
+        out = subprocess.run([str(exe)], input=inp, capture_output=True, text=True, check=True)
+        return [tuple(int(x) for x in line.split()) for line in out.stdout.splitlines()]
+    return run
+
+
+def test_prefill_uses_the_512x256_pair_tiles(choose):
+    (k0, bn0, g0, kt0), (k1, _, g1, _) = choose([(0, 32768, 1, 2560, 148, 0, 0, 0),
+                                                (1, 32768, 1, 2560, 148, 0, 0, 0)])
+    assert (k0, bn0, g0, kt0) == (WIDE, 128, 148, 256) and (k1, g1) == (WIDE, 148)
+
+
+def test_choice_invariants_over_shapes(choose):
+    cases = [(ph, R, M, d, sms, fl, cv, 0)
+             for ph, R, M, d, sms, fl, cv in itertools.product(
+                 (0, 1), (1, 4, 256, 2048, 3000, 32768), (1, 2, 4), (128, 256, 512, 640, 2560, 4096),
+                 (148, 132), (0, 1), (0, 1))]
+    for c, (kind, bn, grid, kt) in zip(cases, choose(cases)):
+        ph, R, M, d, sms, fl, cv, _ = c
+        n_total = M * d if ph == 0 else d
+        assert d % kt == 0, c                        # key tiles never straddle branches
+        assert n_total % bn == 0 and 1 <= grid <= sms, c
+        if fl:                                       # no CTA pairs: single-CTA tiles only
+            assert kind == SINGLE, c
+        if kind != SINGLE:
+            assert grid % 2 == 0, c                  # whole CTA pairs
+        if kind == WIDE:
+            assert d % 256 == 0 and kt == 256, c
+        if kind == PAIR:
+            assert kt == 128 and not (ph == 1 and cv), c   # no pair kernel for the conv's values
+
+
+def test_wide_choice_for_fp8(choose):
+    cases = [(ph, R, M, d, 148, 0, 0, 1) for ph in (0, 1) for R in (1, 6, 513, 32768)
+             for M in (1, 4) for d in (256, 2560)]
+    for c, (kind, bn, grid, kt) in zip(cases, choose(cases)):
+        ph, R, M, d = c[:4]
+        tiles = -(-R // 512) * ((M * d if ph == 0 else d) // 256)
+        assert (kind, bn, kt) == (WIDE, 128, 256) and grid == 2 * min(tiles, 74), c
+
+
+def test_bench_algorithmic_work():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from hashed_gram_embedding_compress_b200 import synth
+    sh = synth.SHAPES["prefill_bf16"]
+    R, S = 32768, 16
+    a = bench.algorithmic(sh)
+    # tokens + S table rows of 160 bytes read and written per row
+    assert a["gather_bytes"] == R * S * 160 * 2 + 8 * 4096 * 4 == 167903232
+    assert a["gemm_flops"] == 2.0 * R * 1280 * (2560 + 2560)
+    # FP8: codes (1 byte per element) and a 4-byte scale per row written instead of bf16 e
+    assert bench.algorithmic(sh, fp8=True)["gather_bytes"] == R * S * 160 + R * 1284 + 8 * 4096 * 4
