@@ -306,7 +306,9 @@ ENGRAM_API int engram_forward(engram_handle *h, const int32_t *tokens, const int
  * Device-resident tables, d <= 4096; not with the FP8 projections or the
  * short convolution on (ENGRAM_ERR_UNSUPPORTED).  Scratch per row: S int64,
  * (M + 1) d (4 + element size) bytes and 4 d_mem bytes, plus the forward's.
- * The dense contractions run through cuBLAS on `stream`.
+ * The dense contractions run through cuBLAS on `stream`.  The first call
+ * creates the handle's cuBLAS context and its scratch (engram_reserve does
+ * not cover the backward's): make it outside any stream capture.
  * Errors: _INVALID, _STATE, _UNSUPPORTED, _OOM, _CUDA.
  */
 ENGRAM_API int engram_backward(engram_handle *h, const int32_t *tokens, const int64_t *idx,
