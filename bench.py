@@ -605,7 +605,8 @@ def run_backward_bench(args, rank, world, dist):
         "gpu_launches": launches,
         "clocks": dict(clk.summary(t_load + 0.5, t_end + 0.15),
                        window="last 1 s of back-to-back warm-up steps and the timed steps"),
-    }
+    } | ({"cpu_baseline": cpu_baseline_backward(P, dout, args.cpu_seconds)}
+         if not args.no_cpu_baseline and world == 1 else {})
 
 
 # ------------------------------------------------------ host-offload leg
@@ -838,6 +839,52 @@ def cpu_baseline(P, budget_s: float):
                           "+short conv" if P["conv"] is not None else "", total_rows, total_t)}
 
 
+def cpu_baseline_backward(P, dout, budget_s: float):
+    """The oracle's backward, as it stands, on a bounded sample of the same
+    workload: compress + hash on every position; gather, the exact derivative
+    and the table-gradient scatter on the first n rows, n grown until the
+    sample takes about `budget_s` seconds.  tokens/s as in cpu_baseline."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    sh = P["sh"]
+    t0 = time.perf_counter()
+    c, z, mult, primes = oracle.forward_indices(P["tokens"].numpy(), P["comp_map"].numpy(),
+                                                sh.cvocab, sh.orders, sh.heads, P["hash_seed"],
+                                                sh.rows_target, t_begin=sh.t_begin)
+    t_hash = (time.perf_counter() - t0) / sh.rows_out
+
+    def to_np(t):
+        t = t.detach().contiguous().cpu()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    wk, wv = to_np(P["w_k"]), to_np(P["w_v"])
+    nq, nk = P["nq"].cpu().numpy(), P["nk"].cpu().numpy()
+    n, total_rows, total_t = 4, 0, 0.0
+    while total_t < budget_s and total_rows < sh.rows_out:
+        rows = np.arange(total_rows, min(sh.rows_out, total_rows + n))
+        zr = z[rows]
+        mini = [to_np(t[torch.from_numpy(zr[:, s]).to(t.device)]) for s, t in enumerate(P["tables"])]
+        zz = np.tile(np.arange(len(rows))[:, None], (1, sh.num_tables))
+        rs = torch.from_numpy(rows)
+        hr = to_np(P["h"][rs.to(P["h"].device)])
+        gr = dout[rs.to(dout.device)].double().cpu().numpy()
+        t0 = time.perf_counter()
+        e = oracle.gather(mini, zz)
+        b = oracle.backward(e, wk, wv, nq, nk, hr, gr, 1e-6, round_dkv=sh.dtype == "bf16")
+        oracle.table_grad(b["de"], zz, [len(rows)] * sh.num_tables, sh.d_head)
+        total_t += time.perf_counter() - t0
+        total_rows += len(rows)
+        n *= 2
+    per_row = t_hash + total_t / total_rows
+    return {"value": 1.0 / per_row, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "compress+hash on all %d positions; gather+backward+table scatter on the "
+                      "first %d rows (%.1f s); single-threaded C, fp64" % (
+                          sh.rows_out, total_rows, total_t)}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -847,12 +894,20 @@ def run_reference(args, rank, world):
               args.short_conv, args.fp8)
     sh = P["sh"]
     budget = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    if args.backward:
+        from hashed_gram_embedding_compress_b200 import synth
+        dout = synth.make_grad_out(sh, P["seeds"], device=P["h"].device)
+        leg = lambda: cpu_baseline_backward(P, dout, budget)  # noqa: E731
+        metric = "Engram backward tokens/s (gradients of h, W_K, W_V, RMSNorm weights, tables)"
+    else:
+        leg = lambda: cpu_baseline(P, budget)  # noqa: E731
+        metric = METRIC
     for _ in range(args.warmup):
-        cpu_baseline(P, budget)
-    vals = [cpu_baseline(P, budget) for _ in range(args.steps)]
+        leg()
+    vals = [leg() for _ in range(args.steps)]
     v = statistics.median(x["value"] for x in vals)
     return {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
+        "impl": "reference", "metric": metric, "value": v, "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sh.rows_out / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",

@@ -91,3 +91,30 @@ def test_bench_algorithmic_work():
     assert a["gemm_flops"] == 2.0 * R * 1280 * (2560 + 2560)
     # FP8: codes (1 byte per element) and a 4-byte scale per row written instead of bf16 e
     assert bench.algorithmic(sh, fp8=True)["gather_bytes"] == R * S * 160 + R * 1284 + 8 * 4096 * 4
+
+
+def _cpu_problem():
+    import oracle
+    from hashed_gram_embedding_compress_b200 import synth
+    sh = synth.SHAPES["tiny_f32"]
+    seeds = synth.stream_seeds(sh)
+    primes = oracle.table_primes(sh.rows_target, sh.num_tables)
+    w_k, w_v, nq, nk = synth.make_weights(sh, seeds)
+    P = dict(sh=sh, tokens=synth.make_tokens(sh, seeds), comp_map=synth.make_comp_map(sh, seeds),
+             hash_seed=synth.make_hash_seed(seeds), w_k=w_k, w_v=w_v, nq=nq, nk=nk,
+             tables=synth.make_tables([int(p) for p in primes], sh.d_head, sh.dtype, seeds,
+                                      device="cpu"),
+             h=synth.make_hidden(sh, seeds), conv=None)
+    return P, synth.make_grad_out(sh, seeds)
+
+
+def test_cpu_baselines_run_the_oracle_on_a_bounded_sample():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    P, dout = _cpu_problem()
+    f = bench.cpu_baseline(P, 0.3)
+    b = bench.cpu_baseline_backward(P, dout, 0.3)
+    for r in (f, b):
+        assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
+    assert "backward" in b["sample"] and "backward" not in f["sample"]
