@@ -91,6 +91,31 @@ def test_bench_algorithmic_work():
     assert a["gemm_flops"] == 2.0 * R * 1280 * (2560 + 2560)
     # FP8: codes (1 byte per element) and a 4-byte scale per row written instead of bf16 e
     assert bench.algorithmic(sh, fp8=True)["gather_bytes"] == R * S * 160 + R * 1284 + 8 * 4096 * 4
+    # the step's unavoidable bytes: tokens, each addressed row once, h in, out, W once
+    assert a["step_bytes"] == 8 * 4096 * 4 + R * S * 160 + 2 * R * 2560 * 2 + 2 * 2560 * 1280 * 2
+    r = bench.step_roofline(a, 0.5, 6500.0, 1600.0)
+    t_mma = a["gemm_flops"] / 1.6e15 * 1e3
+    assert r["bound"] == "tensor" and abs(r["time_ms"] - t_mma) < 1e-12
+    assert abs(r["frac"] - t_mma / 0.5) < 1e-12
+
+
+def test_reference_arm_runs_the_oracle_without_the_library():
+    """bench.py --impl reference times the oracle alone: the library's shared
+    object is never loaded in its process."""
+    import subprocess
+    import sys
+    code = (
+        "import sys, types; sys.path.insert(0, %r); import bench\n"
+        "a = types.SimpleNamespace(workload='tiny_f32', rows_target=None, short_conv=False,\n"
+        "    fp8=False, backward=False, steps=1, warmup=0, cpu_seconds=0.2)\n"
+        "r = bench.run_reference(a, 0, 1)\n"
+        "assert r['impl'] == 'reference' and r['value'] > 0 and r['ms_per_step'] > 0\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "assert 'libengram' not in maps and '_engram_oracle' in maps\n"
+        "print('ok')\n" % ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         timeout=300, env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert out.returncode == 0 and "ok" in out.stdout, out.stderr[-2000:]
 
 
 def _cpu_problem():
