@@ -56,11 +56,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         if p.wait() != 0:
             raise RuntimeError("nvcc failed on " + src)
     tmp = LIB + ".tmp%d" % os.getpid()
-    # cuBLAS: the backward's plain GEMMs (the process's already-loaded copy is used when
-    # torch has loaded one; else the toolkit's)
     subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
-                           "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-lcublas",
-                           "-Xlinker", "-rpath=" + os.path.join(CUDA_HOME, "lib64")])
+                           "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-lpthread"])
     os.replace(tmp, LIB)
     return LIB
 

@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <thread>
 #include <string>
 #include <utility>
 #include <vector>
@@ -63,16 +64,22 @@ void free_dev(T*& p) {
   p = nullptr;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+}  // namespace
+
+namespace engram {
+
+// The driver's tensor-map encoder, looked up once (a function-local static:
+// its initialisation is thread-safe).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+  }();
   return fn;
 }
 
@@ -81,7 +88,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // the box's row bytes (128-byte rows: 128-byte swizzle, 64-byte rows: 64-byte
 // swizzle).
 int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
-             int box_rows, int box_cols = 64, int esz = 2) {
+             int box_rows, int box_cols, int esz) {
   auto fn = encode_fn();
   if (!fn) return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const CUtensorMapDataType dt = esz == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
@@ -100,7 +107,9 @@ int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, i
   return ENGRAM_OK;
 }
 
-int bn_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
+}  // namespace engram
+
+namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -194,10 +203,62 @@ HashArgs hash_args(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T
   return a;
 }
 
+void free_host_gather(engram_handle* h) {
+  delete h->hg;  // waits for its queued jobs
+  h->hg = nullptr;
+  for (int i = 0; i < 2; ++i) {
+    if (h->h_count[i]) cudaFreeHost(h->h_count[i]);
+    if (h->h_list[i]) cudaFreeHost(h->h_list[i]);
+    if (h->h_bounce[i]) cudaFreeHost(h->h_bounce[i]);
+    h->h_count[i] = nullptr;
+    h->h_list[i] = nullptr;
+    h->h_bounce[i] = nullptr;
+  }
+}
+
+// Pinned buffers, copy stream, events and threads of the host-thread route
+// for `entries` (row, table) lookups per prefetch.
+int ensure_host_gather(engram_handle* h, int64_t entries) {
+  const size_t row_bytes = (size_t)h->cfg.d_head * h->elt;
+  for (int i = 0; i < 2; ++i) {
+    if (!h->h_count[i])
+      CK(h, cudaHostAlloc((void**)&h->h_count[i], 2 * sizeof(unsigned long long),
+                          cudaHostAllocDefault));
+    if (!h->h_list[i])
+      CK(h, cudaHostAlloc((void**)&h->h_list[i], (size_t)entries * sizeof(int2),
+                          cudaHostAllocDefault));
+    if (!h->h_bounce[i])
+      CK(h, cudaHostAlloc((void**)&h->h_bounce[i], (size_t)entries * row_bytes,
+                          cudaHostAllocDefault));
+    if (!h->ev_list[i]) CK(h, cudaEventCreateWithFlags(&h->ev_list[i], cudaEventDisableTiming));
+  }
+  if (!h->copy_stream) CK(h, cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+  if (!h->hg) {
+    int n = h->pf_workers;
+    if (n <= 0) {
+      const int hw = (int)std::thread::hardware_concurrency();
+      n = std::max(1, std::min(8, hw / 2));
+    }
+    h->hg = new (std::nothrow) HostGather(h->device, n);
+    if (!h->hg) return fail(h, ENGRAM_ERR_OOM, "host gather threads");
+  }
+  return ENGRAM_OK;
+}
+
 int ensure_prefetch_scratch(engram_handle* h, int64_t rows) {
-  if (rows <= h->pf_cap_rows) return ENGRAM_OK;
+  if (rows <= h->pf_cap_rows) {
+    if (h->pf_mode == ENGRAM_PREFETCH_HOST_THREADS)
+      return ensure_host_gather(h, h->pf_cap_rows * h->S);
+    return ENGRAM_OK;
+  }
+  // growing frees the staging buffers, which a pending prefetch has filled
+  if (h->n_prefetch != h->n_consumed)
+    return fail(h, ENGRAM_ERR_STATE,
+                "a larger batch while a prefetch is pending; engram_reserve the largest batch "
+                "first, or run engram_forward first");
   // the staging buffers may still be in use by queued work
   CK(h, cudaDeviceSynchronize());
+  free_host_gather(h);
   free_dev(h->d_keys);
   free_dev(h->d_vals);
   free_dev(h->d_uniq);
@@ -223,11 +284,8 @@ int ensure_prefetch_scratch(engram_handle* h, int64_t rows) {
   for (int s = 0; s < h->S; ++s) bound[s] = entries;
   CK(h, cudaMemcpy(h->d_stage_bound, bound, h->S * sizeof(int64_t), cudaMemcpyHostToDevice));
   for (int i = 0; i < 2; ++i) {
-    if (!h->d_hot_hits[i]) {
-      CK(h, cudaMalloc(&h->d_hot_hits[i], sizeof(unsigned long long)));
-      CK(h, cudaMemset(h->d_hot_hits[i], 0, sizeof(unsigned long long)));
-    }
-    CK(h, cudaMalloc(&h->d_count[i], sizeof(unsigned long long)));
+    CK(h, cudaMalloc(&h->d_count[i], 2 * sizeof(unsigned long long)));
+    CK(h, cudaMemset(h->d_count[i], 0, 2 * sizeof(unsigned long long)));
     CK(h, cudaMalloc(&h->d_remap[i], (size_t)entries * sizeof(int64_t)));
     CK(h, cudaMalloc(&h->d_staging[i], (size_t)entries * row_bytes));
     CK(h, cudaMalloc(&h->d_stage_tables[i], h->S * sizeof(void*)));
@@ -236,6 +294,7 @@ int ensure_prefetch_scratch(engram_handle* h, int64_t rows) {
     CK(h, cudaMemcpy(h->d_stage_tables[i], ptrs, h->S * sizeof(void*), cudaMemcpyHostToDevice));
   }
   h->pf_cap_rows = rows;
+  if (h->pf_mode == ENGRAM_PREFETCH_HOST_THREADS) return ensure_host_gather(h, entries);
   return ENGRAM_OK;
 }
 
@@ -346,7 +405,7 @@ int engram_create(const engram_config* cfg, engram_handle** out) {
                           cudaMemcpyHostToDevice));
          CK(h, cudaMalloc(&h->d_err, sizeof(unsigned)));
          CK(h, cudaMemset(h->d_err, 0, sizeof(unsigned)));
-         CK(h, cudaMalloc(&h->d_tables, S * sizeof(void*)));
+         CK(h, cudaMalloc(&h->d_tables, (size_t)S * kMaxShards * sizeof(void*)));
          CK(h, cudaMalloc(&h->d_wqk, (size_t)c.branches * c.d_hidden * sizeof(float)));
          for (int i = 0; i < 2; ++i) {
            CK(h, cudaEventCreateWithFlags(&h->ev_ready[i], cudaEventDisableTiming));
@@ -365,6 +424,11 @@ void engram_destroy(engram_handle* h) {
   cudaGetDevice(&cur);
   cudaSetDevice(h->device);
   cudaDeviceSynchronize();
+  free_host_gather(h);  // joins the prefetch threads
+  cudaDeviceSynchronize();
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  for (int i = 0; i < 2; ++i)
+    if (h->ev_list[i]) cudaEventDestroy(h->ev_list[i]);
   free_dev(h->d_map);
   free_dev(h->d_primes);
   free_dev(h->d_barrett);
@@ -381,7 +445,6 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->bw_dkv);
   free_dev(h->bw_de);
   free_dev(h->bw_partials);
-  if (h->blas) cublasDestroy(h->blas);
   free_dev(h->e8);
   free_dev(h->se8);
   free_dev(h->d_conv_w);
@@ -398,7 +461,6 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->d_hot_keys);
   free_dev(h->d_hot_slots);
   free_dev(h->d_hot_rows);
-  for (int i = 0; i < 2; ++i) free_dev(h->d_hot_hits[i]);
   for (int i = 0; i < 2; ++i) {
     free_dev(h->d_count[i]);
     free_dev(h->d_remap[i]);
@@ -444,6 +506,7 @@ int engram_set_params(engram_handle* h, const void* const* tables, const void* w
     }
   }
   CK(h, cudaMemcpy(h->d_tables, dev_tab, h->S * sizeof(void*), cudaMemcpyHostToDevice));
+  h->shards = 1;
   CK(h, launch_mul(norm_q, norm_k, h->d_wqk, (int64_t)M * d, 0));
   CK(h, cudaDeviceSynchronize());
   h->w_k = w_k;
@@ -461,6 +524,58 @@ int engram_set_params(engram_handle* h, const void* const* tables, const void* w
   }
   h->have_params = true;
   if (h->fp8) return quantize_weights(h, 0);  // the new weights' E4M3 copy
+  return ENGRAM_OK;
+}
+
+int engram_set_table_shards(engram_handle* h, int32_t shards, const void* const* ptrs) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!h->have_params) return fail(h, ENGRAM_ERR_STATE, "engram_set_params first");
+  if (h->cfg.table_location != ENGRAM_DEVICE)
+    return fail(h, ENGRAM_ERR_UNSUPPORTED, "row-sharded tables are device tables");
+  if (shards < 1 || shards > kMaxShards)
+    return fail(h, ENGRAM_ERR_INVALID, "shards must lie in [1, " + std::to_string(kMaxShards) + "]");
+  if (!ptrs) return fail(h, ENGRAM_ERR_INVALID, "null shard array");
+  for (int i = 0; i < h->S * shards; ++i) {
+    if (!ptrs[i] || !aligned16(ptrs[i]))
+      return fail(h, ENGRAM_ERR_INVALID, "shard pointers must be non-null and 16-byte aligned");
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ptrs[i]) != cudaSuccess || at.type != cudaMemoryTypeDevice) {
+      cudaGetLastError();
+      return fail(h, ENGRAM_ERR_INVALID, "shard pointers must be device memory (own or a peer's)");
+    }
+  }
+  // the previous pointers may still be read by queued work
+  CK(h, cudaDeviceSynchronize());
+  CK(h, cudaMemcpy(h->d_tables, ptrs, (size_t)h->S * shards * sizeof(void*),
+                   cudaMemcpyHostToDevice));
+  h->shards = shards;
+  return ENGRAM_OK;
+}
+
+int engram_ipc_handle(engram_handle* h, const void* ptr, void* handle) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!ptr || !handle) return fail(h, ENGRAM_ERR_INVALID, "null pointer");
+  cudaIpcMemHandle_t mh;
+  CK(h, cudaIpcGetMemHandle(&mh, const_cast<void*>(ptr)));
+  static_assert(sizeof(mh) == ENGRAM_IPC_HANDLE_BYTES, "IPC handle size");
+  std::memcpy(handle, &mh, sizeof(mh));
+  return ENGRAM_OK;
+}
+
+int engram_ipc_open(engram_handle* h, const void* handle, void** ptr) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!handle || !ptr) return fail(h, ENGRAM_ERR_INVALID, "null pointer");
+  cudaIpcMemHandle_t mh;
+  std::memcpy(&mh, handle, sizeof(mh));
+  CK(h, cudaSetDevice(h->device));
+  CK(h, cudaIpcOpenMemHandle(ptr, mh, cudaIpcMemLazyEnablePeerAccess));
+  return ENGRAM_OK;
+}
+
+int engram_ipc_close(engram_handle* h, void* ptr) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!ptr) return fail(h, ENGRAM_ERR_INVALID, "null pointer");
+  CK(h, cudaIpcCloseMemHandle(ptr));
   return ENGRAM_OK;
 }
 
@@ -575,6 +690,7 @@ int engram_gather(engram_handle* h, const int64_t* idx, int64_t rows, void* e, v
   if (!idx || !e || !aligned16(e)) return fail(h, ENGRAM_ERR_INVALID, "null or misaligned buffer");
   GatherArgs g{};
   g.tables = h->d_tables;
+  g.shards = h->shards;
   g.primes = h->d_primes;
   g.idx = idx;
   g.e = e;
@@ -679,12 +795,28 @@ int engram_build_hot_cache(engram_handle* h, const int32_t* tokens, int32_t B, i
 int engram_prefetch_hot_hits(engram_handle* h, int64_t* hits) {
   if (!h || !hits) return ENGRAM_ERR_INVALID;
   *hits = 0;
-  if (h->n_prefetch == 0 || !h->d_hot_hits[(h->n_prefetch - 1) & 1]) return ENGRAM_OK;
+  if (h->n_prefetch == 0 || !h->d_count[(h->n_prefetch - 1) & 1]) return ENGRAM_OK;
   CK(h, cudaDeviceSynchronize());
-  unsigned long long v = 0;
-  CK(h, cudaMemcpy(&v, h->d_hot_hits[(h->n_prefetch - 1) & 1], sizeof(v),
-                   cudaMemcpyDeviceToHost));
-  *hits = (int64_t)v;
+  unsigned long long v[2] = {0, 0};
+  CK(h, cudaMemcpy(v, h->d_count[(h->n_prefetch - 1) & 1], sizeof(v), cudaMemcpyDeviceToHost));
+  *hits = (int64_t)v[1];
+  return ENGRAM_OK;
+}
+
+int engram_set_prefetch(engram_handle* h, int32_t mode, int32_t workers) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (h->cfg.table_location != ENGRAM_PINNED_HOST)
+    return fail(h, ENGRAM_ERR_STATE, "engram_set_prefetch needs ENGRAM_PINNED_HOST tables");
+  if (mode != ENGRAM_PREFETCH_HOST_THREADS && mode != ENGRAM_PREFETCH_ZERO_COPY)
+    return fail(h, ENGRAM_ERR_INVALID, "unknown prefetch mode");
+  if (workers < 0 || workers > 4096) return fail(h, ENGRAM_ERR_INVALID, "workers outside [0, 4096]");
+  if (h->n_prefetch != h->n_consumed)
+    return fail(h, ENGRAM_ERR_STATE, "a prefetch is pending; run engram_forward first");
+  // threads of the old setting finish and leave; the next prefetch starts new ones
+  delete h->hg;
+  h->hg = nullptr;
+  h->pf_mode = mode;
+  h->pf_workers = workers;
   return ENGRAM_OK;
 }
 
@@ -703,6 +835,7 @@ int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t 
   if ((rc = ensure_prefetch_scratch(h, rows))) return rc;
   cudaStream_t st = (cudaStream_t)side_stream;
   const int slot = (int)(h->n_prefetch & 1);
+  const bool host_threads = h->pf_mode == ENGRAM_PREFETCH_HOST_THREADS;
   // the staging slot must no longer be read by the forward that used it last
   if (h->n_prefetch >= 2) CK(h, cudaStreamWaitEvent(st, h->ev_consumed[slot], 0));
   if (rows > 0) {
@@ -725,24 +858,49 @@ int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t 
   a.row_bytes = h->cfg.d_head * h->elt;
   a.staging = h->d_staging[slot];
   a.sms = h->sms;
-  a.fetch_blocks = h->sms * 8;
+  a.fetch_blocks = h->pf_workers > 0 ? h->pf_workers : h->sms;
   if (h->n_hot > 0) {
     a.hot_keys = h->d_hot_keys;
     a.hot_slots = h->d_hot_slots;
     a.hot_cap = h->hot_cap;
     a.hot_rows = h->d_hot_rows;
   }
-  a.hot_hits = h->d_hot_hits[slot];
-  CK(h, launch_prefetch(a, st));
-  h->launches += rows > 0 ? 5 : 1;
-  CK(h, cudaEventRecord(h->ev_ready[slot], st));
+  CK(h, launch_prefetch_index(a, st));
+  h->launches += rows > 0 ? (h->n_hot > 0 ? 5 : 4) : 1;
+  if (host_threads) {
+    // the row list goes to the host; reader threads gather the rows and the
+    // copy engines send them (ev_ready is recorded after the last copy)
+    const int64_t entries = rows * h->S;
+    CK(h, cudaMemcpyAsync(h->h_count[slot], h->d_count[slot], 2 * sizeof(unsigned long long),
+                          cudaMemcpyDeviceToHost, st));
+    if (entries > 0)
+      CK(h, cudaMemcpyAsync(h->h_list[slot], h->d_uniq, (size_t)entries * sizeof(int2),
+                            cudaMemcpyDeviceToHost, st));
+    CK(h, cudaEventRecord(h->ev_list[slot], st));
+    HostGatherJob job;
+    job.slot = slot;
+    job.idx_ready = h->ev_list[slot];
+    job.count = h->h_count[slot];
+    job.list = h->h_list[slot];
+    job.tables = h->tables;
+    job.row_bytes = a.row_bytes;
+    job.bounce = h->h_bounce[slot];
+    job.staging = (char*)h->d_staging[slot];
+    job.copy_stream = h->copy_stream;
+    job.done = h->ev_ready[slot];
+    h->hg->submit(job);
+  } else {
+    CK(h, launch_prefetch_fetch(a, st));
+    h->launches += rows > 0 ? 1 : 0;
+    CK(h, cudaEventRecord(h->ev_ready[slot], st));
+  }
   h->pf_rows[slot] = rows;
   ++h->n_prefetch;
   if (unique_rows) {
-    unsigned long long n = 0;
-    CK(h, cudaMemcpyAsync(&n, h->d_count[slot], sizeof(n), cudaMemcpyDeviceToHost, st));
+    unsigned long long n[2] = {0, 0};
+    CK(h, cudaMemcpyAsync(n, h->d_count[slot], sizeof(n), cudaMemcpyDeviceToHost, st));
     CK(h, cudaStreamSynchronize(st));
-    *unique_rows = rows > 0 ? (int64_t)n : 0;
+    *unique_rows = rows > 0 ? (int64_t)(n[0] + n[1]) : 0;
   }
   return ENGRAM_OK;
 }
@@ -764,6 +922,15 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     slot = (int)(h->n_consumed & 1);
     if (h->pf_rows[slot] != R)
       return fail(h, ENGRAM_ERR_INVALID, "forward shape differs from the pending prefetch");
+  }
+  if (host_tables && h->hg) {
+    // the host-thread route: its copies and ev_ready[slot] are enqueued by
+    // the reader threads; wait until they are
+    std::string msg;
+    const cudaError_t ge = h->hg->wait_issued(slot, &msg);
+    if (ge != cudaSuccess)
+      return fail(h, ge == cudaErrorMemoryAllocation ? ENGRAM_ERR_OOM : ENGRAM_ERR_CUDA,
+                  "prefetch: " + msg);
   }
   if (R == 0) {
     if (host_tables) {
@@ -809,10 +976,12 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   if (host_tables) {
     CK(h, cudaStreamWaitEvent(st, h->ev_ready[slot], 0));
     ga.tables = h->d_stage_tables[slot];
+    ga.shards = 1;
     ga.primes = h->d_stage_bound;
     ga.idx = h->d_remap[slot];
   } else {
     ga.tables = h->d_tables;
+    ga.shards = h->shards;
     ga.primes = h->d_primes;
     ga.idx = idx;
   }
@@ -822,6 +991,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     HashGatherArgs hg{};
     hg.hash = hash_args(h, tokens, B, T, t_begin, nullptr);
     hg.tables = h->d_tables;
+    hg.shards = h->shards;
     hg.e = h->e;
     hg.q = h->e8;
     hg.scale = h->se8;
@@ -994,28 +1164,63 @@ int ensure_bw_scratch(engram_handle* h, int64_t rows, int grid) {
     CK(h, cudaMalloc(&h->bw_partials, (size_t)grid * 2 * M * d * sizeof(float)));
     h->bw_part_blocks = grid;
   }
-  if (!h->blas) {
-    if (cublasCreate(&h->blas) != CUBLAS_STATUS_SUCCESS) {
-      h->blas = nullptr;
-      return fail(h, ENGRAM_ERR_CUDA, "cublasCreate failed");
-    }
-  }
   return ENGRAM_OK;
 }
 
-// Column-major C[m x n] = alpha op(A) op(B) + beta C with A, B in the handle's
-// dtype and C fp32, fp32 accumulation (no TF32 for fp32 operands).
-int gemm(engram_handle* h, bool ta, bool tb, int m, int n, int k, const void* A, int lda,
-         const void* B, int ldb, float beta, float* C, int ldc) {
-  const float alpha = 1.f;
-  const bool bf16 = h->cfg.dtype == ENGRAM_BF16;
-  const cudaDataType_t t = bf16 ? CUDA_R_16BF : CUDA_R_32F;
-  const cublasStatus_t st = cublasGemmEx(
-      h->blas, ta ? CUBLAS_OP_T : CUBLAS_OP_N, tb ? CUBLAS_OP_T : CUBLAS_OP_N, m, n, k, &alpha, A,
-      t, lda, B, t, ldb, &beta, C, CUDA_R_32F, ldc,
-      bf16 ? CUBLAS_COMPUTE_32F : CUBLAS_COMPUTE_32F_PEDANTIC, CUBLAS_GEMM_DEFAULT);
-  if (st != CUBLAS_STATUS_SUCCESS)
-    return fail(h, ENGRAM_ERR_CUDA, "cublasGemmEx failed (status " + std::to_string((int)st) + ")");
+// K splits of a reduce-add contraction: the count that fills the most of
+// `rounds` rounds of CTA pairs (1-8 rounds), at least 8 K blocks per split.
+void choose_splits(GemmArgs& g, int pairs) {
+  const int kb_total = (g.K + 63) / 64;
+  const int mn = gemm_pair_tiles(GemmArgs{g.M, g.N, g.K, 0, 0, 1, 1, 0, nullptr});
+  int best = 1;
+  double best_util = (double)mn / (((mn + pairs - 1) / pairs) * (double)pairs);
+  for (int rounds = 1; rounds <= 8; ++rounds) {
+    const int sp = std::min(std::max(1, rounds * pairs / mn), std::max(1, kb_total / 8));
+    const int tiles = mn * sp;
+    const double util = (double)tiles / (((tiles + pairs - 1) / pairs) * (double)pairs);
+    if (util > best_util + 1e-9) {
+      best_util = util;
+      best = sp;
+    }
+  }
+  g.kb_per_split = (kb_total + best - 1) / best;
+  g.splits = (kb_total + g.kb_per_split - 1) / g.kb_per_split;
+}
+
+// D (=|+=) A B^T on the tensor cores; see GemmArgs.  a_mn / b_mn: the
+// operand is stored MN-major ([K, rows]).
+int gemm_bf16(engram_handle* h, bool a_mn, bool b_mn, bool add, const void* A, int64_t a_rows,
+              int64_t a_cols, const void* B0, int64_t b0_rows, const void* B1, int64_t b1_rows,
+              int64_t b_cols, float* D, int64_t d_rows, int64_t d_cols, GemmArgs g,
+              cudaStream_t st) {
+  GemmMaps mp;
+  int rc;
+  if ((rc = make_map(h, &mp.a, A, a_cols, a_rows, a_mn ? 64 : 128, 64))) return rc;
+  if ((rc = make_map(h, &mp.b0, B0, b_cols, b0_rows, b_mn ? 64 : 128, 64))) return rc;
+  if ((rc = make_map(h, &mp.b1, B1 ? B1 : B0, b_cols, B1 ? b1_rows : b0_rows, b_mn ? 64 : 128,
+                     64)))
+    return rc;
+  if ((rc = make_map(h, &mp.d, D, d_cols, d_rows, 32, 32, 4))) return rc;
+  g.err = h->d_err;
+  const int pairs = h->sms / 2;
+  if (add) {
+    choose_splits(g, pairs);
+  } else {
+    g.splits = 1;
+    g.kb_per_split = (g.K + 63) / 64;
+  }
+  const int tiles = gemm_pair_tiles(g);
+  CK(h, launch_gemm_pair(a_mn, b_mn, add, mp, g, 2 * std::min(tiles, pairs), st));
+  h->launches += 1;
+  return ENGRAM_OK;
+}
+
+int gemm_f32(engram_handle* h, const float* A, int64_t a_m, int64_t a_k, const float* B,
+             int64_t b_n, int64_t b_k, float* D, int64_t ldd, int M, int N, int K, bool add,
+             cudaStream_t st) {
+  GemmF32Args g{A, a_m, a_k, B, b_n, b_k, D, ldd, M, N, K, add};
+  CK(h, launch_gemm_f32(g, st));
+  h->launches += 1;
   return ENGRAM_OK;
 }
 
@@ -1045,14 +1250,12 @@ int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx,
     return fail(h, ENGRAM_ERR_INVALID, "h, dout and dh must be non-null and 16-byte aligned");
   if (!idx && !tokens) return fail(h, ENGRAM_ERR_INVALID, "need tokens or idx");
   if (dtables)
-    for (int s = 0; s < S; ++s)
+    for (int s = 0; s < S * h->shards; ++s)
       if (!dtables[s]) return fail(h, ENGRAM_ERR_INVALID, "null table-gradient pointer");
   cudaStream_t st = (cudaStream_t)stream;
-  const int grid = gate_bw_grid(M, d, R);
+  const int grid = gate_bw_grid(M, d, R, h->elt);
   if ((rc = ensure_scratch(h, R))) return rc;
   if ((rc = ensure_bw_scratch(h, R, grid))) return rc;
-  if (cublasSetStream(h->blas, st) != CUBLAS_STATUS_SUCCESS)
-    return fail(h, ENGRAM_ERR_CUDA, "cublasSetStream failed");
   const bool prof = h->bprof_armed;
   h->bprof_armed = false;
   auto mark = [&](int i) -> cudaError_t {
@@ -1069,6 +1272,7 @@ int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx,
   }
   GatherArgs ga{};
   ga.tables = h->d_tables;
+  ga.shards = h->shards;
   ga.primes = h->d_primes;
   ga.idx = z;
   ga.e = h->e;
@@ -1082,12 +1286,31 @@ int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx,
 
   // k and v recomputed (Eq. 3): kv [R, (M+1) d] = e [W_K; W_V]^T
   const int nkv = (M + 1) * d;
-  const char* dkv = static_cast<const char*>(h->bw_dkv);
-  if ((rc = gemm(h, true, false, M * d, (int)R, dm, h->w_k, dm, h->e, dm, 0.f, h->bw_kv, nkv)))
-    return rc;
-  if ((rc = gemm(h, true, false, d, (int)R, dm, h->w_v, dm, h->e, dm, 0.f,
-                 h->bw_kv + (int64_t)M * d, nkv)))
-    return rc;
+  const bool bf16 = h->cfg.dtype == ENGRAM_BF16;
+  const int Md = M * d;
+  const void* dkv = h->bw_dkv;  // [R, (M + 1) d] in the handle's dtype
+  if (bf16) {
+    GemmArgs g{};
+    g.M = (int)R;
+    g.K = dm;
+    g.kb_split = 1 << 30;
+    g.N = Md;
+    if ((rc = gemm_bf16(h, false, false, false, h->e, R, dm, h->w_k, Md, nullptr, 0, dm, h->bw_kv,
+                        R, nkv, g, st)))
+      return rc;
+    g.N = d;
+    g.d_col0 = Md;
+    if ((rc = gemm_bf16(h, false, false, false, h->e, R, dm, h->w_v, d, nullptr, 0, dm, h->bw_kv,
+                        R, nkv, g, st)))
+      return rc;
+  } else {
+    const float* e32 = (const float*)h->e;
+    if ((rc = gemm_f32(h, e32, dm, 1, (const float*)h->w_k, dm, 1, h->bw_kv, nkv, (int)R, Md, dm,
+                       false, st)) ||
+        (rc = gemm_f32(h, e32, dm, 1, (const float*)h->w_v, dm, 1, h->bw_kv + Md, nkv, (int)R, d,
+                       dm, false, st)))
+      return rc;
+  }
   CK(h, mark(2));
 
   // gate and residual backward: dh, dk, dv, RMSNorm weight gradients
@@ -1100,6 +1323,7 @@ int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx,
   a.dh = dhid;
   a.dkv = h->bw_dkv;
   a.partials = h->bw_partials;
+  a.err = h->d_err;
   a.R = R;
   a.M = M;
   a.d = d;
@@ -1114,26 +1338,63 @@ int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx,
   }
   CK(h, mark(3));
 
-  // weight gradients (Eq. 3 transposed): dW_K += dk^T e, dW_V += dv^T e
-  if (dw_k && (rc = gemm(h, false, true, dm, M * d, (int)R, h->e, dm, dkv, nkv, 1.f, dw_k, dm)))
-    return rc;
-  if (dw_v && (rc = gemm(h, false, true, dm, d, (int)R, h->e, dm,
-                         dkv + (int64_t)M * d * h->elt, nkv, 1.f, dw_v, dm)))
-    return rc;
+  // weight gradients (Eq. 3 transposed): dW_K += dk^T e, dW_V += dv^T e, a
+  // contraction over the rows (both operands MN-major)
+  if (bf16) {
+    GemmArgs g{};
+    g.N = dm;
+    g.K = (int)R;
+    g.kb_split = 1 << 30;
+    if (dw_k) {
+      g.M = Md;
+      if ((rc = gemm_bf16(h, true, true, true, dkv, R, nkv, h->e, R, nullptr, 0, dm, dw_k, Md, dm,
+                          g, st)))
+        return rc;
+    }
+    if (dw_v) {
+      g.M = d;
+      g.a_off = Md;
+      if ((rc = gemm_bf16(h, true, true, true, dkv, R, nkv, h->e, R, nullptr, 0, dm, dw_v, d, dm,
+                          g, st)))
+        return rc;
+    }
+  } else {
+    const float* dkv32 = (const float*)h->bw_dkv;
+    const float* e32 = (const float*)h->e;
+    if (dw_k && (rc = gemm_f32(h, dkv32, 1, nkv, e32, 1, dm, dw_k, dm, Md, dm, (int)R, true, st)))
+      return rc;
+    if (dw_v &&
+        (rc = gemm_f32(h, dkv32 + Md, 1, nkv, e32, 1, dm, dw_v, dm, d, dm, (int)R, true, st)))
+      return rc;
+  }
   CK(h, mark(4));
 
-  // memory-vector gradient de = [dk dv] [W_K; W_V], then the table rows (Eq. 2 transposed)
+  // memory-vector gradient de = [dk dv] [W_K; W_V] (B MN-major, its K range
+  // from the two weight tensors), then the table rows (Eq. 2 transposed)
   if (dtables) {
-    if ((rc = gemm(h, false, false, dm, (int)R, M * d, h->w_k, dm, dkv, nkv, 0.f, h->bw_de, dm)))
-      return rc;
-    if ((rc = gemm(h, false, false, dm, (int)R, d, h->w_v, dm, dkv + (int64_t)M * d * h->elt, nkv,
-                   1.f, h->bw_de, dm)))
-      return rc;
+    if (bf16) {
+      GemmArgs g{};
+      g.M = (int)R;
+      g.N = dm;
+      g.K = nkv;
+      g.kb_split = Md / 64;
+      if ((rc = gemm_bf16(h, false, true, false, dkv, R, nkv, h->w_k, Md, h->w_v, d, dm, h->bw_de,
+                          R, dm, g, st)))
+        return rc;
+    } else {
+      const float* dkv32 = (const float*)h->bw_dkv;
+      if ((rc = gemm_f32(h, dkv32, nkv, 1, (const float*)h->w_k, 1, dm, h->bw_de, dm, (int)R, dm,
+                         Md, false, st)) ||
+          (rc = gemm_f32(h, dkv32 + Md, nkv, 1, (const float*)h->w_v, 1, dm, h->bw_de, dm, (int)R,
+                         dm, d, true, st)))
+        return rc;
+    }
     TableGradArgs tg{};
     tg.de = h->bw_de;
     tg.idx = z;
     tg.primes = h->d_primes;
-    for (int s = 0; s < S; ++s) tg.dtables[s] = dtables[s];
+    for (int s = 0; s < S * h->shards; ++s) tg.dtables[s] = dtables[s];
+    tg.shards = h->shards;
     tg.err = h->d_err;
     tg.rows = R;
     tg.S = S;

@@ -3,12 +3,11 @@
 // weights, scratch and prefetch state.  Internal to libengram.so.
 #pragma once
 
-#include <cublas_v2.h>
-
 #include <string>
 
 #include "../../include/engram.h"
 #include "engram_internal.cuh"
+#include "host_gather.cuh"
 
 struct engram_handle {
   engram_config cfg{};
@@ -28,7 +27,8 @@ struct engram_handle {
   // borrowed parameters
   bool have_params = false;
   const void* tables[engram::kMaxTables] = {};
-  const void** d_tables = nullptr;  // device array of S table pointers
+  const void** d_tables = nullptr;  // device array of S x shards table (shard) pointers
+  int shards = 1;                   // row shards per table (engram_set_table_shards)
   const void* w_k = nullptr;
   const void* w_v = nullptr;
   float* d_wqk = nullptr;           // norm_q * norm_k, [M, d]
@@ -68,7 +68,7 @@ struct engram_handle {
   uint32_t set_cap = 0;
   unsigned long long* d_keys = nullptr;
   int32_t* d_vals = nullptr;
-  unsigned long long* d_count[2] = {nullptr, nullptr};
+  unsigned long long* d_count[2] = {nullptr, nullptr};  // [2] each: host-table rows, hot rows
   int2* d_uniq = nullptr;
   int64_t* d_remap[2] = {nullptr, nullptr};
   void* d_staging[2] = {nullptr, nullptr};
@@ -78,7 +78,16 @@ struct engram_handle {
   cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
   int64_t pf_rows[2] = {0, 0};
   uint64_t n_prefetch = 0, n_consumed = 0;
-  unsigned long long* d_hot_hits[2] = {nullptr, nullptr};  // per prefetch slot
+  // how step 5 moves the rows (engram_set_prefetch): host threads + copy
+  // engines, or zero-copy loads on a few CTAs
+  int pf_mode = ENGRAM_PREFETCH_HOST_THREADS;
+  int pf_workers = 0;                           // 0: the default for the mode
+  engram::HostGather* hg = nullptr;             // host-thread route
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_list[2] = {nullptr, nullptr};  // the row list has reached the host
+  unsigned long long* h_count[2] = {nullptr, nullptr};  // pinned [2]
+  int2* h_list[2] = {nullptr, nullptr};         // pinned [rows*S]
+  char* h_bounce[2] = {nullptr, nullptr};       // pinned [rows*S, row_bytes]
 
   // hot-row cache in HBM in front of the host tables (engram_build_hot_cache)
   int64_t n_hot = 0;
@@ -87,8 +96,7 @@ struct engram_handle {
   int32_t* d_hot_slots = nullptr;            // [hot_cap] cache slot per bucket
   void* d_hot_rows = nullptr;                // [n_hot, row_bytes]
 
-  // backward (engram_backward): scratch sized for bw_cap_rows, cuBLAS for its
-  // dense GEMMs (k and v recomputed, weight and memory-vector gradients)
+  // backward (engram_backward): scratch sized for bw_cap_rows
   int64_t bw_cap_rows = 0;
   int64_t* bw_idx = nullptr;       // [rows, S]
   float* bw_kv = nullptr;          // [rows, (M + 1) d]
@@ -96,7 +104,6 @@ struct engram_handle {
   float* bw_de = nullptr;          // [rows, d_mem]
   float* bw_partials = nullptr;    // [bw_part_blocks][2][M][d]
   int bw_part_blocks = 0;
-  cublasHandle_t blas = nullptr;
 
   // instrumentation
   int64_t launches = 0;
@@ -106,3 +113,17 @@ struct engram_handle {
   cudaEvent_t bprof[6] = {};  // stages of the next engram_backward
   bool bprof_armed = false;
 };
+
+namespace engram {
+
+// 2-D row-major tensor map of `rows` rows x `cols` elements of esz bytes (2:
+// bf16, 4: fp32, 1: E4M3 codes) with a box of box_cols x box_rows; a box row
+// of 128 bytes gets the 128-byte swizzle, any other the 64-byte one.  On
+// failure the message goes to h->last_error.
+int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
+             int box_rows, int box_cols = 64, int esz = 2);
+
+// Index into the handle's W tensor maps (map_wk, map_wv) of a box width.
+inline int bn_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
+
+}  // namespace engram

@@ -18,6 +18,7 @@ constexpr unsigned kDevErrTimeout = 4u;  // a bounded mbarrier wait expired
 constexpr int kMaxTables = 64;
 constexpr int kMaxOrders = 4;
 constexpr int kMaxBranches = 4;
+constexpr int kMaxShards = 8;  // row shards per table (engram_set_table_shards)
 
 // Everything the compress+hash kernel needs (section 2.2, Eq. 1).
 struct HashArgs {
@@ -33,8 +34,11 @@ struct HashArgs {
 };
 
 // Row gather (Eq. 2).  Tables are addressed through a device array of S pointers.
+// Row-sharded tables: row z of table s lives in shard z % shards at local row
+// z / shards; `tables` then holds S x shards pointers, table-major.
 struct GatherArgs {
-  const void* const* tables;  // device array [S] of table base pointers
+  const void* const* tables;  // device array [S x shards] of table (shard) base pointers
+  int32_t shards;             // 1: whole tables
   const int64_t* primes;      // [S]
   const int64_t* idx;         // [rows, S]
   void* e;                    // [rows, S*d_head]
@@ -47,7 +51,8 @@ struct GatherArgs {
 // Hash and gather in one pass (Eq. 1 then Eq. 2), for device-resident tables.
 struct HashGatherArgs {
   HashArgs hash;              // idx is unused: the indices stay on chip
-  const void* const* tables;  // device array [S] of table base pointers
+  const void* const* tables;  // device array [S x shards] of table (shard) base pointers
+  int32_t shards;             // 1: whole tables
   void* e;                    // [rows, S*d_head]
   uint8_t* q;                 // E4M3 form: codes [rows, S*d_head] (bf16 tables)
   float* scale;               // E4M3 form: power-of-two scale per row
@@ -98,6 +103,7 @@ struct GateBwArgs {
   void* dh;             // [R, M, d] gradient of h, same dtype
   void* dkv;            // [R, (M + 1) d] dk of each branch, then dv, same dtype
   float* partials;      // [grid][2][M][d] per-CTA sums for the RMSNorm weight gradients
+  unsigned* err;        // device error word (a bounded wait that expired)
   int64_t R;
   int32_t M, d;
   bool bf16;
@@ -109,14 +115,16 @@ struct TableGradArgs {
   const float* de;               // [rows, S * d_head]
   const int64_t* idx;            // [rows, S]
   const int64_t* primes;         // [S] (indices outside a table are skipped and flagged)
-  float* dtables[kMaxTables];    // fp32 [primes[s], d_head] each
+  float* dtables[kMaxTables * kMaxShards];  // fp32 [rows of the shard, d_head], table-major
   unsigned* err;
   int64_t rows;
   int32_t S, d_head;
+  int32_t shards;                // 1: whole tables
 };
 
 size_t gate_bw_smem(int M, int d);
-int gate_bw_grid(int M, int d, int64_t R);
+size_t gate_bw_ring_smem(int M, int d, int elt);
+int gate_bw_grid(int M, int d, int64_t R, int elt);
 // d <= 4096 and gate_bw_smem(M, d) within the per-CTA shared memory limit.
 cudaError_t launch_gate_backward(const GateBwArgs& a, int grid, cudaStream_t stream);
 // dnorm_q[i] += sum_b partials[b][0][i], dnorm_k[i] += sum_b partials[b][1][i]
@@ -133,21 +141,20 @@ struct PrefetchArgs {
   unsigned long long* keys;     // [cap] open-addressing set, cap a power of two >= 2*rows*S
   int32_t* vals;                // [cap] staging slot of each occupied bucket
   uint32_t cap;
-  unsigned long long* count;    // distinct rows found
-  int2* uniq;                   // [rows*S] (slot s, row z) of each staging slot
+  unsigned long long* count;    // [2]: distinct rows from the host tables, from the hot cache
+  int2* uniq;                   // [rows*S] per staging slot: (s, z) at the front, (-1, cache
+                                // slot) at the back
   int64_t* remapped;            // [rows, S] staging slot of each index
   const void* const* tables;    // device array [S] of pinned host table pointers
   int32_t row_bytes;
   void* staging;                // [rows*S, row_bytes] device
   int sms;
-  int fetch_blocks;             // grid cap of the PCIe copy kernel
-  // hot-row cache in HBM (null hot_keys: none): rows found there are copied
-  // from HBM instead of over PCIe
+  int fetch_blocks;             // grid of the zero-copy fetch kernel
+  // hot-row cache in HBM (null hot_keys: none): its rows are copied from HBM
   const unsigned long long* hot_keys;  // [hot_cap] open-addressing set of (s << 40 | z)
   const int32_t* hot_slots;     // [hot_cap] cache slot of each occupied bucket
   uint32_t hot_cap;             // power of two
   const void* hot_rows;         // [cached rows, row_bytes]
-  unsigned long long* hot_hits; // distinct rows of this prefetch served from the cache
 };
 
 // Hot-row cache building blocks (host-resident tables).
@@ -181,7 +188,12 @@ cudaError_t launch_conv_taps(const float* conv_w, const float* norm_w, int d, fl
 // dilation 1..4; scale is scratch [B*T, M] fp32.  Two launches: the RMS
 // scale per (position, branch), then the convolution and residual.
 cudaError_t launch_short_conv(const ConvArgs& a, int dilation, float* scale, cudaStream_t stream);
-cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream);
+// Steps 1-4 of the prefetch: distinct rows, staging slots, remapped indices,
+// hot rows copied from the cache.
+cudaError_t launch_prefetch_index(const PrefetchArgs& a, cudaStream_t stream);
+// Step 5 by zero-copy loads: the count[0] rows of the host tables listed at
+// the front of uniq, on a.fetch_blocks CTAs.
+cudaError_t launch_prefetch_fetch(const PrefetchArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t stream);
 cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);
 
@@ -215,6 +227,45 @@ cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArg
 // 128 in phase 0).  Phases 0-2 as above.
 cudaError_t launch_proj_gate_pair(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
                                   cudaStream_t stream);
+
+// Dense contractions of the backward (bf16 operands, fp32 accumulation):
+// D[m, n] (= or +=) sum_k A(m, k) B(n, k), m < M, n < N, k < K.  A K-major A
+// is stored [rows, K] (map box 64 x 128, 128-byte swizzle), an MN-major A
+// [K, rows] (box 64 x 64); the same for B.  B's K range may come from two
+// tensors: K blocks (of 64) below kb_split from map b0, the rest from map b1
+// at K - 64 kb_split.  D is fp32 (map box 32 x 32, 128-byte swizzle), n = 0 at
+// column d_col0.  With `add` the tiles reduce-add into D, and K may be split
+// over `splits` tiles of kb_per_split K blocks each.
+struct GemmArgs {
+  int32_t M, N, K;
+  int32_t a_off;          // first A row (K-major) or column (MN-major) used
+  int32_t kb_split;       // K blocks read from map b0
+  int32_t splits, kb_per_split;
+  int32_t d_col0;
+  unsigned* err;
+};
+struct GemmMaps {
+  CUtensorMap a, b0, b1, d;
+};
+// Tiles of 256 x 256 (one per CTA pair and round) times the K splits.
+int gemm_pair_tiles(const GemmArgs& g);
+// grid = 2 x pairs (even).
+cudaError_t launch_gemm_pair(bool a_mn, bool b_mn, bool add, const GemmMaps& maps,
+                             const GemmArgs& g, int grid, cudaStream_t stream);
+
+// fp32 form (SIMT FFMA, 64 x 64 tiles) with strided operands:
+// D[m * ldd + n] (= or +=) sum_k A[m * a_m + k * a_k] B[n * b_n + k * b_k].
+struct GemmF32Args {
+  const float* A;
+  int64_t a_m, a_k;
+  const float* B;
+  int64_t b_n, b_k;
+  float* D;
+  int64_t ldd;
+  int32_t M, N, K;
+  bool add;
+};
+cudaError_t launch_gemm_f32(const GemmF32Args& g, cudaStream_t stream);
 
 // The bf16 projection kernel of one phase (0 keys, 1 values) for R rows.
 enum class ProjKernel { Wide, Pair, Single };

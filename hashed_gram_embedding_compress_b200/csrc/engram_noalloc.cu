@@ -10,8 +10,6 @@
 // produce e with engram_hash and engram_gather into its own buffers), and the
 // only scratch, the key phase's per-row partial sums, lives in a fixed array
 // in the library's device image.
-#include <cudaTypedefs.h>
-
 #include <cmath>
 #include <mutex>
 #include <string>
@@ -63,33 +61,6 @@ int partials_address(engram_handle* h, float4** out) {
   *out = reinterpret_cast<float4*>(g_partials_dev[dev]);
   return ENGRAM_OK;
 }
-
-int encode_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
-               int box_rows, int box_cols) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1u, 1u};
-  const CUtensorMapSwizzle sw =
-      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return fail(h, ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-  return ENGRAM_OK;
-}
-
-int map_slot(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -161,41 +132,41 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
     const int kphase = (phase == 1 && out == hid) ? 2 : phase;
     if (pc.kind == ProjKernel::Pair) {
       if (!have_pair) {
-        if ((rc = encode_map(h, &pair.e, e, h->d_mem, R, 128, 64)) ||
-            (rc = encode_map(h, &pair.h, hid, hcols, R, 128, 32)) ||
-            (rc = encode_map(h, &pair.out, out, hcols, R, 32, 32)))
+        if ((rc = make_map(h, &pair.e, e, h->d_mem, R, 128, 64)) ||
+            (rc = make_map(h, &pair.h, hid, hcols, R, 128, 32)) ||
+            (rc = make_map(h, &pair.out, out, hcols, R, 32, 32)))
           return rc;
         have_pair = true;
       }
-      pair.w = wmaps[map_slot(pc.bn)];
+      pair.w = wmaps[bn_index(pc.bn)];
       ProjMaps pm = pair;
       // in place: per-warp reduce-adds of 32 rows x 64 columns
-      if (kphase == 2 && (rc = encode_map(h, &pm.out, out, hcols, R, 32, 64))) return rc;
+      if (kphase == 2 && (rc = make_map(h, &pm.out, out, hcols, R, 32, 64))) return rc;
       if ((ce = launch_proj_gate_pair(kphase, pm, g, pc.grid, st)))
         return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
     } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
-        if ((rc = encode_map(h, &wide.e, e, h->d_mem, R, 256, 64)) ||
-            (rc = encode_map(h, &wide.h, hid, hcols, R, 256, 32)) ||
-            (rc = encode_map(h, &wide.out, out, hcols, R, 32, 32)))
+        if ((rc = make_map(h, &wide.e, e, h->d_mem, R, 256, 64)) ||
+            (rc = make_map(h, &wide.h, hid, hcols, R, 256, 32)) ||
+            (rc = make_map(h, &wide.out, out, hcols, R, 32, 32)))
           return rc;
         have_wide = true;
       }
-      wide.w = wmaps[map_slot(pc.bn)];
+      wide.w = wmaps[bn_index(pc.bn)];
       ProjMaps wl = wide;
       // in place: per-warp reduce-adds of 32 rows x 64 columns
-      if (kphase == 2 && (rc = encode_map(h, &wl.out, out, hcols, R, 32, 64))) return rc;
+      if (kphase == 2 && (rc = make_map(h, &wl.out, out, hcols, R, 32, 64))) return rc;
       if ((ce = launch_proj_gate_wide(kphase, wl, g, pc.grid, st)))
         return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
     } else {
       if (!have_single) {
-        if ((rc = encode_map(h, &single.e, e, h->d_mem, R, 128, 64)) ||
-            (rc = encode_map(h, &single.h, hid, hcols, R, 128, 64)) ||
-            (rc = encode_map(h, &single.out, out, hcols, R, 128, 64)))
+        if ((rc = make_map(h, &single.e, e, h->d_mem, R, 128, 64)) ||
+            (rc = make_map(h, &single.h, hid, hcols, R, 128, 64)) ||
+            (rc = make_map(h, &single.out, out, hcols, R, 128, 64)))
           return rc;
         have_single = true;
       }
-      single.w = wmaps[map_slot(pc.bn)];
+      single.w = wmaps[bn_index(pc.bn)];
       if ((ce = launch_proj_gate_sm100(phase, pc.bn, single, g, pc.grid, st)))
         return fail(h, ENGRAM_ERR_CUDA, cudaGetErrorString(ce));
     }

@@ -15,13 +15,17 @@
 //     u_q = dqn w_q:  dh = dout + rh u_q - rh^3 / d h (u_q . h),
 //     u_k = dkn w_k:  dk = rk u_k - rk^3 / d k (u_k . k).
 //
-// gate_backward_kernel: a CTA per row at a time (grid-stride), 256 threads,
-// each holding PER elements of the row (column tid + 256 j) in registers; the
-// two row reductions per branch are block reductions.  dw_q and dw_k are
+// gate_backward_ring_kernel: a CTA of 256 threads per row at a time
+// (grid-stride, two CTAs per SM); thread 0 streams the rows' h, dout and kv
+// into a ring of three shared-memory slots with bulk copies two rows ahead,
+// so the loads of the next rows overlap the reductions of the current one.
+// The two row reductions per branch are block reductions.  dw_q and dw_k are
 // summed per CTA in shared memory (each thread owns its columns) and reduced
 // over the CTAs in a fixed order by dnorm_reduce_kernel (deterministic).
+// gate_backward_kernel is the same arithmetic with the row in registers and
+// no ring, for rows too long for three slots.
 // table_grad_kernel adds the slices of de into fp32 table gradients.
-#include "engram_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace engram {
 
@@ -154,6 +158,171 @@ __global__ void __launch_bounds__(kBwThreads) gate_backward_kernel(GateBwArgs a)
   for (int64_t i = tid; i < 2LL * M * d; i += kBwThreads) part[i] = s_dwq[i];
 }
 
+constexpr int kRing = 3;
+
+// Bytes of one ring slot: h and dout rows (element size elt) and the kv row (fp32).
+__host__ __device__ inline size_t ring_slot_bytes(int M, int d, int elt) {
+  return (size_t)2 * M * d * elt + (size_t)(M + 1) * d * 4;
+}
+
+template <int PER>
+__global__ void __launch_bounds__(kBwThreads) gate_backward_ring_kernel(GateBwArgs a) {
+  extern __shared__ __align__(128) unsigned char smraw[];
+  const int d = a.d, M = a.M, tid = threadIdx.x;
+  const int elt = a.bf16 ? 2 : 4;
+  const int64_t nkv = (int64_t)(M + 1) * d;
+  const float inv_d = 1.f / (float)d;
+  const uint32_t hb = (uint32_t)M * d * elt, kvb = (uint32_t)nkv * 4;
+  const size_t slot_bytes = ring_slot_bytes(M, d, elt);
+  unsigned char* ring = smraw;
+  float* red = reinterpret_cast<float*>(ring + kRing * slot_bytes);   // [2][8 warps][4]
+  float* s_dwq = red + 64;                                           // [M][d]
+  float* s_dwk = s_dwq + (int64_t)M * d;                             // [M][d]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_dwk + (int64_t)M * d);  // [kRing]
+  volatile int* flag = reinterpret_cast<volatile int*>(full + kRing);
+  for (int64_t i = tid; i < 2LL * M * d; i += kBwThreads) s_dwq[i] = 0.f;
+  if (tid == 0) {
+    for (int i = 0; i < kRing; ++i) sm100::mbar_init(sm100::smem_u32(full + i), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // row i of this CTA is blockIdx.x + i gridDim.x, staged in slot i % kRing
+  const int64_t n_rows = a.R > blockIdx.x ? (a.R - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  int64_t issued = 0;  // rows whose copies thread 0 has issued
+  auto issue_next = [&]() {
+    if (issued >= n_rows) return;
+    const int64_t r = blockIdx.x + issued * (int64_t)gridDim.x;
+    const int slot = (int)(issued % kRing);
+    const uint32_t bar = sm100::smem_u32(full + slot);
+    const uint32_t dst = sm100::smem_u32(ring + slot * slot_bytes);
+    sm100::mbar_expect_tx(bar, 2 * hb + kvb);
+    sm100::bulk_load(dst, (const char*)a.h + r * hb, hb, bar);
+    sm100::bulk_load(dst + hb, (const char*)a.dout + r * hb, hb, bar);
+    sm100::bulk_load(dst + 2 * hb, a.kv + r * nkv, kvb, bar);
+    ++issued;
+  };
+  // bounded wait for the copies of row i (thread 0)
+  auto wait_row = [&](int64_t i) -> bool {
+    const uint32_t bar = sm100::smem_u32(full + (i % kRing));
+    const uint32_t par = (uint32_t)(i / kRing) & 1u;
+    if (sm100::mbar_try_wait(bar, par)) return true;
+    const uint64_t t0 = sm100::globaltimer();
+    while (!sm100::mbar_try_wait(bar, par))
+      if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) return false;
+    return true;
+  };
+  if (tid == 0)
+    for (int i = 0; i < kRing - 1; ++i) issue_next();
+  int rb = 0;  // which half of `red` the next reduction uses
+  // sum of N values over the block with one barrier: the halves of `red`
+  // alternate, so a reduction never overwrites values still being read
+  auto bsum = [&](float* x, int N) {
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int n = 0; n < N; ++n)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x[n] += __shfl_xor_sync(0xffffffffu, x[n], o);
+    float* rr = red + rb * 32;
+    if (lane == 0)
+      for (int n = 0; n < N; ++n) rr[warp * 4 + n] = x[n];
+    __syncthreads();
+    for (int n = 0; n < N; ++n) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kBwThreads / 32; ++w) t += rr[w * 4 + n];
+      x[n] = t;
+    }
+    rb ^= 1;
+  };
+  int64_t i = 0;
+  for (; i < n_rows; ++i) {
+    const int64_t r = blockIdx.x + i * (int64_t)gridDim.x;
+    if (tid == 0) {
+      issue_next();  // row i + kRing - 1, into the slot row i - 1 left
+      const bool ok = wait_row(i);
+      *flag = ok ? 1 : 0;
+      if (!ok) atomicOr(a.err, kDevErrTimeout);
+    }
+    __syncthreads();
+    if (!*flag) break;
+    const unsigned char* slot = ring + (i % kRing) * slot_bytes;
+    const void* hs = slot;
+    const void* gs = slot + hb;
+    const float* kv = reinterpret_cast<const float*>(slot + 2 * hb);
+    float dv[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) dv[j] = 0.f;
+    for (int m = 0; m < M; ++m) {
+      const int64_t base = (r * M + m) * (int64_t)d;
+      const int sb = m * d;
+      const float* wq = a.w_q + (int64_t)m * d;
+      const float* wk = a.w_k + (int64_t)m * d;
+      float sums[4] = {0.f, 0.f, 0.f, 0.f};  // sum h^2, sum k^2, sum (h w_q)(k w_k), dout . v
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int c = tid + kBwThreads * j;
+        if (c < d) {
+          const float h = load_elt(hs, sb + c, a.bf16), k = kv[sb + c];
+          const float g = load_elt(gs, sb + c, a.bf16), v = kv[M * d + c];
+          sums[0] += h * h;
+          sums[1] += k * k;
+          sums[2] += (h * __ldg(wq + c)) * (k * __ldg(wk + c));
+          sums[3] += g * v;
+        }
+      }
+      bsum(sums, 4);
+      const float rh = rsqrtf(sums[0] * inv_d + a.eps);
+      const float rk = rsqrtf(sums[1] * inv_d + a.eps);
+      const float alpha = 1.f / (1.f + __expf(-sums[2] * rh * rk * a.inv_sqrt_d));
+      const float ds = sums[3] * alpha * (1.f - alpha);
+      const float cq = ds * rk * a.inv_sqrt_d;  // dqn_c = cq k_c w_k,c
+      const float ck = ds * rh * a.inv_sqrt_d;  // dkn_c = ck h_c w_q,c
+      float u[2] = {0.f, 0.f};                  // u_q . h, u_k . k
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int c = tid + kBwThreads * j;
+        if (c < d) {
+          const float h = load_elt(hs, sb + c, a.bf16), k = kv[sb + c];
+          const float g = load_elt(gs, sb + c, a.bf16);
+          const float q_w = __ldg(wq + c), k_w = __ldg(wk + c);
+          const float dqn = cq * k * k_w, dkn = ck * h * q_w;
+          s_dwq[sb + c] += dqn * h * rh;
+          s_dwk[sb + c] += dkn * k * rk;
+          u[0] += dqn * q_w * h;
+          u[1] += dkn * k_w * k;
+          dv[j] += alpha * g;
+        }
+      }
+      bsum(u, 2);
+      const float th = rh * rh * rh * inv_d * u[0], tk = rk * rk * rk * inv_d * u[1];
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int c = tid + kBwThreads * j;
+        if (c < d) {
+          const float h = load_elt(hs, sb + c, a.bf16), k = kv[sb + c];
+          const float g = load_elt(gs, sb + c, a.bf16);
+          const float q_w = __ldg(wq + c), k_w = __ldg(wk + c);
+          const float dqn = cq * k * k_w, dkn = ck * h * q_w;
+          store_elt(a.dh, base + c, g + rh * dqn * q_w - th * h, a.bf16);
+          store_elt(a.dkv, r * nkv + sb + c, rk * dkn * k_w - tk * k, a.bf16);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int c = tid + kBwThreads * j;
+      if (c < d) store_elt(a.dkv, r * nkv + (int64_t)M * d + c, dv[j], a.bf16);
+    }
+    __syncthreads();  // slot i % kRing is read by no thread any more
+  }
+  __syncthreads();
+  float* part = a.partials + (int64_t)blockIdx.x * 2 * M * d;
+  for (int64_t j = tid; j < 2LL * M * d; j += kBwThreads) part[j] = s_dwq[j];
+  // after a timeout: the copies still in flight land before the CTA leaves
+  // (each waited for a bounded time)
+  if (tid == 0)
+    for (int64_t k = i; k < issued; ++k) (void)wait_row(k);
+}
+
 // dnorm_q[i] += sum over CTAs b of partials[b][0][i], dnorm_k likewise, in
 // order of b (one thread per column).
 __global__ void dnorm_reduce_kernel(const float* partials, int nblocks, int64_t n, float* dnorm_q,
@@ -184,7 +353,16 @@ __global__ void table_grad_kernel(TableGradArgs a) {
       if (c == 0) atomicOr(a.err, kDevErrIndex);
       continue;
     }
-    atomicAdd(a.dtables[s] + z * a.d_head + c, a.de[i]);
+    float* dst;
+    if (a.shards == 1) {
+      dst = a.dtables[s] + z * a.d_head;
+    } else {
+      // row-sharded: owner z % N at local row z / N (z < 2^31)
+      const uint32_t q = (uint32_t)z / (uint32_t)a.shards;
+      dst = a.dtables[s * a.shards + (int)((uint32_t)z - q * (uint32_t)a.shards)] +
+            (int64_t)q * a.d_head;
+    }
+    atomicAdd(dst + c, a.de[i]);
   }
 }
 
@@ -229,10 +407,18 @@ int resident(size_t smem) {
 }  // namespace
 
 // One CTA per resident slot on every SM (each loops over rows), at most R.
-int gate_bw_grid(int M, int d, int64_t R) {
+int gate_bw_grid(int M, int d, int64_t R, int elt) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t rsm = gate_bw_ring_smem(M, d, elt);
+  if (rsm <= 232448) {
+    // the ring kernel: as many CTAs per SM as its shared memory allows (<= 2)
+    const int64_t per_sm = rsm <= 113 * 1024 ? 2 : 1;
+    int64_t grid = (int64_t)sms * per_sm;
+    if (grid > R) grid = R;
+    return grid < 1 ? 1 : (int)grid;
+  }
   const size_t smem = gate_bw_smem(M, d);
   const int per = (d + kBwThreads - 1) / kBwThreads;
   const int per_sm = per <= 1   ? resident<1>(smem)
@@ -246,8 +432,37 @@ int gate_bw_grid(int M, int d, int64_t R) {
   return grid < 1 ? 1 : (int)grid;
 }
 
+size_t gate_bw_ring_smem(int M, int d, int elt) {
+  return kRing * ring_slot_bytes(M, d, elt) + 64 * sizeof(float) + 2 * (size_t)M * d * 4 +
+         kRing * 8 + 16;
+}
+
+namespace {
+
+template <int PER>
+cudaError_t launch_ring(const GateBwArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  auto kern = gate_backward_ring_kernel<PER>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kBwThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_gate_backward(const GateBwArgs& a, int grid, cudaStream_t stream) {
   if (a.R == 0) return cudaSuccess;
+  const size_t rsm = gate_bw_ring_smem(a.M, a.d, a.bf16 ? 2 : 4);
+  if (rsm <= 232448) {
+    const int per = (a.d + kBwThreads - 1) / kBwThreads;
+    if (per <= 1) return launch_ring<1>(a, grid, rsm, stream);
+    if (per <= 2) return launch_ring<2>(a, grid, rsm, stream);
+    if (per <= 4) return launch_ring<4>(a, grid, rsm, stream);
+    if (per <= 8) return launch_ring<8>(a, grid, rsm, stream);
+    if (per <= 12) return launch_ring<12>(a, grid, rsm, stream);
+    if (per <= 16) return launch_ring<16>(a, grid, rsm, stream);
+    return cudaErrorInvalidValue;
+  }
   const size_t smem = gate_bw_smem(a.M, a.d);
   if (smem > 232448) return cudaErrorInvalidValue;
   const int per = (a.d + kBwThreads - 1) / kBwThreads;

@@ -103,13 +103,20 @@ __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
 // One thread per 16-byte chunk of e.  Consecutive threads cover consecutive
 // chunks of one table row (a 160-byte bf16 row is 10 chunks), so each warp
 // reads whole rows and writes a contiguous run of e.
+// Address of row z of table s: whole tables, or row-sharded ones (owner z %
+// N, local row z / N; z < 2^31).
+__device__ __forceinline__ const char* row_addr(const char* const* tab, int s, uint64_t z,
+                                                int shards, int64_t row_bytes) {
+  if (shards == 1) return tab[s] + z * (uint64_t)row_bytes;
+  const uint32_t zz = (uint32_t)z, q = zz / (uint32_t)shards;
+  return tab[s * shards + (int)(zz - q * (uint32_t)shards)] + (uint64_t)q * (uint64_t)row_bytes;
+}
+
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
-  __shared__ const char* s_tab[kMaxTables];
+  __shared__ const char* s_tab[kMaxTables * kMaxShards];
   __shared__ int64_t s_prime[kMaxTables];
-  for (int i = threadIdx.x; i < a.S; i += blockDim.x) {
-    s_tab[i] = (const char*)a.tables[i];
-    s_prime[i] = a.primes[i];
-  }
+  for (int i = threadIdx.x; i < a.S * a.shards; i += blockDim.x) s_tab[i] = (const char*)a.tables[i];
+  for (int i = threadIdx.x; i < a.S; i += blockDim.x) s_prime[i] = a.primes[i];
   __syncthreads();
   const uint32_t cpr = (uint32_t)(a.row_bytes >> 4);  // chunks per table row
   const uint32_t S = (uint32_t)a.S;
@@ -123,7 +130,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
     const int64_t z = __ldg(a.idx + rs);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (z >= 0 && z < s_prime[s]) {
-      v = ld_stream_16(s_tab[s] + z * a.row_bytes + c * 16);
+      v = ld_stream_16(row_addr(s_tab, (int)s, (uint64_t)z, a.shards, a.row_bytes) + c * 16);
     } else if (c == 0) {
       atomicOr(a.err, kDevErrIndex);
     }
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
   __shared__ uint64_t s_prime[kMaxTables];
   __shared__ uint64_t s_inv[kMaxTables];
   __shared__ int32_t s_order_of_slot[kMaxTables];
-  __shared__ const char* s_tab[kMaxTables];
+  __shared__ const char* s_tab[kMaxTables * kMaxShards];
   __shared__ const char* s_src[kFusedThreads];  // source row of (row, slot)
   const int S = a.S;
   for (int i = threadIdx.x; i < S * a.max_order; i += blockDim.x) s_mult[i] = a.mult[i];
@@ -153,8 +160,8 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
     s_prime[i] = (uint64_t)a.primes[i];
     s_inv[i] = a.barrett[i];
     s_order_of_slot[i] = a.orders[i / a.heads];
-    s_tab[i] = (const char*)g.tables[i];
   }
+  for (int i = threadIdx.x; i < S * g.shards; i += blockDim.x) s_tab[i] = (const char*)g.tables[i];
   __syncthreads();
 
   const uint32_t Tout = (uint32_t)(a.T - a.t_begin);
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
     const int t = a.t_begin + (int)(row - (uint32_t)b * Tout);
     const uint64_t z = hash_slot(a, a.tokens + (int64_t)b * a.T, t, s_order_of_slot[s],
                                  s_mult + s * a.max_order, s_prime[s], s_inv[s]);
-    s_src[threadIdx.x] = s_tab[s] + z * (uint64_t)g.row_bytes;
+    s_src[threadIdx.x] = row_addr(s_tab, s, z, g.shards, g.row_bytes);
   }
   __syncthreads();
 
@@ -209,7 +216,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_e4m3_kernel(HashGat
   __shared__ uint64_t s_prime[kMaxTables];
   __shared__ uint64_t s_inv[kMaxTables];
   __shared__ int32_t s_order_of_slot[kMaxTables];
-  __shared__ const char* s_tab[kMaxTables];
+  __shared__ const char* s_tab[kMaxTables * kMaxShards];
   __shared__ const char* s_src[kFusedThreads];  // source row of (row, slot)
   const int S = a.S;
   for (int i = threadIdx.x; i < S * a.max_order; i += blockDim.x) s_mult[i] = a.mult[i];
@@ -217,8 +224,8 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_e4m3_kernel(HashGat
     s_prime[i] = (uint64_t)a.primes[i];
     s_inv[i] = a.barrett[i];
     s_order_of_slot[i] = a.orders[i / a.heads];
-    s_tab[i] = (const char*)g.tables[i];
   }
+  for (int i = threadIdx.x; i < S * g.shards; i += blockDim.x) s_tab[i] = (const char*)g.tables[i];
   __syncthreads();
 
   const uint32_t Tout = (uint32_t)(a.T - a.t_begin);
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_e4m3_kernel(HashGat
     const int t = a.t_begin + (int)(row - (uint32_t)b * Tout);
     const uint64_t z = hash_slot(a, a.tokens + (int64_t)b * a.T, t, s_order_of_slot[s],
                                  s_mult + s * a.max_order, s_prime[s], s_inv[s]);
-    s_src[threadIdx.x] = s_tab[s] + z * (uint64_t)g.row_bytes;
+    s_src[threadIdx.x] = row_addr(s_tab, s, z, g.shards, g.row_bytes);
   }
   __syncthreads();
 

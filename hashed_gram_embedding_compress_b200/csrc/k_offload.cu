@@ -7,23 +7,30 @@
 // paper's Table 4 run sends every retrieval over PCIe, and notes that the
 // traffic scales with the active rows, not the table size.
 //
-// Steps (all on the prefetch stream):
+// Steps 1-4 run on the prefetch stream:
 //   1. clear an open-addressing set of 64-bit keys (slot s << 40 | row z);
 //   2. insert every (s, z[r, s]) with atomicCAS: one key per distinct row;
-//   3. number the occupied buckets with an atomic counter: a staging slot per
-//      distinct row, and a list of (s, z) per slot;
+//   3. number the occupied buckets: a staging slot per distinct row.  Rows
+//      held in the HBM hot-row cache take slots from the back of the staging
+//      buffer (count[1]), all others from the front (count[0]), with a list
+//      of (s, z) per front slot and of the cache slot per back slot;
 //   4. remap every index to its staging slot (a lookup, no waiting on other
-//      threads: the slot numbers are final after step 3);
-//   5. copy each distinct row once from pinned host memory (zero-copy loads
-//      over PCIe, 16 bytes per thread, whole rows per run of threads) into
-//      the HBM staging buffer.
+//      threads: the slot numbers are final after step 3), and copy the hot
+//      rows from the cache into their back slots (HBM to HBM).
+// Step 5 moves the front slots' rows, each distinct row once, from pinned
+// host memory into the HBM staging buffer, by one of two routes:
+//   - host threads read the rows into a pinned bounce buffer and the copy
+//     engines send it over PCIe in large copies (engram_host_gather.cu): no
+//     SM takes part, so the transfer runs beside any compute;
+//   - fetch_kernel reads them through the mapped host address (zero-copy
+//     loads over PCIe, 16 bytes per load, eight in flight per thread) on a
+//     capped number of CTAs.
 // The forward then gathers from the staging buffer with the remapped indices.
 //
 // Hot-row cache (the paper's cache hierarchy over a Zipfian access pattern,
 // section 2.5): engram_build_hot_cache counts the rows calibration tokens
-// address (count_kernel), keeps the most frequent ones in HBM
-// (hot_insert_kernel, hot_copy_kernel), and step 5 then copies a cached row
-// from HBM instead of over PCIe.
+// address (count_kernel) and keeps the most frequent ones in HBM
+// (hot_insert_kernel, hot_copy_kernel).
 #include "engram_internal.cuh"
 
 namespace engram {
@@ -47,7 +54,7 @@ __global__ void clear_kernel(unsigned long long* keys, int32_t* vals, uint32_t c
     keys[i] = kEmpty;
     if (vals) vals[i] = -1;
   }
-  if (count && blockIdx.x == 0 && threadIdx.x == 0) *count = 0;
+  if (count && blockIdx.x == 0 && threadIdx.x < 2) count[threadIdx.x] = 0;
 }
 
 // Linear probing; the set holds at least twice as many buckets as inserted
@@ -67,14 +74,37 @@ __global__ void insert_kernel(const int64_t* idx, int64_t n, int32_t S, unsigned
   }
 }
 
-__global__ void number_kernel(const unsigned long long* keys, int32_t* vals, uint32_t cap,
-                              unsigned long long* count, int2* uniq) {
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < cap; i += gridDim.x * blockDim.x) {
-    const unsigned long long k = keys[i];
+// Cache slot of key in the hot-row table, or -1.
+__device__ __forceinline__ int32_t hot_lookup(const unsigned long long* keys, const int32_t* slots,
+                                              uint32_t mask, unsigned long long key) {
+  uint32_t b = mix_bucket(key, mask);
+  for (uint32_t probe = 0; probe <= mask; ++probe) {
+    const unsigned long long k = keys[b];
+    if (k == key) return slots[b];
+    if (k == kEmpty) return -1;
+    b = (b + 1) & mask;
+  }
+  return -1;
+}
+
+// Staging slot per distinct key: rows from the host tables count up from the
+// front (count[0]; uniq = (s, z)), rows in the hot-row cache down from the
+// back (count[1]; uniq = (-1, cache slot)).  At most `entries` keys exist, so
+// the two ranges never meet.
+__global__ void number_kernel(PrefetchArgs a) {
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < a.cap; i += gridDim.x * blockDim.x) {
+    const unsigned long long k = a.keys[i];
     if (k == kEmpty) continue;
-    const int32_t slot = (int32_t)atomicAdd(count, 1ull);
-    vals[i] = slot;
-    uniq[slot] = make_int2((int)(k >> 40), (int)(k & 0xFFFFFFFFFFull));
+    const int32_t hot = a.hot_keys ? hot_lookup(a.hot_keys, a.hot_slots, a.hot_cap - 1, k) : -1;
+    int64_t slot;
+    if (hot >= 0) {
+      slot = a.rows * a.S - 1 - (int64_t)atomicAdd(a.count + 1, 1ull);
+      a.uniq[slot] = make_int2(-1, hot);
+    } else {
+      slot = (int64_t)atomicAdd(a.count, 1ull);
+      a.uniq[slot] = make_int2((int)(k >> 40), (int)(k & 0xFFFFFFFFFFull));
+    }
+    a.vals[i] = (int32_t)slot;
   }
 }
 
@@ -108,44 +138,51 @@ __device__ __forceinline__ uint4 ld_host_16(const void* p) {
   return v;
 }
 
-// Cache slot of key in the hot-row table, or -1.
-__device__ __forceinline__ int32_t hot_lookup(const unsigned long long* keys, const int32_t* slots,
-                                              uint32_t mask, unsigned long long key) {
-  uint32_t b = mix_bucket(key, mask);
-  for (uint32_t probe = 0; probe <= mask; ++probe) {
-    const unsigned long long k = keys[b];
-    if (k == key) return slots[b];
-    if (k == kEmpty) return -1;
-    b = (b + 1) & mask;
+// The hot rows of this prefetch, copied from the cache (HBM) into their
+// staging slots at the back of the buffer; one thread per 16-byte chunk.
+__global__ void hot_fill_kernel(PrefetchArgs a) {
+  const int cpr = a.row_bytes >> 4;
+  const int64_t n_hot = (int64_t)a.count[1];
+  const int64_t first = a.rows * a.S - n_hot;
+  char* staging = (char*)a.staging;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_hot * cpr;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = first + i / cpr;
+    const int c = (int)(i % cpr);
+    const int2 e = a.uniq[u];
+    *reinterpret_cast<uint4*>(staging + u * a.row_bytes + c * 16) = __ldg(
+        reinterpret_cast<const uint4*>((const char*)a.hot_rows + (int64_t)e.y * a.row_bytes + c * 16));
   }
-  return -1;
 }
 
-// One thread per 16-byte chunk of a distinct row; threads past the distinct
-// count (known only on the device) return at once.  A row held in the hot
-// cache is copied from HBM, any other over PCIe.
+// Zero-copy route of step 5: the front slots' rows read through the mapped
+// host address.  Chunk i = 16 bytes of a row; a thread keeps eight chunks,
+// gridDim x blockDim apart, in flight at once (PCIe latency is microseconds,
+// so few CTAs need many loads outstanding).
 __global__ void fetch_kernel(PrefetchArgs a) {
   const int cpr = a.row_bytes >> 4;
-  const int64_t total = (int64_t)(*a.count) * cpr;
+  const int64_t total = (int64_t)a.count[0] * cpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   char* staging = (char*)a.staging;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t u = i / cpr;
-    const int c = (int)(i - u * cpr);
-    const int2 sz = a.uniq[u];
-    int32_t hot = -1;
-    if (a.hot_keys) {
-      const unsigned long long key = ((unsigned long long)sz.x << 40) | (unsigned long long)sz.y;
-      hot = hot_lookup(a.hot_keys, a.hot_slots, a.hot_cap - 1, key);
-      if (hot >= 0 && c == 0) atomicAdd(a.hot_hits, 1ull);
+  constexpr int kInFlight = 8;
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < total;
+       i0 += stride * kInFlight) {
+    uint4 v[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const int64_t i = i0 + k * stride;
+      if (i < total) {
+        const int64_t u = i / cpr;
+        const int c = (int)(i - u * cpr);
+        const int2 sz = a.uniq[u];
+        v[k] = ld_host_16((const char*)a.tables[sz.x] + (int64_t)sz.y * a.row_bytes + c * 16);
+      }
     }
-    uint4 v;
-    if (hot >= 0)
-      v = __ldg(reinterpret_cast<const uint4*>((const char*)a.hot_rows +
-                                               (int64_t)hot * a.row_bytes + c * 16));
-    else
-      v = ld_host_16((const char*)a.tables[sz.x] + (int64_t)sz.y * a.row_bytes + c * 16);
-    *reinterpret_cast<uint4*>(staging + u * a.row_bytes + c * 16) = v;
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const int64_t i = i0 + k * stride;
+      if (i < total) *reinterpret_cast<uint4*>(staging + i * 16) = v[k];
+    }
   }
 }
 
@@ -209,24 +246,31 @@ int blocks_for(int64_t n, int threads, int cap) {
 
 }  // namespace
 
-cudaError_t launch_prefetch(const PrefetchArgs& a, cudaStream_t stream) {
+cudaError_t launch_prefetch_index(const PrefetchArgs& a, cudaStream_t stream) {
   const int n = 256;
   const int cap_blocks = a.sms * 16;
   const int64_t entries = a.rows * a.S;
   clear_kernel<<<blocks_for(a.cap, n, cap_blocks), n, 0, stream>>>(a.keys, a.vals, a.cap, a.count);
-  if (a.hot_hits) {
-    cudaError_t e = cudaMemsetAsync(a.hot_hits, 0, sizeof(unsigned long long), stream);
-    if (e != cudaSuccess) return e;
-  }
   if (entries > 0) {
     insert_kernel<<<blocks_for(entries, n, cap_blocks), n, 0, stream>>>(a.idx, entries, a.S,
                                                                        a.keys, a.cap - 1);
-    number_kernel<<<blocks_for(a.cap, n, cap_blocks), n, 0, stream>>>(a.keys, a.vals, a.cap,
-                                                                     a.count, a.uniq);
+    number_kernel<<<blocks_for(a.cap, n, cap_blocks), n, 0, stream>>>(a);
     remap_kernel<<<blocks_for(entries, n, cap_blocks), n, 0, stream>>>(
         a.idx, entries, a.S, a.keys, a.vals, a.cap - 1, a.remapped);
+    if (a.hot_keys)
+      hot_fill_kernel<<<blocks_for(entries * (a.row_bytes >> 4), n, a.sms * 4), n, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefetch_fetch(const PrefetchArgs& a, cudaStream_t stream) {
+  const int n = 256;
+  const int64_t entries = a.rows * a.S;
+  if (entries > 0) {
     // at most `entries` distinct rows
-    fetch_kernel<<<blocks_for(entries * (a.row_bytes >> 4), n, a.fetch_blocks), n, 0, stream>>>(a);
+    const int64_t per_block = (int64_t)n * 8;
+    fetch_kernel<<<blocks_for(entries * (a.row_bytes >> 4), (int)per_block, a.fetch_blocks), n, 0,
+                   stream>>>(a);
   }
   return cudaGetLastError();
 }

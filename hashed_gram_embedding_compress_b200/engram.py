@@ -21,8 +21,10 @@ ENGRAM_F32, ENGRAM_BF16 = 0, 1
 ENGRAM_DEVICE, ENGRAM_PINNED_HOST = 0, 1
 ENGRAM_OK, ENGRAM_ERR_INVALID, ENGRAM_ERR_BOUNDS, ENGRAM_ERR_CUDA = 0, 1, 2, 3
 ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_UNSUPPORTED, ENGRAM_ERR_STATE = 4, 5, 6, 7
-MAX_ORDERS, MAX_TABLES, MAX_BRANCHES = 4, 64, 4
+MAX_ORDERS, MAX_TABLES, MAX_BRANCHES, MAX_SHARDS = 4, 64, 4, 8
+IPC_HANDLE_BYTES = 64
 ENGRAM_FLAG_NO_CTA_PAIRS = 1
+ENGRAM_PREFETCH_HOST_THREADS, ENGRAM_PREFETCH_ZERO_COPY = 0, 1
 
 #: every symbol include/engram.h declares
 EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last_error",
@@ -31,7 +33,9 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_profile_next_forward", "engram_kernel_launches",
            "engram_project_gate_noalloc", "engram_selftest_timeout", "engram_set_short_conv",
            "engram_build_hot_cache", "engram_prefetch_hot_hits", "engram_set_fp8",
-           "engram_quantize_e4m3", "engram_backward", "engram_profile_next_backward")
+           "engram_quantize_e4m3", "engram_backward", "engram_profile_next_backward",
+           "engram_set_prefetch", "engram_set_table_shards", "engram_ipc_handle",
+           "engram_ipc_open", "engram_ipc_close")
 
 
 class engram_config(ctypes.Structure):
@@ -78,6 +82,11 @@ def _load():
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
         "engram_forward": ([H, P, P, i32, i32, i32, P, P, P, P, P], ctypes.c_int),
         "engram_prefetch": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
+        "engram_set_prefetch": ([H, i32, i32], ctypes.c_int),
+        "engram_set_table_shards": ([H, i32, P], ctypes.c_int),
+        "engram_ipc_handle": ([H, P, P], ctypes.c_int),
+        "engram_ipc_open": ([H, P, P], ctypes.c_int),
+        "engram_ipc_close": ([H, P], ctypes.c_int),
         "engram_check_errors": ([H, P], ctypes.c_int),
         "engram_profile_next_forward": ([H, P, i32], ctypes.c_int),
         "engram_profile_next_backward": ([H, P, i32], ctypes.c_int),
@@ -186,6 +195,33 @@ class Engram:
         self._check(lib.engram_set_short_conv(self._h, _ptr(conv_w), _ptr(norm_w), kernel_size,
                                               dilation, _stream_ptr(stream)))
 
+    def set_table_shards(self, shards):
+        """Row-sharded tables: shards[s][j] = shard j of table s (a tensor, or a
+        device pointer as int), row z of table s at local row z // N of shard
+        z % N."""
+        N = len(shards[0])
+        flat = [x for row in shards for x in row]
+        if len(shards) != self.S or any(len(row) != N for row in shards):
+            raise EngramError(ENGRAM_ERR_INVALID, "shards must be S lists of N entries")
+        arr = (ctypes.c_void_p * len(flat))(*[_ptr(x) for x in flat])
+        self._check(lib.engram_set_table_shards(self._h, N, ctypes.cast(arr, ctypes.c_void_p)))
+        self._shards = flat  # borrowed: keep alive
+
+    def ipc_handle(self, t) -> bytes:
+        """Inter-process handle of the allocation that starts at t (64 bytes)."""
+        buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+        self._check(lib.engram_ipc_handle(self._h, _ptr(t), buf))
+        return buf.raw
+
+    def ipc_open(self, handle: bytes) -> int:
+        """Map another process's allocation; returns its device pointer here."""
+        p = ctypes.c_void_p()
+        self._check(lib.engram_ipc_open(self._h, ctypes.c_char_p(handle), ctypes.byref(p)))
+        return p.value
+
+    def ipc_close(self, ptr: int):
+        self._check(lib.engram_ipc_close(self._h, ptr))
+
     def set_fp8(self, enable: bool = True, stream=None):
         """Projections on E4M3 operands (section 2.4), or back to bf16."""
         self._check(lib.engram_set_fp8(self._h, 1 if enable else 0, _stream_ptr(stream)))
@@ -234,6 +270,14 @@ class Engram:
                                         ctypes.byref(n) if want_count else None))
         return n.value if want_count else None
 
+    def set_prefetch(self, mode: str = "host_threads", workers: int = 0):
+        """Route of the prefetch's copy from host tables: "host_threads" (host
+        threads + copy engines) or "zero_copy" (a kernel of `workers` CTAs);
+        workers = 0 takes the route's default."""
+        m = {"host_threads": ENGRAM_PREFETCH_HOST_THREADS,
+             "zero_copy": ENGRAM_PREFETCH_ZERO_COPY}[mode]
+        self._check(lib.engram_set_prefetch(self._h, m, workers))
+
     def build_hot_cache(self, tokens, max_rows: int, t_begin=0, stream=None):
         """Keep the max_rows rows the calibration tokens address most often in HBM."""
         B, T = tokens.shape
@@ -264,8 +308,27 @@ class Engram:
         return int(lib.engram_kernel_launches(self._h))
 
     def project_gate_noalloc(self, e, h, out, alpha=None, stream=None):
-        """Projection + gate from caller-supplied memory vectors; allocates nothing."""
-        self._check(lib.engram_project_gate_noalloc(self._h, _ptr(e), e.shape[0], _ptr(h),
+        """Projection + gate from caller-supplied memory vectors; allocates nothing.
+
+        e [rows, d_mem], h and out [rows, M, d] in the handle's dtype, alpha
+        fp32 [rows, M] or None; all contiguous on the handle's device.  The
+        library encodes its tensor maps from these sizes, so they are checked
+        here before the call."""
+        rows = e.shape[0] if e.dim() == 2 else -1
+        dt = torch.float32 if self.cfg.dtype == ENGRAM_F32 else torch.bfloat16
+        M, d = self.cfg.branches, self.cfg.d_hidden
+        want = [("e", e, (rows, self.d_mem), dt), ("h", h, (rows, M, d), dt),
+                ("out", out, (rows, M, d), dt)]
+        if alpha is not None:
+            want.append(("alpha", alpha, (rows, M), torch.float32))
+        for name, t, shape, dtype in want:
+            if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous() \
+                    or not t.is_cuda:
+                raise EngramError(ENGRAM_ERR_INVALID,
+                                  "project_gate_noalloc: %s must be a contiguous CUDA tensor of "
+                                  "shape %s and dtype %s (got %s %s)"
+                                  % (name, shape, dtype, tuple(t.shape), t.dtype))
+        self._check(lib.engram_project_gate_noalloc(self._h, _ptr(e), rows, _ptr(h),
                                                     _ptr(out), _ptr(alpha), _stream_ptr(stream)))
 
     def selftest_timeout(self, stream=None) -> int:

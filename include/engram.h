@@ -53,6 +53,8 @@ extern "C" {
 #define ENGRAM_MAX_ORDERS 4   /* n-gram orders per module            */
 #define ENGRAM_MAX_TABLES 64  /* orders x heads                      */
 #define ENGRAM_MAX_BRANCHES 4 /* M of the multi-branch form (Eq. 6)  */
+#define ENGRAM_MAX_SHARDS 8   /* row shards per table (engram_set_table_shards) */
+#define ENGRAM_IPC_HANDLE_BYTES 64
 
 /* element types */
 #define ENGRAM_F32 0
@@ -64,6 +66,10 @@ extern "C" {
 
 /* config flags */
 #define ENGRAM_FLAG_NO_CTA_PAIRS 1 /* bf16 projection on single-CTA tiles only */
+
+/* how engram_prefetch moves rows from host tables (engram_set_prefetch) */
+#define ENGRAM_PREFETCH_HOST_THREADS 0 /* host threads + copy engines (default) */
+#define ENGRAM_PREFETCH_ZERO_COPY 1    /* device loads through the mapped address */
 
 /* status codes */
 #define ENGRAM_OK 0
@@ -190,6 +196,41 @@ ENGRAM_API int engram_set_short_conv(engram_handle *h, const float *conv_w, cons
                                      int32_t kernel_size, int32_t dilation, void *stream);
 
 /*
+ * Row-sharded tables (section 2.5, Figure 2a: for training, the paper spreads
+ * the embedding tables over the GPUs and exchanges the active rows).  Row z
+ * of table s lives in shard z mod N at local row floor(z / N), so shard j of
+ * table s has ceil((primes[s] - j) / N) rows of d_head elements.  Every
+ * kernel that reads a table row (the forward's gather, engram_gather, the
+ * backward's recomputation) and the backward's table-gradient scatter
+ * address the owner's shard directly; with shards on other GPUs of the
+ * node (pointers from engram_ipc_open) those are peer loads and remote
+ * atomic adds over NVLink, so no request or row exchange step is needed.
+ *  shards  N in [1, ENGRAM_MAX_SHARDS].
+ *  ptrs    host array of S x N device pointers, table by table: ptrs[s N + j]
+ *          = shard j of table s, in the handle's dtype, 16-byte aligned; own
+ *          or a peer's memory.  Borrowed: must outlive the handle.
+ * Replaces the tables given to engram_set_params until the next
+ * engram_set_params.  Device-resident tables only (ENGRAM_ERR_UNSUPPORTED
+ * otherwise).  Waits for all device work first.
+ * Errors: _INVALID, _STATE (engram_set_params first), _UNSUPPORTED, _CUDA.
+ */
+ENGRAM_API int engram_set_table_shards(engram_handle *h, int32_t shards, const void *const *ptrs);
+
+/*
+ * CUDA inter-process handles for the shards of the other GPUs (plumbing of
+ * engram_set_table_shards across processes; no counterpart in the paper).
+ * engram_ipc_handle writes the ENGRAM_IPC_HANDLE_BYTES-byte handle of the
+ * device allocation that starts at `ptr` (on the handle's device) into
+ * `handle`; another process passes those bytes to engram_ipc_open, which maps
+ * the allocation into its own device's address space (peer access enabled)
+ * and returns the pointer; engram_ipc_close unmaps it.
+ * Errors: _INVALID, _CUDA.
+ */
+ENGRAM_API int engram_ipc_handle(engram_handle *h, const void *ptr, void *handle);
+ENGRAM_API int engram_ipc_open(engram_handle *h, const void *handle, void **ptr);
+ENGRAM_API int engram_ipc_close(engram_handle *h, void *ptr);
+
+/*
  * FP8 projections (section 2.4: the value projection and the M key
  * projections computed as one dense FP8 matmul).  enable = 1: every later
  * engram_forward multiplies an E4M3 form of e by an E4M3 copy of [W_K; W_V]
@@ -297,17 +338,24 @@ ENGRAM_API int engram_forward(engram_handle *h, const int32_t *tokens, const int
  *  hid     device [rows, M, d] dtype: the forward's h.
  *  dout    device [rows, M, d] dtype.
  *  dhid    device [rows, M, d] dtype: written with dL/dh.
- *  dw_k    device fp32 [M, d, d_mem] or NULL, accumulated (+=).
- *  dw_v    device fp32 [d, d_mem] or NULL, accumulated.
+ *  dw_k    device fp32 [M, d, d_mem] or NULL, accumulated (+=); the sum over
+ *          rows is split into parts added in an order that varies between
+ *          runs (last-bit differences).
+ *  dw_v    device fp32 [d, d_mem] or NULL, accumulated the same way.
  *  dnorm_q, dnorm_k  device fp32 [M, d] or NULL, accumulated.
  *  dtables host array of S device pointers to fp32 [primes[s], d_head]
  *          table gradients, accumulated (atomic adds: the order of additions
- *          into one row varies between runs); or NULL.
+ *          into one row varies between runs); or NULL.  With row-sharded
+ *          tables (engram_set_table_shards) it holds S x N pointers, table
+ *          by table, shard j of table s's gradient having the rows of its
+ *          table shard; row z's gradient is added into its owner's shard
+ *          (a peer's memory when the shard lives on another GPU).
  * Device-resident tables, d <= 4096; not with the FP8 projections or the
  * short convolution on (ENGRAM_ERR_UNSUPPORTED).  Scratch per row: S int64,
  * (M + 1) d (4 + element size) bytes and 4 d_mem bytes, plus the forward's.
- * The dense contractions run through cuBLAS on `stream`.  The first call
- * creates the handle's cuBLAS context and its scratch (engram_reserve does
+ * The dense contractions run on the library's own kernels on `stream`
+ * (tcgen05 tensor-core tiles for bf16, FFMA tiles for fp32).  The first call
+ * creates its scratch (engram_reserve does
  * not cover the backward's): make it outside any stream capture.
  * Errors: _INVALID, _STATE, _UNSUPPORTED, _OOM, _CUDA.
  */
@@ -321,15 +369,43 @@ ENGRAM_API int engram_backward(engram_handle *h, const int32_t *tokens, const in
  * Deterministic prefetch for host-resident tables (section 2.5, Figure 2b):
  * hash the tokens of an upcoming step, de-duplicate the addressed rows per
  * table, and copy each distinct row once from pinned host memory over PCIe
- * into a device staging buffer, all on `side_stream`.  The next
- * engram_forward with the same tokens reads the staged rows; its stream waits
- * for this prefetch through an event, so the copy overlaps whatever runs on
- * other streams meanwhile.  ENGRAM_PINNED_HOST handles only.
+ * into a device staging buffer.  The hashing and de-duplication run on
+ * `side_stream`; the copy follows the route engram_set_prefetch chose (by
+ * default host threads and the copy engines, no SM involved).  The call
+ * returns without waiting for the copy.  The next engram_forward with the
+ * same tokens reads the staged rows; its stream waits for this prefetch
+ * through an event (with the host-thread route, engram_forward first waits
+ * on the host until the copies have been enqueued), so the transfer overlaps
+ * whatever runs on other streams meanwhile.  At most two prefetches may be
+ * pending (staging is double-buffered).  ENGRAM_PINNED_HOST handles only.
  * *unique_rows (host, may be NULL) receives the number of distinct rows once
- * the prefetch has completed (this synchronises side_stream when non-NULL).
+ * the de-duplication has completed (this synchronises side_stream when
+ * non-NULL).  Pinned host memory of the host-thread route: 2 x (16 + 8 +
+ * d_head x element size) bytes per (row, table) of the largest batch.
+ * Errors: _INVALID, _STATE (engram_set_params first; more than two pending),
+ * _OOM, _CUDA.
  */
 ENGRAM_API int engram_prefetch(engram_handle *h, const int32_t *tokens, int32_t B, int32_t T,
                     int32_t t_begin, void *side_stream, int64_t *unique_rows);
+
+/*
+ * The route of engram_prefetch's copy from the host tables (section 2.5: the
+ * paper fetches the rows asynchronously over PCIe while earlier blocks
+ * compute, but does not say how).
+ *  mode  ENGRAM_PREFETCH_HOST_THREADS: `workers` host threads (0: up to 8,
+ *        half the host's hardware threads) read the distinct rows into a
+ *        pinned bounce buffer and the copy engines send it to the device in
+ *        chunks of about 1 MB; no SM takes part, so the transfer runs beside
+ *        any compute.  Random 160-byte reads from host DRAM set its rate.
+ *        ENGRAM_PREFETCH_ZERO_COPY: a kernel of `workers` CTAs (0: one per SM)
+ *        on side_stream loads the rows through the tables' mapped device
+ *        address, 16 bytes per load; those CTAs occupy SMs for the whole
+ *        transfer.
+ * Both routes stage the same bytes, so results do not depend on the mode.
+ * No prefetch may be pending (ENGRAM_ERR_STATE).  ENGRAM_PINNED_HOST handles
+ * only.  Errors: _INVALID, _STATE.
+ */
+ENGRAM_API int engram_set_prefetch(engram_handle *h, int32_t mode, int32_t workers);
 
 /*
  * Hot-row cache for host-resident tables (section 2.5: the accesses follow

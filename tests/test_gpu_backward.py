@@ -144,6 +144,26 @@ def test_prefill_full_size_sampled():
         assert torch.isfinite(g[k]).all() and g[k].abs().max() > 0
 
 
+def test_prefill_full_size_sampled_rows_every_gradient():
+    """The benchmarked workload and launch configuration (32 768 rows) with
+    dL/dout zero outside a sample of rows: a row whose dout is zero has zero
+    dk and dv (dv sums alpha dout over the branches, and d alpha = dout . v),
+    so the weight, RMSNorm-weight and table gradients of the whole call equal
+    the oracle's backward over the sampled rows alone, and dh is zero on every
+    other row."""
+    p = Problem(synth.SHAPES["prefill_bf16"])
+    m = p.engram()
+    rows = p.sample_rows(40, seed=5)
+    mask = torch.zeros((p.shape.rows_out, 1, 1), device="cuda", dtype=torch.bfloat16)
+    mask[torch.from_numpy(rows).cuda()] = 1
+    dout = synth.make_grad_out(p.shape, p.seeds, device="cuda") * mask
+    dh, g = run_backward(p, m, dout)
+    check_all(p, dh, g, dout, rows=rows)
+    others = torch.ones(p.shape.rows_out, dtype=torch.bool, device="cuda")
+    others[torch.from_numpy(rows).cuda()] = False
+    assert (dh[others] == 0).all()
+
+
 def test_unsupported_modes():
     from hashed_gram_embedding_compress_b200 import engram as eg
     p = Problem(REDUCED.replace(T=40))

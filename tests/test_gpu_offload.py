@@ -1,9 +1,11 @@
 """Host-resident tables: deterministic prefetch over PCIe (section 2.5, Fig. 2b).
 
 The prefetch hashes the tokens ahead, de-duplicates the addressed rows, copies
-each distinct row once from pinned host memory into an HBM staging buffer on a
-side stream, and the forward gathers from there.  Its results must equal the
-device-resident path bit for bit (same rows, same kernels after the gather).
+each distinct row once from pinned host memory into an HBM staging buffer
+(host threads + copy engines, or zero-copy loads on a few CTAs), and the
+forward gathers from there.  Its results must equal the device-resident path
+bit for bit (same rows, same kernels after the gather), whichever route moved
+the rows.
 """
 import numpy as np
 import pytest
@@ -21,12 +23,17 @@ def _pair(shape):
     return host, dev_tables
 
 
-def test_prefetch_then_forward_equals_device_tables():
+ROUTES = [("host_threads", 0), ("host_threads", 1), ("zero_copy", 16), ("zero_copy", 0)]
+
+
+@pytest.mark.parametrize("route", ROUTES)
+def test_prefetch_then_forward_equals_device_tables(route):
     from hashed_gram_embedding_compress_b200 import engram as eg
     sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=1500, rows_target=1 << 18)
     p, dev_tables = _pair(sh)
     assert p.tables[0].is_pinned()
     m = p.engram()
+    m.set_prefetch(*route)
     # reference: the same inputs with device-resident tables
     md = eg.Engram(eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=p.comp_map,
                                   orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
@@ -56,11 +63,13 @@ def test_prefetch_then_forward_equals_device_tables():
     assert out_close(to_oracle(out[rs]), o_o, "bf16") <= 1e-3
 
 
-def test_double_buffered_prefetch_and_call_order():
+@pytest.mark.parametrize("route", ROUTES[::2])
+def test_double_buffered_prefetch_and_call_order(route):
     from hashed_gram_embedding_compress_b200 import engram as eg
     sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=300, rows_target=1 << 16, d_hidden=256)
     p, dev_tables = _pair(sh)
     m = p.engram()
+    m.set_prefetch(*route)
     tok_a = p.tokens.cuda()
     tok_b = torch.flip(p.tokens, dims=[1]).contiguous().cuda()
     with pytest.raises(eg.EngramError) as ei:
@@ -99,14 +108,16 @@ def _expected_hits(p, calib_z, step_z, max_rows):
     return sum(1 for k in step.tolist() if k in hot)
 
 
-@pytest.mark.parametrize("max_rows", [1000, 10 ** 7])
-def test_hot_row_cache_serves_rows_and_keeps_results(max_rows):
+@pytest.mark.parametrize("max_rows,route", [(1000, ROUTES[0]), (10 ** 7, ROUTES[0]),
+                                            (1000, ROUTES[2])])
+def test_hot_row_cache_serves_rows_and_keeps_results(max_rows, route):
     from hashed_gram_embedding_compress_b200 import engram as eg
     import oracle
     sh = synth.SHAPES["prefill_bf16"].replace(B=2, T=1200, rows_target=1 << 17, d_hidden=256)
     p, _ = _pair(sh)
     m0 = p.engram()
     m1 = p.engram()
+    m1.set_prefetch(*route)
     side = torch.cuda.Stream()
     # calibrate on other tokens of the same distribution (the step's own
     # indices would overstate the hits)
@@ -136,3 +147,79 @@ def test_hot_row_cache_needs_host_tables():
     with pytest.raises(eg.EngramError) as ei:
         m.build_hot_cache(p.tokens.cuda(), 10)
     assert ei.value.code == eg.ENGRAM_ERR_STATE
+
+
+def test_set_prefetch_rejects_bad_modes_and_pending_prefetches():
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["prefill_bf16"].replace(B=1, T=64, rows_target=1031, d_hidden=256)
+    p, _ = _pair(sh)
+    m = p.engram()
+    with pytest.raises(eg.EngramError) as ei:
+        m._check(eg.lib.engram_set_prefetch(m._h, 7, 0))
+    assert ei.value.code == eg.ENGRAM_ERR_INVALID
+    side = torch.cuda.Stream()
+    tok = p.tokens.cuda()
+    m.prefetch(tok, stream=side)
+    with pytest.raises(eg.EngramError) as ei:
+        m.set_prefetch("zero_copy")
+    assert ei.value.code == eg.ENGRAM_ERR_STATE
+    m.forward(tok, p.h, torch.empty_like(p.h))
+    m.set_prefetch("zero_copy")
+    d = Problem(synth.SHAPES["tiny_f32"]).engram()
+    with pytest.raises(eg.EngramError) as ei:
+        d.set_prefetch("host_threads")
+    assert ei.value.code == eg.ENGRAM_ERR_STATE
+
+
+def test_offload_workload_shapes_against_the_oracle():
+    """The host-offloaded workload's own shapes: B = 4 x T = 8192 tokens,
+    vocab 128000 -> 98560, 16 host tables of 160-byte rows (primes >= 2^21
+    here, 5.4 GB pinned, instead of the benchmark's 100 GB), M = 4 branches of
+    d = 4096.  Two steps run the benchmark's pipeline (the next step's
+    prefetch issued before the current forward) with the host-thread route;
+    every index is checked against the oracle's distinct-row count, alpha and
+    out against the oracle on sampled rows, and the zero-copy route must give
+    the same bytes."""
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["offload"].replace(rows_target=1 << 21)
+    p = Problem(sh)
+    assert p.tables[0].is_pinned() and sh.branches == 4 and sh.d_hidden == 4096
+    tok = [p.tokens.cuda(), torch.flip(p.tokens, dims=[1]).contiguous().cuda()]
+    side = torch.cuda.Stream()
+    outs = {}
+    for route in (("host_threads", 0), ("zero_copy", 0)):
+        m = p.engram()
+        m.set_prefetch(*route)
+        m.reserve(sh.rows_out)
+        n0 = m.prefetch(tok[0], stream=side, want_count=True)
+        want = sum(len(np.unique(p.z[:, s])) for s in range(sh.num_tables))
+        assert n0 == want
+        res = []
+        for k in range(2):
+            if k + 1 < len(tok):
+                m.prefetch(tok[k + 1], stream=side)  # next step's rows, overlapped
+            out = torch.empty_like(p.h)
+            alpha = torch.empty((sh.rows_out, sh.branches), device="cuda")
+            m.forward(tok[k], p.h, out, alpha=alpha)
+            res.append((out, alpha))
+        torch.cuda.synchronize()
+        assert m.check_errors() == 0
+        outs[route[0]] = res
+    for (o1, a1), (o2, a2) in zip(outs["host_threads"], outs["zero_copy"]):
+        assert torch.equal(o1, o2) and torch.equal(a1, a2)
+    out, alpha = outs["host_threads"][0]
+    rows = p.sample_rows(24)
+    _, a_o, _, o_o = p.oracle_forward(rows)
+    rs = torch.from_numpy(rows).cuda()
+    assert rel_l2(alpha[rs].double().cpu(), a_o) <= 1e-3
+    assert out_close(to_oracle(out[rs]), o_o, "bf16") <= 1e-3
+    # the second step (reversed sequences) against a device-table forward of the same tokens
+    md = eg.Engram(eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=p.comp_map,
+                                  orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
+                                  d_hidden=sh.d_hidden, branches=sh.branches, dtype=sh.dtype,
+                                  table_rows_target=sh.rows_target, hash_seed=p.hash_seed))
+    md.set_params([t.cuda() for t in p.tables], p.w_k, p.w_v, p.norm_q, p.norm_k)
+    ref = torch.empty_like(p.h)
+    md.forward(tok[1], p.h, ref)
+    torch.cuda.synchronize()
+    assert torch.equal(outs["host_threads"][1][0], ref)
