@@ -78,6 +78,9 @@ def parse():
     ap.add_argument("--hot-rows", type=int, default=0,
                     help="offload workload: rows of the HBM hot-row cache in front of the host "
                          "tables, chosen from 4 calibration batches of other tokens (0: none)")
+    ap.add_argument("--load-seconds", type=float, default=1.5,
+                    help="back-to-back steps before the timed ones, so that the clock sampler "
+                         "sees the loaded state (0 for profiling captures)")
     ap.add_argument("--rows-target", type=int, default=None,
                     help="smaller tables for profiling captures (same kernel shapes); "
                          "not the benchmarked workload")
@@ -328,7 +331,7 @@ def run_ours(args, rank, world, dist):
     # keep the GPU under the same back-to-back load for >= 1.5 s before the
     # timed steps, so that the clock sampler sees the loaded state
     t_load = time.monotonic()
-    while time.monotonic() - t_load < 1.5:
+    while time.monotonic() - t_load < args.load_seconds:
         for _ in range(50):
             step()
         torch.cuda.synchronize()
@@ -343,21 +346,28 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    # the timed steps carry no stage events: an event between two launches
+    # would serialise the launches that otherwise overlap (the key launch
+    # starts during the gather, the value launch during the key launch)
     t0.record(stream)
     for k in range(K):
-        if graph is None:
-            m.profile_next_forward(evs[k])
         step()
     t1.record(stream)
     torch.cuda.synchronize()
     t_end = time.monotonic()
+    launches = m.kernel_launches() - launches0
+    if graph is not None:
+        launches = per_replay * K  # replays do not pass through the library's counter
+    # stage times: the same steps again, each with events between its launches
+    if graph is None:
+        for k in range(K):
+            m.profile_next_forward(evs[k])
+            step()
+        torch.cuda.synchronize()
     time.sleep(0.3)
     clk.__exit__(None, None, None)
     if dist:
         dist.barrier()
-    launches = m.kernel_launches() - launches0
-    if graph is not None:
-        launches = per_replay * K  # replays do not pass through the library's counter
     ms = max_over_ranks(t0.elapsed_time(t1), dist, device)
     if graph is None:
         stage = [[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(NEV - 1)] for k in range(K)]
@@ -484,6 +494,8 @@ def run_ours(args, rank, world, dist):
         "gpu_launches": launches,
         "clocks": dict(clk.summary(t_load + 0.5, t_end + 0.15),
                        window="last 1 s of back-to-back warm-up steps and the timed steps"),
+        "stages_note": "stage times from a second pass of the same steps with events between "
+                       "the launches (which serialises them); ms_per_step has no events",
     }
     if args.short_conv:
         res["config"]["workload"] += (" + ShortConv (Eq. 5: W=4, dilation %d, RMSNorm, SiLU, "
@@ -549,7 +561,7 @@ def run_backward_bench(args, rank, world, dist):
     if m.check_errors(stream) != 0:
         raise RuntimeError("device error during warm-up")
     t_load = time.monotonic()
-    while time.monotonic() - t_load < 1.5:
+    while time.monotonic() - t_load < args.load_seconds:
         for _ in range(5):
             step()
         torch.cuda.synchronize()
@@ -733,22 +745,21 @@ def run_offload(args):
         def measure(route):
             """One route of the prefetch's copy: alone, then pipelined."""
             m.set_prefetch(*route)
-            # the prefetch alone: issue to staged rows ready (host clock around
-            # prefetch + forward, less the forward's own event time)
+            # the prefetch alone (host clock from the call until its rows are
+            # staged), then the forward from the staged rows (CUDA events)
             uniq, t_pf, t_fw, hits = [], [], [], []
             for k in range(K):
                 torch.cuda.synchronize()
                 w0 = time.perf_counter()
-                f0, f1 = ev(), ev()
                 m.prefetch(toks[k], stream=side)
+                m.prefetch_wait()
+                t_pf.append((time.perf_counter() - w0) * 1e3)
+                f0, f1 = ev(), ev()
                 f0.record(main)
-                m.forward(toks[k], h, h, stream=main)  # waits for the staged rows
+                m.forward(toks[k], h, h, stream=main)
                 f1.record(main)
                 torch.cuda.synchronize()
-                w1 = time.perf_counter()
-                fw = f0.elapsed_time(f1)
-                t_fw.append(fw)
-                t_pf.append((w1 - w0) * 1e3 - fw)
+                t_fw.append(f0.elapsed_time(f1))
             for k in range(3):
                 uniq.append(m.prefetch(toks[k], stream=side, want_count=True))
                 hits.append(m.prefetch_hot_hits())

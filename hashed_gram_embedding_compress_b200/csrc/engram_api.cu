@@ -107,6 +107,29 @@ int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, i
   return ENGRAM_OK;
 }
 
+int cached_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
+               int box_rows, int box_cols, int esz) {
+  for (const auto& e : h->map_cache) {
+    if (e.base == base && e.cols == cols && e.rows == rows && e.box_rows == box_rows &&
+        e.box_cols == box_cols && e.esz == esz) {
+      *m = e.map;
+      return ENGRAM_OK;
+    }
+  }
+  const int rc = make_map(h, m, base, cols, rows, box_rows, box_cols, esz);
+  if (rc) return rc;
+  auto& e = h->map_cache[h->map_cache_next];
+  h->map_cache_next = (h->map_cache_next + 1) % engram_handle::kMapCache;
+  e.base = base;
+  e.cols = cols;
+  e.rows = rows;
+  e.box_rows = box_rows;
+  e.box_cols = box_cols;
+  e.esz = esz;
+  e.map = *m;
+  return ENGRAM_OK;
+}
+
 }  // namespace engram
 
 namespace {
@@ -820,6 +843,19 @@ int engram_set_prefetch(engram_handle* h, int32_t mode, int32_t workers) {
   return ENGRAM_OK;
 }
 
+int engram_prefetch_wait(engram_handle* h) {
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (h->n_prefetch == h->n_consumed) return fail(h, ENGRAM_ERR_STATE, "no prefetch is pending");
+  const int slot = (int)(h->n_consumed & 1);
+  if (h->hg) {
+    std::string msg;
+    const cudaError_t ge = h->hg->wait_issued(slot, &msg);
+    if (ge != cudaSuccess) return fail(h, ENGRAM_ERR_CUDA, "prefetch: " + msg);
+  }
+  CK(h, cudaEventSynchronize(h->ev_ready[slot]));
+  return ENGRAM_OK;
+}
+
 int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T, int32_t t_begin,
                     void* side_stream, int64_t* unique_rows) {
   if (!h) return ENGRAM_ERR_INVALID;
@@ -1029,6 +1065,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   g.d_mem = h->d_mem;
   g.eps = h->cfg.eps;
   g.inv_sqrt_d = (float)(1.0 / std::sqrt((double)h->cfg.d_hidden));
+  // the key launch overlaps the gather's tail and the value launch the key's
+  g.pdl = 1;
   if (conv) {
     g.vals = h->conv_v;
     g.vv = h->conv_vv;
@@ -1089,46 +1127,46 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     const int kphase = phase == 0 ? 0 : conv ? 3 : out == hid ? 2 : 1;
     if (pc.kind == ProjKernel::Pair) {
       if (!have_pair) {
-        if ((rc = make_map(h, &pair.e, h->e, h->d_mem, R, 128))) return rc;
-        if ((rc = make_map(h, &pair.h, hid, hcols, R, 128, 32))) return rc;
-        if ((rc = make_map(h, &pair.out, out, hcols, R, 32, 32))) return rc;  // per-warp boxes
+        if ((rc = cached_map(h, &pair.e, h->e, h->d_mem, R, 128))) return rc;
+        if ((rc = cached_map(h, &pair.h, hid, hcols, R, 128, 32))) return rc;
+        if ((rc = cached_map(h, &pair.out, out, hcols, R, 32, 32))) return rc;  // per-warp boxes
         have_pair = true;
       }
       pair.w = wmaps[bn_index(pc.bn)];  // each CTA of a pair loads 128 of the tile's 256 W rows
       ProjMaps pm = pair;
       // in place: per-warp reduce-adds of 32 rows x 64 columns
-      if (kphase == 2 && (rc = make_map(h, &pm.out, out, hcols, R, 32, 64))) return rc;
+      if (kphase == 2 && (rc = cached_map(h, &pm.out, out, hcols, R, 32, 64))) return rc;
       CK(h, launch_proj_gate_pair(kphase, pm, g, pc.grid, st));
     } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if (fp8) {
-          if ((rc = make_map(h, &wide.e, h->e8, h->d_mem, R, 256, 128, 1))) return rc;
-        } else if ((rc = make_map(h, &wide.e, h->e, h->d_mem, R, 256))) {
+          if ((rc = cached_map(h, &wide.e, h->e8, h->d_mem, R, 256, 128, 1))) return rc;
+        } else if ((rc = cached_map(h, &wide.e, h->e, h->d_mem, R, 256))) {
           return rc;
         }
-        if ((rc = make_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
-        if ((rc = make_map(h, &wide.out, out, hcols, R, 32, 32))) return rc;
+        if ((rc = cached_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
+        if ((rc = cached_map(h, &wide.out, out, hcols, R, 32, 32))) return rc;
         have_wide = true;
       }
       wide.w = fp8 ? (phase == 0 ? h->map_wk8 : h->map_wv8) : wmaps[bn_index(pc.bn)];
       if (kphase == 2) {
         // in place: per-warp reduce-adds of 32 rows x 64 columns
         ProjMaps wr = wide;
-        if ((rc = make_map(h, &wr.out, out, hcols, R, 32, 64))) return rc;
+        if ((rc = cached_map(h, &wr.out, out, hcols, R, 32, 64))) return rc;
         CK(h, launch_proj_gate_wide(kphase, wr, g, pc.grid, st, fp8));
       } else if (kphase == 3) {
         // v leaves through per-warp TMA stores of 32 x 32 fp32 boxes
         ProjMaps wv = wide;
-        if ((rc = make_map(h, &wv.out, h->conv_v, g.d, R, 32, 32, 4))) return rc;
+        if ((rc = cached_map(h, &wv.out, h->conv_v, g.d, R, 32, 32, 4))) return rc;
         CK(h, launch_proj_gate_wide(kphase, wv, g, pc.grid, st, fp8));
       } else {
         CK(h, launch_proj_gate_wide(kphase, wide, g, pc.grid, st, fp8));
       }
     } else {
       if (!have_single) {
-        if ((rc = make_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;
-        if ((rc = make_map(h, &single.h, hid, hcols, R, 128))) return rc;
-        if ((rc = make_map(h, &single.out, out, hcols, R, 128))) return rc;
+        if ((rc = cached_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;
+        if ((rc = cached_map(h, &single.h, hid, hcols, R, 128))) return rc;
+        if ((rc = cached_map(h, &single.out, out, hcols, R, 128))) return rc;
         have_single = true;
       }
       single.w = wmaps[bn_index(pc.bn)];
@@ -1251,7 +1289,8 @@ int engram_backward(engram_handle* h, const int32_t* tokens, const int64_t* idx,
   if (!idx && !tokens) return fail(h, ENGRAM_ERR_INVALID, "need tokens or idx");
   if (dtables)
     for (int s = 0; s < S * h->shards; ++s)
-      if (!dtables[s]) return fail(h, ENGRAM_ERR_INVALID, "null table-gradient pointer");
+      if (!dtables[s] || !aligned16(dtables[s]))
+        return fail(h, ENGRAM_ERR_INVALID, "table-gradient pointers must be non-null and 16-byte aligned");
   cudaStream_t st = (cudaStream_t)stream;
   const int grid = gate_bw_grid(M, d, R, h->elt);
   if ((rc = ensure_scratch(h, R))) return rc;

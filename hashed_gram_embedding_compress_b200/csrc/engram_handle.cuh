@@ -105,6 +105,18 @@ struct engram_handle {
   float* bw_partials = nullptr;    // [bw_part_blocks][2][M][d]
   int bw_part_blocks = 0;
 
+  // tensor maps of the per-call operands (e, h, out), keyed by their
+  // arguments: a repeated call shape encodes nothing on the host
+  struct MapEntry {
+    const void* base = nullptr;
+    int64_t cols = 0, rows = 0;
+    int box_rows = 0, box_cols = 0, esz = 0;
+    CUtensorMap map;
+  };
+  static constexpr int kMapCache = 32;
+  MapEntry map_cache[kMapCache];
+  int map_cache_next = 0;
+
   // instrumentation
   int64_t launches = 0;
   cudaEvent_t prof[6] = {};
@@ -122,6 +134,9 @@ namespace engram {
 // failure the message goes to h->last_error.
 int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
              int box_rows, int box_cols = 64, int esz = 2);
+// make_map through the handle's cache of recently encoded maps.
+int cached_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
+               int box_rows, int box_cols = 64, int esz = 2);
 
 // Index into the handle's W tensor maps (map_wk, map_wv) of a box width.
 inline int bn_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }

@@ -20,6 +20,20 @@ constexpr int kMaxOrders = 4;
 constexpr int kMaxBranches = 4;
 constexpr int kMaxShards = 8;  // row shards per table (engram_set_table_shards)
 
+#ifdef __CUDACC__
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel on the
+// stream runs; griddep_wait() blocks until that kernel has completed and its
+// memory is visible, griddep_launch_dependents() lets the next such kernel
+// start.  Both are no-ops in a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
+
 // Everything the compress+hash kernel needs (section 2.2, Eq. 1).
 struct HashArgs {
   const int32_t* tokens;   // [B, T] raw ids
@@ -77,6 +91,11 @@ struct GateArgs {
   int32_t key_tile;     // width of the key-phase tiles that wrote `partials`
   float eps;
   float inv_sqrt_d;
+  // 1: launch with programmatic dependent launch.  The key phase then waits
+  // for the previous kernel (the gather) before reading e and lets the value
+  // phase start early; the value phase's epilogue waits for the key phase
+  // before it reads the partial sums or writes out.
+  int32_t pdl;
 };
 
 // Short convolution and residual (Eq. 5) over B sequences of T positions.

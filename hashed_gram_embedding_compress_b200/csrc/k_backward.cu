@@ -339,15 +339,19 @@ __global__ void dnorm_reduce_kernel(const float* partials, int nblocks, int64_t 
   }
 }
 
-// dtab[s][idx[r][s]][c] += de[r][s d_h + c]: one thread per element of de.
+// dtab[s][idx[r][s]][c..c+3] += de[r][s d_h + c..c+3]: one thread per four
+// elements of de, added by one 16-byte vector reduction in L2 (d_head is a
+// multiple of 4 and the gradient rows 16-byte aligned).
 __global__ void table_grad_kernel(TableGradArgs a) {
-  const int64_t per_row = (int64_t)a.S * a.d_head;
+  const int32_t q_per_row = a.d_head >> 2;  // float4 per table row
+  const int64_t per_row = (int64_t)a.S * q_per_row;
   const int64_t total = a.rows * per_row;
+  const float4* de4 = reinterpret_cast<const float4*>(a.de);
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / per_row;
     const int32_t rem = (int32_t)(i - r * per_row);
-    const int32_t s = rem / a.d_head, c = rem - s * a.d_head;
+    const int32_t s = rem / q_per_row, c = (rem - s * q_per_row) * 4;
     const int64_t z = a.idx[r * a.S + s];
     if (z < 0 || z >= a.primes[s]) {
       if (c == 0) atomicOr(a.err, kDevErrIndex);
@@ -362,7 +366,10 @@ __global__ void table_grad_kernel(TableGradArgs a) {
       dst = a.dtables[s * a.shards + (int)((uint32_t)z - q * (uint32_t)a.shards)] +
             (int64_t)q * a.d_head;
     }
-    atomicAdd(dst + c, a.de[i]);
+    const float4 v = __ldg(de4 + i);
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
   }
 }
 
@@ -484,7 +491,8 @@ cudaError_t launch_dnorm_reduce(const float* partials, int nblocks, int64_t n, f
 }
 
 cudaError_t launch_table_grad(const TableGradArgs& a, cudaStream_t stream) {
-  const int64_t total = a.rows * a.S * a.d_head;
+  if (a.d_head % 4) return cudaErrorInvalidValue;
+  const int64_t total = a.rows * a.S * (a.d_head / 4);
   if (total == 0) return cudaSuccess;
   table_grad_kernel<<<grid_cap(total, 256), 256, 0, stream>>>(a);
   return cudaGetLastError();

@@ -113,6 +113,7 @@ __device__ __forceinline__ const char* row_addr(const char* const* tab, int s, u
 }
 
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
+  griddep_launch_dependents();  // the key phase may set up while this runs
   __shared__ const char* s_tab[kMaxTables * kMaxShards];
   __shared__ int64_t s_prime[kMaxTables];
   for (int i = threadIdx.x; i < a.S * a.shards; i += blockDim.x) s_tab[i] = (const char*)a.tables[i];
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(GatherArgs a) {
 constexpr int kFusedThreads = 256;
 
 __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherArgs g) {
+  griddep_launch_dependents();  // the key phase may set up while this runs
   const HashArgs& a = g.hash;
   __shared__ uint64_t s_mult[kMaxTables * kMaxOrders];
   __shared__ uint64_t s_prime[kMaxTables];
@@ -211,6 +213,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
 // flight together), reduces the row's largest magnitude over the warp and
 // writes the row's codes (half the bytes of e) and its scale.
 __global__ void __launch_bounds__(kFusedThreads) hash_gather_e4m3_kernel(HashGatherArgs g) {
+  griddep_launch_dependents();  // the key phase may set up while this runs
   const HashArgs& a = g.hash;
   __shared__ uint64_t s_mult[kMaxTables * kMaxOrders];
   __shared__ uint64_t s_prime[kMaxTables];

@@ -150,6 +150,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // the partner's barriers are initialised before any signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (PHASE == 0) {
+    // e (and its scales) come from the previous kernel; once it is complete
+    // the value phase may launch
+    griddep_wait();
+    griddep_launch_dependents();
+  }
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------- e / W producer
@@ -299,6 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // the key phase's partial sums are complete (and h no longer read by it)
+    if (PHASE >= 1) griddep_wait();
     const int quarter = warp & 3, colhalf = warp >> 2;
     const int r = quarter * 32 + lane;  // tile row of this thread (within the CTA)
     uint32_t hpos = 0;                  // ring position of the tile's first entry
@@ -601,13 +609,15 @@ cudaError_t launch_pair(const ProjMaps& maps, const GateArgs& g, int grid, cudaS
   lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = SMEM;
   lc.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = at;
-  lc.numAttrs = 1;
+  lc.numAttrs = g.pdl ? 2 : 1;
   e = cudaLaunchKernelEx(&lc, kern, maps.e, maps.w, maps.h, maps.out, g);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

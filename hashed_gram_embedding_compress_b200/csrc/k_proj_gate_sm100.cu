@@ -131,6 +131,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (PHASE == 0) {
+    // e (and its scales) come from the previous kernel; once it is complete
+    // the value phase may launch
+    griddep_wait();
+    griddep_launch_dependents();
+  }
 
   if (warp == 4) {
     // ------------------------------------------------- e / W producer (TMA)
@@ -241,6 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // the key phase's partial sums are complete (and h no longer read by it)
+    if (PHASE >= 1) griddep_wait();
     // Thread (warp w, lane l) owns tile row r = 32w + l: TMEM lane r and
     // row r of every h sub-tile in shared memory.
     const int r = warp * 32 + lane;
@@ -428,7 +436,18 @@ cudaError_t launch_bn(const ProjMaps& maps, const GateArgs& g, int grid, cudaStr
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg<BN>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, Cfg<BN>::SMEM, stream>>>(maps.e, maps.w, maps.h, maps.out, g);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = Cfg<BN>::SMEM;
+  lc.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = g.pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&lc, kern, maps.e, maps.w, maps.h, maps.out, g);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

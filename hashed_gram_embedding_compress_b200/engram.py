@@ -35,7 +35,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_build_hot_cache", "engram_prefetch_hot_hits", "engram_set_fp8",
            "engram_quantize_e4m3", "engram_backward", "engram_profile_next_backward",
            "engram_set_prefetch", "engram_set_table_shards", "engram_ipc_handle",
-           "engram_ipc_open", "engram_ipc_close")
+           "engram_ipc_open", "engram_ipc_close", "engram_prefetch_wait")
 
 
 class engram_config(ctypes.Structure):
@@ -83,6 +83,7 @@ def _load():
         "engram_forward": ([H, P, P, i32, i32, i32, P, P, P, P, P], ctypes.c_int),
         "engram_prefetch": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_set_prefetch": ([H, i32, i32], ctypes.c_int),
+        "engram_prefetch_wait": ([H], ctypes.c_int),
         "engram_set_table_shards": ([H, i32, P], ctypes.c_int),
         "engram_ipc_handle": ([H, P, P], ctypes.c_int),
         "engram_ipc_open": ([H, P, P], ctypes.c_int),
@@ -257,7 +258,8 @@ class Engram:
         B, T = tokens.shape
         arr = None
         if dtables is not None:
-            arr = ctypes.cast((ctypes.c_void_p * self.S)(*[t.data_ptr() for t in dtables]),
+            # S pointers, or S x N with row-sharded tables
+            arr = ctypes.cast((ctypes.c_void_p * len(dtables))(*[t.data_ptr() for t in dtables]),
                               ctypes.c_void_p)
         self._check(lib.engram_backward(self._h, _ptr(tokens), _ptr(idx), B, T, t_begin, _ptr(h),
                                         _ptr(dout), _ptr(dh), _ptr(dw_k), _ptr(dw_v),
@@ -269,6 +271,10 @@ class Engram:
         self._check(lib.engram_prefetch(self._h, _ptr(tokens), B, T, t_begin, _stream_ptr(stream),
                                         ctypes.byref(n) if want_count else None))
         return n.value if want_count else None
+
+    def prefetch_wait(self):
+        """Block until the oldest pending prefetch's rows are in device memory."""
+        self._check(lib.engram_prefetch_wait(self._h))
 
     def set_prefetch(self, mode: str = "host_threads", workers: int = 0):
         """Route of the prefetch's copy from host tables: "host_threads" (host

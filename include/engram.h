@@ -343,8 +343,9 @@ ENGRAM_API int engram_forward(engram_handle *h, const int32_t *tokens, const int
  *          runs (last-bit differences).
  *  dw_v    device fp32 [d, d_mem] or NULL, accumulated the same way.
  *  dnorm_q, dnorm_k  device fp32 [M, d] or NULL, accumulated.
- *  dtables host array of S device pointers to fp32 [primes[s], d_head]
- *          table gradients, accumulated (atomic adds: the order of additions
+ *  dtables host array of S device pointers (16-byte aligned) to fp32
+ *          [primes[s], d_head] table gradients, accumulated (atomic adds: the
+ *          order of additions
  *          into one row varies between runs); or NULL.  With row-sharded
  *          tables (engram_set_table_shards) it holds S x N pointers, table
  *          by table, shard j of table s's gradient having the rows of its
@@ -387,6 +388,15 @@ ENGRAM_API int engram_backward(engram_handle *h, const int32_t *tokens, const in
  */
 ENGRAM_API int engram_prefetch(engram_handle *h, const int32_t *tokens, int32_t B, int32_t T,
                     int32_t t_begin, void *side_stream, int64_t *unique_rows);
+
+/*
+ * Block the calling host thread until the rows of the oldest pending
+ * prefetch (the one the next engram_forward reads) are in device memory.
+ * Not needed for correctness (engram_forward orders itself after the
+ * prefetch); for callers that time or schedule the transfer.
+ * Errors: _STATE (no prefetch pending), _CUDA.
+ */
+ENGRAM_API int engram_prefetch_wait(engram_handle *h);
 
 /*
  * The route of engram_prefetch's copy from the host tables (section 2.5: the

@@ -159,10 +159,14 @@ def test_set_prefetch_rejects_bad_modes_and_pending_prefetches():
     assert ei.value.code == eg.ENGRAM_ERR_INVALID
     side = torch.cuda.Stream()
     tok = p.tokens.cuda()
+    with pytest.raises(eg.EngramError) as ei:
+        m.prefetch_wait()  # nothing pending
+    assert ei.value.code == eg.ENGRAM_ERR_STATE
     m.prefetch(tok, stream=side)
     with pytest.raises(eg.EngramError) as ei:
         m.set_prefetch("zero_copy")
     assert ei.value.code == eg.ENGRAM_ERR_STATE
+    m.prefetch_wait()
     m.forward(tok, p.h, torch.empty_like(p.h))
     m.set_prefetch("zero_copy")
     d = Problem(synth.SHAPES["tiny_f32"]).engram()
