@@ -165,22 +165,76 @@ __host__ __device__ inline size_t ring_slot_bytes(int M, int d, int elt) {
   return (size_t)2 * M * d * elt + (size_t)(M + 1) * d * 4;
 }
 
-template <int PER>
-__global__ void __launch_bounds__(kBwThreads) gate_backward_ring_kernel(GateBwArgs a) {
+// Eight consecutive elements of a row, as fp32: bf16 (one 16-byte load) or
+// fp32 (two).
+template <bool BF16>
+__device__ __forceinline__ void load8(const void* base, int64_t i, float (&x)[8]) {
+  if (BF16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = __uint_as_float(w[j] << 16);
+      x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i);
+    const float4 u = p[0], v = p[1];
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+    x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+  }
+}
+
+__device__ __forceinline__ void load8f(const float* p, float (&x)[8]) {
+  const float4 u = reinterpret_cast<const float4*>(p)[0], v = reinterpret_cast<const float4*>(p)[1];
+  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+  x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+}
+
+__device__ __forceinline__ void ldg8f(const float* p, float (&x)[8]) {
+  const float4 u = __ldg(reinterpret_cast<const float4*>(p)),
+               v = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+  x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store8(void* base, int64_t i, const float (&x)[8]) {
+  if (BF16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = (uint32_t)bf16_rne(x[2 * j]) | ((uint32_t)bf16_rne(x[2 * j + 1]) << 16);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(base) + i) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + i);
+    p[0] = make_float4(x[0], x[1], x[2], x[3]);
+    p[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+}
+
+// One CTA per row at a time, one thread per 8 consecutive columns (blockDim
+// = d / 8 rounded up to whole warps), the row's h, dout, k and v of a branch
+// held in registers across the three passes of the branch.
+template <bool BF16>
+__global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
   extern __shared__ __align__(128) unsigned char smraw[];
   const int d = a.d, M = a.M, tid = threadIdx.x;
-  const int elt = a.bf16 ? 2 : 4;
+  const int nwarps = blockDim.x >> 5;
+  const int c0 = tid * 8;       // this thread's columns [c0, c0 + 8)
+  const bool act = c0 < d;
+  constexpr int elt = BF16 ? 2 : 4;
   const int64_t nkv = (int64_t)(M + 1) * d;
   const float inv_d = 1.f / (float)d;
   const uint32_t hb = (uint32_t)M * d * elt, kvb = (uint32_t)nkv * 4;
   const size_t slot_bytes = ring_slot_bytes(M, d, elt);
   unsigned char* ring = smraw;
-  float* red = reinterpret_cast<float*>(ring + kRing * slot_bytes);   // [2][8 warps][4]
-  float* s_dwq = red + 64;                                           // [M][d]
+  float* red = reinterpret_cast<float*>(ring + kRing * slot_bytes);   // [2][32 warps][4]
+  float* s_dwq = red + 256;                                          // [M][d]
   float* s_dwk = s_dwq + (int64_t)M * d;                             // [M][d]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_dwk + (int64_t)M * d);  // [kRing]
   volatile int* flag = reinterpret_cast<volatile int*>(full + kRing);
-  for (int64_t i = tid; i < 2LL * M * d; i += kBwThreads) s_dwq[i] = 0.f;
+  for (int64_t i = tid; i < 2LL * M * d; i += blockDim.x) s_dwq[i] = 0.f;
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) sm100::mbar_init(sm100::smem_u32(full + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -221,14 +275,13 @@ __global__ void __launch_bounds__(kBwThreads) gate_backward_ring_kernel(GateBwAr
     for (int n = 0; n < N; ++n)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) x[n] += __shfl_xor_sync(0xffffffffu, x[n], o);
-    float* rr = red + rb * 32;
+    float* rr = red + rb * 128;
     if (lane == 0)
       for (int n = 0; n < N; ++n) rr[warp * 4 + n] = x[n];
     __syncthreads();
     for (int n = 0; n < N; ++n) {
       float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < kBwThreads / 32; ++w) t += rr[w * 4 + n];
+      for (int w = 0; w < nwarps; ++w) t += rr[w * 4 + n];
       x[n] = t;
     }
     rb ^= 1;
@@ -248,25 +301,27 @@ __global__ void __launch_bounds__(kBwThreads) gate_backward_ring_kernel(GateBwAr
     const void* hs = slot;
     const void* gs = slot + hb;
     const float* kv = reinterpret_cast<const float*>(slot + 2 * hb);
-    float dv[PER];
+    float v[8], dv[8];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) dv[j] = 0.f;
+    for (int j = 0; j < 8; ++j) v[j] = dv[j] = 0.f;
+    if (act) load8f(kv + (int64_t)M * d + c0, v);
     for (int m = 0; m < M; ++m) {
       const int64_t base = (r * M + m) * (int64_t)d;
       const int sb = m * d;
-      const float* wq = a.w_q + (int64_t)m * d;
-      const float* wk = a.w_k + (int64_t)m * d;
+      float h[8], k[8], g[8], wq[8], wk[8];
       float sums[4] = {0.f, 0.f, 0.f, 0.f};  // sum h^2, sum k^2, sum (h w_q)(k w_k), dout . v
+      if (act) {
+        load8<BF16>(hs, sb + c0, h);
+        load8<BF16>(gs, sb + c0, g);
+        load8f(kv + sb + c0, k);
+        ldg8f(a.w_q + sb + c0, wq);
+        ldg8f(a.w_k + sb + c0, wk);
 #pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int c = tid + kBwThreads * j;
-        if (c < d) {
-          const float h = load_elt(hs, sb + c, a.bf16), k = kv[sb + c];
-          const float g = load_elt(gs, sb + c, a.bf16), v = kv[M * d + c];
-          sums[0] += h * h;
-          sums[1] += k * k;
-          sums[2] += (h * __ldg(wq + c)) * (k * __ldg(wk + c));
-          sums[3] += g * v;
+        for (int j = 0; j < 8; ++j) {
+          sums[0] += h[j] * h[j];
+          sums[1] += k[j] * k[j];
+          sums[2] += (h[j] * wq[j]) * (k[j] * wk[j]);
+          sums[3] += g[j] * v[j];
         }
       }
       bsum(sums, 4);
@@ -277,46 +332,47 @@ __global__ void __launch_bounds__(kBwThreads) gate_backward_ring_kernel(GateBwAr
       const float cq = ds * rk * a.inv_sqrt_d;  // dqn_c = cq k_c w_k,c
       const float ck = ds * rh * a.inv_sqrt_d;  // dkn_c = ck h_c w_q,c
       float u[2] = {0.f, 0.f};                  // u_q . h, u_k . k
+      float dqn[8], dkn[8];
+      if (act) {
+        float aq[8], ak[8];
+        load8f(s_dwq + sb + c0, aq);
+        load8f(s_dwk + sb + c0, ak);
 #pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int c = tid + kBwThreads * j;
-        if (c < d) {
-          const float h = load_elt(hs, sb + c, a.bf16), k = kv[sb + c];
-          const float g = load_elt(gs, sb + c, a.bf16);
-          const float q_w = __ldg(wq + c), k_w = __ldg(wk + c);
-          const float dqn = cq * k * k_w, dkn = ck * h * q_w;
-          s_dwq[sb + c] += dqn * h * rh;
-          s_dwk[sb + c] += dkn * k * rk;
-          u[0] += dqn * q_w * h;
-          u[1] += dkn * k_w * k;
-          dv[j] += alpha * g;
+        for (int j = 0; j < 8; ++j) {
+          dqn[j] = cq * k[j] * wk[j];
+          dkn[j] = ck * h[j] * wq[j];
+          aq[j] += dqn[j] * h[j] * rh;
+          ak[j] += dkn[j] * k[j] * rk;
+          u[0] += dqn[j] * wq[j] * h[j];
+          u[1] += dkn[j] * wk[j] * k[j];
+          dv[j] += alpha * g[j];
         }
+        float4* pq = reinterpret_cast<float4*>(s_dwq + sb + c0);
+        float4* pk = reinterpret_cast<float4*>(s_dwk + sb + c0);
+        pq[0] = make_float4(aq[0], aq[1], aq[2], aq[3]);
+        pq[1] = make_float4(aq[4], aq[5], aq[6], aq[7]);
+        pk[0] = make_float4(ak[0], ak[1], ak[2], ak[3]);
+        pk[1] = make_float4(ak[4], ak[5], ak[6], ak[7]);
       }
       bsum(u, 2);
       const float th = rh * rh * rh * inv_d * u[0], tk = rk * rk * rk * inv_d * u[1];
+      if (act) {
+        float oh[8], ok_[8];
 #pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int c = tid + kBwThreads * j;
-        if (c < d) {
-          const float h = load_elt(hs, sb + c, a.bf16), k = kv[sb + c];
-          const float g = load_elt(gs, sb + c, a.bf16);
-          const float q_w = __ldg(wq + c), k_w = __ldg(wk + c);
-          const float dqn = cq * k * k_w, dkn = ck * h * q_w;
-          store_elt(a.dh, base + c, g + rh * dqn * q_w - th * h, a.bf16);
-          store_elt(a.dkv, r * nkv + sb + c, rk * dkn * k_w - tk * k, a.bf16);
+        for (int j = 0; j < 8; ++j) {
+          oh[j] = g[j] + rh * dqn[j] * wq[j] - th * h[j];
+          ok_[j] = rk * dkn[j] * wk[j] - tk * k[j];
         }
+        store8<BF16>(a.dh, base + c0, oh);
+        store8<BF16>(a.dkv, r * nkv + sb + c0, ok_);
       }
     }
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int c = tid + kBwThreads * j;
-      if (c < d) store_elt(a.dkv, r * nkv + (int64_t)M * d + c, dv[j], a.bf16);
-    }
+    if (act) store8<BF16>(a.dkv, r * nkv + (int64_t)M * d + c0, dv);
     __syncthreads();  // slot i % kRing is read by no thread any more
   }
   __syncthreads();
   float* part = a.partials + (int64_t)blockIdx.x * 2 * M * d;
-  for (int64_t j = tid; j < 2LL * M * d; j += kBwThreads) part[j] = s_dwq[j];
+  for (int64_t j = tid; j < 2LL * M * d; j += blockDim.x) part[j] = s_dwq[j];
   // after a timeout: the copies still in flight land before the CTA leaves
   // (each waited for a bounded time)
   if (tid == 0)
@@ -419,9 +475,22 @@ int gate_bw_grid(int M, int d, int64_t R, int elt) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const size_t rsm = gate_bw_ring_smem(M, d, elt);
-  if (rsm <= 232448) {
-    // the ring kernel: as many CTAs per SM as its shared memory allows (<= 2)
-    const int64_t per_sm = rsm <= 113 * 1024 ? 2 : 1;
+  if (rsm <= 232448 && d % 8 == 0 && ((d / 8 + 31) / 32) * 32 <= 1024) {
+    // the ring kernel: as many CTAs per SM as its registers and shared memory allow
+    int per_sm = 1;
+    const int threads = ((d / 8 + 31) / 32) * 32;
+    auto occ = [&](auto kern) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm) ==
+              cudaSuccess &&
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, rsm) == cudaSuccess)
+        return;
+      per_sm = 1;
+    };
+    if (elt == 2)
+      occ(gate_backward_ring_kernel<true>);
+    else
+      occ(gate_backward_ring_kernel<false>);
+    if (per_sm < 1) per_sm = 1;
     int64_t grid = (int64_t)sms * per_sm;
     if (grid > R) grid = R;
     return grid < 1 ? 1 : (int)grid;
@@ -440,18 +509,20 @@ int gate_bw_grid(int M, int d, int64_t R, int elt) {
 }
 
 size_t gate_bw_ring_smem(int M, int d, int elt) {
-  return kRing * ring_slot_bytes(M, d, elt) + 64 * sizeof(float) + 2 * (size_t)M * d * 4 +
+  return kRing * ring_slot_bytes(M, d, elt) + 256 * sizeof(float) + 2 * (size_t)M * d * 4 +
          kRing * 8 + 16;
 }
 
 namespace {
 
-template <int PER>
+int ring_threads(int d) { return ((d / 8 + 31) / 32) * 32; }
+
+template <bool BF16>
 cudaError_t launch_ring(const GateBwArgs& a, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = gate_backward_ring_kernel<PER>;
+  auto kern = gate_backward_ring_kernel<BF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kBwThreads, smem, stream>>>(a);
+  kern<<<grid, ring_threads(a.d), smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -460,16 +531,8 @@ cudaError_t launch_ring(const GateBwArgs& a, int grid, size_t smem, cudaStream_t
 cudaError_t launch_gate_backward(const GateBwArgs& a, int grid, cudaStream_t stream) {
   if (a.R == 0) return cudaSuccess;
   const size_t rsm = gate_bw_ring_smem(a.M, a.d, a.bf16 ? 2 : 4);
-  if (rsm <= 232448) {
-    const int per = (a.d + kBwThreads - 1) / kBwThreads;
-    if (per <= 1) return launch_ring<1>(a, grid, rsm, stream);
-    if (per <= 2) return launch_ring<2>(a, grid, rsm, stream);
-    if (per <= 4) return launch_ring<4>(a, grid, rsm, stream);
-    if (per <= 8) return launch_ring<8>(a, grid, rsm, stream);
-    if (per <= 12) return launch_ring<12>(a, grid, rsm, stream);
-    if (per <= 16) return launch_ring<16>(a, grid, rsm, stream);
-    return cudaErrorInvalidValue;
-  }
+  if (rsm <= 232448 && a.d % 8 == 0 && ring_threads(a.d) <= 1024)
+    return a.bf16 ? launch_ring<true>(a, grid, rsm, stream) : launch_ring<false>(a, grid, rsm, stream);
   const size_t smem = gate_bw_smem(a.M, a.d);
   if (smem > 232448) return cudaErrorInvalidValue;
   const int per = (a.d + kBwThreads - 1) / kBwThreads;

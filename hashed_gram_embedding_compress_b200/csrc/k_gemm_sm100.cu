@@ -87,9 +87,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb_total = (g.K + kBK - 1) / kBK;
   const int num_tiles = mt * nt * g.splits;
   const int first_tile = (int)(blockIdx.x >> 1), tile_step = (int)(gridDim.x >> 1);
-  // tile -> (m block, n block, K range); neighbouring tiles share their m block
+  // tile -> (m block, n block, K range).  The K split is the slowest index:
+  // the tiles running at one time share their K range, so each K slab of A
+  // and B is read from HBM about once and then from L2 by the other tiles;
+  // neighbouring tiles share their m block.
   auto tile_coords = [&](int tile, int& m_blk, int& n_blk, int& kb0, int& kb1) {
-    const int split = tile % g.splits, mn = tile / g.splits;
+    const int split = tile / (mt * nt), mn = tile - split * (mt * nt);
     m_blk = mn / nt;
     n_blk = mn - m_blk * nt;
     kb0 = split * g.kb_per_split;
