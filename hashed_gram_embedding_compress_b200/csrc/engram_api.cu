@@ -139,10 +139,12 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 int ensure_scratch(engram_handle* h, int64_t rows) {
   if (rows <= h->cap_rows) return ENGRAM_OK;
   free_dev(h->e);
+  free_dev(h->e_alt);
   free_dev(h->partials);
   h->cap_rows = 0;
   const int64_t key_tiles = (int64_t)h->cfg.branches * h->cfg.d_hidden / 64;
   CK(h, cudaMalloc(&h->e, (size_t)rows * h->d_mem * h->elt));
+  CK(h, cudaMalloc(&h->e_alt, (size_t)rows * h->d_mem * h->elt));
   CK(h, cudaMalloc(&h->partials, (size_t)rows * key_tiles * sizeof(float4)));
   h->cap_rows = rows;
   return ENGRAM_OK;
@@ -152,9 +154,13 @@ int ensure_fp8_scratch(engram_handle* h, int64_t rows) {
   if (rows <= h->fp8_cap_rows) return ENGRAM_OK;
   free_dev(h->e8);
   free_dev(h->se8);
+  free_dev(h->e8_alt);
+  free_dev(h->se8_alt);
   h->fp8_cap_rows = 0;
   CK(h, cudaMalloc(&h->e8, (size_t)rows * h->d_mem));
   CK(h, cudaMalloc(&h->se8, (size_t)rows * sizeof(float)));
+  CK(h, cudaMalloc(&h->e8_alt, (size_t)rows * h->d_mem));
+  CK(h, cudaMalloc(&h->se8_alt, (size_t)rows * sizeof(float)));
   h->fp8_cap_rows = rows;
   return ENGRAM_OK;
 }
@@ -460,6 +466,7 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->d_tables);
   free_dev(h->d_wqk);
   free_dev(h->e);
+  free_dev(h->e_alt);
   free_dev(h->partials);
   free_dev(h->d_w8);
   free_dev(h->d_sw8);
@@ -470,6 +477,8 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->bw_partials);
   free_dev(h->e8);
   free_dev(h->se8);
+  free_dev(h->e8_alt);
+  free_dev(h->se8_alt);
   free_dev(h->d_conv_w);
   free_dev(h->d_conv_nw);
   free_dev(h->d_conv_taps);
@@ -986,6 +995,12 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   if ((rc = ensure_scratch(h, R))) return rc;
   const bool fp8 = h->fp8;  // E4M3 operands for the projections (bf16 handles only)
   if (fp8 && (rc = ensure_fp8_scratch(h, R))) return rc;
+  // this call's e buffers (alternating between calls)
+  const bool flip = h->e_flip != 0;
+  h->e_flip ^= 1;
+  void* const E = flip ? h->e_alt : h->e;
+  uint8_t* const E8 = flip ? h->e8_alt : h->e8;
+  float* const SE8 = flip ? h->se8_alt : h->se8;
   const bool prof = h->prof_armed;
   h->prof_armed = false;
   auto mark = [&](int i) -> cudaError_t {
@@ -1004,7 +1019,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
 
   // steps 1-4: indices, then the gathered memory vectors e
   GatherArgs ga{};
-  ga.e = h->e;
+  ga.e = E;
   ga.err = h->d_err;
   ga.rows = R;
   ga.S = h->S;
@@ -1028,10 +1043,11 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     hg.hash = hash_args(h, tokens, B, T, t_begin, nullptr);
     hg.tables = h->d_tables;
     hg.shards = h->shards;
-    hg.e = h->e;
-    hg.q = h->e8;
-    hg.scale = h->se8;
+    hg.e = E;
+    hg.q = E8;
+    hg.scale = SE8;
     hg.row_bytes = ga.row_bytes;
+    hg.pdl = 1;  // overlaps the previous call's value launch (other e buffer)
     CK(h, mark(1));
     // FP8: e leaves the gather as E4M3 codes and row scales
     CK(h, fp8 ? launch_hash_gather_e4m3(hg, st) : launch_hash_gather(hg, st));
@@ -1039,7 +1055,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     CK(h, mark(1));
     CK(h, launch_gather(ga, st));
     if (fp8) {
-      CK(h, launch_quantize_e4m3(h->e, R, h->d_mem, h->e8, h->se8, st));
+      CK(h, launch_quantize_e4m3(E, R, h->d_mem, E8, SE8, st));
       h->launches += 1;
     }
   }
@@ -1097,9 +1113,9 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   };
   if (h->cfg.dtype == ENGRAM_F32) {
     g.key_tile = kF32Tile;
-    CK(h, launch_proj_gate_f32(0, (const float*)h->e, (const float*)h->w_k, g, st));
+    CK(h, launch_proj_gate_f32(0, (const float*)E, (const float*)h->w_k, g, st));
     CK(h, mark(3));
-    CK(h, launch_proj_gate_f32(conv ? 3 : 1, (const float*)h->e, (const float*)h->w_v, g, st));
+    CK(h, launch_proj_gate_f32(conv ? 3 : 1, (const float*)E, (const float*)h->w_v, g, st));
     CK(h, mark(4));
     h->launches += 2;
     if (conv) return short_conv(kF32Tile);
@@ -1113,7 +1129,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   ProjMaps single, wide, pair;
   bool have_single = false, have_wide = false, have_pair = false;
   int value_tile = 0;
-  if (fp8) g.s_row = h->se8;
+  if (fp8) g.s_row = SE8;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
     // the E4M3 operands run on the 512 x 256 CTA-pair kernel only
@@ -1127,7 +1143,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     const int kphase = phase == 0 ? 0 : conv ? 3 : out == hid ? 2 : 1;
     if (pc.kind == ProjKernel::Pair) {
       if (!have_pair) {
-        if ((rc = cached_map(h, &pair.e, h->e, h->d_mem, R, 128))) return rc;
+        if ((rc = cached_map(h, &pair.e, E, h->d_mem, R, 128))) return rc;
         if ((rc = cached_map(h, &pair.h, hid, hcols, R, 128, 32))) return rc;
         if ((rc = cached_map(h, &pair.out, out, hcols, R, 32, 32))) return rc;  // per-warp boxes
         have_pair = true;
@@ -1140,8 +1156,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     } else if (pc.kind == ProjKernel::Wide) {
       if (!have_wide) {
         if (fp8) {
-          if ((rc = cached_map(h, &wide.e, h->e8, h->d_mem, R, 256, 128, 1))) return rc;
-        } else if ((rc = cached_map(h, &wide.e, h->e, h->d_mem, R, 256))) {
+          if ((rc = cached_map(h, &wide.e, E8, h->d_mem, R, 256, 128, 1))) return rc;
+        } else if ((rc = cached_map(h, &wide.e, E, h->d_mem, R, 256))) {
           return rc;
         }
         if ((rc = cached_map(h, &wide.h, hid, hcols, R, 256, 32))) return rc;
@@ -1164,7 +1180,7 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
       }
     } else {
       if (!have_single) {
-        if ((rc = cached_map(h, &single.e, h->e, h->d_mem, R, 128))) return rc;
+        if ((rc = cached_map(h, &single.e, E, h->d_mem, R, 128))) return rc;
         if ((rc = cached_map(h, &single.h, hid, hcols, R, 128))) return rc;
         if ((rc = cached_map(h, &single.out, out, hcols, R, 128))) return rc;
         have_single = true;

@@ -51,10 +51,17 @@ struct engram_handle {
   int64_t fp8_cap_rows = 0;
   uint8_t* e8 = nullptr;       // [rows, d_mem] codes of e
   float* se8 = nullptr;        // [rows] scales of e
+  uint8_t* e8_alt = nullptr;
+  float* se8_alt = nullptr;
 
-  // scratch, sized for cap_rows emitted positions
+  // scratch, sized for cap_rows emitted positions.  The forward alternates
+  // between two buffers of e (e, e_alt; e8/se8 and their twins for FP8), so a
+  // call's gather may run while the previous call's value launch still reads
+  // the other one.
   int64_t cap_rows = 0;
   void* e = nullptr;
+  void* e_alt = nullptr;
+  int e_flip = 0;
   float4* partials = nullptr;
   // short-convolution scratch, sized for conv_cap_rows
   int64_t conv_cap_rows = 0;

@@ -72,6 +72,11 @@ struct HashGatherArgs {
   float* scale;               // E4M3 form: power-of-two scale per row
   int32_t row_bytes;          // d_head * element size, a multiple of 16
   int32_t rows_per_block;     // set by the launcher
+  // 1: launch with programmatic dependent launch, so that the kernel runs
+  // while the previous kernel on the stream (the previous call's value
+  // launch, which reads the other e buffer) finishes; each block waits for
+  // that kernel before it exits, so the next launch still sees it complete.
+  int32_t pdl;
 };
 
 // Projection + gate epilogue arguments (Eq. 3, 4, 6).

@@ -165,64 +165,70 @@ __host__ __device__ inline size_t ring_slot_bytes(int M, int d, int elt) {
   return (size_t)2 * M * d * elt + (size_t)(M + 1) * d * 4;
 }
 
-// Eight consecutive elements of a row, as fp32: bf16 (one 16-byte load) or
-// fp32 (two).
+using u64 = unsigned long long;
+
+// Four consecutive elements as two packed fp32 pairs: bf16 (one 8-byte load)
+// or fp32 (one 16-byte load).
 template <bool BF16>
-__device__ __forceinline__ void load8(const void* base, int64_t i, float (&x)[8]) {
+__device__ __forceinline__ void load4(const void* base, int64_t i, u64& p0, u64& p1) {
   if (BF16) {
-    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + i);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x[2 * j] = __uint_as_float(w[j] << 16);
-      x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
+    const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + i);
+    p0 = sm100::bf16x2_to_f2(u.x);
+    p1 = sm100::bf16x2_to_f2(u.y);
   } else {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i);
-    const float4 u = p[0], v = p[1];
-    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-    x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(base) + i);
+    p0 = sm100::f2_pack(u.x, u.y);
+    p1 = sm100::f2_pack(u.z, u.w);
   }
 }
 
-__device__ __forceinline__ void load8f(const float* p, float (&x)[8]) {
-  const float4 u = reinterpret_cast<const float4*>(p)[0], v = reinterpret_cast<const float4*>(p)[1];
-  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-  x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+__device__ __forceinline__ void load4f(const float* p, u64& p0, u64& p1) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  p0 = sm100::f2_pack(u.x, u.y);
+  p1 = sm100::f2_pack(u.z, u.w);
 }
 
-__device__ __forceinline__ void ldg8f(const float* p, float (&x)[8]) {
-  const float4 u = __ldg(reinterpret_cast<const float4*>(p)),
-               v = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-  x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+__device__ __forceinline__ void ldg4f(const float* p, u64& p0, u64& p1) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  p0 = sm100::f2_pack(u.x, u.y);
+  p1 = sm100::f2_pack(u.z, u.w);
 }
 
 template <bool BF16>
-__device__ __forceinline__ void store8(void* base, int64_t i, const float (&x)[8]) {
+__device__ __forceinline__ void store4(void* base, int64_t i, u64 p0, u64 p1) {
+  const float2 a = sm100::f2_unpack(p0), b = sm100::f2_unpack(p1);
   if (BF16) {
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      w[j] = (uint32_t)bf16_rne(x[2 * j]) | ((uint32_t)bf16_rne(x[2 * j + 1]) << 16);
-    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(base) + i) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(base) + i) =
+        make_uint2(sm100::pack2(a.x, a.y), sm100::pack2(b.x, b.y));
   } else {
-    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + i);
-    p[0] = make_float4(x[0], x[1], x[2], x[3]);
-    p[1] = make_float4(x[4], x[5], x[6], x[7]);
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + i) = make_float4(a.x, a.y, b.x, b.y);
   }
 }
 
-// One CTA per row at a time, one thread per 8 consecutive columns (blockDim
-// = d / 8 rounded up to whole warps), the row's h, dout, k and v of a branch
-// held in registers across the three passes of the branch.
-template <bool BF16>
+__device__ __forceinline__ u64 f2s(float x) {  // {x, x}
+  return sm100::f2_pack(__float_as_uint(x), __float_as_uint(x));
+}
+__device__ __forceinline__ float f2sum(u64 p) {
+  const float2 v = sm100::f2_unpack(p);
+  return v.x + v.y;
+}
+
+// One CTA per row at a time.  Thread t owns columns [4t, 4t + 4) and
+// [4t + 4T, 4t + 4T + 4) (T = blockDim.x = d / 8 rounded up to whole warps),
+// so every shared-memory load of a warp reads consecutive words; the branch's
+// h, dout, k and v stay in registers as packed fp32 pairs (fma.rn.f32x2)
+// through the three passes.  The derivative is arranged to share products:
+// with kw = k w_k and hw = h w_q, u_q . h = cq sum(kw hw) and u_k . k =
+// ck sum(kw hw) = the first reduction's third sum times cq or ck: one block
+// reduction per branch.  M1: one branch, whose weight-gradient sums stay in
+// registers.
+template <bool BF16, bool M1>
 __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
   extern __shared__ __align__(128) unsigned char smraw[];
-  const int d = a.d, M = a.M, tid = threadIdx.x;
-  const int nwarps = blockDim.x >> 5;
-  const int c0 = tid * 8;       // this thread's columns [c0, c0 + 8)
-  const bool act = c0 < d;
+  const int d = a.d, M = a.M, tid = threadIdx.x, T = blockDim.x;
+  const int nwarps = T >> 5;
+  const int cA = 4 * tid, cB = 4 * tid + 4 * T;  // this thread's two groups of 4 columns
+  const bool actA = cA < d, actB = cB < d;
   constexpr int elt = BF16 ? 2 : 4;
   const int64_t nkv = (int64_t)(M + 1) * d;
   const float inv_d = 1.f / (float)d;
@@ -230,16 +236,30 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
   const size_t slot_bytes = ring_slot_bytes(M, d, elt);
   unsigned char* ring = smraw;
   float* red = reinterpret_cast<float*>(ring + kRing * slot_bytes);   // [2][32 warps][4]
-  float* s_dwq = red + 256;                                          // [M][d]
+  float* s_dwq = red + 256;                                          // [M][d] (M > 1)
   float* s_dwk = s_dwq + (int64_t)M * d;                             // [M][d]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_dwk + (int64_t)M * d);  // [kRing]
   volatile int* flag = reinterpret_cast<volatile int*>(full + kRing);
-  for (int64_t i = tid; i < 2LL * M * d; i += blockDim.x) s_dwq[i] = 0.f;
+  if (!M1)
+    for (int64_t i = tid; i < 2LL * M * d; i += T) s_dwq[i] = 0.f;
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) sm100::mbar_init(sm100::smem_u32(full + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // the branch's RMSNorm weights; with one branch the weight-gradient sums
+  // stay in registers
+  u64 WQ[4] = {0, 0, 0, 0}, WK[4] = {0, 0, 0, 0}, DQ[4] = {0, 0, 0, 0}, DK[4] = {0, 0, 0, 0};
+  auto load_w = [&](int m) {
+    if (actA) {
+      ldg4f(a.w_q + m * d + cA, WQ[0], WQ[1]);
+      ldg4f(a.w_k + m * d + cA, WK[0], WK[1]);
+    }
+    if (actB) {
+      ldg4f(a.w_q + m * d + cB, WQ[2], WQ[3]);
+      ldg4f(a.w_k + m * d + cB, WK[2], WK[3]);
+    }
+  };
   // row i of this CTA is blockIdx.x + i gridDim.x, staged in slot i % kRing
   const int64_t n_rows = a.R > blockIdx.x ? (a.R - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   int64_t issued = 0;  // rows whose copies thread 0 has issued
@@ -301,29 +321,34 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     const void* hs = slot;
     const void* gs = slot + hb;
     const float* kv = reinterpret_cast<const float*>(slot + 2 * hb);
-    float v[8], dv[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = dv[j] = 0.f;
-    if (act) load8f(kv + (int64_t)M * d + c0, v);
+    u64 V[4] = {0, 0, 0, 0}, DV[4] = {0, 0, 0, 0};
+    if (actA) load4f(kv + (int64_t)M * d + cA, V[0], V[1]);
+    if (actB) load4f(kv + (int64_t)M * d + cB, V[2], V[3]);
     for (int m = 0; m < M; ++m) {
       const int64_t base = (r * M + m) * (int64_t)d;
       const int sb = m * d;
-      float h[8], k[8], g[8], wq[8], wk[8];
-      float sums[4] = {0.f, 0.f, 0.f, 0.f};  // sum h^2, sum k^2, sum (h w_q)(k w_k), dout . v
-      if (act) {
-        load8<BF16>(hs, sb + c0, h);
-        load8<BF16>(gs, sb + c0, g);
-        load8f(kv + sb + c0, k);
-        ldg8f(a.w_q + sb + c0, wq);
-        ldg8f(a.w_k + sb + c0, wk);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          sums[0] += h[j] * h[j];
-          sums[1] += k[j] * k[j];
-          sums[2] += (h[j] * wq[j]) * (k[j] * wk[j]);
-          sums[3] += g[j] * v[j];
-        }
+      load_w(m);  // L1-resident after the first rows
+      u64 H[4] = {0, 0, 0, 0}, G[4] = {0, 0, 0, 0}, K[4] = {0, 0, 0, 0};
+      if (actA) {
+        load4<BF16>(hs, sb + cA, H[0], H[1]);
+        load4<BF16>(gs, sb + cA, G[0], G[1]);
+        load4f(kv + sb + cA, K[0], K[1]);
       }
+      if (actB) {
+        load4<BF16>(hs, sb + cB, H[2], H[3]);
+        load4<BF16>(gs, sb + cB, G[2], G[3]);
+        load4f(kv + sb + cB, K[2], K[3]);
+      }
+      // sum h^2, sum k^2, sum (h w_q)(k w_k), dout . v
+      u64 s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        s0 = sm100::f2_fma(H[p], H[p], s0);
+        s1 = sm100::f2_fma(K[p], K[p], s1);
+        s2 = sm100::f2_fma(sm100::f2_mul(H[p], WQ[p]), sm100::f2_mul(K[p], WK[p]), s2);
+        s3 = sm100::f2_fma(G[p], V[p], s3);
+      }
+      float sums[4] = {f2sum(s0), f2sum(s1), f2sum(s2), f2sum(s3)};
       bsum(sums, 4);
       const float rh = rsqrtf(sums[0] * inv_d + a.eps);
       const float rk = rsqrtf(sums[1] * inv_d + a.eps);
@@ -331,48 +356,83 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
       const float ds = sums[3] * alpha * (1.f - alpha);
       const float cq = ds * rk * a.inv_sqrt_d;  // dqn_c = cq k_c w_k,c
       const float ck = ds * rh * a.inv_sqrt_d;  // dkn_c = ck h_c w_q,c
-      float u[2] = {0.f, 0.f};                  // u_q . h, u_k . k
-      float dqn[8], dkn[8];
-      if (act) {
-        float aq[8], ak[8];
-        load8f(s_dwq + sb + c0, aq);
-        load8f(s_dwk + sb + c0, ak);
+      // dw_q += cq rh h kw; dw_k += ck rk k hw; dv += alpha dout
+      const u64 cqr = f2s(cq * rh), ckr = f2s(ck * rk), al = f2s(alpha);
+      float U[1] = {f2sum(s2)};  // sum kw hw (this thread's part) is s2
+      if (M1) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          dqn[j] = cq * k[j] * wk[j];
-          dkn[j] = ck * h[j] * wq[j];
-          aq[j] += dqn[j] * h[j] * rh;
-          ak[j] += dkn[j] * k[j] * rk;
-          u[0] += dqn[j] * wq[j] * h[j];
-          u[1] += dkn[j] * wk[j] * k[j];
-          dv[j] += alpha * g[j];
+        for (int p = 0; p < 4; ++p) {
+          const u64 hk = sm100::f2_mul(H[p], K[p]);
+          DQ[p] = sm100::f2_fma(cqr, sm100::f2_mul(hk, WK[p]), DQ[p]);
+          DK[p] = sm100::f2_fma(ckr, sm100::f2_mul(hk, WQ[p]), DK[p]);
         }
-        float4* pq = reinterpret_cast<float4*>(s_dwq + sb + c0);
-        float4* pk = reinterpret_cast<float4*>(s_dwk + sb + c0);
-        pq[0] = make_float4(aq[0], aq[1], aq[2], aq[3]);
-        pq[1] = make_float4(aq[4], aq[5], aq[6], aq[7]);
-        pk[0] = make_float4(ak[0], ak[1], ak[2], ak[3]);
-        pk[1] = make_float4(ak[4], ak[5], ak[6], ak[7]);
+      } else {
+        u64 aq[4], ak[4];
+        if (actA) {
+          load4f(s_dwq + sb + cA, aq[0], aq[1]);
+          load4f(s_dwk + sb + cA, ak[0], ak[1]);
+        }
+        if (actB) {
+          load4f(s_dwq + sb + cB, aq[2], aq[3]);
+          load4f(s_dwk + sb + cB, ak[2], ak[3]);
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const u64 hk = sm100::f2_mul(H[p], K[p]);
+          aq[p] = sm100::f2_fma(cqr, sm100::f2_mul(hk, WK[p]), aq[p]);
+          ak[p] = sm100::f2_fma(ckr, sm100::f2_mul(hk, WQ[p]), ak[p]);
+        }
+        if (actA) {
+          store4<false>(s_dwq, sb + cA, aq[0], aq[1]);
+          store4<false>(s_dwk, sb + cA, ak[0], ak[1]);
+        }
+        if (actB) {
+          store4<false>(s_dwq, sb + cB, aq[2], aq[3]);
+          store4<false>(s_dwk, sb + cB, ak[2], ak[3]);
+        }
       }
-      bsum(u, 2);
-      const float th = rh * rh * rh * inv_d * u[0], tk = rk * rk * rk * inv_d * u[1];
-      if (act) {
-        float oh[8], ok_[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          oh[j] = g[j] + rh * dqn[j] * wq[j] - th * h[j];
-          ok_[j] = rk * dkn[j] * wk[j] - tk * k[j];
-        }
-        store8<BF16>(a.dh, base + c0, oh);
-        store8<BF16>(a.dkv, r * nkv + sb + c0, ok_);
+      for (int p = 0; p < 4; ++p) DV[p] = sm100::f2_fma(al, G[p], DV[p]);
+      // the first reduction already summed kw hw (s2) over the block
+      U[0] = sums[2];
+      const float th = rh * rh * rh * inv_d * (cq * U[0]);
+      const float tk = rk * rk * rk * inv_d * (ck * U[0]);
+      // dh = dout + (rh cq) kw w_q - th h;  dk = (rk ck) hw w_k - tk k
+      const u64 a_h = f2s(rh * cq), a_k = f2s(rk * ck), m_th = f2s(-th), m_tk = f2s(-tk);
+      u64 OH[4], OK[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const u64 ww = sm100::f2_mul(WQ[p], WK[p]);
+        OH[p] = sm100::f2_fma(m_th, H[p], sm100::f2_fma(a_h, sm100::f2_mul(K[p], ww), G[p]));
+        OK[p] = sm100::f2_fma(m_tk, K[p], sm100::f2_mul(a_k, sm100::f2_mul(H[p], ww)));
+      }
+      if (actA) {
+        store4<BF16>(a.dh, base + cA, OH[0], OH[1]);
+        store4<BF16>(a.dkv, r * nkv + sb + cA, OK[0], OK[1]);
+      }
+      if (actB) {
+        store4<BF16>(a.dh, base + cB, OH[2], OH[3]);
+        store4<BF16>(a.dkv, r * nkv + sb + cB, OK[2], OK[3]);
       }
     }
-    if (act) store8<BF16>(a.dkv, r * nkv + (int64_t)M * d + c0, dv);
+    if (actA) store4<BF16>(a.dkv, r * nkv + (int64_t)M * d + cA, DV[0], DV[1]);
+    if (actB) store4<BF16>(a.dkv, r * nkv + (int64_t)M * d + cB, DV[2], DV[3]);
     __syncthreads();  // slot i % kRing is read by no thread any more
   }
   __syncthreads();
   float* part = a.partials + (int64_t)blockIdx.x * 2 * M * d;
-  for (int64_t j = tid; j < 2LL * M * d; j += blockDim.x) part[j] = s_dwq[j];
+  if (M1) {
+    if (actA) {
+      store4<false>(part, cA, DQ[0], DQ[1]);
+      store4<false>(part, d + cA, DK[0], DK[1]);
+    }
+    if (actB) {
+      store4<false>(part, cB, DQ[2], DQ[3]);
+      store4<false>(part, d + cB, DK[2], DK[3]);
+    }
+  } else {
+    for (int64_t j = tid; j < 2LL * M * d; j += T) part[j] = s_dwq[j];
+  }
   // after a timeout: the copies still in flight land before the CTA leaves
   // (each waited for a bounded time)
   if (tid == 0)
@@ -487,9 +547,9 @@ int gate_bw_grid(int M, int d, int64_t R, int elt) {
       per_sm = 1;
     };
     if (elt == 2)
-      occ(gate_backward_ring_kernel<true>);
+      occ(gate_backward_ring_kernel<true, false>);
     else
-      occ(gate_backward_ring_kernel<false>);
+      occ(gate_backward_ring_kernel<false, false>);
     if (per_sm < 1) per_sm = 1;
     int64_t grid = (int64_t)sms * per_sm;
     if (grid > R) grid = R;
@@ -517,9 +577,9 @@ namespace {
 
 int ring_threads(int d) { return ((d / 8 + 31) / 32) * 32; }
 
-template <bool BF16>
+template <bool BF16, bool M1>
 cudaError_t launch_ring(const GateBwArgs& a, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = gate_backward_ring_kernel<BF16>;
+  auto kern = gate_backward_ring_kernel<BF16, M1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, ring_threads(a.d), smem, stream>>>(a);
@@ -532,7 +592,10 @@ cudaError_t launch_gate_backward(const GateBwArgs& a, int grid, cudaStream_t str
   if (a.R == 0) return cudaSuccess;
   const size_t rsm = gate_bw_ring_smem(a.M, a.d, a.bf16 ? 2 : 4);
   if (rsm <= 232448 && a.d % 8 == 0 && ring_threads(a.d) <= 1024)
-    return a.bf16 ? launch_ring<true>(a, grid, rsm, stream) : launch_ring<false>(a, grid, rsm, stream);
+    return a.bf16 ? (a.M == 1 ? launch_ring<true, true>(a, grid, rsm, stream)
+                              : launch_ring<true, false>(a, grid, rsm, stream))
+                  : (a.M == 1 ? launch_ring<false, true>(a, grid, rsm, stream)
+                              : launch_ring<false, false>(a, grid, rsm, stream));
   const size_t smem = gate_bw_smem(a.M, a.d);
   if (smem > 232448) return cudaErrorInvalidValue;
   const int per = (a.d + kBwThreads - 1) / kBwThreads;

@@ -205,6 +205,9 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
       if (i < nchunks) dst[i] = v[k];
     }
   }
+  // the previous kernel (which this one may have overlapped) is complete
+  // before this block, and so this kernel, completes
+  if (threadIdx.x == 0) griddep_wait();
 }
 
 // Hash, gather and E4M3 quantisation fused (the FP8 projections): the hash
@@ -260,6 +263,7 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_e4m3_kernel(HashGat
     };
     quant_row_warp(chunk, C, g.q + (int64_t)(row0 + rl) * C * 8, g.scale + row0 + rl, lane);
   }
+  if (threadIdx.x == 0) griddep_wait();  // as in hash_gather_kernel
 }
 
 // E4M3 codes and scales of bf16 rows (the quantiser on its own: for W when
@@ -327,7 +331,17 @@ cudaError_t launch_hash_gather(const HashGatherArgs& a, cudaStream_t stream) {
   if (fill < rb) rb = fill < 1 ? 1 : fill;
   HashGatherArgs b = a;
   b.rows_per_block = (int32_t)rb;
-  hash_gather_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(b);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)((rows + rb - 1) / rb));
+  lc.blockDim = dim3(kFusedThreads);
+  lc.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = b.pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&lc, hash_gather_kernel, b);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -346,7 +360,17 @@ cudaError_t launch_hash_gather_e4m3(const HashGatherArgs& a, cudaStream_t stream
   if (fill < rb) rb = fill < 1 ? 1 : fill;
   HashGatherArgs b = a;
   b.rows_per_block = (int32_t)rb;
-  hash_gather_e4m3_kernel<<<(unsigned)((rows + rb - 1) / rb), kFusedThreads, 0, stream>>>(b);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)((rows + rb - 1) / rb));
+  lc.blockDim = dim3(kFusedThreads);
+  lc.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = b.pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&lc, hash_gather_e4m3_kernel, b);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the value phase may launch
     griddep_wait();
     griddep_launch_dependents();
+  } else {
+    // the next call's gather (which writes the other e buffer) may start
+    griddep_launch_dependents();
   }
 
   if (warp == 4) {
