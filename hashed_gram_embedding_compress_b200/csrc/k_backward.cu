@@ -299,24 +299,31 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     if (lane == 0)
       for (int n = 0; n < N; ++n) rr[warp * 4 + n] = x[n];
     __syncthreads();
-    for (int n = 0; n < N; ++n) {
-      float t = 0.f;
-      for (int w = 0; w < nwarps; ++w) t += rr[w * 4 + n];
-      x[n] = t;
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < nwarps; ++w) {
+      const float4 q = reinterpret_cast<const float4*>(rr)[w];
+      t.x += q.x;
+      t.y += q.y;
+      t.z += q.z;
+      t.w += q.w;
     }
+    x[0] = t.x;
+    if (N > 1) x[1] = t.y;
+    if (N > 2) x[2] = t.z;
+    if (N > 3) x[3] = t.w;
     rb ^= 1;
   };
   int64_t i = 0;
   for (; i < n_rows; ++i) {
     const int64_t r = blockIdx.x + i * (int64_t)gridDim.x;
     if (tid == 0) {
-      issue_next();  // row i + kRing - 1, into the slot row i - 1 left
       const bool ok = wait_row(i);
       *flag = ok ? 1 : 0;
       if (!ok) atomicOr(a.err, kDevErrTimeout);
     }
-    __syncthreads();
+    __syncthreads();  // every thread is done with row i - 1, and row i is here
     if (!*flag) break;
+    if (tid == 0) issue_next();  // row i + kRing - 1, into the slot row i - 1 left
     const unsigned char* slot = ring + (i % kRing) * slot_bytes;
     const void* hs = slot;
     const void* gs = slot + hb;
@@ -417,7 +424,6 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     }
     if (actA) store4<BF16>(a.dkv, r * nkv + (int64_t)M * d + cA, DV[0], DV[1]);
     if (actB) store4<BF16>(a.dkv, r * nkv + (int64_t)M * d + cB, DV[2], DV[3]);
-    __syncthreads();  // slot i % kRing is read by no thread any more
   }
   __syncthreads();
   float* part = a.partials + (int64_t)blockIdx.x * 2 * M * d;
