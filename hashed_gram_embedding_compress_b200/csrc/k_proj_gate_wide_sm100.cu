@@ -171,15 +171,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // the partner's barriers are initialised before any signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  if (PHASE == 0) {
-    // e (and its scales) come from the previous kernel; once it is complete
-    // the value phase may launch
-    griddep_wait();
-    griddep_launch_dependents();
-  } else {
-    // the next call's gather (which writes the other e buffer) may start
-    griddep_launch_dependents();
-  }
+  // Programmatic dependent launch.  Key phase: e (and its scales) come from
+  // the previous kernel; the producers wait for it (the e/W producer after
+  // issuing the first tile's W boxes, which do not depend on it) and then let
+  // the value phase launch.  Value phase: the next call's gather (which
+  // writes the other e buffer) may start at once.
+  if (PHASE != 0) griddep_launch_dependents();
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------- e / W producer
@@ -190,20 +187,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    // key phase: the first tile's first stages of W go out before the wait
+    // for the previous kernel (every stage is free at this point)
+    int pre = 0;
+    if (PHASE == 0 && first_tile < num_tiles) {
+      pre = num_kb < STAGES ? num_kb : STAGES;
+      const int b_row = (first_tile % num_n) * kCols + (int)rank * (kCols / 2);
+      if (lane == 0) {
+        for (int kb = 0; kb < pre; ++kb) {
+          if (leader) mbar_expect_tx(full_bar(kb), 2 * STAGE_BYTES);
+          tma_load_2d_pair(sB + kb * B_BYTES, &map_w, peer_addr(full_bar(kb), 0), kb * BK, b_row);
+        }
+      }
+      __syncwarp();
+    }
+    if (PHASE == 0) {
+      griddep_wait();
+      griddep_launch_dependents();
+    }
     for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
       const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
       const int a_row = m_blk * 2 * kRows + (int)rank * kRows;
       const int b_row = n_blk * kCols + (int)rank * (kCols / 2);
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (lane == 0) ok = wait_ready(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+        const bool early = tile == first_tile && kb < pre;  // W already on its way
+        if (!early) {
+          if (lane == 0) ok = wait_ready(empty_bar(stage), phase ^ 1u, abort_flag, g.err);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+        }
         if (lane == 0) {
           // the leader's full barrier counts the bytes of both CTAs
           const uint32_t fb = peer_addr(full_bar(stage), 0);
-          if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          if (!early && leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
           tma_load_2d_pair(sA + stage * A_BYTES, &map_e, fb, kb * BK, a_row);
-          tma_load_2d_pair(sB + stage * B_BYTES, &map_w, fb, kb * BK, b_row);
+          if (!early) tma_load_2d_pair(sB + stage * B_BYTES, &map_w, fb, kb * BK, b_row);
         }
         __syncwarp();
         if (++stage == STAGES) {
@@ -220,6 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kHWarp) {
     // -------------------------------------------------- h sub-tile producer
     if (lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&map_h) : "memory");
+    // h may still be written by the kernel before the previous kernel
+    if (PHASE == 0) griddep_wait();
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
