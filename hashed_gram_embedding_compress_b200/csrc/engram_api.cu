@@ -1130,13 +1130,11 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   bool have_single = false, have_wide = false, have_pair = false;
   int value_tile = 0;
   if (fp8) g.s_row = SE8;
-  int key_grid = -1;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
     // the E4M3 operands run on the 512 x 256 CTA-pair kernel only
     const ProjChoice pc = fp8 ? wide_proj(phase, R, g.M, g.d, h->sms)
-                              : choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv, key_grid);
-    if (phase == 0) key_grid = pc.grid;
+                              : choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv);
     if (fp8) g.s_col = h->d_sw8 + (phase == 0 ? 0 : (int64_t)g.M * g.d);
     if (phase == 0) g.key_tile = pc.key_tile;
     if (phase == 1) value_tile = pc.key_tile;

@@ -318,13 +318,8 @@ inline ProjChoice wide_proj(int phase, int64_t R, int M, int d, int sms) {
   return {ProjKernel::Wide, 128, 2 * (int)(tiles < pairs ? tiles : pairs), 256};
 }
 
-// key_grid (value phase): CTAs of the key launch.  When the 256 x 256 pair
-// tiles of the value launch fit on the SMs the key launch leaves free, they
-// are chosen: the value launch, started early (programmatic dependent
-// launch), then streams W_V and e beside the key launch and only its
-// epilogue waits for the keys (short calls such as decode).
 inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int flags,
-                              bool conv = false, int key_grid = -1) {
+                              bool conv = false) {
   const int n_total = phase == 0 ? M * d : d;
   const int pairs = sms / 2;
   const bool pairs_ok = !(flags & ENGRAM_FLAG_NO_CTA_PAIRS) && n_total % 256 == 0;
@@ -344,8 +339,6 @@ inline ProjChoice choose_proj(int phase, int64_t R, int M, int d, int sms, int f
     const int64_t tiles = (R + 255) / 256 * (n_total / 256);
     const int64_t cost = (tiles + pairs - 1) / pairs * 256 * 10;
     const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
-    if (phase == 1 && key_grid >= 0 && tiles <= pairs && key_grid + grid <= sms)
-      return {ProjKernel::Pair, 128, grid, 128};
     if (cost < best_cost) {
       best_cost = cost;
       best = {ProjKernel::Pair, 128, grid, 128};

@@ -248,7 +248,14 @@ def test_in_place_update_and_empty_batch():
     h2 = p.h.clone()
     m.forward(p.tokens.cuda(), h2, h2)  # out aliases h
     torch.cuda.synchronize()
-    assert torch.equal(h2, out_ref)
+    # in place the CTA-pair value kernels add bf16(alpha v) into h (a second
+    # rounding, RN(h + RN(alpha v))); out of place every value kernel writes
+    # RN(h + alpha v): equal, or one rounding step apart on a few elements
+    same = (h2 == out_ref).float().mean().item()
+    assert same > 0.98 and rel_l2(h2.double(), out_ref.double()) <= 1e-3
+    rows = np.arange(sh.rows_out)
+    _, _, _, o_ref = p.oracle_forward(rows)
+    assert out_close(to_oracle(h2), o_ref, "bf16") <= 1e-3
     empty = torch.empty((0, 5), dtype=torch.int32, device="cuda")
     m.forward(empty, h2[:0], h2[:0])
     m.hash(empty, torch.empty((0, sh.num_tables), dtype=torch.int64, device="cuda"))
