@@ -446,18 +446,33 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
 }
 
 // dnorm_q[i] += sum over CTAs b of partials[b][0][i], dnorm_k likewise, in
-// order of b (one thread per column).
-__global__ void dnorm_reduce_kernel(const float* partials, int nblocks, int64_t n, float* dnorm_q,
-                                    float* dnorm_k) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 2 * n;
-       i += (int64_t)gridDim.x * blockDim.x) {
+// a fixed order (deterministic): a block of 32 x 8 threads takes 32
+// consecutive columns; thread (x, y) sums the CTAs b = y, y + 8, ... in
+// order (the 32 columns of one b are one coalesced 128-byte read), then the
+// 8 partial sums of a column are added in order of y.
+__global__ void __launch_bounds__(256) dnorm_reduce_kernel(const float* partials, int nblocks,
+                                                           int64_t n, float* dnorm_q,
+                                                           float* dnorm_k) {
+  __shared__ float part[8][33];
+  const int x = threadIdx.x & 31, y = threadIdx.x >> 5;
+  for (int64_t c0 = (int64_t)blockIdx.x * 32; c0 < 2 * n; c0 += (int64_t)gridDim.x * 32) {
+    const int64_t i = c0 + x;
     float s = 0.f;
-    for (int b = 0; b < nblocks; ++b) s += partials[(int64_t)b * 2 * n + i];
-    if (i < n) {
-      if (dnorm_q) dnorm_q[i] += s;
-    } else if (dnorm_k) {
-      dnorm_k[i - n] += s;
+    if (i < 2 * n)
+      for (int b = y; b < nblocks; b += 8) s += partials[(int64_t)b * 2 * n + i];
+    part[y][x] = s;
+    __syncthreads();
+    if (y == 0 && i < 2 * n) {
+      float t = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t += part[k][x];
+      if (i < n) {
+        if (dnorm_q) dnorm_q[i] += t;
+      } else if (dnorm_k) {
+        dnorm_k[i - n] += t;
+      }
     }
+    __syncthreads();
   }
 }
 
@@ -617,8 +632,12 @@ cudaError_t launch_gate_backward(const GateBwArgs& a, int grid, cudaStream_t str
 cudaError_t launch_dnorm_reduce(const float* partials, int nblocks, int64_t n, float* dnorm_q,
                                 float* dnorm_k, cudaStream_t stream) {
   if (n == 0 || (!dnorm_q && !dnorm_k)) return cudaSuccess;
-  dnorm_reduce_kernel<<<grid_cap(2 * n, 256), 256, 0, stream>>>(partials, nblocks, n, dnorm_q,
-                                                                 dnorm_k);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t blocks = (2 * n + 31) / 32;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  dnorm_reduce_kernel<<<(unsigned)blocks, 256, 0, stream>>>(partials, nblocks, n, dnorm_q, dnorm_k);
   return cudaGetLastError();
 }
 
