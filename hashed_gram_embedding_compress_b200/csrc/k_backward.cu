@@ -275,7 +275,7 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     sm100::bulk_load(dst + 2 * hb, a.kv + r * nkv, kvb, bar);
     ++issued;
   };
-  // bounded wait for the copies of row i (thread 0)
+  // bounded wait for the copies of row i
   auto wait_row = [&](int64_t i) -> bool {
     const uint32_t bar = sm100::smem_u32(full + (i % kRing));
     const uint32_t par = (uint32_t)(i / kRing) & 1u;
@@ -285,11 +285,17 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
       if (sm100::globaltimer() - t0 > sm100::kWaitLimitNs) return false;
     return true;
   };
-  if (tid == 0)
+  if (tid == 0) {
+    *flag = 1;
     for (int i = 0; i < kRing - 1; ++i) issue_next();
+  }
+  if (M1) load_w(0);
+  __syncthreads();
   int rb = 0;  // which half of `red` the next reduction uses
   // sum of N values over the block with one barrier: the halves of `red`
-  // alternate, so a reduction never overwrites values still being read
+  // alternate, so a reduction never overwrites values still being read (a
+  // thread writes a half again only after the next row's barrier, which every
+  // thread reaches after reading this half)
   auto bsum = [&](float* x, int N) {
     const int lane = tid & 31, warp = tid >> 5;
     for (int n = 0; n < N; ++n)
@@ -313,17 +319,17 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     if (N > 3) x[3] = t.w;
     rb ^= 1;
   };
+  // One barrier per row (the block reduction's).  Every thread waits for row
+  // i's copies itself; after row i's barrier every thread has finished with
+  // row i - 1's slot, so thread 0 then refills it with row i + kRing - 1.  A
+  // timed-out wait is acted on after the barrier, by every thread alike.
   int64_t i = 0;
   for (; i < n_rows; ++i) {
     const int64_t r = blockIdx.x + i * (int64_t)gridDim.x;
-    if (tid == 0) {
-      const bool ok = wait_row(i);
-      *flag = ok ? 1 : 0;
-      if (!ok) atomicOr(a.err, kDevErrTimeout);
+    if (!wait_row(i)) {
+      *flag = 0;
+      atomicOr(a.err, kDevErrTimeout);
     }
-    __syncthreads();  // every thread is done with row i - 1, and row i is here
-    if (!*flag) break;
-    if (tid == 0) issue_next();  // row i + kRing - 1, into the slot row i - 1 left
     const unsigned char* slot = ring + (i % kRing) * slot_bytes;
     const void* hs = slot;
     const void* gs = slot + hb;
@@ -331,10 +337,11 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     u64 V[4] = {0, 0, 0, 0}, DV[4] = {0, 0, 0, 0};
     if (actA) load4f(kv + (int64_t)M * d + cA, V[0], V[1]);
     if (actB) load4f(kv + (int64_t)M * d + cB, V[2], V[3]);
+    bool stop = false;
     for (int m = 0; m < M; ++m) {
       const int64_t base = (r * M + m) * (int64_t)d;
       const int sb = m * d;
-      load_w(m);  // L1-resident after the first rows
+      if (!M1) load_w(m);  // L1-resident after the first rows
       u64 H[4] = {0, 0, 0, 0}, G[4] = {0, 0, 0, 0}, K[4] = {0, 0, 0, 0};
       if (actA) {
         load4<BF16>(hs, sb + cA, H[0], H[1]);
@@ -357,6 +364,13 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
       }
       float sums[4] = {f2sum(s0), f2sum(s1), f2sum(s2), f2sum(s3)};
       bsum(sums, 4);
+      if (m == 0) {
+        if (!*flag) {  // a wait timed out: leave before any store of this row
+          stop = true;
+          break;
+        }
+        if (tid == 0) issue_next();  // row i + kRing - 1, into the slot row i - 1 left
+      }
       const float rh = rsqrtf(sums[0] * inv_d + a.eps);
       const float rk = rsqrtf(sums[1] * inv_d + a.eps);
       const float alpha = 1.f / (1.f + __expf(-sums[2] * rh * rk * a.inv_sqrt_d));
@@ -422,6 +436,7 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
         store4<BF16>(a.dkv, r * nkv + sb + cB, OK[2], OK[3]);
       }
     }
+    if (stop) break;
     if (actA) store4<BF16>(a.dkv, r * nkv + (int64_t)M * d + cA, DV[0], DV[1]);
     if (actB) store4<BF16>(a.dkv, r * nkv + (int64_t)M * d + cB, DV[2], DV[3]);
   }
