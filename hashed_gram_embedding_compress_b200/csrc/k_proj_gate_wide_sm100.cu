@@ -31,7 +31,10 @@
 // h ring), 2 = values when out aliases h (the residual update in place): the
 // epilogue stages bf16(alpha v) for 64 columns at a time and adds it into out
 // with a TMA reduce-add, so h never passes through shared memory; the sum is rounded once more
-// (RN(h + RN(alpha v)) instead of RN(h + alpha v)); 3 = values for the short
+// (RN(h + RN(alpha v)) instead of RN(h + alpha v)); with one branch the
+// whole tile is read out of TMEM (half staged, half kept in registers) before
+// the first reduce-add, so the accumulators are free again within a fraction
+// of the time the reduce-adds take (bf16 operands); 3 = values for the short
 // convolution (Eq. 5): v in fp32 and its sum of squares per row and tile,
 // plus alpha; h is not read.
 // FP8 form (section 2.4, the projections as one dense FP8 matmul): e and W
@@ -531,11 +534,107 @@ __global__ void __launch_bounds__(kThreads, 1)
           vals_chunk(q + 1, vb, va);
         }
         if (valid) g.vv[(int64_t)n_blk * R + row] = svv;
+      } else if (PHASE == 2 && !F8 && M == 1) {
+        // out aliases h, one branch (bf16 operands; the E4M3 form takes the
+        // general path below): the whole tile leaves TMEM before any
+        // reduce-add is issued.  bf16(alpha v) of chunks 0-3 (columns 0-127)
+        // is staged in the warp's two 4 KB buffers and that of chunks 4-7 kept
+        // packed in registers; the accumulators are released, then the four
+        // 32 x 64 reduce-adds go out (the last two once the first two have
+        // read their buffers) while the next tile's MMAs run.
+        uint8_t* stage0 = hbuf + warp * 8192;
+        const float a = al[0];
+        const unsigned long long a2 = f2_pack(__float_as_uint(a), __float_as_uint(a));
+        uint32_t keep[2][32];
+        // the previous tile's reduces have read the buffers
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        __syncwarp();
+        tmem_ld32_async(taddr + H_COLS, vb);  // chunk 1 (chunk 0 is on its way into va)
+#pragma unroll
+        for (int p = 0; p < NQ / 2; ++p) {
+          const int q = 2 * p;
+          tmem_wait32(va);
+          tmem_wait32(vb);
+          __syncwarp();
+          uint32_t ow[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* v = c < 4 ? va : vb;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int e = (c & 3) * 8 + 2 * j;
+              const float2 o = f2_unpack(f2_mul(a2, f2_pack(v[e], v[e + 1])));
+              ow[4 * c + j] = pack2(o.x, o.y);
+            }
+          }
+          if (g.delta && valid) {
+            float4* dp = reinterpret_cast<float4*>(g.delta + (int64_t)row * d + n0 + q * H_COLS);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const uint32_t* v = c < 8 ? va : vb;
+              const int e = (c & 7) * 4;
+              dp[c] = make_float4(a * __uint_as_float(v[e]), a * __uint_as_float(v[e + 1]),
+                                  a * __uint_as_float(v[e + 2]), a * __uint_as_float(v[e + 3]));
+            }
+          }
+          __syncwarp();
+          if (q + 2 < NQ) {
+            tmem_ld32_async(taddr + (q + 2) * H_COLS, va);
+            tmem_ld32_async(taddr + (q + 3) * H_COLS, vb);
+          } else {
+            tc_fence_before();  // last TMEM read done: release the accumulators
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(peer_addr(tempty_bar, 0));
+          }
+          if (p < 2) {
+            uint8_t* st = stage0 + p * 4096;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(st + sw128_off(lane, c)) =
+                  make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) keep[p - 2][i] = ow[i];
+          }
+        }
+        // a warp whose rows all lie past R commits empty groups instead
+        const bool any = row0 + wrow0 < R;
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            if (any)
+              tma_reduce_add_2d(&map_out, smem_u32(stage0 + b * 4096), n0 + b * 2 * H_COLS,
+                                row0 + wrow0);
+            else
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          // buffer b has been read by its first reduce (the other may be pending)
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
+          uint8_t* st = stage0 + b * 4096;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(st + sw128_off(lane, c)) =
+                make_uint4(keep[b][4 * c], keep[b][4 * c + 1], keep[b][4 * c + 2], keep[b][4 * c + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (any)
+              tma_reduce_add_2d(&map_out, smem_u32(st), n0 + (2 + b) * 2 * H_COLS, row0 + wrow0);
+            else
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+        }
       } else if (PHASE == 2) {
-        // out aliases h: add bf16(alpha v) into it with TMA reduce-add, two
-        // 32-column chunks per operation (32 rows x 64 columns, 4 KB,
-        // 128-byte swizzle); each warp stages in one of two buffers (the h
-        // ring is unused in this phase)
+        // out aliases h, several branches: add bf16(alpha_m v) into each
+        // branch with TMA reduce-add, two 32-column chunks per operation (32
+        // rows x 64 columns, 4 KB, 128-byte swizzle); each warp stages in one
+        // of two buffers (the h ring is unused in this phase)
         uint8_t* stage0 = hbuf + warp * 8192;
         int sbuf = 0;
         __syncwarp();
