@@ -636,7 +636,8 @@ def run_backward_bench(args, rank, world, dist):
                    "global_batch": R * world, "seq_len": sh.T,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: inputs larger than L2"},
-        "roofline": {"kernel": "cuBLAS GEMMs (k, v recomputed; dW; de) of the backward",
+        "roofline": {"kernel": "the library's tcgen05 contractions of the backward "
+                               "(gemm_pair_kernel: k and v recomputed; dW; de)",
                      "bound": "tensor", "achieved": gemm_flops / gemm_s / 1e12,
                      "peak": tflops_burst, "unit": "TFLOP/s",
                      "frac": gemm_flops / gemm_s / 1e12 / tflops_burst, "traffic": None,
