@@ -289,34 +289,45 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     *flag = 1;
     for (int i = 0; i < kRing - 1; ++i) issue_next();
   }
-  if (M1) load_w(0);
   __syncthreads();
   int rb = 0;  // which half of `red` the next reduction uses
-  // sum of N values over the block with one barrier: the halves of `red`
-  // alternate, so a reduction never overwrites values still being read (a
-  // thread writes a half again only after the next row's barrier, which every
-  // thread reaches after reading this half)
-  auto bsum = [&](float* x, int N) {
+  // Sum of the four values x[0..3] over the block with one barrier, every
+  // thread getting the four totals.  Within a warp the four sums share one
+  // shuffle tree: after the exchanges across lane bits 4 and 3 each lane
+  // carries one of the four values (v = 2 bit4 + bit3), whose sum over the
+  // remaining lane bits the last three exchanges complete.  Warp w's totals go
+  // to red; after the barrier lane l < nwarps takes warp l's four and the same
+  // tree sums them over the warps, and four shuffles hand the totals to every
+  // lane.  The halves of `red` alternate, so a reduction never overwrites
+  // values still being read (a thread writes a half again only after the next
+  // row's barrier, which every thread reaches after reading this half).
+  auto tree4 = [](float x0, float x1, float x2, float x3, int lane) -> float {
+    const bool b4 = lane & 16, b3 = lane & 8;
+    float k0 = b4 ? x2 : x0, k1 = b4 ? x3 : x1;
+    const float s0 = b4 ? x0 : x2, s1 = b4 ? x1 : x3;
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    float c = b3 ? k1 : k0;
+    c += __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+    c += __shfl_xor_sync(0xffffffffu, c, 4);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    return c;  // the total of value 2 bit4 + bit3 over the warp's lanes
+  };
+  auto bsum = [&](float* x) {
     const int lane = tid & 31, warp = tid >> 5;
-    for (int n = 0; n < N; ++n)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) x[n] += __shfl_xor_sync(0xffffffffu, x[n], o);
+    const int v = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+    const float c = tree4(x[0], x[1], x[2], x[3], lane);
     float* rr = red + rb * 128;
-    if (lane == 0)
-      for (int n = 0; n < N; ++n) rr[warp * 4 + n] = x[n];
+    if ((lane & 7) == 0) rr[warp * 4 + v] = c;
     __syncthreads();
-    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = 0; w < nwarps; ++w) {
-      const float4 q = reinterpret_cast<const float4*>(rr)[w];
-      t.x += q.x;
-      t.y += q.y;
-      t.z += q.z;
-      t.w += q.w;
-    }
-    x[0] = t.x;
-    if (N > 1) x[1] = t.y;
-    if (N > 2) x[2] = t.z;
-    if (N > 3) x[3] = t.w;
+    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane < nwarps) q = reinterpret_cast<const float4*>(rr)[lane];
+    const float t = tree4(q.x, q.y, q.z, q.w, lane);
+    x[0] = __shfl_sync(0xffffffffu, t, 0);
+    x[1] = __shfl_sync(0xffffffffu, t, 8);
+    x[2] = __shfl_sync(0xffffffffu, t, 16);
+    x[3] = __shfl_sync(0xffffffffu, t, 24);
     rb ^= 1;
   };
   // One barrier per row (the block reduction's).  Every thread waits for row
@@ -341,7 +352,7 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     for (int m = 0; m < M; ++m) {
       const int64_t base = (r * M + m) * (int64_t)d;
       const int sb = m * d;
-      if (!M1) load_w(m);  // L1-resident after the first rows
+      load_w(m);  // L1-resident after the first rows
       u64 H[4] = {0, 0, 0, 0}, G[4] = {0, 0, 0, 0}, K[4] = {0, 0, 0, 0};
       if (actA) {
         load4<BF16>(hs, sb + cA, H[0], H[1]);
@@ -363,7 +374,7 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
         s3 = sm100::f2_fma(G[p], V[p], s3);
       }
       float sums[4] = {f2sum(s0), f2sum(s1), f2sum(s2), f2sum(s3)};
-      bsum(sums, 4);
+      bsum(sums);
       if (m == 0) {
         if (!*flag) {  // a wait timed out: leave before any store of this row
           stop = true;
