@@ -141,8 +141,10 @@ int ensure_scratch(engram_handle* h, int64_t rows) {
   free_dev(h->e);
   free_dev(h->e_alt);
   free_dev(h->partials);
+  free_dev(h->alpha_scratch);
   h->cap_rows = 0;
   const int64_t key_tiles = (int64_t)h->cfg.branches * h->cfg.d_hidden / 64;
+  CK(h, cudaMalloc(&h->alpha_scratch, (size_t)rows * h->cfg.branches * sizeof(float)));
   CK(h, cudaMalloc(&h->e, (size_t)rows * h->d_mem * h->elt));
   CK(h, cudaMalloc(&h->e_alt, (size_t)rows * h->d_mem * h->elt));
   CK(h, cudaMalloc(&h->partials, (size_t)rows * key_tiles * sizeof(float4)));
@@ -468,6 +470,7 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->e);
   free_dev(h->e_alt);
   free_dev(h->partials);
+  free_dev(h->alpha_scratch);
   free_dev(h->d_w8);
   free_dev(h->d_sw8);
   free_dev(h->bw_idx);
@@ -1138,6 +1141,15 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     if (fp8) g.s_col = h->d_sw8 + (phase == 0 ? 0 : (int64_t)g.M * g.d);
     if (phase == 0) g.key_tile = pc.key_tile;
     if (phase == 1) value_tile = pc.key_tile;
+    if (phase == 1 && !conv && pc.kind != ProjKernel::Wide) {
+      // short calls: alpha is formed once per row between the launches, so
+      // that the value CTAs (many per row block) do not each sum the same
+      // partials after the key launch completes
+      float* adst = alpha ? alpha : h->alpha_scratch;
+      CK(h, launch_row_alpha(g, adst, st));
+      h->launches += 1;
+      g.alpha_in = adst;
+    }
     // values: 3 = v for the short convolution; 2 = in place (out aliases h,
     // alpha v is added into out); 1 = out = h + alpha v
     const int kphase = phase == 0 ? 0 : conv ? 3 : out == hid ? 2 : 1;

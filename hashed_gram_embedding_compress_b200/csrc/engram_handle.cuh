@@ -63,6 +63,7 @@ struct engram_handle {
   void* e_alt = nullptr;
   int e_flip = 0;
   float4* partials = nullptr;
+  float* alpha_scratch = nullptr;  // [rows, M]: alpha formed once per row at short calls
   // short-convolution scratch, sized for conv_cap_rows
   int64_t conv_cap_rows = 0;
   float* conv_v = nullptr;      // [rows, d] v = W_V e

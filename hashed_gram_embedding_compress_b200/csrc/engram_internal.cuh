@@ -86,6 +86,9 @@ struct GateArgs {
   const float* w_qk;    // [M, d]: norm_q * norm_k (the two RMSNorm weights multiply)
   float4* partials;     // [num key tiles][R]: (sum k^2, sum h w_q w_k k, sum h^2, 0)
   float* alpha;         // [R, M] or null
+  // [R, M] alpha already formed from the partial sums (launch_row_alpha), or
+  // null: the value phase forms it itself from `partials`
+  const float* alpha_in;
   float* delta;         // [R, M, d] or null
   float* vals;          // phase 3: v = W_V e, fp32 [R, d]
   float* vv;            // phase 3: sum of v^2 per value tile and row, [d / value tile][R]
@@ -239,6 +242,11 @@ struct ProjMaps {
 };
 cudaError_t launch_proj_gate_sm100(int phase, int bn, const ProjMaps& maps, const GateArgs& g,
                                    int grid, cudaStream_t stream);
+// alpha[R, M] from the key phase's partial sums (g.partials, g.key_tile):
+// the value phase of a short call then reads it instead of every value CTA
+// summing the same partials.  Launched between the key and value launches
+// with programmatic dependent launch when g.pdl.
+cudaError_t launch_row_alpha(const GateArgs& g, float* alpha, cudaStream_t stream);
 // 512 x 256 tiles on CTA pairs (tcgen05 cta_group::2); grid = 2 x pairs.
 // phase 0 keys, 1 values, 2 values added in place (out aliases h), 3 values
 // for the short convolution.  f8: e and W are E4M3 codes (maps of uint8 with

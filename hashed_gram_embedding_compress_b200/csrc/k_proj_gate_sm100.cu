@@ -272,17 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int mb = 0; mb < kMaxBranches; ++mb) {
           al[mb] = 0.f;
           if (mb < M && valid) {
-            float skk = 0.f, shk = 0.f, shh = 0.f;
-            for (int tb = mb * tiles_per_branch; tb < (mb + 1) * tiles_per_branch; ++tb) {
-              const float4 p = g.partials[(int64_t)tb * R + row];
-              skk += p.x;
-              shk += p.y;
-              shh += p.z;
+            if (g.alpha_in) {
+              al[mb] = g.alpha_in[(int64_t)row * M + mb];
+            } else {
+              al[mb] = row_alpha<1>(g.partials, R, row, mb, tiles_per_branch, d, g.eps,
+                                    g.inv_sqrt_d);
+              if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
             }
-            const float rh = 1.0f / sqrtf(shh / (float)d + g.eps);
-            const float rk = 1.0f / sqrtf(skk / (float)d + g.eps);
-            al[mb] = sigmoid_f(shk * rh * rk * g.inv_sqrt_d);
-            if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
           }
         }
       }
@@ -454,7 +450,40 @@ cudaError_t launch_bn(const ProjMaps& maps, const GateArgs& g, int grid, cudaStr
   return cudaGetLastError();
 }
 
+// One thread per (branch, row), rows fastest: the warp's loads of a tile's
+// partials are one coalesced 512-byte read.  Blocks of 128 threads: a short
+// call's blocks then occupy few SMs while they wait for the key launch (more,
+// smaller blocks measured slower: they held SMs the value launch needed).
+__global__ void __launch_bounds__(128) row_alpha_kernel(GateArgs g, float* alpha) {
+  griddep_launch_dependents();  // the value launch may set up and stream its operands
+  griddep_wait();               // the key launch's partial sums are complete
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)g.R * g.M) return;
+  const int mb = (int)(i / g.R);
+  const int64_t row = i - (int64_t)mb * g.R;
+  alpha[row * g.M + mb] = row_alpha<16>(g.partials, g.R, row, mb, g.d / g.key_tile, g.d, g.eps,
+                                        g.inv_sqrt_d);
+}
+
 }  // namespace
+
+cudaError_t launch_row_alpha(const GateArgs& g, float* alpha, cudaStream_t stream) {
+  if (g.R == 0) return cudaSuccess;
+  if (!alpha || g.key_tile <= 0 || g.d % g.key_tile) return cudaErrorInvalidValue;
+  const int64_t n = (int64_t)g.R * g.M;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)((n + 127) / 128));
+  lc.blockDim = dim3(128);
+  lc.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = g.pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&lc, row_alpha_kernel, g, alpha);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 int sm100_stages(int bn) {
   return bn == 256 ? Cfg<256>::STAGES : bn == 128 ? Cfg<128>::STAGES : Cfg<64>::STAGES;

@@ -382,17 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int mb = 0; mb < kMaxBranches; ++mb) {
           al[mb] = 0.f;
           if (mb < M && valid) {
-            float skk = 0.f, shk = 0.f, shh = 0.f;
-            for (int tb = mb * tiles_per_branch; tb < (mb + 1) * tiles_per_branch; ++tb) {
-              const float4 p = g.partials[(int64_t)tb * R + row];
-              skk += p.x;
-              shk += p.y;
-              shh += p.z;
+            if (g.alpha_in) {
+              al[mb] = g.alpha_in[(int64_t)row * M + mb];
+            } else {
+              al[mb] = row_alpha<1>(g.partials, R, row, mb, tiles_per_branch, d, g.eps, g.inv_sqrt_d);
+              if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
             }
-            const float rh = 1.0f / sqrtf(shh / (float)d + g.eps);
-            const float rk = 1.0f / sqrtf(skk / (float)d + g.eps);
-            al[mb] = sigmoid_f(shk * rh * rk * g.inv_sqrt_d);
-            if (g.alpha && n_blk == 0) g.alpha[(int64_t)row * M + mb] = al[mb];
           }
         }
       }

@@ -342,6 +342,55 @@ __device__ __forceinline__ unsigned long long bf16x2_to_f2(uint32_t w) {
 
 __device__ __forceinline__ float sigmoid_f(float s) { return 1.0f / (1.0f + expf(-s)); }
 
+// Sums of the key phase's partials (sum k^2, sum h w k, sum h^2) of one row
+// over tiles [t0, t1) of partials [tiles][R], added in tile order; the loads
+// go out kBatch at a time, so a row of many tiles (several branches at a
+// short call) costs a few memory round trips instead of one per tile.
+template <int kBatch>
+__device__ __forceinline__ void sum_partials(const float4* partials, int64_t R, int64_t row,
+                                             int t0, int t1, float& skk, float& shk, float& shh) {
+  int tb = t0;
+  for (; tb + kBatch <= t1; tb += kBatch) {
+    float4 p[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) p[i] = partials[(int64_t)(tb + i) * R + row];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      skk += p[i].x;
+      shk += p[i].y;
+      shh += p[i].z;
+    }
+  }
+  if (tb < t1) {
+    float4 p[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      if (tb + i < t1) p[i] = partials[(int64_t)(tb + i) * R + row];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      if (tb + i < t1) {
+        skk += p[i].x;
+        shk += p[i].y;
+        shh += p[i].z;
+      }
+  }
+}
+
+// alpha of branch mb of one row (Eq. 4 / Eq. 6) from the key phase's
+// per-tile partial sums: the same arithmetic, in the same order, wherever it
+// is formed.
+template <int kBatch>
+__device__ __forceinline__ float row_alpha(const float4* partials, int64_t R, int64_t row, int mb,
+                                           int tiles_per_branch, int d, float eps,
+                                           float inv_sqrt_d) {
+  float skk = 0.f, shk = 0.f, shh = 0.f;
+  sum_partials<kBatch>(partials, R, row, mb * tiles_per_branch, (mb + 1) * tiles_per_branch, skk,
+                       shk, shh);
+  const float rh = 1.0f / sqrtf(shh / (float)d + eps);
+  const float rk = 1.0f / sqrtf(skk / (float)d + eps);
+  return sigmoid_f(shk * rh * rk * inv_sqrt_d);
+}
+
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
