@@ -1133,11 +1133,29 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
   bool have_single = false, have_wide = false, have_pair = false;
   int value_tile = 0;
   if (fp8) g.s_row = SE8;
+  int key_grid = 0;
   for (int phase = 0; phase < 2; ++phase) {
     const CUtensorMap* wmaps = phase == 0 ? h->map_wk : h->map_wv;
     // the E4M3 operands run on the 512 x 256 CTA-pair kernel only
-    const ProjChoice pc = fp8 ? wide_proj(phase, R, g.M, g.d, h->sms)
-                              : choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv);
+    ProjChoice pc = fp8 ? wide_proj(phase, R, g.M, g.d, h->sms)
+                        : choose_proj(phase, R, g.M, g.d, h->sms, h->cfg.flags, conv);
+    if (phase == 0) key_grid = pc.grid;
+    if (phase == 1 && pc.kind != ProjKernel::Wide && key_grid < h->sms) {
+      // Short calls: the value CTAs stream their operands beside the key
+      // launch, on the SMs that it and the row alpha kernel (whose blocks,
+      // launched before, wait on SMs too) leave free.  A value CTA beyond
+      // those would start only when a key CTA leaves and end the step late,
+      // so the launch takes at most the free SMs, each then taking up to two
+      // tiles (both mainloops run before alpha is ready).
+      const int alpha_blocks = conv ? 0 : (int)((R * g.M + 127) / 128);
+      const int free_sms = h->sms - key_grid - alpha_blocks;
+      const int64_t n_total = g.d;
+      const int64_t tiles = pc.kind == ProjKernel::Pair ? (R + 255) / 256 * (n_total / 256)
+                                                        : (R + 127) / 128 * (n_total / pc.bn);
+      const int unit = pc.kind == ProjKernel::Pair ? 2 : 1;  // CTAs per tile
+      const int cap = free_sms / unit * unit;
+      if (cap >= unit && pc.grid > cap && tiles * unit <= 2 * (int64_t)cap) pc.grid = cap;
+    }
     if (fp8) g.s_col = h->d_sw8 + (phase == 0 ? 0 : (int64_t)g.M * g.d);
     if (phase == 0) g.key_tile = pc.key_tile;
     if (phase == 1) value_tile = pc.key_tile;
