@@ -38,9 +38,11 @@ using sm100::f2_unpack;
 
 constexpr int kTaps = 4;
 
-// x sigmoid(x) with the fast exponential and reciprocal (relative error a few
-// ulp of fp32, far inside the 1e-5 bound of the fp32 path)
-__device__ __forceinline__ float silu_f(float x) { return x * __frcp_rn(1.0f + __expf(-x)); }
+// x sigmoid(x) = x / (1 + e^-x) with the fast exponential and the fast
+// division (a few ulp of fp32, far inside the 1e-5 bound of the fp32 path; a
+// denominator beyond 2^126, x below about -87, gives 0 where the true value
+// is below 1e-36)
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 __device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
   unsigned long long d;
