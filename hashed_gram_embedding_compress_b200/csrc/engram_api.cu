@@ -457,6 +457,7 @@ void engram_destroy(engram_handle* h) {
   cudaDeviceSynchronize();
   free_host_gather(h);  // joins the prefetch threads
   cudaDeviceSynchronize();
+  engram::free_host_io(h);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   for (int i = 0; i < 2; ++i)
     if (h->ev_list[i]) cudaEventDestroy(h->ev_list[i]);

@@ -91,6 +91,17 @@ struct engram_handle {
   int pf_mode = ENGRAM_PREFETCH_HOST_THREADS;
   int pf_workers = 0;                           // 0: the default for the mode
   engram::HostGather* hg = nullptr;             // host-thread route
+  // engram_forward_host: device staging of two calls (so that one call's
+  // host-to-device copies overlap the previous call's device-to-host ones),
+  // the two copy streams and their events
+  void* io_h[2] = {nullptr, nullptr};
+  int32_t* io_tok[2] = {nullptr, nullptr};
+  float* io_alpha[2] = {nullptr, nullptr};
+  size_t io_h_bytes = 0, io_tok_bytes = 0, io_alpha_bytes = 0;
+  cudaStream_t io_in = nullptr, io_out = nullptr;
+  cudaEvent_t io_ev_in[2] = {nullptr, nullptr}, io_ev_comp[2] = {nullptr, nullptr},
+              io_ev_out[2] = {nullptr, nullptr};
+  int io_flip = 0;
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ev_list[2] = {nullptr, nullptr};  // the row list has reached the host
   unsigned long long* h_count[2] = {nullptr, nullptr};  // pinned [2]
@@ -145,6 +156,9 @@ int make_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, i
 // make_map through the handle's cache of recently encoded maps.
 int cached_map(engram_handle* h, CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
                int box_rows, int box_cols = 64, int esz = 2);
+
+// Frees what engram_forward_host allocated (after a device synchronise).
+void free_host_io(engram_handle* h);
 
 // Index into the handle's W tensor maps (map_wk, map_wv) of a box width.
 inline int bn_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : 2; }

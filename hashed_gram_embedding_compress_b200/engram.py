@@ -35,7 +35,8 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_build_hot_cache", "engram_prefetch_hot_hits", "engram_set_fp8",
            "engram_quantize_e4m3", "engram_backward", "engram_profile_next_backward",
            "engram_set_prefetch", "engram_set_table_shards", "engram_ipc_handle",
-           "engram_ipc_open", "engram_ipc_close", "engram_prefetch_wait")
+           "engram_ipc_open", "engram_ipc_close", "engram_prefetch_wait",
+           "engram_forward_host")
 
 
 class engram_config(ctypes.Structure):
@@ -81,6 +82,7 @@ def _load():
         "engram_hash": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
         "engram_forward": ([H, P, P, i32, i32, i32, P, P, P, P, P], ctypes.c_int),
+        "engram_forward_host": ([H, P, i32, i32, i32, P, P, P, P], ctypes.c_int),
         "engram_prefetch": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_set_prefetch": ([H, i32, i32], ctypes.c_int),
         "engram_prefetch_wait": ([H], ctypes.c_int),
@@ -250,6 +252,28 @@ class Engram:
         B, T = tokens.shape
         self._check(lib.engram_forward(self._h, _ptr(tokens), _ptr(idx), B, T, t_begin, _ptr(h),
                                        _ptr(out), _ptr(alpha), _ptr(delta), _stream_ptr(stream)))
+
+    def forward_host(self, tokens, h, out, t_begin=0, alpha=None, stream=None):
+        """The forward from host tensors (tokens int32 [B, T], h and out [rows, M, d],
+        alpha fp32 [rows, M] or None; pinned for overlapped copies): the library
+        stages them on the device and copies the result back; `stream` waits for it."""
+        for name, t in (("tokens", tokens), ("h", h), ("out", out), ("alpha", alpha)):
+            if t is not None and (t.is_cuda or not t.is_contiguous()):
+                raise EngramError(ENGRAM_ERR_INVALID, name + " must be a contiguous host tensor")
+        B, T = tokens.shape
+        rows = B * (T - t_begin)
+        M, d = self.cfg.branches, self.cfg.d_hidden
+        if tuple(h.shape) != (rows, M, d) or tuple(out.shape) != (rows, M, d):
+            raise EngramError(ENGRAM_ERR_INVALID, "h and out must have shape (rows, M, d)")
+        if alpha is not None and tuple(alpha.shape) != (rows, M):
+            raise EngramError(ENGRAM_ERR_INVALID, "alpha must have shape (rows, M)")
+        dt = torch.float32 if self.cfg.dtype == ENGRAM_F32 else torch.bfloat16
+        if (tokens.dtype != torch.int32 or h.dtype != dt or out.dtype != dt
+                or (alpha is not None and alpha.dtype != torch.float32)):
+            raise EngramError(ENGRAM_ERR_INVALID, "dtypes: tokens int32, h and out %s, alpha "
+                              "float32" % dt)
+        self._check(lib.engram_forward_host(self._h, _ptr(tokens), B, T, t_begin, _ptr(h),
+                                            _ptr(out), _ptr(alpha), _stream_ptr(stream)))
 
     def backward(self, tokens, h, dout, dh, dw_k=None, dw_v=None, dnorm_q=None, dnorm_k=None,
                  dtables=None, idx=None, t_begin=0, stream=None):

@@ -322,6 +322,30 @@ ENGRAM_API int engram_forward(engram_handle *h, const int32_t *tokens, const int
                    float *delta, void *stream);
 
 /*
+ * engram_forward from HOST buffers: the call copies tokens and h to device
+ * staging owned by the handle (on an internal stream), runs engram_forward
+ * there in place on `stream`, and copies the result to out (and alpha) on a
+ * second internal stream; `stream` then waits for those copies, so work
+ * issued on it after the call (a synchronise, an event) sees out.  The
+ * handle keeps two stagings and alternates them, so the host-to-device copies
+ * of one call overlap the device-to-host copies of the call before it: a loop
+ * of calls moves both directions over PCIe at once.
+ *  tokens  host int32 [B, T].
+ *  hid     host [rows, M, d] dtype, rows = B*(T-t_begin); read by the call's
+ *          copy, so it must stay unchanged until `stream` passes the call.
+ *  out     host [rows, M, d] dtype (may be hid itself).
+ *  alpha   host fp32 [rows, M] or NULL.
+ * Host buffers should be pinned (cudaHostAlloc / cudaHostRegister); pageable
+ * ones work but their copies do not overlap.  The staging grows on demand
+ * (the call then waits for the handle's earlier copies).  Device-resident
+ * tables, or host tables with a pending engram_prefetch of the same tokens.
+ * Errors: _INVALID, _STATE, _OOM, _CUDA (those of engram_forward included).
+ */
+ENGRAM_API int engram_forward_host(engram_handle *h, const int32_t *tokens, int32_t B, int32_t T,
+                        int32_t t_begin, const void *hid, void *out, float *alpha,
+                        void *stream);
+
+/*
  * Backward of engram_forward (training): the exact derivative of
  * out = h + alpha v (Eq. 3, 4, 6) for a loss whose gradient with respect to
  * out is dout, for the same tokens (or idx) and h.  The pages give only the
