@@ -2,9 +2,9 @@
 //
 // "Conditional Memory via Scalable Lookup", section 2.3 Eq. (3)-(4) and
 // section 2.4 Eq. (6) give the forward; this file holds the hand-written
-// kernels of its exact derivative (the dense contractions, k and v recomputed
-// and the weight and memory-vector gradients, are library GEMMs issued by the
-// ABI layer):
+// kernels of its exact derivative apart from the dense contractions (k and v
+// recomputed, the weight and memory-vector gradients), which run on the
+// CTA-pair tcgen05 GEMM of k_gemm_sm100.cu, issued by the ABI layer:
 //
 //   per row r and branch m, with k = W_K^(m) e, v = W_V e,
 //   rh = (mean(h^2) + eps)^-1/2, rk likewise, qn = h rh w_q, kn = k rk w_k,
@@ -15,13 +15,14 @@
 //     u_q = dqn w_q:  dh = dout + rh u_q - rh^3 / d h (u_q . h),
 //     u_k = dkn w_k:  dk = rk u_k - rk^3 / d k (u_k . k).
 //
-// gate_backward_ring_kernel: a CTA of 256 threads per row at a time
+// gate_backward_ring_kernel: a CTA of d / 8 threads per row at a time
 // (grid-stride, two CTAs per SM); thread 0 streams the rows' h, dout and kv
 // into a ring of three shared-memory slots with bulk copies two rows ahead,
 // so the loads of the next rows overlap the reductions of the current one.
-// The two row reductions per branch are block reductions.  dw_q and dw_k are
-// summed per CTA in shared memory (each thread owns its columns) and reduced
-// over the CTAs in a fixed order by dnorm_reduce_kernel (deterministic).
+// One block reduction (of four sums) and one barrier per branch and row.
+// dw_q and dw_k are summed per CTA (in registers with one branch, else in
+// shared memory; each thread owns its columns) and reduced over the CTAs in a
+// fixed order by dnorm_reduce_kernel (deterministic).
 // gate_backward_kernel is the same arithmetic with the row in registers and
 // no ring, for rows too long for three slots.
 // table_grad_kernel adds the slices of de into fp32 table gradients.
