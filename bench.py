@@ -597,16 +597,12 @@ def run_backward_bench(args, rank, world, dist):
     h_h, g_h = h.cpu().pin_memory(), dout.cpu().pin_memory()
     dh_h = torch.empty_like(h_h).pin_memory()
     tok_h = P["tokens"].pin_memory()
-    tok_b, h_b, g_b = torch.empty_like(tok_d), torch.empty_like(h), torch.empty_like(dout)
 
     def e2e_step():
-        tok_b.copy_(tok_h, non_blocking=True)
-        h_b.copy_(h_h, non_blocking=True)
-        g_b.copy_(g_h, non_blocking=True)
-        m.backward(tok_b, h_b, g_b, dh, t_begin=sh.t_begin, stream=stream, **g)
+        # through the host-buffer entry point (tokens, h, dout in; dh back)
+        m.backward_host(tok_h, h_h, g_h, dh_h, t_begin=sh.t_begin, stream=stream, **g)
         if dist:
             dp.all_reduce_dense([g["dw_k"], g["dw_v"], g["dnorm_q"], g["dnorm_k"]])
-        dh_h.copy_(dh, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -652,7 +648,9 @@ def run_backward_bench(args, rank, world, dist):
                       "weight_grads": st[3], "de_and_table_grads": st[4]},
         "e2e": {"value": R * world * E / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": tok_h.numel() * 4 + 2 * h_h.numel() * h_h.element_size(),
-                "d2h_bytes_per_step": dh_h.numel() * dh_h.element_size(), "steps": E},
+                "d2h_bytes_per_step": dh_h.numel() * dh_h.element_size(), "steps": E,
+                "path": "engram_backward_host: C ABI call on pinned host buffers (tokens, h, "
+                        "dL/dout in; dh back), copies inside the timed region"},
         "gpu_launches": launches,
         "clocks": dict(clk.summary(t_load + 0.5, t_end + 0.15),
                        window="last 1 s of back-to-back warm-up steps and the timed steps"),

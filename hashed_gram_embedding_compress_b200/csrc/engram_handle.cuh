@@ -102,6 +102,12 @@ struct engram_handle {
   cudaEvent_t io_ev_in[2] = {nullptr, nullptr}, io_ev_comp[2] = {nullptr, nullptr},
               io_ev_out[2] = {nullptr, nullptr};
   int io_flip = 0;
+  // engram_backward_host: h, dout and dh of two calls
+  void* bio_h[2] = {nullptr, nullptr};
+  void* bio_dout[2] = {nullptr, nullptr};
+  void* bio_dh[2] = {nullptr, nullptr};
+  int32_t* bio_tok[2] = {nullptr, nullptr};
+  size_t bio_bytes = 0, bio_tok_bytes = 0;
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ev_list[2] = {nullptr, nullptr};  // the row list has reached the host
   unsigned long long* h_count[2] = {nullptr, nullptr};  // pinned [2]

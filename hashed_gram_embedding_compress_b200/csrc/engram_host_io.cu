@@ -83,9 +83,50 @@ int ensure_io(engram_handle* h, size_t h_bytes, size_t tok_bytes, size_t alpha_b
   return ENGRAM_OK;
 }
 
+// The backward's stagings (h, dout, dh of rows x M x d; tokens), grown as
+// ensure_io grows the forward's.
+int ensure_bio(engram_handle* h, size_t bytes, size_t tok_bytes) {
+  int rc = ensure_io(h, 0, 0, 0);  // streams and events
+  if (rc) return rc;
+  if (bytes > h->bio_bytes || tok_bytes > h->bio_tok_bytes) {
+    IO_CK(h, cudaStreamSynchronize(h->io_in));
+    IO_CK(h, cudaStreamSynchronize(h->io_out));
+    if (bytes > h->bio_bytes) {
+      h->bio_bytes = 0;
+      for (int i = 0; i < 2; ++i) {
+        for (void** b : {&h->bio_h[i], &h->bio_dout[i], &h->bio_dh[i]}) {
+          cudaFree(*b);
+          *b = nullptr;
+          IO_CK(h, cudaMalloc(b, bytes));
+        }
+      }
+      h->bio_bytes = bytes;
+    }
+    if (tok_bytes > h->bio_tok_bytes) {
+      h->bio_tok_bytes = 0;
+      for (int i = 0; i < 2; ++i) {
+        cudaFree(h->bio_tok[i]);
+        h->bio_tok[i] = nullptr;
+        IO_CK(h, cudaMalloc(&h->bio_tok[i], tok_bytes));
+      }
+      h->bio_tok_bytes = tok_bytes;
+    }
+  }
+  return ENGRAM_OK;
+}
+
 }  // namespace
 
 void free_host_io(engram_handle* h) {
+  for (int i = 0; i < 2; ++i) {
+    for (void** b : {&h->bio_h[i], &h->bio_dout[i], &h->bio_dh[i]}) {
+      cudaFree(*b);
+      *b = nullptr;
+    }
+    cudaFree(h->bio_tok[i]);
+    h->bio_tok[i] = nullptr;
+  }
+  h->bio_bytes = h->bio_tok_bytes = 0;
   for (int i = 0; i < 2; ++i) {
     cudaFree(h->io_h[i]);
     cudaFree(h->io_tok[i]);
@@ -143,6 +184,45 @@ int engram_forward_host(engram_handle* h, const int32_t* tokens, int32_t B, int3
                              h->io_out));
   IO_CK(h, cudaEventRecord(h->io_ev_out[slot], h->io_out));
   // work after this call on `stream` sees out (and alpha)
+  IO_CK(h, cudaStreamWaitEvent(st, h->io_ev_out[slot], 0));
+  return ENGRAM_OK;
+}
+
+int engram_backward_host(engram_handle* h, const int32_t* tokens, int32_t B, int32_t T,
+                         int32_t t_begin, const void* hid, const void* dout, void* dhid,
+                         float* dw_k, float* dw_v, float* dnorm_q, float* dnorm_k,
+                         float* const* dtables, void* stream) {
+  using namespace engram;
+  if (!h) return ENGRAM_ERR_INVALID;
+  if (!tokens || !hid || !dout || !dhid)
+    return io_fail(h, ENGRAM_ERR_INVALID,
+                   "engram_backward_host: tokens, h, dout and dh must be non-null");
+  if (B < 0 || T <= 0 || t_begin < 0 || t_begin >= T)
+    return io_fail(h, ENGRAM_ERR_INVALID, "engram_backward_host: need B >= 0 and 0 <= t_begin < T");
+  const int64_t R = (int64_t)B * (T - t_begin);
+  if (R == 0) return ENGRAM_OK;
+  const size_t bytes = (size_t)R * h->cfg.branches * h->cfg.d_hidden * h->elt;
+  const size_t tok_bytes = (size_t)B * T * sizeof(int32_t);
+  int rc = ensure_bio(h, bytes, tok_bytes);
+  if (rc) return rc;
+  const int slot = h->io_flip;
+  h->io_flip ^= 1;
+  cudaStream_t st = (cudaStream_t)stream;
+  IO_CK(h, cudaStreamWaitEvent(h->io_in, h->io_ev_out[slot], 0));
+  IO_CK(h, cudaMemcpyAsync(h->bio_tok[slot], tokens, tok_bytes, cudaMemcpyHostToDevice, h->io_in));
+  IO_CK(h, cudaMemcpyAsync(h->bio_h[slot], hid, bytes, cudaMemcpyHostToDevice, h->io_in));
+  IO_CK(h, cudaMemcpyAsync(h->bio_dout[slot], dout, bytes, cudaMemcpyHostToDevice, h->io_in));
+  IO_CK(h, cudaEventRecord(h->io_ev_in[slot], h->io_in));
+  IO_CK(h, cudaStreamWaitEvent(st, h->io_ev_in[slot], 0));
+  rc = engram_backward(h, h->bio_tok[slot], nullptr, B, T, t_begin, h->bio_h[slot],
+                       h->bio_dout[slot], h->bio_dh[slot], dw_k, dw_v, dnorm_q, dnorm_k, dtables,
+                       stream);
+  if (rc) return rc;
+  IO_CK(h, cudaEventRecord(h->io_ev_comp[slot], st));
+  IO_CK(h, cudaStreamWaitEvent(h->io_out, h->io_ev_comp[slot], 0));
+  IO_CK(h, cudaMemcpyAsync(dhid, h->bio_dh[slot], bytes, cudaMemcpyDeviceToHost, h->io_out));
+  IO_CK(h, cudaEventRecord(h->io_ev_out[slot], h->io_out));
+  // work after this call on `stream` sees dh
   IO_CK(h, cudaStreamWaitEvent(st, h->io_ev_out[slot], 0));
   return ENGRAM_OK;
 }

@@ -36,7 +36,7 @@ EXPORTS = ("engram_create", "engram_destroy", "engram_config_size", "engram_last
            "engram_quantize_e4m3", "engram_backward", "engram_profile_next_backward",
            "engram_set_prefetch", "engram_set_table_shards", "engram_ipc_handle",
            "engram_ipc_open", "engram_ipc_close", "engram_prefetch_wait",
-           "engram_forward_host")
+           "engram_forward_host", "engram_backward_host")
 
 
 class engram_config(ctypes.Structure):
@@ -83,6 +83,8 @@ def _load():
         "engram_gather": ([H, P, i64, P, P], ctypes.c_int),
         "engram_forward": ([H, P, P, i32, i32, i32, P, P, P, P, P], ctypes.c_int),
         "engram_forward_host": ([H, P, i32, i32, i32, P, P, P, P], ctypes.c_int),
+        "engram_backward_host": ([H, P, i32, i32, i32, P, P, P, P, P, P, P, P, P],
+                                 ctypes.c_int),
         "engram_prefetch": ([H, P, i32, i32, i32, P, P], ctypes.c_int),
         "engram_set_prefetch": ([H, i32, i32], ctypes.c_int),
         "engram_prefetch_wait": ([H], ctypes.c_int),
@@ -288,6 +290,31 @@ class Engram:
         self._check(lib.engram_backward(self._h, _ptr(tokens), _ptr(idx), B, T, t_begin, _ptr(h),
                                         _ptr(dout), _ptr(dh), _ptr(dw_k), _ptr(dw_v),
                                         _ptr(dnorm_q), _ptr(dnorm_k), arr, _stream_ptr(stream)))
+
+    def backward_host(self, tokens, h, dout, dh, dw_k=None, dw_v=None, dnorm_q=None,
+                      dnorm_k=None, dtables=None, t_begin=0, stream=None):
+        """The backward from host tensors (tokens, h, dout in; dh out; pinned for
+        overlapped copies); the weight and table gradients stay device tensors."""
+        for name, t in (("tokens", tokens), ("h", h), ("dout", dout), ("dh", dh)):
+            if t.is_cuda or not t.is_contiguous():
+                raise EngramError(ENGRAM_ERR_INVALID, name + " must be a contiguous host tensor")
+        B, T = tokens.shape
+        rows = B * (T - t_begin)
+        M, d = self.cfg.branches, self.cfg.d_hidden
+        dt = torch.float32 if self.cfg.dtype == ENGRAM_F32 else torch.bfloat16
+        for name, t in (("h", h), ("dout", dout), ("dh", dh)):
+            if tuple(t.shape) != (rows, M, d) or t.dtype != dt:
+                raise EngramError(ENGRAM_ERR_INVALID, "%s must be %s of shape (rows, M, d)" % (name, dt))
+        if tokens.dtype != torch.int32:
+            raise EngramError(ENGRAM_ERR_INVALID, "tokens must be int32")
+        arr = None
+        if dtables is not None:
+            arr = ctypes.cast((ctypes.c_void_p * len(dtables))(*[t.data_ptr() for t in dtables]),
+                              ctypes.c_void_p)
+        self._check(lib.engram_backward_host(self._h, _ptr(tokens), B, T, t_begin, _ptr(h),
+                                             _ptr(dout), _ptr(dh), _ptr(dw_k), _ptr(dw_v),
+                                             _ptr(dnorm_q), _ptr(dnorm_k), arr,
+                                             _stream_ptr(stream)))
 
     def prefetch(self, tokens, t_begin=0, stream=None, want_count=False):
         B, T = tokens.shape

@@ -391,6 +391,24 @@ ENGRAM_API int engram_backward(engram_handle *h, const int32_t *tokens, const in
                                void *stream);
 
 /*
+ * engram_backward from HOST buffers, as engram_forward_host is to
+ * engram_forward: tokens, h and dout are copied to device staging owned by
+ * the handle (internal stream), the backward runs there on `stream`, and dh is
+ * copied back (second internal stream); `stream` then waits for that copy.
+ * Consecutive calls alternate two stagings, so one call's copies in overlap
+ * the previous call's copy out.
+ *  tokens, hid, dout  host, as engram_backward's device arguments; read by the
+ *                     call's copies, unchanged until `stream` passes the call.
+ *  dhid               host [rows, M, d] dtype.
+ *  dw_k, dw_v, dnorm_q, dnorm_k, dtables  DEVICE buffers, as engram_backward.
+ * Host buffers should be pinned.  Errors: those of engram_backward.
+ */
+ENGRAM_API int engram_backward_host(engram_handle *h, const int32_t *tokens, int32_t B, int32_t T,
+                         int32_t t_begin, const void *hid, const void *dout, void *dhid,
+                         float *dw_k, float *dw_v, float *dnorm_q, float *dnorm_k,
+                         float *const *dtables, void *stream);
+
+/*
  * Deterministic prefetch for host-resident tables (section 2.5, Figure 2b):
  * hash the tokens of an upcoming step, de-duplicate the addressed rows per
  * table, and copy each distinct row once from pinned host memory over PCIe

@@ -83,3 +83,28 @@ def test_host_buffers_reject_device_tensors_and_bad_shapes():
     with pytest.raises(eg.EngramError) as ei:
         m.forward_host(p.tokens, p.h.cpu().float(), torch.empty_like(p.h).cpu().float())
     assert ei.value.code == eg.ENGRAM_ERR_INVALID
+
+
+def test_backward_host_buffers_equal_device_backward():
+    """engram_backward_host: h and dout in, dh out through host buffers, two
+    calls back to back; dh equal to the device-buffer backward bit for bit and
+    the weight gradients accumulated once per call."""
+    p = Problem(SHAPE)
+    sh = p.shape
+    M, d, dm = sh.branches, sh.d_hidden, sh.d_mem
+    m = p.engram()
+    dout = synth.make_grad_out(sh, p.seeds, device="cpu")
+    tok_h, h_h, g_h = p.tokens.pin_memory(), p.h.cpu().pin_memory(), dout.pin_memory()
+    dh1, dh2 = torch.empty_like(h_h).pin_memory(), torch.empty_like(h_h).pin_memory()
+    dw_v = torch.zeros((d, dm), device="cuda")
+    m.backward_host(tok_h, h_h, g_h, dh1, dw_v=dw_v)
+    m.backward_host(tok_h, h_h, g_h, dh2, dw_v=dw_v)
+    torch.cuda.synchronize()
+    assert m.check_errors() == 0
+    ref = torch.empty_like(p.h)
+    dw_ref = torch.zeros((d, dm), device="cuda")
+    m.backward(p.tokens.cuda(), p.h, dout.cuda(), ref, dw_v=dw_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(dh1, ref.cpu()) and torch.equal(dh2, ref.cpu())
+    # two accumulations of the same gradient (the contraction's order may vary in the last bits)
+    assert rel_l2((dw_v / 2).double().cpu(), dw_ref.double().cpu()) < 1e-6
