@@ -257,9 +257,10 @@ def step_roofline(A, ms_step, hbm_gbs, tflops):
             "peak_tflops": tflops, "peak_gbs": hbm_gbs}
 
 
-def kernel_traffic(name="traffic.json"):
-    """DRAM bytes per step of the projection kernel (key + value launches)
-    from a committed ncu capture, or None once its source has changed."""
+def kernel_traffic(name="traffic.json", key="proj_gate_bytes_per_step"):
+    """DRAM bytes from a committed ncu capture (by default those of the
+    projection kernel's key + value launches per step), or None once the
+    captured kernel's source has changed."""
     p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
@@ -269,7 +270,7 @@ def kernel_traffic(name="traffic.json"):
         h.update(open(os.path.join(ROOT, f), "rb").read())
     if d.get("source_sha256_16") != h.hexdigest()[:16]:
         return None
-    return d.get("proj_gate_bytes_per_step")
+    return d.get(key)
 
 
 def max_over_ranks(x: float, dist, device) -> float:
@@ -429,7 +430,12 @@ def run_ours(args, rank, world, dist):
     gemm_s = (st_mean[2] + st_mean[3]) / 1e3
     gemm_tflops = A["gemm_flops"] / gemm_s / 1e12
     fused = sh.table_location == "device"  # one hash + gather kernel: its time is stage 1
-    gather_gbs = A["gather_bytes"] / ((st_mean[0] + st_mean[1] if fused else st_mean[1]) / 1e3) / 1e9
+    gather_s = (st_mean[0] + st_mean[1] if fused else st_mean[1]) / 1e3
+    gather_gbs = A["gather_bytes"] / gather_s / 1e9
+    # the DRAM bytes the fused kernel moves in the step (row over-fetch and the
+    # write-back of the value launch's dirty h included), from an ncu capture
+    gather_traffic = (kernel_traffic("traffic_gather.json", "dram_bytes_per_launch")
+                      if fused and not args.fp8 and args.workload == WORKLOAD else None)
     traffic = None if args.fp8 else kernel_traffic()
     res = {
         "metric": METRIC,
@@ -477,6 +483,9 @@ def run_ours(args, rank, world, dist):
             "frac_of_hbm": gather_gbs / hbm,
             "peak_gbs": hbm,
             "bytes_per_step": A["gather_bytes"],
+            "traffic": gather_traffic,
+            "traffic_frac_of_hbm": (gather_traffic / gather_s / 1e9 / hbm
+                                    if gather_traffic else None),
         },
         "stages_ms": ({"hash_gather": st_mean[0] + st_mean[1]} if fused else
                       {"hash": st_mean[0], "gather": st_mean[1]}) |
