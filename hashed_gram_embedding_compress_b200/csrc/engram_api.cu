@@ -1213,7 +1213,8 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
       if (!have_single) {
         if ((rc = cached_map(h, &single.e, E, h->d_mem, R, 128))) return rc;
         if ((rc = cached_map(h, &single.h, hid, hcols, R, 128))) return rc;
-        if ((rc = cached_map(h, &single.out, out, hcols, R, 128))) return rc;
+        // the value epilogue stores per warp: 32-row boxes
+        if ((rc = cached_map(h, &single.out, out, hcols, R, 32))) return rc;
         have_single = true;
       }
       single.w = wmaps[bn_index(pc.bn)];

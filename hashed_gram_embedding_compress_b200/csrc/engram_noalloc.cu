@@ -162,7 +162,7 @@ extern "C" int engram_project_gate_noalloc(engram_handle* h, const void* e, int6
       if (!have_single) {
         if ((rc = make_map(h, &single.e, e, h->d_mem, R, 128, 64)) ||
             (rc = make_map(h, &single.h, hid, hcols, R, 128, 64)) ||
-            (rc = make_map(h, &single.out, out, hcols, R, 128, 64)))
+            (rc = make_map(h, &single.out, out, hcols, R, 32, 64)))
           return rc;
         have_single = true;
       }

@@ -28,7 +28,7 @@
 //   warps 0-3   epilogue: tcgen05.ld 32 columns at a time (warp w owns TMEM
 //               lanes 32w..32w+31, i.e. rows of the tile), fused gate math
 //               against h in shared memory; the value phase writes out over h
-//               in place and stores it with TMA.
+//               in place and each warp stores its 32 rows with TMA.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel records
 // kDevErrTimeout, every role leaves its loop, outstanding MMAs are drained and
 // TMEM is freed before the CTA exits.
@@ -57,7 +57,7 @@ struct Cfg {
                                     ? 8
                                     : ((229376 - H_SLOTS * H_BYTES) / STAGE_BYTES);
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 3 * H_SLOTS + 1;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * H_SLOTS + 1;
   static constexpr uint32_t BAR_BYTES = 8 * NUM_BARS + 16;
   static constexpr size_t SMEM =
       1024 + (size_t)STAGES * STAGE_BYTES + (size_t)H_SLOTS * H_BYTES + BAR_BYTES;
@@ -88,8 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   auto hfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + s); };
   auto hempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + H_SLOTS + s); };
-  auto hdone_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + 2 * H_SLOTS + s); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4 + 3 * H_SLOTS);
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4 + 2 * H_SLOTS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -114,8 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < H_SLOTS; ++s) {
       mbar_init(hfull_bar(s), 1);
-      mbar_init(hempty_bar(s), PHASE == 0 ? 4 : 1);
-      mbar_init(hdone_bar(s), 4);
+      mbar_init(hempty_bar(s), 4);  // every epilogue warp releases its rows
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -255,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Thread (warp w, lane l) owns tile row r = 32w + l: TMEM lane r and
     // row r of every h sub-tile in shared memory.
     const int r = warp * 32 + lane;
-    int pending = -1;  // value phase, warp 0: slot whose TMA store may still read it
+    int pending = -1;  // value phase: slot whose TMA store (this warp's rows) may still read it
     int acc = 0, hslot = 0;
     uint32_t acc_phase = 0, hphase = 0;
     bool ok = true;
@@ -381,22 +379,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_async_smem();  // generic-proxy writes -> visible to the TMA store
             __syncwarp();
-            if (lane == 0) mbar_arrive(hdone_bar(hslot));
-            if (warp == 0) {
-              if (lane == 0) {
-                ok = wait_ready(hdone_bar(hslot), hphase, abort_flag, g.err);
-                if (ok) {
-                  tma_store_2d(&map_out, sH + hslot * H_BYTES, mb * d + n0 + q * 64, m_blk * BM);
-                  // hand back the previous slot once its store has read it;
-                  // this one stays with its store in flight
-                  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                  if (pending >= 0) mbar_arrive(hempty_bar(pending));
-                  pending = hslot;
-                }
-              }
-              ok = __shfl_sync(0xffffffffu, ok, 0);
-              if (!ok) break;
+            if (lane == 0) {
+              // this warp's 32 rows of the slot (map_out has 32-row boxes;
+              // rows past R are clipped, a warp with none commits an empty
+              // group), then hand back the previous slot once this warp's
+              // store of it has read it
+              if (m_blk * BM + warp * 32 < R)
+                tma_store_2d(&map_out, sH + hslot * H_BYTES + warp * 32 * 128,
+                             mb * d + n0 + q * 64, m_blk * BM + warp * 32);
+              else
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+              asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+              if (pending >= 0) mbar_arrive(hempty_bar(pending));
             }
+            pending = hslot;
             if (++hslot == H_SLOTS) {
               hslot = 0;
               hphase ^= 1u;
@@ -414,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
-    if (PHASE == 1 && warp == 0 && lane == 0) {
+    if (PHASE == 1 && lane == 0) {
       asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
       if (pending >= 0 && ok) mbar_arrive(hempty_bar(pending));
     }
