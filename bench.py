@@ -462,7 +462,11 @@ def run_ours(args, rank, world, dist):
             "cuda_graph": bool(graph is not None),
         },
         "roofline": {
-            "kernel": "proj_gate_wide_kernel: key + in-place value launches per step (tcgen05, CTA pairs)",
+            "kernel": ("proj_gate_pair_kernel (keys, 256 x 256 CTA-pair tiles) + row_alpha_kernel "
+                       "+ proj_gate_kernel (values, 128 x 64 single-CTA tiles), tcgen05"
+                       if sh.rows_out <= 4096 else
+                       "proj_gate_wide_kernel: key + in-place value launches per step (tcgen05, "
+                       "CTA pairs)"),
             "bound": "tensor",
             "achieved": gemm_tflops,
             "peak": tflops_burst,
