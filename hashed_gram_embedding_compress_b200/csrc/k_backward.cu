@@ -237,12 +237,20 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
   const size_t slot_bytes = ring_slot_bytes(M, d, elt);
   unsigned char* ring = smraw;
   float* red = reinterpret_cast<float*>(ring + kRing * slot_bytes);   // [2][32 warps][4]
-  float* s_dwq = red + 256;                                          // [M][d] (M > 1)
-  float* s_dwk = s_dwq + (int64_t)M * d;                             // [M][d]
+  // M > 1: the weight-gradient sums [M][d] each; one branch (sums in
+  // registers): the RMSNorm weights w_q, w_k [d] each, read there every row
+  float* s_dwq = red + 256;
+  float* s_dwk = s_dwq + (int64_t)M * d;
   uint64_t* full = reinterpret_cast<uint64_t*>(s_dwk + (int64_t)M * d);  // [kRing]
   volatile int* flag = reinterpret_cast<volatile int*>(full + kRing);
-  if (!M1)
+  if (!M1) {
     for (int64_t i = tid; i < 2LL * M * d; i += T) s_dwq[i] = 0.f;
+  } else {
+    for (int i = tid; i < d; i += T) {
+      s_dwq[i] = __ldg(a.w_q + i);
+      s_dwk[i] = __ldg(a.w_k + i);
+    }
+  }
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) sm100::mbar_init(sm100::smem_u32(full + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -252,6 +260,17 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
   // stay in registers
   u64 WQ[4] = {0, 0, 0, 0}, WK[4] = {0, 0, 0, 0}, DQ[4] = {0, 0, 0, 0}, DK[4] = {0, 0, 0, 0};
   auto load_w = [&](int m) {
+    if (M1) {  // from shared memory (two CTAs' rows and the ring leave little L1)
+      if (actA) {
+        load4f(s_dwq + cA, WQ[0], WQ[1]);
+        load4f(s_dwk + cA, WK[0], WK[1]);
+      }
+      if (actB) {
+        load4f(s_dwq + cB, WQ[2], WQ[3]);
+        load4f(s_dwk + cB, WK[2], WK[3]);
+      }
+      return;
+    }
     if (actA) {
       ldg4f(a.w_q + m * d + cA, WQ[0], WQ[1]);
       ldg4f(a.w_k + m * d + cA, WK[0], WK[1]);
@@ -353,7 +372,7 @@ __global__ void __maxnreg__(96) gate_backward_ring_kernel(GateBwArgs a) {
     for (int m = 0; m < M; ++m) {
       const int64_t base = (r * M + m) * (int64_t)d;
       const int sb = m * d;
-      load_w(m);  // L1-resident after the first rows
+      load_w(m);  // shared memory with one branch, else L1
       u64 H[4] = {0, 0, 0, 0}, G[4] = {0, 0, 0, 0}, K[4] = {0, 0, 0, 0};
       if (actA) {
         load4<BF16>(hs, sb + cA, H[0], H[1]);
