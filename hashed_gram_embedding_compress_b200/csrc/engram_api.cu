@@ -137,6 +137,14 @@ namespace {
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 int ensure_scratch(engram_handle* h, int64_t rows) {
+  if (!h->fused_sync && h->cfg.dtype == ENGRAM_BF16 && h->cfg.d_hidden % 256 == 0) {
+    // the fused short-call kernel's counters (zero before its first launch,
+    // zeroed again by every launch on its way out) and its v hand-off buffer
+    CK(h, cudaMalloc(&h->fused_vt, (size_t)h->cfg.d_hidden * 256 * sizeof(float)));
+    CK(h, cudaMalloc(&h->fused_sync, engram::kFusedSyncWords * sizeof(unsigned)));
+    CK(h, cudaMemset(h->fused_sync, 0, engram::kFusedSyncWords * sizeof(unsigned)));
+    CK(h, cudaDeviceSynchronize());
+  }
   if (rows <= h->cap_rows) return ENGRAM_OK;
   free_dev(h->e);
   free_dev(h->e_alt);
@@ -370,7 +378,8 @@ int engram_create(const engram_config* cfg, engram_handle** out) {
   if (c.table_location != ENGRAM_DEVICE && c.table_location != ENGRAM_PINNED_HOST)
     return fail(nullptr, ENGRAM_ERR_INVALID, "bad table_location");
   if (c.pad_id < -1) return fail(nullptr, ENGRAM_ERR_INVALID, "pad_id must be >= -1");
-  if (c.flags & ~ENGRAM_FLAG_NO_CTA_PAIRS) return fail(nullptr, ENGRAM_ERR_INVALID, "unknown flags");
+  if (c.flags & ~(ENGRAM_FLAG_NO_CTA_PAIRS | ENGRAM_FLAG_NO_FUSED_SHORT))
+    return fail(nullptr, ENGRAM_ERR_INVALID, "unknown flags");
   const int S = c.num_orders * c.heads;
   const int64_t d_mem = (int64_t)S * c.d_head;
   if (d_mem > (1 << 20)) return fail(nullptr, ENGRAM_ERR_INVALID, "d_mem too large");
@@ -472,6 +481,8 @@ void engram_destroy(engram_handle* h) {
   free_dev(h->e_alt);
   free_dev(h->partials);
   free_dev(h->alpha_scratch);
+  free_dev(h->fused_sync);
+  free_dev(h->fused_vt);
   free_dev(h->d_w8);
   free_dev(h->d_sw8);
   free_dev(h->bw_idx);
@@ -954,6 +965,25 @@ int engram_prefetch(engram_handle* h, const int32_t* tokens, int32_t B, int32_t 
   return ENGRAM_OK;
 }
 
+namespace {
+
+// Whether a bf16 call of R rows takes the one-launch short-call kernel: at
+// most 256 rows, d a multiple of 256, at most four branches, CTA pairs
+// allowed, and all nkey + nval clusters resident at once.
+bool use_fused(engram_handle* h, int64_t R, int* nkey, int* nval) {
+  const int M = h->cfg.branches, d = h->cfg.d_hidden;
+  if (h->cfg.dtype != ENGRAM_BF16 || R > 256 || M > engram::kMaxBranches || d % 256 != 0)
+    return false;
+  if (h->cfg.flags & (ENGRAM_FLAG_NO_CTA_PAIRS | ENGRAM_FLAG_NO_FUSED_SHORT)) return false;
+  if (!h->fused_sync) return false;
+  if (h->fused_clusters < 0) h->fused_clusters = engram::fused_max_clusters();
+  *nkey = M * d / 256;
+  *nval = d / 128;
+  return *nkey + *nval <= h->fused_clusters;
+}
+
+}  // namespace
+
 int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, int32_t B,
                    int32_t T, int32_t t_begin, const void* hid, void* out, float* alpha,
                    float* delta, void* stream) {
@@ -1126,10 +1156,30 @@ int engram_forward(engram_handle* h, const int32_t* tokens, const int64_t* idx, 
     CK(h, mark(5));
     return ENGRAM_OK;
   }
+  const int64_t hcols = (int64_t)g.M * g.d;
+  int nkey = 0, nval = 0;
+  if (!conv && !fp8 && use_fused(h, R, &nkey, &nval)) {
+    // Short calls: keys, alpha and values in one launch, the value CTAs
+    // taking alpha from the key CTAs' partial sums through counters
+    FusedMaps fm;
+    if ((rc = cached_map(h, &fm.e, E, h->d_mem, R, 128))) return rc;
+    if ((rc = cached_map(h, &fm.h, hid, hcols, R, 128, 32))) return rc;
+    if ((rc = cached_map(h, &fm.out, out, hcols, R, 32, 32))) return rc;  // per-warp boxes
+    fm.wk = h->map_wk[bn_index(128)];  // each CTA of a key pair: 128 of the tile's 256 W rows
+    fm.wv = h->map_wv[bn_index(64)];   // each CTA of a value pair: 64 of 128
+    g.key_tile = 128;
+    g.sync = h->fused_sync;
+    g.vt = h->fused_vt;
+    CK(h, launch_proj_gate_fused(fm, g, nkey, nval, st));
+    h->launches += 1;
+    CK(h, mark(3));
+    CK(h, mark(4));
+    CK(h, mark(5));
+    return ENGRAM_OK;
+  }
   // Tensor maps are built for whichever kernel each phase uses (choose_proj):
   // 512 x 256 tiles on CTA pairs when the tile count fills every pair at least
   // once, else 256 x 256 pair tiles or single-CTA 128-row tiles by cost.
-  const int64_t hcols = (int64_t)g.M * g.d;
   ProjMaps single, wide, pair;
   bool have_single = false, have_wide = false, have_pair = false;
   int value_tile = 0;

@@ -64,6 +64,9 @@ struct engram_handle {
   int e_flip = 0;
   float4* partials = nullptr;
   float* alpha_scratch = nullptr;  // [rows, M]: alpha formed once per row at short calls
+  unsigned* fused_sync = nullptr;  // counters of the one-launch short-call kernel
+  float* fused_vt = nullptr;       // its v hand-off buffer, d x 256 fp32
+  int fused_clusters = -1;         // its clusters resident at once (-1: not yet asked)
   // short-convolution scratch, sized for conv_cap_rows
   int64_t conv_cap_rows = 0;
   float* conv_v = nullptr;      // [rows, d] v = W_V e

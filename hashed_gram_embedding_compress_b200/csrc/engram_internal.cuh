@@ -99,6 +99,10 @@ struct GateArgs {
   int32_t key_tile;     // width of the key-phase tiles that wrote `partials`
   float eps;
   float inv_sqrt_d;
+  // one launch for steps 5-7 of a short call (launch_proj_gate_fused): [0],
+  // [1] key CTAs done per 128-row half, [2] CTAs done; zero between launches
+  unsigned* sync;
+  float* vt;            // fused short-call kernel: v handed to the key CTAs, [d / 4][256][4]
   // 1: launch with programmatic dependent launch.  The key phase then waits
   // for the previous kernel (the gather) before reading e and lets the value
   // phase start early; the value phase's epilogue waits for the key phase
@@ -259,6 +263,26 @@ cudaError_t launch_proj_gate_wide(int phase, const ProjMaps& maps, const GateArg
 // 128 in phase 0).  Phases 0-2 as above.
 cudaError_t launch_proj_gate_pair(int phase, const ProjMaps& maps, const GateArgs& g, int grid,
                                   cudaStream_t stream);
+
+// Steps 5-7 of a short call (R <= 256, bf16, d a multiple of 256, M <= 4) in
+// one launch of nkey = M d / 256 key clusters and nval = d / 128 value
+// clusters (CTA pairs); out = h + alpha v (out may alias h); g.partials,
+// g.sync (kFusedSyncWords, zeroed), g.vt (d x 256 fp32), g.alpha and g.delta
+// as for the other kernels.  Every CTA must be resident at once: 2 (nkey +
+// nval) CTAs at one per SM, nkey + nval <= fused_max_clusters().
+constexpr int kFusedSyncWords = 16;
+struct FusedMaps {
+  CUtensorMap e;    // e [R, d_mem], boxes of 128 rows x 64
+  CUtensorMap wk;   // W_K [M d, d_mem], boxes of 128 rows x 64
+  CUtensorMap wv;   // W_V [d, d_mem], boxes of 64 rows x 64
+  CUtensorMap h;    // h [R, M d], boxes of 128 rows x 32
+  CUtensorMap out;  // out [R, M d], boxes of 32 rows x 32
+};
+cudaError_t launch_proj_gate_fused(const FusedMaps& maps, const GateArgs& g, int nkey, int nval,
+                                   cudaStream_t stream);
+// Clusters of the fused kernel that can be resident at once on this device (0
+// if unknown).
+int fused_max_clusters();
 
 // Dense contractions of the backward (bf16 operands, fp32 accumulation):
 // D[m, n] (= or +=) sum_k A(m, k) B(n, k), m < M, n < N, k < K.  A K-major A

@@ -376,6 +376,16 @@ __device__ __forceinline__ void sum_partials(const float4* partials, int64_t R, 
   }
 }
 
+// alpha of one row and branch from its sums over the d columns: sum k^2,
+// sum (h w_q w_k) k and sum h^2 (RMSNorm of h and k, their dot product over
+// sqrt(d), sigmoid).
+__device__ __forceinline__ float alpha_from_sums(float skk, float shk, float shh, int d, float eps,
+                                                 float inv_sqrt_d) {
+  const float rh = 1.0f / sqrtf(shh / (float)d + eps);
+  const float rk = 1.0f / sqrtf(skk / (float)d + eps);
+  return sigmoid_f(shk * rh * rk * inv_sqrt_d);
+}
+
 // alpha of branch mb of one row (Eq. 4 / Eq. 6) from the key phase's
 // per-tile partial sums: the same arithmetic, in the same order, wherever it
 // is formed.
@@ -386,9 +396,7 @@ __device__ __forceinline__ float row_alpha(const float4* partials, int64_t R, in
   float skk = 0.f, shk = 0.f, shh = 0.f;
   sum_partials<kBatch>(partials, R, row, mb * tiles_per_branch, (mb + 1) * tiles_per_branch, skk,
                        shk, shh);
-  const float rh = 1.0f / sqrtf(shh / (float)d + eps);
-  const float rk = 1.0f / sqrtf(skk / (float)d + eps);
-  return sigmoid_f(shk * rh * rk * inv_sqrt_d);
+  return alpha_from_sums(skk, shk, shh, d, eps, inv_sqrt_d);
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {

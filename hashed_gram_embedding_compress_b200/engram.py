@@ -24,6 +24,7 @@ ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT, ENGRAM_ERR_UNSUPPORTED, ENGRAM_ERR_STATE = 4
 MAX_ORDERS, MAX_TABLES, MAX_BRANCHES, MAX_SHARDS = 4, 64, 4, 8
 IPC_HANDLE_BYTES = 64
 ENGRAM_FLAG_NO_CTA_PAIRS = 1
+ENGRAM_FLAG_NO_FUSED_SHORT = 2
 ENGRAM_PREFETCH_HOST_THREADS, ENGRAM_PREFETCH_ZERO_COPY = 0, 1
 
 #: every symbol include/engram.h declares

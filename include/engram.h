@@ -66,6 +66,7 @@ extern "C" {
 
 /* config flags */
 #define ENGRAM_FLAG_NO_CTA_PAIRS 1 /* bf16 projection on single-CTA tiles only */
+#define ENGRAM_FLAG_NO_FUSED_SHORT 2 /* short calls: separate key, alpha and value launches */
 
 /* how engram_prefetch moves rows from host tables (engram_set_prefetch) */
 #define ENGRAM_PREFETCH_HOST_THREADS 0 /* host threads + copy engines (default) */
@@ -115,9 +116,13 @@ typedef struct engram_handle engram_handle;
  *                  out.  Accumulation is always fp32.
  *  eps             RMSNorm epsilon (the pages give none; 1e-6 is typical).
  *  table_location  ENGRAM_DEVICE or ENGRAM_PINNED_HOST.
- *  flags           0, or ENGRAM_FLAG_NO_CTA_PAIRS to keep the bf16 projection
- *                  on single-CTA 128-row tiles (by default 512 x 256 tiles on
- *                  CTA pairs are used when they fill the GPU).  Both give the
+ *  flags           0, or an OR of: ENGRAM_FLAG_NO_CTA_PAIRS to keep the bf16
+ *                  projection on single-CTA 128-row tiles (by default 512 x
+ *                  256 tiles on CTA pairs are used when they fill the GPU);
+ *                  ENGRAM_FLAG_NO_FUSED_SHORT to run calls of at most 256 rows
+ *                  as separate key, alpha and value launches (by default one
+ *                  launch does all three when d is a multiple of 256, M <= 4
+ *                  and its CTAs fit on the GPU at once).  All choices give the
  *                  same results up to fp32 summation order.
  */
 typedef struct engram_config {

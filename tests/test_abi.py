@@ -69,7 +69,7 @@ def _cfg(eg, **kw):
     (dict(primes=[101, 1, 103, 107]), "table sizes"),
     (dict(comp_map=torch.arange(100)), "comp_map"),
     (dict(pad_id=-2), "pad_id"),
-    (dict(flags=2), "unknown flags"),
+    (dict(flags=4), "unknown flags"),
 ])
 def test_invalid_configs_rejected_before_any_cuda_call(eg, kw, msg):
     cfg = _cfg(eg, **kw)
