@@ -102,7 +102,7 @@ struct GateArgs {
   // one launch for steps 5-7 of a short call (launch_proj_gate_fused): [0],
   // [1] key CTAs done per 128-row half, [2] CTAs done; zero between launches
   unsigned* sync;
-  float* vt;            // fused short-call kernel: v handed to the key CTAs, [d / 4][256][4]
+  float* vt;            // fused short-call kernel: v handed to the key CTAs, [2 row halves][d / 4][128][4]
   // 1: launch with programmatic dependent launch.  The key phase then waits
   // for the previous kernel (the gather) before reading e and lets the value
   // phase start early; the value phase's epilogue waits for the key phase

@@ -26,7 +26,8 @@
 //                               global memory, stored by TMA per warp.
 //   clusters [nkey, nkey+nval)  value tiles: 128 columns of v (nval = d / 128);
 //                               the epilogue writes v (fp32) to a scratch laid
-//                               out [d / 4][256 rows][4], counts itself done on
+//                               out [2 row halves][d / 4][128 rows][4], counts
+//                               itself done on
 //                               its row half's counter and leaves.
 // Only the key CTAs touch h: each reads and writes its own block, so the
 // in-place update (out aliasing h) needs no ordering between CTAs.  The value
@@ -80,7 +81,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = kEpiThreads + 3 * 32;         // 352
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1, kHWarp = kEpiWarps + 2;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;  // k (or v) and, in key CTAs, h w_q w_k
 constexpr int NQ = (kKeyCols / 2) / H_COLS;            // 32-column chunks per key epilogue warp
 constexpr int kSegBatch = 20;                          // partial-sum loads in flight per row
 constexpr int NUM_BARS = 2 * STAGES + 5;
@@ -326,10 +327,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           // generic-proxy writes of other CTAs, read by bulk copies
           asm volatile("fence.proxy.async.global;" ::: "memory");
+          // the block is contiguous in the [2][d / 4][128][4] layout: four copies
           mbar_expect_tx(vfull_bar, VT_CHUNKS * VT_CHUNK);
-          const float* src = g.vt + ((int64_t)(j0 / 4) * (2 * kRows) + row0) * 4;
-          for (int c = 0; c < VT_CHUNKS; ++c)
-            bulk_load(sA + c * VT_CHUNK, src + (int64_t)c * (2 * kRows) * 4, VT_CHUNK, vfull_bar);
+          const float* src = g.vt + (int64_t)((int)rank * (d / 4) + j0 / 4) * kRows * 4;
+          constexpr uint32_t kPart = VT_CHUNKS * VT_CHUNK / 4;
+          for (int c = 0; c < 4; ++c)
+            bulk_load(sA + c * kPart, src + (int64_t)c * (kPart / 4), kPart, vfull_bar);
           wait_drain(vfull_bar, 0);
         }
         wait_drain(hfull_bar, 0);  // no copy of this CTA is in flight when it leaves
@@ -346,24 +349,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool valid = row < R;
     const bool rows_in = row0 + quarter * 32 < R;  // this warp has a row inside R
     bool ok = true;
-    if (lane == 0) ok = wait_ready(tfull_bar, 0, abort_flag, g.err);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
     if (key) {
-      if (lane == 0 && ok) ok = wait_ready(hfull_bar, 0, abort_flag, g.err);
+      if (lane == 0) ok = wait_ready(hfull_bar, 0, abort_flag, g.err);
       ok = __shfl_sync(0xffffffffu, ok, 0);
+      float skk = 0.f, shk = 0.f, shh = 0.f;
+      // this warp's TMEM lanes: columns [0, 256) hold k, [256, 512) h w_q w_k
+      const uint32_t tl = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t tk = tl + (uint32_t)(half * (kKeyCols / 2));
+      const uint32_t thw = tl + (uint32_t)(kKeyCols + half * (kKeyCols / 2));
       if (ok) {
-        tc_fence_after();
-        const uint32_t taddr =
-            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * (kKeyCols / 2));
+        // while the MMAs run: h w_q w_k of this row's 128 columns into TMEM,
+        // and the row's sum of h^2 (both in the pair kernel's order).  Chunk
+        // q: columns 128 half + 32 q of the tile, h box 4 half + q.
         const float* wcol = wbuf + half * (kKeyCols / 2);
-        float skk = 0.f, shk = 0.f, shh = 0.f;
-        uint32_t va[32], vb[32];
-        // chunk q: columns 128 half + 32 q of the tile, h box 4 half + q; the
-        // next chunk's TMEM load is in flight while this one is used
-        auto key_chunk = [&](int q, uint32_t(&v)[32], uint32_t(&vn)[32]) {
-          tmem_wait32(v);
-          __syncwarp();
-          if (q + 1 < NQ) tmem_ld32_async(taddr + (q + 1) * H_COLS, vn);
+#pragma unroll 1
+        for (int q = 0; q < NQ; ++q) {
           const uint8_t* hs = khbuf + (half * NQ + q) * KH_BOX;
           const float4* wp = reinterpret_cast<const float4*>(wcol + q * H_COLS);
           uint4 hu[4];
@@ -372,8 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 4; ++c) hu[c] = *reinterpret_cast<const uint4*>(hs + sw64_off(r, c));
 #pragma unroll
           for (int c = 0; c < 8; ++c) wv[c] = wp[c];
-          // packed fp32 pairs, two accumulators per sum (the pair kernel's order)
-          unsigned long long akk[2] = {0ull, 0ull}, ahh[2] = {0ull, 0ull}, ahk[2] = {0ull, 0ull};
+          unsigned long long ahh[2] = {0ull, 0ull};
+          uint32_t hwv[32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint32_t hw[4] = {hu[c].x, hu[c].y, hu[c].z, hu[c].w};
@@ -381,29 +381,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 4; ++j) {
               const int e = c * 8 + 2 * j;  // elements e, e+1 of the chunk
               const unsigned long long h2 = bf16x2_to_f2(hw[j]);
-              const unsigned long long k2 = f2_pack(v[e], v[e + 1]);
               const float4 wq = wv[e / 4];
               const unsigned long long w2 =
                   (j & 1) ? f2_pack(__float_as_uint(wq.z), __float_as_uint(wq.w))
                           : f2_pack(__float_as_uint(wq.x), __float_as_uint(wq.y));
-              akk[j & 1] = f2_fma(k2, k2, akk[j & 1]);
               ahh[j & 1] = f2_fma(h2, h2, ahh[j & 1]);
-              ahk[j & 1] = f2_fma(f2_mul(h2, w2), k2, ahk[j & 1]);
+              const float2 p = f2_unpack(f2_mul(h2, w2));
+              hwv[e] = __float_as_uint(p.x);
+              hwv[e + 1] = __float_as_uint(p.y);
             }
           }
-          const float2 kk0 = f2_unpack(akk[0]), kk1 = f2_unpack(akk[1]);
           const float2 hh0 = f2_unpack(ahh[0]), hh1 = f2_unpack(ahh[1]);
+          shh += (hh0.x + hh0.y) + (hh1.x + hh1.y);
+          __syncwarp();
+          tmem_st32(thw + q * H_COLS, hwv);
+        }
+        tmem_wait_st();
+      }
+      if (lane == 0 && ok) ok = wait_ready(tfull_bar, 0, abort_flag, g.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) {
+        tc_fence_after();
+        // sum k^2 and sum (h w_q w_k) k: packed fp32 pairs, two accumulators
+        // per sum, chunk sums added in order (the pair kernel's arithmetic)
+        uint32_t kv[32], hv[32];
+#pragma unroll 1
+        for (int q = 0; q < NQ; ++q) {
+          __syncwarp();
+          tmem_ld32_async(tk + q * H_COLS, kv);
+          tmem_ld32_async(thw + q * H_COLS, hv);
+          tmem_wait32(kv);
+          tmem_wait32(hv);
+          unsigned long long akk[2] = {0ull, 0ull}, ahk[2] = {0ull, 0ull};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int e = c * 8 + 2 * j;
+              const unsigned long long k2 = f2_pack(kv[e], kv[e + 1]);
+              akk[j & 1] = f2_fma(k2, k2, akk[j & 1]);
+              ahk[j & 1] = f2_fma(f2_pack(hv[e], hv[e + 1]), k2, ahk[j & 1]);
+            }
+          const float2 kk0 = f2_unpack(akk[0]), kk1 = f2_unpack(akk[1]);
           const float2 hk0 = f2_unpack(ahk[0]), hk1 = f2_unpack(ahk[1]);
           skk += (kk0.x + kk0.y) + (kk1.x + kk1.y);
-          shh += (hh0.x + hh0.y) + (hh1.x + hh1.y);
           shk += (hk0.x + hk0.y) + (hk1.x + hk1.y);
-        };
-        __syncwarp();
-        tmem_ld32_async(taddr, va);
-#pragma unroll 1
-        for (int q = 0; q < NQ; q += 2) {
-          key_chunk(q, va, vb);
-          key_chunk(q + 1, vb, va);
         }
         // segment (tile, half) of the [M d / 128][R] partial sums
         if (valid)
@@ -473,7 +495,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else {
       // v of this CTA's 128 rows and 64 columns (column half `half` of the
-      // tile) into the [d / 4][256][4] scratch, then count this CTA done
+      // tile) into the [2][d / 4][128][4] scratch, then count this CTA done
+      if (lane == 0) ok = wait_ready(tfull_bar, 0, abort_flag, g.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok) {
         tc_fence_after();
         const uint32_t taddr =
@@ -485,12 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait32(va);
         tmem_wait32(vb);
         if (valid) {
-          float4* vt = reinterpret_cast<float4*>(g.vt) + (int64_t)((n0 + half * 64) / 4) * (2 * kRows) + row;
+          float4* vt = reinterpret_cast<float4*>(g.vt) +
+                       (int64_t)((int)rank * (d / 4) + (n0 + half * 64) / 4) * kRows + r;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const uint32_t* v = c < 8 ? va : vb;
             const int e = (c & 7) * 4;
-            vt[(int64_t)c * (2 * kRows)] =
+            vt[(int64_t)c * kRows] =
                 make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                             __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
