@@ -430,6 +430,9 @@ def run_ours(args, rank, world, dist):
     gemm_s = (st_mean[2] + st_mean[3]) / 1e3
     gemm_tflops = A["gemm_flops"] / gemm_s / 1e12
     fused = sh.table_location == "device"  # one hash + gather kernel: its time is stage 1
+    # calls of at most 256 rows: keys, alpha and values in one launch (stage 2)
+    short_fused = (sh.rows_out <= 256 and sh.dtype == "bf16" and sh.d_hidden % 256 == 0
+                   and sh.branches <= 4 and not args.fp8 and not args.short_conv)
     gather_s = (st_mean[0] + st_mean[1] if fused else st_mean[1]) / 1e3
     gather_gbs = A["gather_bytes"] / gather_s / 1e9
     # the DRAM bytes the fused kernel moves in the step (row over-fetch and the
@@ -462,7 +465,9 @@ def run_ours(args, rank, world, dist):
             "cuda_graph": bool(graph is not None),
         },
         "roofline": {
-            "kernel": ("proj_gate_pair_kernel (keys, 256 x 256 CTA-pair tiles) + row_alpha_kernel "
+            "kernel": ("proj_gate_fused_kernel: keys, alpha and values in one launch (256 x 256 "
+                       "key and 256 x 128 value CTA-pair tiles, tcgen05)" if short_fused else
+                       "proj_gate_pair_kernel (keys, 256 x 256 CTA-pair tiles) + row_alpha_kernel "
                        "+ proj_gate_kernel (values, 128 x 64 single-CTA tiles), tcgen05"
                        if sh.rows_out <= 4096 else
                        "proj_gate_wide_kernel: key + in-place value launches per step (tcgen05, "
@@ -493,7 +498,8 @@ def run_ours(args, rank, world, dist):
         },
         "stages_ms": ({"hash_gather": st_mean[0] + st_mean[1]} if fused else
                       {"hash": st_mean[0], "gather": st_mean[1]}) |
-                     {"key_proj_gate": st_mean[2], "value_proj_gate": st_mean[3]} |
+                     ({"proj_gate": st_mean[2] + st_mean[3]} if short_fused else
+                      {"key_proj_gate": st_mean[2], "value_proj_gate": st_mean[3]}) |
                      ({"short_conv": st_mean[4]} if args.short_conv else {}),
         "e2e": {
             "value": tokens_per_step * world * E / (e2e_ms / 1e3),
