@@ -48,7 +48,7 @@
 // Roles (352 threads per CTA):
 //   warps 0-7   epilogue: warp w owns TMEM lanes 32 (w % 4).. (tile rows) and
 //               column half w / 4 of the tile;
-//   warp 8      TMA producer of e and W (5 stages x 32 KB);
+//   warp 8      TMA producer of e and W (4 stages x 32 KB);
 //   warp 9      TMEM allocator; MMA issuer on the leader (rank 0);
 //   warp 10     key CTAs: loads of the h block and its column weights
 //               w_q * w_k, then (after the mainloop, into the free stage
@@ -68,8 +68,8 @@ constexpr int BK = 64;
 constexpr uint32_t A_BYTES = kRows * BK * 2;           // 16 KB
 constexpr uint32_t KB_BYTES = (kKeyCols / 2) * BK * 2; // 16 KB: a key CTA's half of B
 constexpr uint32_t VB_BYTES = (kValCols / 2) * BK * 2; // 8 KB: a value CTA's half of B
-constexpr int STAGES = 5;
-constexpr uint32_t STAGE_REGION = STAGES * (A_BYTES + KB_BYTES);  // 160 KB
+constexpr int STAGES = 4;
+constexpr uint32_t STAGE_REGION = STAGES * (A_BYTES + KB_BYTES);  // 128 KB
 constexpr int H_COLS = 32;
 constexpr uint32_t KH_BOX = kRows * H_COLS * 2;        // 8 KB: 128 rows x 32 columns
 constexpr int KH_BOXES = kKeyCols / H_COLS;            // 8
