@@ -73,6 +73,10 @@ def parse():
                          "of h, W_K, W_V, the RMSNorm weights and the tables for a seeded dL/dout")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a captured CUDA graph (launch-bound shapes)")
+    ap.add_argument("--graph-steps", type=int, default=1,
+                    help="with --graph: consecutive steps captured in one graph (the launches of "
+                         "one step then overlap the next step's, as in eager calls); --steps "
+                         "must be a multiple of it")
     ap.add_argument("--offload-gb", type=float, default=100.0,
                     help="offload workload: total size of the pinned host tables")
     ap.add_argument("--hot-rows", type=int, default=0,
@@ -307,17 +311,22 @@ def run_ours(args, rank, world, dist):
         m.forward(tok_d, h, h, t_begin=sh.t_begin, stream=torch.cuda.current_stream())
 
     graph = None
+    G = max(1, args.graph_steps) if args.graph else 1
     if args.graph:
+        if args.steps % G:
+            raise SystemExit("--steps must be a multiple of --graph-steps")
         forward_once()
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         n0 = m.kernel_launches()
         with torch.cuda.graph(graph):
-            forward_once()
+            for _ in range(G):
+                forward_once()
         per_replay = m.kernel_launches() - n0  # kernels each replay launches
         torch.cuda.synchronize()
 
     def step():
+        # one replay covers G steps (G = 1 without a graph)
         if graph is not None:
             graph.replay()
         else:
@@ -351,14 +360,14 @@ def run_ours(args, rank, world, dist):
     # would serialise the launches that otherwise overlap (the key launch
     # starts during the gather, the value launch during the key launch)
     t0.record(stream)
-    for k in range(K):
+    for k in range(K // G):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
     t_end = time.monotonic()
     launches = m.kernel_launches() - launches0
     if graph is not None:
-        launches = per_replay * K  # replays do not pass through the library's counter
+        launches = per_replay * (K // G)  # replays do not pass through the library's counter
     # stage times: the same steps again, each with events between its launches
     if graph is None:
         for k in range(K):
@@ -463,6 +472,7 @@ def run_ours(args, rank, world, dist):
                      sum(t.numel() * t.element_size() for t in P["tables"]) / 1e9),
             "residual": "in place: out aliases h (H <- H + alpha v)",
             "cuda_graph": bool(graph is not None),
+            "graph_steps": G if graph is not None else None,
         },
         "roofline": {
             "kernel": ("proj_gate_fused_kernel: keys, alpha and values in one launch (256 x 256 "
