@@ -137,3 +137,20 @@ def test_in_place_steps_match_repeated_out_of_place_updates():
     torch.cuda.synchronize()
     assert m.check_errors() == 0
     assert torch.equal(h_in, cur)
+
+
+@pytest.mark.parametrize("B,T,t_begin,M,d,flags,launches", [
+    (257, 3, 2, 2, 256, 0, 4),    # 257 rows: more than one 256-row block
+    (64, 3, 2, 2, 384, 0, 4),     # d not a multiple of 256
+    (64, 3, 2, 2, 256, 2, 4),     # ENGRAM_FLAG_NO_FUSED_SHORT
+    (64, 3, 2, 2, 256, 1, 4),     # ENGRAM_FLAG_NO_CTA_PAIRS
+    (256, 3, 2, 4, 512, 0, 2),    # taken
+])
+def test_which_calls_take_the_one_launch_path(B, T, t_begin, M, d, flags, launches):
+    sh = synth.SHAPES["decode_mb"].replace(B=B, T=T, t_begin=t_begin, branches=M, d_hidden=d,
+                                           rows_target=1031)
+    p = Problem(sh)
+    m = p.engram(flags=flags)
+    out, a, dl, n = _forward(p, m)
+    assert n == launches
+    _check_oracle(p, p.sample_rows(48), out, a, dl)
