@@ -547,7 +547,10 @@ def run_ours(args, rank, world, dist):
     if args.rows_target:
         res["config"]["workload"] += " [profiling variant: tables of %d rows]" % args.rows_target
     if args.workload != "prefill_bf16":
-        res["roofline"]["traffic"] = None  # the committed capture is of the prefill shapes
+        # the committed captures: the prefill shapes, and the decode workload's one launch
+        res["roofline"]["traffic"] = (
+            kernel_traffic("traffic_decode.json", "dram_bytes_per_launch")
+            if args.workload == "decode_mb" and short_fused and not args.rows_target else None)
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(P, args.cpu_seconds)
     return res
