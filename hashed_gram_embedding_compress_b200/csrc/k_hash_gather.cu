@@ -188,6 +188,11 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
   const uint32_t nchunks = nslots * cpr;
   // row0 * S * row_bytes < 2^31 * 16 by the launcher's bound
   uint4* dst = reinterpret_cast<uint4*>((char*)g.e + (int64_t)row0 * S * g.row_bytes);
+  // e is written evict-last (the projection launches read it next, with the
+  // same policy), the table rows, read once, evict-first
+  uint64_t keep, once;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(once));
   constexpr int kInFlight = 4;
   for (uint32_t i0 = threadIdx.x; i0 < nchunks; i0 += kInFlight * kFusedThreads) {
     uint4 v[kInFlight];
@@ -196,13 +201,18 @@ __global__ void __launch_bounds__(kFusedThreads) hash_gather_kernel(HashGatherAr
       const uint32_t i = i0 + k * kFusedThreads;
       if (i < nchunks) {
         const uint32_t rs = i / cpr;
-        v[k] = ld_stream_16(s_src[rs] + (i - rs * cpr) * 16);
+        asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                     : "=r"(v[k].x), "=r"(v[k].y), "=r"(v[k].z), "=r"(v[k].w)
+                     : "l"(s_src[rs] + (i - rs * cpr) * 16), "l"(once));
       }
     }
 #pragma unroll
     for (int k = 0; k < kInFlight; ++k) {
       const uint32_t i = i0 + k * kFusedThreads;
-      if (i < nchunks) dst[i] = v[k];
+      if (i < nchunks)
+        asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(dst + i),
+                     "r"(v[k].x), "r"(v[k].y), "r"(v[k].z), "r"(v[k].w), "l"(keep)
+                     : "memory");
     }
   }
   // the previous kernel (which this one may have overlapped) is complete

@@ -208,6 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       griddep_wait();
       griddep_launch_dependents();
     }
+    // e (written by the gather with the same policy, read by about ten CTA
+    // pairs per launch and by both launches) is kept in L2 over the streamed h
+    const uint64_t e_policy = policy_evict_last();
     for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
       const int m_blk = tile / num_n, n_blk = tile - m_blk * num_n;
       const int a_row = m_blk * 2 * kRows + (int)rank * kRows;
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the leader's full barrier counts the bytes of both CTAs
           const uint32_t fb = peer_addr(full_bar(stage), 0);
           if (!early && leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          tma_load_2d_pair(sA + stage * A_BYTES, &map_e, fb, kb * BK, a_row);
+          tma_load_2d_pair_hint(sA + stage * A_BYTES, &map_e, fb, kb * BK, a_row, e_policy);
           if (!early) tma_load_2d_pair(sB + stage * B_BYTES, &map_w, fb, kb * BK, b_row);
         }
         __syncwarp();
