@@ -12,7 +12,10 @@
 // owns rows [128 r, 128 r + 128) of the call), one tile per cluster:
 //   clusters [0, nkey)          key tiles: 256 columns [j0, j0 + 256) of
 //                               branch mb (nkey = M d / 256).  The CTA loads
-//                               its 128 x 256 block of h^(mb) at the start.
+//                               its 128 x 256 block of h^(mb) at the start;
+//                               while its MMAs run, the epilogue warps form
+//                               h w_q w_k into the spare TMEM columns and the
+//                               rows' sums of h^2.
 //                               Epilogue: the per-row partial sums of Eq. (4)
 //                               of each 128-column half tile (the arithmetic
 //                               of the 256 x 256 pair kernel's key phase),
@@ -26,9 +29,10 @@
 //                               global memory, stored by TMA per warp.
 //   clusters [nkey, nkey+nval)  value tiles: 128 columns of v (nval = d / 128);
 //                               the epilogue writes v (fp32) to a scratch laid
-//                               out [2 row halves][d / 4][128 rows][4], counts
-//                               itself done on
-//                               its row half's counter and leaves.
+//                               out [2 row halves][d / 4][128 rows][4] (a key
+//                               CTA's block of v is then contiguous), counts
+//                               itself done on its row half's counter and
+//                               leaves.
 // Only the key CTAs touch h: each reads and writes its own block, so the
 // in-place update (out aliasing h) needs no ordering between CTAs.  The value
 // CTAs' mainloops run beside the key CTAs'; the step costs one mainloop, one
