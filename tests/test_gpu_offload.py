@@ -227,3 +227,41 @@ def test_offload_workload_shapes_against_the_oracle():
     md.forward(tok[1], p.h, ref)
     torch.cuda.synchronize()
     assert torch.equal(outs["host_threads"][1][0], ref)
+
+
+@pytest.mark.parametrize("route", ROUTES[::2])
+def test_prefetch_then_short_multibranch_call(route):
+    """A decode-sized call (256 rows, four branches) on host tables: the rows
+    come through the prefetch staging, then keys, alpha and values run in one
+    launch; results equal the device-resident tables' bit for bit, in place."""
+    from hashed_gram_embedding_compress_b200 import engram as eg
+    sh = synth.SHAPES["decode_mb"].replace(rows_target=1 << 16, d_hidden=512)
+    p, dev_tables = _pair(sh)
+    m = p.engram()
+    m.set_prefetch(*route)
+    md = eg.Engram(eg.make_config(vocab=sh.vocab, cvocab=sh.cvocab, comp_map=p.comp_map,
+                                  orders=sh.orders, heads=sh.heads, d_head=sh.d_head,
+                                  d_hidden=sh.d_hidden, branches=sh.branches, dtype=sh.dtype,
+                                  table_rows_target=sh.rows_target, hash_seed=p.hash_seed))
+    md.set_params(dev_tables, p.w_k, p.w_v, p.norm_q, p.norm_k)
+    tok = p.tokens.cuda()
+    R, M = sh.rows_out, sh.branches
+    ref = p.h.clone()
+    a_ref = torch.empty((R, M), device="cuda")
+    n0 = md.kernel_launches()
+    md.forward(tok, ref, ref, t_begin=sh.t_begin, alpha=a_ref)
+    assert md.kernel_launches() - n0 == 2  # the gather, then the one-launch projections
+
+    side = torch.cuda.Stream()
+    m.prefetch(tok, t_begin=sh.t_begin, stream=side)
+    out = p.h.clone()
+    alpha = torch.empty((R, M), device="cuda")
+    m.forward(tok, out, out, t_begin=sh.t_begin, alpha=alpha)
+    torch.cuda.synchronize()
+    assert m.check_errors() == 0 and md.check_errors() == 0
+    assert torch.equal(out, ref) and torch.equal(alpha, a_ref)
+    rows = p.sample_rows(32)
+    _, a_o, _, o_o = p.oracle_forward(rows)
+    rs = torch.from_numpy(rows).cuda()
+    assert rel_l2(alpha[rs].double().cpu(), a_o) <= 1e-3
+    assert out_close(to_oracle(out[rs]), o_o, "bf16") <= 1e-3
