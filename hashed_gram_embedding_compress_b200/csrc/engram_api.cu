@@ -1578,9 +1578,14 @@ int64_t engram_kernel_launches(const engram_handle* h) { return h ? h->launches 
 
 int engram_selftest_timeout(engram_handle* h, void* stream) {
   if (!h) return ENGRAM_ERR_INVALID;
-  CK(h, launch_wait_timeout_selftest(h->d_err, (cudaStream_t)stream));
-  h->launches += 1;
-  return engram_check_errors(h, stream);
+  // both kinds of bounded wait: an mbarrier, then a count in global memory
+  for (int which = 0; which < 2; ++which) {
+    CK(h, launch_wait_timeout_selftest(h->d_err, which, (cudaStream_t)stream));
+    h->launches += 1;
+    const int rc = engram_check_errors(h, stream);
+    if (rc != ENGRAM_ERR_TIMEOUT) return rc;  // ENGRAM_OK: the wait did not expire
+  }
+  return fail(h, ENGRAM_ERR_TIMEOUT, "both bounded waits expired and were reported");
 }
 
 int engram_check_errors(engram_handle* h, void* stream) {

@@ -225,7 +225,7 @@ cudaError_t launch_prefetch_index(const PrefetchArgs& a, cudaStream_t stream);
 // Step 5 by zero-copy loads: the count[0] rows of the host tables listed at
 // the front of uniq, on a.fetch_blocks CTAs.
 cudaError_t launch_prefetch_fetch(const PrefetchArgs& a, cudaStream_t stream);
-cudaError_t launch_wait_timeout_selftest(unsigned* err, cudaStream_t stream);
+cudaError_t launch_wait_timeout_selftest(unsigned* err, int which, cudaStream_t stream);
 cudaError_t launch_mul(const float* x, const float* y, float* out, int64_t n, cudaStream_t stream);
 
 // fp32 path (SIMT FFMA; 64-column tiles).  phase 0 = key tiles over W_K

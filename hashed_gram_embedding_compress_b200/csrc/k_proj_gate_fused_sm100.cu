@@ -58,6 +58,7 @@
 //               w_q * w_k, then (after the mainloop, into the free stage
 //               buffers) of the v block once the value CTAs are done.
 #include "sm100_ptx.cuh"
+#include "sm100_wait.cuh"
 
 namespace engram {
 
@@ -102,29 +103,6 @@ constexpr int kVCount = 2 * kMaxBranches, kExit = kVCount + 2;
 
 __device__ __forceinline__ void epi_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-}
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Wait until *p >= target, for at most kWaitLimitNs (then raise the CTA's
-// abort flag and kDevErrTimeout).
-static __device__ __noinline__ bool wait_count(const unsigned* p, unsigned target,
-                                               volatile int* abort_flag, unsigned* err) {
-  const uint64_t t0 = globaltimer();
-  while (ld_acquire_u32(p) < target) {
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicOr(err, kDevErrTimeout);
-      return false;
-    }
-    __nanosleep(32);
-  }
-  return true;
 }
 
 // Count this CTA done on *p once the epilogue warps' global writes before the

@@ -520,11 +520,14 @@ ENGRAM_API int engram_profile_next_backward(engram_handle *h, void *const *event
 
 /*
  * Self-test of device-side failure detection.  Launches on `stream` a one-CTA
- * kernel that waits on an mbarrier no thread ever arrives at, with the same
- * bounded wait the tensor-core kernels use (limit 2 s): the wait expires, the
- * kernel records a timeout in the device error word and returns normally.
- * Then behaves as engram_check_errors, so it returns ENGRAM_ERR_TIMEOUT when
- * the mechanism works; the handle and the CUDA context remain usable.
+ * kernel that waits on an mbarrier no thread ever arrives at, then one that
+ * waits on a count in global memory that never reaches its target, with the
+ * same bounded waits the tensor-core kernels use (limit 2 s each): each wait
+ * expires, the kernel records a timeout in the device error word and returns
+ * normally, and the word is read and cleared as engram_check_errors does.
+ * Returns ENGRAM_ERR_TIMEOUT when both waits expired and were reported (the
+ * mechanism works), ENGRAM_OK if one of them was not; the handle and the CUDA
+ * context remain usable.
  */
 ENGRAM_API int engram_selftest_timeout(engram_handle *h, void *stream);
 

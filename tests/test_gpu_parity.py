@@ -287,8 +287,10 @@ def test_out_of_range_tokens_are_reported_not_read():
 
 
 def test_bounded_wait_expiry_is_reported_and_context_survives():
-    # a kernel waits on an mbarrier nothing arrives at: the bounded wait
-    # expires (2 s), the timeout is reported, and the next forward is exact
+    # a kernel waits on an mbarrier nothing arrives at, another on a count in
+    # global memory that never reaches its target (the one-launch short-call
+    # kernel's wait): each bounded wait expires (2 s), each timeout is
+    # reported, and the next forward is exact
     from hashed_gram_embedding_compress_b200 import engram as eg
     sh = synth.SHAPES["tiny_f32"]
     p = Problem(sh)
