@@ -73,10 +73,11 @@ def parse():
                          "of h, W_K, W_V, the RMSNorm weights and the tables for a seeded dL/dout")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a captured CUDA graph (launch-bound shapes)")
-    ap.add_argument("--graph-steps", type=int, default=1,
+    ap.add_argument("--graph-steps", type=int, default=None,
                     help="with --graph: consecutive steps captured in one graph (the launches of "
                          "one step then overlap the next step's, as in eager calls); --steps "
-                         "must be a multiple of it")
+                         "must be a multiple of it (default: the largest of 8, 4, 2, 1 that "
+                         "divides --steps)")
     ap.add_argument("--offload-gb", type=float, default=100.0,
                     help="offload workload: total size of the pinned host tables")
     ap.add_argument("--hot-rows", type=int, default=0,
@@ -311,7 +312,10 @@ def run_ours(args, rank, world, dist):
         m.forward(tok_d, h, h, t_begin=sh.t_begin, stream=torch.cuda.current_stream())
 
     graph = None
-    G = max(1, args.graph_steps) if args.graph else 1
+    G = 1
+    if args.graph:
+        G = (max(1, args.graph_steps) if args.graph_steps
+             else next(g for g in (8, 4, 2, 1) if args.steps % g == 0))
     if args.graph:
         if args.steps % G:
             raise SystemExit("--steps must be a multiple of --graph-steps")
