@@ -54,7 +54,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="steps of the end-to-end (host-buffer) measurement; default: enough "
+                         "for ~0.1 s, at least 10, from one untimed step's wall time")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -278,6 +280,24 @@ def kernel_traffic(name="traffic.json", key="proj_gate_bytes_per_step"):
     return d.get(key)
 
 
+def e2e_count(requested, step, dist, target_s=0.1, lo=10, hi=2000) -> int:
+    """Steps of an end-to-end measurement: as requested, else enough for about
+    target_s of work (at least lo), from one more untimed step's wall time; the
+    largest over ranks, so that every rank takes the same steps."""
+    import torch
+    if requested:
+        return max(1, requested)
+    t = time.monotonic()
+    step()
+    torch.cuda.synchronize()
+    n = int(min(hi, max(lo, target_s / max(time.monotonic() - t, 1e-6))))
+    if dist:
+        v = torch.tensor([n], device="cuda", dtype=torch.int64)
+        dist.all_reduce(v, op=dist.ReduceOp.MAX)
+        n = int(v.item())
+    return n
+
+
 def max_over_ranks(x: float, dist, device) -> float:
     """The largest value of x over all ranks (identity without a process group)."""
     if dist is None:
@@ -408,7 +428,6 @@ def run_ours(args, rank, world, dist):
     # through the host-buffer entry point: every step copies its tokens and h
     # from pinned host memory to the device and its out back (the library
     # overlaps one step's copies in with the previous step's copies out)
-    E = max(1, args.e2e_steps)
     tok_h = P["tokens"].pin_memory()
     h_h = h.cpu().pin_memory()
     out_h = torch.empty_like(h_h).pin_memory()
@@ -418,6 +437,7 @@ def run_ours(args, rank, world, dist):
 
     e2e_step()
     torch.cuda.synchronize()
+    E = e2e_count(args.e2e_steps, e2e_step, dist)
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -629,7 +649,6 @@ def run_backward_bench(args, rank, world, dist):
         raise RuntimeError("device error during the timed steps")
 
     # e2e: h and dL/dout in from pinned host memory, dh back, every step
-    E = max(1, args.e2e_steps)
     h_h, g_h = h.cpu().pin_memory(), dout.cpu().pin_memory()
     dh_h = torch.empty_like(h_h).pin_memory()
     tok_h = P["tokens"].pin_memory()
@@ -642,6 +661,7 @@ def run_backward_bench(args, rank, world, dist):
 
     e2e_step()
     torch.cuda.synchronize()
+    E = e2e_count(args.e2e_steps, e2e_step, dist)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(E):
