@@ -256,15 +256,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m_blk = tile / num_n, n0 = (tile - m_blk * num_n) * kCols;
       const int row0 = m_blk * 2 * kRows + (int)rank * kRows;
       // Bring this tile's h into L2 while its MMAs run: the boxes beyond the
-      // smem ring (keys, values) or all of them (values added in place, which
-      // read-modify-write h in L2 from the epilogue).  In place, pace by the
-      // accumulator: prefetch tile i once tile i-1's MMAs are done.
-      if (PHASE == 2 && tix > 0) {
+      // smem ring (keys, values) or, in place with one branch, all of them
+      // (the epilogue read-modify-writes h in L2), paced by the accumulator:
+      // tile i once tile i-1's MMAs are done.  In place with several branches
+      // the h of the tiles in flight (M x 128 KB per CTA) does not fit in L2
+      // beside e, the prefetched lines were evicted before the reduce-adds
+      // reached them and h came from DRAM twice: nothing is prefetched there.
+      const bool prefetch = PHASE != 3 && !(PHASE == 2 && M > 1);
+      if (PHASE == 2 && prefetch && tix > 0) {
         if (lane == 0) ok = wait_ready(tfull_bar, (uint32_t)(tix - 1) & 1u, abort_flag, g.err);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
       }
-      if (PHASE != 3 && lane == 0 && row0 < R) {
+      if (prefetch && lane == 0 && row0 < R) {
         for (int i = PHASE == 2 ? 0 : H_SLOTS; i < nbox; ++i)
           tma_prefetch_l2_2d(&map_h, PHASE == 0 ? n0 + H_COLS * i
                                                 : (i % M) * d + n0 + H_COLS * (i / M),
